@@ -1,0 +1,291 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU needed).
+
+Each test below checks the oracle against something the pages or the
+mathematics fix: the LFSR's maximal period, a block worked out by hand,
+closed-form sums over the full cycle, special inputs with a known answer,
+exact rational arithmetic, and brute-force recovery of a planted seed.
+A plausible slip anywhere in the oracle -- a dropped term, a wrong sign,
+offset, scale, index or bit order, a transposed product -- fails at least
+one of them.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from prng_seeded_decompress_b200 import inputs
+
+
+# ---------------------------------------------------------------- the LFSR
+
+def test_lfsr_maximal_period(oracle_mod):
+    # A 16-bit register with a primitive feedback polynomial (taps 16,14,13,11)
+    # walks through all 2^16 - 1 nonzero states before it repeats; zero is
+    # its fixed point.
+    seen = np.zeros(65536, dtype=bool)
+    st = oracle_mod.lfsr_states(1, 65536)
+    assert st[65535] == 1
+    seen[st[:65535]] = True
+    assert not seen[0] and seen[1:].all()
+    assert oracle_mod.lfsr_next(0) == 0
+
+
+def test_lfsr_is_a_right_shift_register(oracle_mod):
+    # The register shifts right by one; only bit 15 is new.
+    s = np.arange(65536)
+    nxt = np.array([oracle_mod.lfsr_next(int(v)) for v in range(0, 65536, 97)])
+    assert np.array_equal(nxt & 0x7FFF, s[::97] >> 1)
+
+
+def test_lfsr_hand_stepped_from_0xACE1(oracle_mod):
+    # Worked by hand: 0xACE1 = 1010 1100 1110 0001; feedback = b0^b2^b3^b5 =
+    # 1^0^0^1 = 0, so the next state is 0xACE1 >> 1 = 0x5670; then b0^b2^b3^b5
+    # of 0x5670 = 0^0^0^1 = 1 -> 0x2B38 | 0x8000 = 0xAB38; and so on.
+    expect = [0xACE1, 0x5670, 0xAB38, 0x559C, 0x2ACE, 0x1567, 0x8AB3, 0x4559]
+    assert oracle_mod.lfsr_states(0xACE1, 8).tolist() == expect
+
+
+# ------------------------------------------------- the basis U and Eq (1)
+
+# Seed 1 stepped by hand: the single set bit moves right one place per step
+# (1 -> 32768 -> 16384 ... -> 32) while bits 0, 2, 3, 5 are clear; at state 32
+# bit 5 is set, feedback 1, giving 16 | 32768 = 32784; and onwards.
+SEED1_STATES = [1, 32768, 16384, 8192, 4096, 2048, 1024, 512, 256, 128, 64, 32,
+                32784, 16392, 40964, 53250, 26625, 46080, 23040, 11520, 5760,
+                2880, 1440, 33488]
+
+
+def test_seed1_states_by_hand(oracle_mod):
+    assert oracle_mod.lfsr_states(1, 24).tolist() == SEED1_STATES
+
+
+def test_hand_worked_block_c8_p3(oracle_mod):
+    # C=8, P=3, seed 1, q = (3, -5, 7), e = 9.  U[c][p] = (state_{8p+c} -
+    # 32768)/32768 and t = q 2^-9, so W[c] 2^24 = sum_p (state_{8p+c} - 32768) q_p.
+    # By hand for c = 0: (1-32768)*3 + (256-32768)*(-5) + (26625-32768)*7 = 21258.
+    expect = [21258, 256384, 46272, -58784, -275152, -219496, -355508, -194138]
+    fmt = inputs.make_format(1, 8, 8, 3)
+    rec, ep = inputs.pack_records(fmt, [[1]], [[[3, -5, 7]]], [[9]])
+    W = oracle_mod.decompress(fmt, rec, ep)
+    assert (W[0] * 2.0 ** 24).tolist() == expect
+
+
+def test_basis_column_order(oracle_mod):
+    # Column p of U holds states pC .. pC+C-1 (not the row-major reading
+    # U[c][p] = state_{cP+p}).
+    U = oracle_mod.block_basis(1, 8, 3)
+    for p in range(3):
+        col = [(SEED1_STATES[8 * p + c] - 32768) / 32768 for c in range(8)]
+        assert U[:, p].tolist() == col
+
+
+def test_basis_full_cycle_sums(oracle_mod):
+    # Over all 65535 seeds, state_k runs through every nonzero 16-bit value
+    # exactly once, so each entry of U sums to sum_{v=1}^{65535}(v-32768)/32768
+    # = 0 and its squares to 2 * sum_{k=1}^{32767} k^2 / 2^30.  A wrong offset
+    # breaks the first, a wrong scale the second.
+    Uall = oracle_mod.basis_all(8, 3)
+    assert np.array_equal(Uall.sum(axis=0), np.zeros((8, 3)))
+    n = 32767
+    sq = 2 * (n * (n + 1) * (2 * n + 1) // 6) / 2.0 ** 30
+    assert np.allclose((Uall ** 2).sum(axis=0), sq, rtol=0, atol=1e-9)
+    # the 3-bit format's 12x4 basis reaches states up to 47 -- same sums
+    U3 = oracle_mod.basis_all(12, 4)
+    assert np.array_equal(U3.sum(axis=0), np.zeros((12, 4)))
+
+
+def test_basis_entries_are_never_plus_minus_one(oracle_mod):
+    Uall = oracle_mod.basis_all(8, 3)
+    assert Uall.max() == 32767 / 32768 and Uall.min() == -32767 / 32768
+
+
+# ------------------------------------------------------------ coefficients
+
+def test_zero_coefficients_give_zero_block(oracle_mod):
+    fmt = inputs.make_format(3, 24, 8, 3)
+    rng = np.random.default_rng(5)
+    seeds = rng.integers(1, 65536, size=(3, 3))
+    rec, ep = inputs.pack_records(fmt, seeds, np.zeros((3, 3, 3)), np.full((3, 3), 11))
+    assert not oracle_mod.decompress(fmt, rec, ep).any()
+
+
+def test_single_coefficient_is_a_scaled_window(oracle_mod):
+    # Only q_p nonzero: W_blk = q_p 2^-e (window_p - 32768)/32768.
+    fmt = inputs.make_format(1, 12, 12, 4)
+    st = oracle_mod.lfsr_states(4242, 48).astype(np.float64)
+    for p in range(4):
+        q = np.zeros((1, 1, 4), np.int64)
+        q[0, 0, p] = -7
+        rec, ep = inputs.pack_records(fmt, [[4242]], q, [[10]])
+        W = oracle_mod.decompress(fmt, rec, ep)[0]
+        assert np.array_equal(W, -7 * 2.0 ** -10 * (st[12 * p:12 * p + 12] - 32768) / 32768)
+
+
+def test_exponent_scales_by_powers_of_two(oracle_mod):
+    # t = q 2^-e: raising e by one halves every weight exactly.
+    fmt = inputs.make_format(1, 8, 8, 3)
+    ws = []
+    for e in (0, 1, 8, 15):
+        rec, ep = inputs.pack_records(fmt, [[999]], [[[5, -1, 2]]], [[e]])
+        ws.append((e, oracle_mod.decompress(fmt, rec, ep)[0]))
+    base = ws[0][1]
+    for e, w in ws[1:]:
+        assert np.array_equal(w * 2.0 ** e, base)
+
+
+def test_signed_coefficients_extremes(oracle_mod):
+    # q = -8 and q = 7 (the ends of two's-complement int4) against the basis.
+    fmt = inputs.make_format(1, 8, 8, 3)
+    rec, ep = inputs.pack_records(fmt, [[321]], [[[-8, 7, -8]]], [[12]])
+    U = oracle_mod.block_basis(321, 8, 3)
+    W = oracle_mod.decompress(fmt, rec, ep)[0]
+    assert np.array_equal(W, U @ np.array([-8.0, 7.0, -8.0]) * 2.0 ** -12)
+
+
+# ----------------------------------------------------------- record layout
+
+def test_record_layout_by_hand(oracle_mod):
+    # 4-bit format: seed 0xBEEF, q = (-1, 7, -8), e = 11:
+    # 0xBEEF << 16 | 0xF | 0x7 << 4 | 0x8 << 8 | 0xB << 12 = 0xBEEFB87F.
+    fmt = dict(C=8, P=3, K=16, rows=1, cols=8, nb=1, rec_pitch=4, e_pitch=0)
+    rec = np.array([[0xBEEFB87F, 0, 0, 0]], np.uint32)
+    s, q, e = oracle_mod.block_fields(fmt, rec, None, 0, 0)
+    assert (s, q.tolist(), e) == (0xBEEF, [-1, 7, -8], 11)
+    # 3-bit format: seed 0x1234, q = (1, -2, 3, -4) -> nibbles 1, E, 3, C;
+    # exponents 5 (block 0, low nibble) and 10 (block 1, high nibble) -> 0xA5.
+    fmt = dict(C=12, P=4, K=16, rows=1, cols=24, nb=2, rec_pitch=4, e_pitch=16)
+    rec = np.array([[0x1234C3E1, 0x00017777, 0, 0]], np.uint32)
+    ep = np.zeros((1, 16), np.uint8)
+    ep[0, 0] = 0xA5
+    s, q, e = oracle_mod.block_fields(fmt, rec, ep, 0, 0)
+    assert (s, q.tolist(), e) == (0x1234, [1, -2, 3, -4], 5)
+    s, q, e = oracle_mod.block_fields(fmt, rec, ep, 0, 1)
+    assert (s, q.tolist(), e) == (1, [7, 7, 7, 7], 10)
+
+
+@pytest.mark.parametrize("C,P", [inputs.FORMAT_4BIT, inputs.FORMAT_3BIT])
+def test_packing_round_trip(oracle_mod, C, P):
+    L = inputs.make_layer(7, 5 * C + 3, C, P, seed=11, e_range=(0, 15))
+    f = L["fmt"]
+    for r in range(f["rows"]):
+        for b in range(f["nb"]):
+            s, q, e = oracle_mod.block_fields(f, L["rec"], L["eplane"], r, b)
+            assert s == L["seeds"][r, b] and e == L["e"][r, b]
+            assert q.tolist() == L["q"][r, b].tolist()
+
+
+def test_ragged_last_block_is_truncated(oracle_mod):
+    # cols = 3 C + 5: the last block's first 5 weights are kept, the rest dropped.
+    C, P = inputs.FORMAT_3BIT
+    L = inputs.make_layer(2, 3 * C + 5, C, P, seed=3)
+    W = oracle_mod.decompress(L["fmt"], L["rec"], L["eplane"])
+    for r in range(2):
+        wb = oracle_mod.reconstruct_block(L["fmt"], L["rec"], L["eplane"], r, 3)
+        assert np.array_equal(W[r, 3 * C:], wb[:5])
+
+
+# ---------------------------------------------------------------- products
+
+def _layer(oracle_mod, rows, cols, fmt_cp, seed):
+    L = inputs.make_layer(rows, cols, *fmt_cp, seed=seed)
+    W = oracle_mod.decompress(L["fmt"], L["rec"], L["eplane"])
+    return L, W
+
+
+@pytest.mark.parametrize("fmt_cp", [inputs.FORMAT_4BIT, inputs.FORMAT_3BIT])
+def test_gemv_one_hot_picks_a_column(oracle_mod, fmt_cp):
+    L, W = _layer(oracle_mod, 9, 61, fmt_cp, 21)
+    for j in (0, 17, 60):
+        x = np.zeros(61)
+        x[j] = 1.0
+        y, _ = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], x)
+        assert np.array_equal(y, W[:, j])
+
+
+def test_gemv_ones_gives_row_sums(oracle_mod):
+    L, W = _layer(oracle_mod, 6, 40, inputs.FORMAT_4BIT, 8)
+    y, ya = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], np.ones(40))
+    exact = [sum(Fraction(v) for v in row) for row in W]
+    assert [Fraction(v) for v in y] == exact
+    assert np.array_equal(ya, np.abs(W).sum(axis=1))
+
+
+@pytest.mark.parametrize("fmt_cp", [inputs.FORMAT_4BIT, inputs.FORMAT_3BIT])
+def test_gemv_against_exact_rationals(oracle_mod, fmt_cp):
+    # W and x are exact dyadic rationals; the exact product is a Fraction sum.
+    # The fp64 accumulation may differ by at most n 2^-53 sum|w||x|.
+    L, W = _layer(oracle_mod, 5, 96, fmt_cp, 4)
+    _, x = inputs.make_activations((96,), "f16", 7)
+    y, ya = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], x)
+    for r in range(5):
+        exact = sum(Fraction(a) * Fraction(b) for a, b in zip(W[r], x))
+        assert abs(Fraction(y[r]) - exact) <= Fraction(96 * 2.0 ** -53) * Fraction(ya[r])
+
+
+def test_gemv_equals_decompress_then_matmul(oracle_mod):
+    L, W = _layer(oracle_mod, 33, 200, inputs.FORMAT_4BIT, 12)
+    _, x = inputs.make_activations((200,), "f16", 13)
+    y, ya = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], x)
+    assert np.all(np.abs(y - W @ x) <= 1e-13 * ya)
+
+
+def test_gemm_rows_equal_gemv_and_threads_agree(oracle_mod):
+    L, W = _layer(oracle_mod, 17, 50, inputs.FORMAT_3BIT, 14)
+    _, X = inputs.make_activations((4, 50), "bf16", 15)
+    Y1, Ya1 = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], X, threads=1)
+    Y4, Ya4 = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], X, threads=4)
+    assert np.array_equal(Y1, Y4) and np.array_equal(Ya1, Ya4)
+    for m in range(4):
+        y, _ = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], X[m])
+        assert np.array_equal(Y1[m], y)
+
+
+def test_empty_shapes(oracle_mod):
+    for rows, cols in ((0, 16), (4, 0), (0, 0)):
+        f = inputs.make_format(rows, cols, 8, 3)
+        rec = np.zeros((rows, f["rec_pitch"]), np.uint32)
+        assert oracle_mod.decompress(f, rec, None).shape == (rows, cols)
+        y, _ = oracle_mod.gemv(f, rec, None, np.zeros(cols))
+        assert y.shape == (rows,) and not y.any()
+
+
+# ------------------------------------------------------ planted-seed search
+
+@pytest.mark.parametrize("seed,q,e", [(1, (3, -5, 7), 9), (40000, (-8, 0, 7), 12),
+                                      (65535, (1, 2, -3), 8)])
+def test_planted_seed_is_recovered_c8_p3(oracle_mod, seed, q, e):
+    # The encoder's search over all seeds (paperhub.cn thread, replies on the
+    # cost of finding seeds and coefficients) must find a zero-error
+    # reconstruction of a block that was generated from a seed.  Compare the
+    # reconstruction, not (seed, q, e): an even q has more than one encoding.
+    from oracle.search import seed_search
+    fmt = inputs.make_format(1, 8, 8, 3)
+    rec, ep = inputs.pack_records(fmt, [[seed]], [[list(q)]], [[e]])
+    w = oracle_mod.decompress(fmt, rec, ep)[0]
+    s, qh, eh, err, what = seed_search(w, 8, 3)
+    assert err == 0.0 and np.array_equal(what, w)
+
+
+def test_planted_seed_is_recovered_c12_p4(oracle_mod):
+    from oracle.search import seed_search
+    fmt = inputs.make_format(1, 12, 12, 4)
+    rec, ep = inputs.pack_records(fmt, [[31337]], [[[2, -3, 5, -7]]], [[10]])
+    w = oracle_mod.decompress(fmt, rec, ep)[0]
+    s, qh, eh, err, what = seed_search(w, 12, 4)
+    assert err == 0.0 and np.array_equal(what, w)
+    assert (s, qh.tolist(), eh) == (31337, [2, -3, 5, -7], 10)
+
+
+def test_search_prefers_the_better_seed(oracle_mod):
+    # A Gaussian block (no exact encoding) must not be reconstructed worse by
+    # the searched seed than by any of a few fixed seeds with the same rule.
+    from oracle.search import seed_search
+    w = np.random.default_rng(2).standard_normal(8) * 0.02
+    s, q, e, err, what = seed_search(w, 8, 3)
+    assert err > 0 and np.isclose(err, ((w - what) ** 2).sum())
+    for other in (1, 2, 777, 65535):
+        U = oracle_mod.block_basis(other, 8, 3)
+        t = np.linalg.pinv(U) @ w
+        for ee in range(16):
+            qq = np.clip(np.rint(t * 2.0 ** ee), -8, 7)
+            assert ((w - U @ qq * 2.0 ** -ee) ** 2).sum() >= err
