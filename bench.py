@@ -1,0 +1,567 @@
+#!/usr/bin/env python
+"""Benchmark of the SeedLM hot path on B200: fused reconstruction + GEMV.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl seedlm|reference]
+
+Default workload (one step): the four batch-1 GEMVs of one Llama-3-70B-shaped
+decoder layer at 4 bits per weight (C=8, P=3, K=16) -- QKV 10240x8192,
+O 8192x8192, gate+up 57344x8192, down 8192x28672 -- with 80 distinct layer
+copies resident in HBM (34.2 GB compressed, i.e. every down-projection of the
+model) and step k using layer k mod 80, so no step finds its weights in L2.
+Inputs are synthetic (seeded PCG64; seed uniform on [1,65535], q on [-8,7],
+e on [8,12], x ~ N(0,1) in fp16); the run time of the method does not depend
+on the weight values.
+
+Prints ONE JSON line (rank 0).  ``value`` is the FP16-equivalent weight
+throughput (2 bytes per weight processed per second, all ranks); ``e2e`` the
+same through the public API with the activations copied in from pinned host
+memory and the results copied back every step; ``roofline`` the GEMV
+kernel's achieved compressed-byte bandwidth against the measured HBM copy
+bandwidth; ``cpu_baseline`` the fp64 CPU oracle timed on a bounded sample;
+``extras`` the other workloads (square sweep, 3-bit 8B layer, small-M GEMM,
+decompression, dense fp16 GEMV reference point) at one GPU.
+
+``--impl reference`` times the oracle itself (the reference arm of this
+build), on the host cores, on the same workload, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("µs/GEMV and FP16-equiv weight GB/s; achieved % of HBM roofline on "
+          "compressed bytes")
+UNIT = "GB/s (FP16-equivalent weight bytes)"
+FALLBACK_HBM_GBS = 6650.0
+
+LAYER_70B = [("qkv", 10240, 8192), ("o", 8192, 8192), ("gate_up", 57344, 8192),
+             ("down", 8192, 28672)]
+LAYER_8B = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_up", 28672, 4096),
+            ("down", 4096, 14336)]
+WORKLOAD = "llama3-70b decoder layer, 4-bit SeedLM GEMV x4 (QKV, O, gate+up, down)"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the
+    kernel's sources are unchanged since that capture (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh).get(kernel)
+    if not d:
+        return None
+    h = hashlib.sha256()
+    for f in d["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != d["sources_sha256"]:
+        return None
+    return d
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_dev: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            self.h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            except Exception:
+                pass
+            if self.h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[torch_dev]) if vis and vis.split(",")[0].isdigit() \
+                    else torch_dev
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report the failure, do not guess
+            self.error = f"nvml unavailable: {e}"
+            self.nv = None
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def result(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+               "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample(shapes, fmt_cp, rows_per_shape, threads, seed=5):
+    """Time the fp64 oracle on the first rows of each shape; (weights, seconds)."""
+    import numpy as np
+
+    import oracle
+    from prng_seeded_decompress_b200 import inputs
+    oracle.build()
+    weights, secs = 0, 0.0
+    for i, (_, R, N) in enumerate(shapes):
+        r = min(R, rows_per_shape)
+        L = inputs.make_layer(r, N, *fmt_cp, seed=seed + i)
+        _, xv = inputs.make_activations((N,), "f16", 77 + i)
+        t0 = time.perf_counter()
+        oracle.gemv(L["fmt"], L["rec"], L["eplane"], xv, threads=threads)
+        secs += time.perf_counter() - t0
+        weights += r * N
+        del L
+    return weights, secs
+
+
+def cpu_baseline(shapes, fmt_cp, target_s=12.0):
+    threads = os.cpu_count() or 1
+    w0, s0 = oracle_sample(shapes, fmt_cp, threads, threads)
+    rows = max(threads, int(threads * target_s / max(s0, 1e-3)))
+    w, s = oracle_sample(shapes, fmt_cp, rows, threads)
+    return {"value": round(2 * w / s / 1e9, 6), "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"first {rows} rows of each of the 4 layer shapes ({w / 1e6:.1f} M weights,"
+                      f" {s:.1f} s, fp64, {threads} host threads)"}
+
+
+# --------------------------------------------------------------- GPU arm
+
+def make_layer_on_device(torch, shapes, cp, seed):
+    import numpy as np
+
+    from prng_seeded_decompress_b200 import inputs
+    out = []
+    for i, (name, R, N) in enumerate(shapes):
+        L = inputs.make_layer(R, N, *cp, seed=seed + i)
+        rec = torch.from_numpy(L["rec"].view(np.int32)).cuda()
+        ep = torch.from_numpy(L["eplane"]).cuda() if cp[1] == 4 else None
+        out.append(dict(name=name, fmt=L["fmt"], rec=rec, ep=ep, R=R, N=N))
+        del L
+    return out
+
+
+def replicate(torch, layer, copies):
+    res = [layer]
+    for _ in range(copies - 1):
+        res.append([dict(m, rec=m["rec"].clone(), ep=None if m["ep"] is None else m["ep"].clone())
+                    for m in layer])
+    return res
+
+
+def time_region(torch, fn, reps):
+    """Device time of `reps` calls of fn() on the current stream, in ms."""
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for i in range(reps):
+        fn(i)
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def layer_bytes(shapes, cp):
+    """(weights, compressed stored bytes, algorithmic bytes) of one layer pass."""
+    C, P = cp
+    w = comp = alg = 0
+    for _, R, N in shapes:
+        nb = (N + C - 1) // C
+        w += R * N
+        rec_pitch = (nb + 3) // 4 * 4
+        e_pitch = ((nb + 1) // 2 + 15) // 16 * 16 if P == 4 else 0
+        comp += R * (4 * rec_pitch + e_pitch)
+        ideal = (16 + 4 * P + 4) * nb / 8
+        alg += R * ideal + 2 * N + 4 * R
+    return w, comp, alg
+
+
+def extras(torch, sl, args):
+    """The other workloads, one GPU: square sweep, 3-bit 8B layer, small-M
+    GEMM, decompression, dense fp16 GEMV reference point."""
+    import numpy as np
+
+    from prng_seeded_decompress_b200 import inputs
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    out = {}
+
+    # Square sweep (512..2048): 1000 back-to-back calls, a CUDA-graph replay
+    # of 1000 calls, and a cold-L2 rotation over >= 4x L2 of distinct copies.
+    sweep = {}
+    for n in (512, 1024, 2048):
+        layer = make_layer_on_device(torch, [("sq", n, n)], (8, 3), 500 + n)[0]
+        xb, _ = inputs.make_activations((n,), "f16", 600 + n)
+        x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+        y = torch.empty(n, device="cuda")
+        f = sl.Format.from_dict(layer["fmt"])
+        call = lambda i: sl.gemv(f, layer["rec"], None, x, y)  # noqa: E731
+        for i in range(20):
+            call(i)
+        warm = time_region(torch, call, 1000) / 1000 * 1e3
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            call(0)
+            with torch.cuda.graph(g, stream=s):
+                for i in range(1000):
+                    sl.gemv(f, layer["rec"], None, x, y, stream=s)
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        graph = time_region(torch, lambda i: g.replay(), 3) / 3000 * 1e3
+        del g
+        copies = max(2, math.ceil(4 * l2 / layer["rec"].numel() / 4))
+        recs = [layer["rec"].clone() for _ in range(copies)]
+        cold = time_region(torch, lambda i: sl.gemv(f, recs[i % copies], None, x, y),
+                           max(1000, copies)) / max(1000, copies) * 1e3
+        del recs
+        comp = n * layer["fmt"]["rec_pitch"] * 4
+        sweep[f"{n}x{n}"] = {"us_per_call": round(warm, 3), "us_per_call_graph": round(graph, 3),
+                             "us_per_call_cold_l2": round(cold, 3), "cold_copies": copies,
+                             "fp16_equiv_gbs_cold": round(2 * n * n / cold / 1e3, 1),
+                             "compressed_gbs_cold": round(comp / cold / 1e3, 1)}
+    out["square_sweep_4bit"] = sweep
+
+    # 3-bit Llama-3-8B layer: as specified (one layer) and 32 copies (cold).
+    layer = make_layer_on_device(torch, LAYER_8B, (12, 4), 700)
+    xs = {}
+    for _, _, N in LAYER_8B:
+        if N not in xs:
+            xb, _ = inputs.make_activations((N,), "f16", 800 + N)
+            xs[N] = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+    ys = [torch.empty(R, device="cuda") for _, R, _ in LAYER_8B]
+    fmts = [sl.Format.from_dict(m["fmt"]) for m in layer]
+
+    def run_layer(lay):
+        for m, f, y in zip(lay, fmts, ys):
+            sl.gemv(f, m["rec"], m["ep"], xs[m["N"]], y)
+    for i in range(5):
+        run_layer(layer)
+    one = time_region(torch, lambda i: run_layer(layer), 200) / 200 * 1e3
+    copies = replicate(torch, layer, 32)
+    cold = time_region(torch, lambda i: run_layer(copies[i % 32]), 320) / 320 * 1e3
+    del copies
+    w, comp, _ = layer_bytes(LAYER_8B, (12, 4))
+    out["llama3_8b_layer_3bit"] = {
+        "us_per_layer_single_copy": round(one, 2), "us_per_layer_32_copies": round(cold, 2),
+        "us_per_gemv_32_copies": round(cold / 4, 2),
+        "fp16_equiv_gbs": round(2 * w / cold / 1e3, 1),
+        "compressed_gbs": round(comp / cold / 1e3, 1)}
+    del layer
+
+    # Small-M GEMM on the 70B MLP shapes, 4-bit and 3-bit, M in {1,8,16,64}.
+    gemm = {}
+    for cp, tag in (((8, 3), "4bit"), ((12, 4), "3bit")):
+        for name, R, N in (("up_28672x8192", 28672, 8192), ("down_8192x28672", 8192, 28672)):
+            mats = make_layer_on_device(torch, [(name, R, N)], cp, 900 + R)
+            mats = [mats[0], dict(mats[0], rec=mats[0]["rec"].clone(),
+                                  ep=None if mats[0]["ep"] is None else mats[0]["ep"].clone())]
+            f = sl.Format.from_dict(mats[0]["fmt"])
+            for M in (1, 8, 16, 64):
+                Xb, _ = inputs.make_activations((M, N), "bf16", 950 + M)
+                X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+                Y = torch.empty((M, R), device="cuda")
+                fn = lambda i: sl.gemm_smallM(f, mats[i % 2]["rec"], mats[i % 2]["ep"], X, Y)  # noqa
+                fn(0)
+                reps = 20 if M > 1 else 50
+                us = time_region(torch, fn, reps) / reps * 1e3
+                gemm[f"{tag}/{name}/M={M}"] = {"us_per_call": round(us, 2),
+                                               "weights_per_s_e9": round(R * N / us / 1e3, 2)}
+            xb, _ = inputs.make_activations((N,), "bf16", 990)
+            x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            y = torch.empty(R, device="cuda")
+            fn = lambda i: sl.gemv(f, mats[i % 2]["rec"], mats[i % 2]["ep"], x, y)  # noqa
+            fn(0)
+            gemm[f"{tag}/{name}/gemv_bf16"] = {"us_per_call": round(time_region(torch, fn, 50)
+                                                                    / 50 * 1e3, 2)}
+            del mats
+    out["gemm_smallM"] = gemm
+
+    # Decompression of the 70B down projection (fp32 output).
+    m = make_layer_on_device(torch, [("down", 8192, 28672)], (8, 3), 1100)[0]
+    f = sl.Format.from_dict(m["fmt"])
+    W = torch.empty((8192, 28672), device="cuda")
+    sl.decompress(f, m["rec"], None, W)
+    us = time_region(torch, lambda i: sl.decompress(f, m["rec"], None, W), 20) / 20 * 1e3
+    moved = W.numel() * 4 + m["rec"].numel() * 4
+    out["decompress_4bit_8192x28672"] = {"us_per_call": round(us, 1),
+                                        "hbm_gbs_read_plus_write": round(moved / us / 1e3, 1)}
+    del W, m
+
+    # Dense fp16 GEMV (in-house) on the 70B layer shapes, 4 rotating copies.
+    rng = np.random.default_rng(3)
+    dense = []
+    for name, R, N in LAYER_70B:
+        Wh = torch.from_numpy((rng.standard_normal((R, N), dtype=np.float32) * 0.02)
+                              .astype(np.float16).view(np.int16)).cuda().view(torch.float16)
+        dense.append((Wh, [Wh] + [Wh.clone() for _ in range(3)]))
+    xsd = {N: torch.randn(N, device="cuda").half() for N in (8192, 28672)}
+    ysd = [torch.empty(R, device="cuda") for _, R, _ in LAYER_70B]
+
+    def dense_layer(i):
+        for (Wh, cps), (_, R, N), y in zip(dense, LAYER_70B, ysd):
+            sl.dense_gemv_f16(cps[i % 4], xsd[N], y)
+    for i in range(4):
+        dense_layer(i)
+    us = time_region(torch, dense_layer, 40) / 40 * 1e3
+    w, _, _ = layer_bytes(LAYER_70B, (8, 3))
+    out["dense_fp16_gemv_70b_layer"] = {"us_per_layer": round(us, 2),
+                                       "hbm_gbs": round(2 * w / us / 1e3, 1)}
+    del dense
+    return out
+
+
+def seedlm_arm(args):
+    import numpy as np
+    import torch
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from prng_seeded_decompress_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    from prng_seeded_decompress_b200 import inputs, seedlm as sl
+    sl.init()
+    hbm_peak, peak_kind = load_peaks()
+
+    shapes, cp = LAYER_70B, (8, 3)
+    t0 = time.time()
+    base = make_layer_on_device(torch, shapes, cp, seed=1000 + rank)
+    layers = replicate(torch, base, args.layers)
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] {args.layers} layer copies resident "
+        f"({sum(m['rec'].numel() * 4 for lay in layers for m in lay) / 1e9:.1f} GB) "
+        f"in {time.time() - t0:.1f} s")
+    xs = {}
+    for _, _, N in shapes:
+        if N not in xs:
+            xb, _ = inputs.make_activations((N,), "f16", 2000 + N)
+            xs[N] = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+    ys = [torch.empty(R, device="cuda") for _, R, _ in shapes]
+    fmts = [sl.Format.from_dict(m["fmt"]) for m in base]
+
+    def step(k):
+        lay = layers[k % args.layers]
+        for m, f, y in zip(lay, fmts, ys):
+            sl.gemv(f, m["rec"], m["ep"], xs[m["N"]], y)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    n0 = sl.launch_count()
+    with ClockSampler(local_rank) as clk:
+        ms = time_region(torch, step, args.steps)
+    launches = sl.launch_count() - n0
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    w, comp, alg = layer_bytes(shapes, cp)
+    secs = ms / 1e3
+    value = 2 * w * args.steps * world / secs / 1e9
+    achieved = alg * args.steps / secs / 1e9          # per launch avg bytes / avg duration
+    comp_gbs = comp * args.steps / secs / 1e9
+
+    # End to end through the public API: activations in from pinned host
+    # memory and results back every step.
+    hx = {N: xs[N].cpu().pin_memory() for N in xs}
+    hy = [torch.empty(R, dtype=torch.float32).pin_memory() for _, R, _ in shapes]
+    dx = {N: torch.empty_like(xs[N]) for N in xs}
+    h2d = sum(hx[N].numel() * 2 for _, _, N in shapes)   # one input per GEMV
+    d2h = sum(R * 4 for _, R, _ in shapes)
+
+    def e2e_step(k):
+        lay = layers[k % args.layers]
+        for m, f, y, hyy in zip(lay, fmts, ys, hy):
+            dx[m["N"]].copy_(hx[m["N"]], non_blocking=True)
+            sl.gemv(f, m["rec"], m["ep"], dx[m["N"]], y)
+            hyy.copy_(y, non_blocking=True)
+
+    for k in range(args.warmup):
+        e2e_step(k)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e2e_ms = time_region(torch, e2e_step, args.steps)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = 2 * w * args.steps * world / (e2e_ms / 1e3) / 1e9
+
+    traffic = profile_traffic("gemv_c8_kernel")
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+        "data": "synthetic (seeded PCG64 records and N(0,1) fp16 activations; runtime does not "
+                "depend on weight values)",
+        "config": {"workload": WORKLOAD, "format": "C=8, P=3, K=16 (32 bits per 8 weights)",
+                   "shapes": {n: [R, N] for n, R, N in shapes}, "batch": 1,
+                   "layer_copies_resident": args.layers,
+                   "resident_compressed_gb": round(comp * args.layers / 1e9, 2),
+                   "l2": "inputs larger than L2: each step reads one layer copy "
+                         f"({comp / 1e6:.0f} MB) of {args.layers} resident",
+                   "parallelism": f"replicas x{world} (independent layer stacks per GPU)"},
+        "us_per_gemv": round(ms * 1e3 / (args.steps * len(shapes)), 3),
+        "compressed_gbs": round(comp_gbs, 1),
+        "hbm_roofline_pct": round(100 * comp_gbs / hbm_peak, 2),
+        "hbm_roofline_pct_of_8tbs_spec": round(100 * comp_gbs / 8000, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "kernel": "gemv_c8_kernel",
+                     "traffic": None if traffic is None else traffic["bytes_per_launch"],
+                     "algorithmic_bytes_per_launch": round(alg / len(shapes))},
+        "clocks": clk.result(),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": int(launches),
+    }
+    del layers, base
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extras:
+        result["extras"] = extras(torch, sl, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(shapes, cp, target_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def reference_arm(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    shapes, cp = LAYER_70B, (8, 3)
+    threads = os.cpu_count() or 1
+    # One step = the oracle on the first `rows` rows of each of the 4 shapes,
+    # sized so that one step takes about `--ref-step-seconds`.
+    w0, s0 = oracle_sample(shapes, cp, threads, threads)
+    rows = max(threads, int(threads * args.ref_step_seconds / max(s0, 1e-3)))
+    for _ in range(args.warmup):
+        oracle_sample(shapes, cp, rows, threads)
+    tot_w, tot_s = 0, 0.0
+    for _ in range(args.steps):
+        w, s = oracle_sample(shapes, cp, rows, threads)
+        tot_w += w
+        tot_s += s
+    value = 2 * tot_w / tot_s / 1e9
+    sample = (f"first {rows} rows of each of the 4 layer shapes per step "
+              f"({tot_w / args.steps / 1e6:.1f} M weights), fp64, {threads} host threads")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded PCG64 records and N(0,1) fp16 activations)",
+        "config": {"workload": WORKLOAD, "format": "C=8, P=3, K=16 (32 bits per 8 weights)",
+                   "shapes": {n: [R, N] for n, R, N in shapes}, "batch": 1,
+                   "parallelism": "host threads (rows split)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("seedlm", "reference"), default="seedlm")
+    ap.add_argument("--layers", type=int, default=80, help="distinct layer copies resident")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=1.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        seedlm_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,145 @@
+/*
+ * seedlm.h -- C ABI of libseedlm.so: SeedLM weight reconstruction fused with
+ * the matrix-vector and small-batch matrix products that consume it, on B200
+ * (sm_100a).
+ *
+ * The operation (SeedLM: Compressing LLM Weights into Seeds of Pseudo-Random
+ * Generators -- abstract on the paperdance.org card; "Approach" on the
+ * atlas.scime.ai summary): a weight matrix W (rows x cols) is cut along each
+ * row into blocks of C weights.  Each block is stored as a 16-bit seed, P
+ * signed 4-bit coefficients q_p and one 4-bit exponent e shared by the block.
+ * The seed starts a 16-bit Fibonacci LFSR (taps 16,14,13,11):
+ *     bit = (s ^ s>>2 ^ s>>3 ^ s>>5) & 1 ;  s <- (s >> 1) | (bit << 15)
+ * with state_0 = seed; U is the C x P matrix U[c][p] = (state_{pC+c} - 32768)
+ * / 32768, and the block is W_blk = U t with t_p = q_p 2^-e (Eq (1) as the
+ * paperhub.cn review thread names it: U and t are the compression matrices).
+ * At inference W is never stored: each call rebuilds the blocks on the fly and
+ * consumes them at once (same thread, the authors' reply on how inference uses
+ * s and t).  Every rebuilt weight is an integer below 2^20 times 2^-(15+e), so
+ * it is exact in fp32.
+ *
+ * Supported formats: (C, P, K) = (8, 3, 16) -- 32 bits per 8 weights, 4 bits
+ * per weight -- and (12, 4, 16) -- 36 bits per 12 weights, 3 bits per weight.
+ *
+ * Record layout (the pages give none; this is the library's reading):
+ *   rec: one uint32 per block, blocks of a row in column order, row r at
+ *        rec + r * rec_pitch.  bits [16,32) seed; bits [4p, 4p+4) q_p for
+ *        p < P, two's complement.  (8,3): e in bits [12,16).
+ *   eplane (only for (12,4)): the exponents, row r at eplane + r * e_pitch,
+ *        block b in byte b/2, low nibble for even b.
+ *   Blocks run along a row; the last block of a row may extend past `cols`,
+ *   its weights beyond `cols` are dropped (as if x were zero-padded).
+ *   Records between nb and rec_pitch are padding and are never used.
+ *   A seed of 0 is accepted and gives the LFSR's fixed point (all states 0,
+ *   U = -1 everywhere).
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers, unless a function says HOST.
+ *     The caller owns every buffer; the library allocates no device memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; the call returns once it is enqueued.
+ *   - Return value 0 = success, negative = error (SEEDLM_E*), with no work
+ *     enqueued when the arguments are rejected.  Nothing aborts or prints.
+ *   - Alignment: rec must be 16-byte aligned (rec_pitch is a multiple of 4,
+ *     so every row is); x and X 2-byte aligned; y, Y and W 4-byte aligned.
+ *   - Results are fp32.  Decompression is bit-exact.  Products accumulate in
+ *     fp32 in a fixed order per shape, so repeated calls give identical bits;
+ *     the error against the exact product stays within 1e-5 * sum_j |W_rj x_j|
+ *     for the shapes this library targets.
+ */
+#ifndef SEEDLM_H
+#define SEEDLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Only the functions below are exported from libseedlm.so. */
+#if defined(__GNUC__)
+#define SEEDLM_API __attribute__((visibility("default")))
+#else
+#define SEEDLM_API
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* seedlm_stream;
+
+typedef struct seedlm_format {
+  int32_t C, P, K;    /* (8,3,16) or (12,4,16); others -> SEEDLM_EUNSUPPORTED     */
+  int32_t rows;       /* rows of W (outputs of the product), >= 0                 */
+  int32_t cols;       /* cols of W (inputs of the product), >= 0                  */
+  int32_t nb;         /* blocks per row; must equal ceil(cols / C)                */
+  int32_t rec_pitch;  /* uint32 records from one row to the next: >= nb, % 4 == 0 */
+  int32_t e_pitch;    /* (12,4): bytes per exponent-plane row, >= ceil(nb / 2);   */
+                      /* (8,3): ignored                                           */
+} seedlm_format;
+
+/* Activation element types. */
+enum { SEEDLM_F16 = 0, SEEDLM_BF16 = 1 };
+
+/* Error codes. */
+enum {
+  SEEDLM_OK = 0,
+  SEEDLM_EINVAL = -1,       /* null or misaligned pointer, bad size or field   */
+  SEEDLM_EUNSUPPORTED = -2, /* format or size outside what the kernels handle  */
+  SEEDLM_ECUDA = -3         /* a CUDA call failed; see seedlm_last_cuda_error  */
+};
+
+/* Prepares the current device (kernel attributes).  Idempotent; every entry
+ * point calls it on first use of a device, so calling it is optional, but a
+ * caller that captures CUDA graphs should call it once per device first. */
+SEEDLM_API int seedlm_init(void);
+
+/* W = decompressed weights, rows x cols, row-major with leading dimension ldw
+ * (floats, >= cols).  Bit-exact.  (Eq (1) of the paperhub.cn thread, applied
+ * to every block.) */
+SEEDLM_API int seedlm_decompress(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                      float* W, int64_t ldw, seedlm_stream stream);
+
+/* y = W x (batch 1).  x: cols elements of type x_dtype (SEEDLM_F16 or
+ * SEEDLM_BF16); y: rows fp32.  The blocks are rebuilt on the fly and never
+ * written out (paperhub.cn thread, authors' replies on inference and on the
+ * custom decoding that avoids full-precision weights in memory).  cols up to
+ * 56,320 (4-bit) or 40,960 (3-bit): x is held in shared memory as fp32. */
+SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                const void* x, int x_dtype, float* y, seedlm_stream stream);
+
+/* Y = X W^T for a small batch: X is M x cols (row-major, type x_dtype), Y is
+ * M x rows fp32 (row-major).  1 <= M <= 64. */
+SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                       const void* X, int x_dtype, int M, float* Y, seedlm_stream stream);
+
+/* Reference point, not part of the method: y = W x with W dense fp16
+ * (rows x cols, row-major, leading dimension ldw halves, 16-byte aligned with
+ * ldw % 8 == 0), x fp16 (cols), y fp32 (rows). */
+SEEDLM_API int seedlm_dense_gemv_f16(int32_t rows, int32_t cols, const uint16_t* W, int64_t ldw,
+                          const uint16_t* x, float* y, seedlm_stream stream);
+
+/* Bytes of compressed storage one row needs at the ideal packing
+ * ((K + 4P + 4) * nb / 8, no pitch padding) and as laid out (4 * rec_pitch +
+ * e_pitch).  HOST function; returns -1 on a bad format. */
+SEEDLM_API int64_t seedlm_row_bytes_ideal(const seedlm_format* fmt);
+SEEDLM_API int64_t seedlm_row_bytes_stored(const seedlm_format* fmt);
+
+/* Static description of an error code (never NULL). */
+SEEDLM_API const char* seedlm_strerror(int code);
+
+/* The cudaError_t of the last SEEDLM_ECUDA on this host thread (0 if none). */
+SEEDLM_API int seedlm_last_cuda_error(void);
+
+/* Number of kernel launches this library has enqueued since load (all
+ * threads); used to count the library's launches in a timed region. */
+SEEDLM_API int64_t seedlm_launch_count(void);
+
+/* Releases nothing that outlives the process today; kept for symmetry with
+ * seedlm_init.  Safe to call more than once. */
+SEEDLM_API void seedlm_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEEDLM_H */

@@ -1,0 +1,197 @@
+// abi.cu -- the extern "C" entry points of libseedlm.so: argument checks,
+// per-device setup and dispatch to the kernels.  See include/seedlm.h for the
+// contract of every function.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "seedlm_internal.h"
+
+namespace seedlm {
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+std::atomic<int64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ready[kMaxDevices] = {};
+
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return record_cuda_error(err);
+  if (dev < 0 || dev >= kMaxDevices) return SEEDLM_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (!g_dev_ready[dev]) {
+    DeviceInfo d{};
+    d.device = dev;
+    if ((err = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) !=
+            cudaSuccess ||
+        (err = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                      dev)) != cudaSuccess ||
+        (err = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) !=
+            cudaSuccess ||
+        (err = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) !=
+            cudaSuccess)
+      return record_cuda_error(err);
+    // The kernels are built for sm_100a only.
+    if (d.cc_major != 10 || d.cc_minor != 0) return SEEDLM_EUNSUPPORTED;
+    g_dev[dev] = d;
+    g_dev_ready[dev] = true;
+  }
+  *out = g_dev[dev];
+  return SEEDLM_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_format(const seedlm_format* f) {
+  if (!f) return SEEDLM_EINVAL;
+  const bool c8 = f->C == 8 && f->P == 3 && f->K == 16;
+  const bool c12 = f->C == 12 && f->P == 4 && f->K == 16;
+  if (!c8 && !c12) return SEEDLM_EUNSUPPORTED;
+  if (f->rows < 0 || f->cols < 0) return SEEDLM_EINVAL;
+  if (f->nb != (f->cols + f->C - 1) / f->C) return SEEDLM_EINVAL;
+  if (f->rec_pitch < f->nb || f->rec_pitch % 4 != 0) return SEEDLM_EINVAL;
+  if (c12 && f->e_pitch < (f->nb + 1) / 2) return SEEDLM_EINVAL;
+  return SEEDLM_OK;
+}
+
+int check_planes(const seedlm_format* f, const uint32_t* rec, const uint8_t* eplane) {
+  if (f->rows == 0 || f->nb == 0) return SEEDLM_OK;
+  if (!rec || !aligned(rec, 16)) return SEEDLM_EINVAL;
+  if (f->P == 4 && !eplane) return SEEDLM_EINVAL;
+  return SEEDLM_OK;
+}
+
+}  // namespace
+
+int record_cuda_error(cudaError_t err) {
+  if (err == cudaSuccess) return SEEDLM_OK;
+  g_last_cuda_error = (int)err;
+  return SEEDLM_ECUDA;
+}
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int allow_max_smem(const void* kernel, const DeviceInfo& dev) {
+  static std::mutex m;
+  static std::set<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(m);
+  if (done.count({kernel, dev.device})) return SEEDLM_OK;
+  cudaError_t err =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
+  if (err != cudaSuccess) return record_cuda_error(err);
+  done.insert({kernel, dev.device});
+  return SEEDLM_OK;
+}
+
+}  // namespace seedlm
+
+using namespace seedlm;
+
+extern "C" {
+
+int seedlm_init(void) {
+  DeviceInfo d;
+  return device_info(&d);
+}
+
+int seedlm_decompress(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                      float* W, int64_t ldw, seedlm_stream stream) {
+  int rc = check_format(fmt);
+  if (rc) return rc;
+  if ((rc = check_planes(fmt, rec, eplane))) return rc;
+  if (fmt->rows == 0 || fmt->cols == 0) return SEEDLM_OK;
+  if (!W || !aligned(W, 4) || ldw < fmt->cols) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  return launch_decompress(*fmt, rec, eplane, W, ldw, (cudaStream_t)stream, dev);
+}
+
+int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                const void* x, int x_dtype, float* y, seedlm_stream stream) {
+  int rc = check_format(fmt);
+  if (rc) return rc;
+  if ((rc = check_planes(fmt, rec, eplane))) return rc;
+  if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
+  if (fmt->rows == 0) return SEEDLM_OK;
+  if (!y || !aligned(y, 4)) return SEEDLM_EINVAL;
+  if (fmt->cols > 0 && (!x || !aligned(x, 2))) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  if (fmt->cols == 0)
+    return record_cuda_error(
+        cudaMemsetAsync(y, 0, (size_t)fmt->rows * sizeof(float), (cudaStream_t)stream));
+  return launch_gemv(*fmt, rec, eplane, static_cast<const uint16_t*>(x),
+                     x_dtype == SEEDLM_BF16, y, (cudaStream_t)stream, dev);
+}
+
+int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                       const void* X, int x_dtype, int M, float* Y, seedlm_stream stream) {
+  int rc = check_format(fmt);
+  if (rc) return rc;
+  if ((rc = check_planes(fmt, rec, eplane))) return rc;
+  if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
+  if (M < 1 || M > 64) return SEEDLM_EINVAL;
+  if (fmt->rows == 0) return SEEDLM_OK;
+  if (!Y || !aligned(Y, 4)) return SEEDLM_EINVAL;
+  if (fmt->cols > 0 && (!X || !aligned(X, 2))) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  if (fmt->cols == 0)
+    return record_cuda_error(
+        cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), (cudaStream_t)stream));
+  return launch_gemm_small(*fmt, rec, eplane, static_cast<const uint16_t*>(X),
+                           x_dtype == SEEDLM_BF16, M, Y, (cudaStream_t)stream, dev);
+}
+
+int seedlm_dense_gemv_f16(int32_t rows, int32_t cols, const uint16_t* W, int64_t ldw,
+                          const uint16_t* x, float* y, seedlm_stream stream) {
+  if (rows < 0 || cols < 0 || ldw < cols || ldw % 8 != 0) return SEEDLM_EINVAL;
+  if (rows == 0) return SEEDLM_OK;
+  if (!y || !aligned(y, 4)) return SEEDLM_EINVAL;
+  if (cols > 0 && (!W || !aligned(W, 16) || !x || !aligned(x, 2))) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  if (cols == 0)
+    return record_cuda_error(
+        cudaMemsetAsync(y, 0, (size_t)rows * sizeof(float), (cudaStream_t)stream));
+  return launch_dense_gemv_f16(rows, cols, W, ldw, x, y, (cudaStream_t)stream, dev);
+}
+
+int64_t seedlm_row_bytes_ideal(const seedlm_format* fmt) {
+  if (check_format(fmt)) return -1;
+  const int64_t bits = (int64_t)(fmt->K + 4 * fmt->P + 4) * fmt->nb;
+  return (bits + 7) / 8;
+}
+
+int64_t seedlm_row_bytes_stored(const seedlm_format* fmt) {
+  if (check_format(fmt)) return -1;
+  return 4 * (int64_t)fmt->rec_pitch + (fmt->P == 4 ? (int64_t)fmt->e_pitch : 0);
+}
+
+const char* seedlm_strerror(int code) {
+  switch (code) {
+    case SEEDLM_OK: return "success";
+    case SEEDLM_EINVAL: return "invalid argument (null or misaligned pointer, bad size or field)";
+    case SEEDLM_EUNSUPPORTED: return "unsupported format, size or device";
+    case SEEDLM_ECUDA: return "a CUDA call failed (see seedlm_last_cuda_error)";
+    default: return "unknown error code";
+  }
+}
+
+int seedlm_last_cuda_error(void) { return g_last_cuda_error; }
+
+int64_t seedlm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void seedlm_shutdown(void) {}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// seedlm_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/seedlm.h"
+
+namespace seedlm {
+
+struct DeviceInfo {
+  int device;
+  int num_sms;
+  int max_smem_optin;  // bytes of dynamic shared memory a block may opt into
+  int cc_major, cc_minor;
+};
+
+// Records err as this thread's last CUDA error; SEEDLM_OK or SEEDLM_ECUDA.
+int record_cuda_error(cudaError_t err);
+// Counts one kernel launch (process-wide).
+void count_launch();
+// Lets `kernel` use all the dynamic shared memory the device allows; done once
+// per kernel and device, outside any stream capture the caller may start later.
+int allow_max_smem(const void* kernel, const DeviceInfo& dev);
+
+size_t gemv_smem_bytes(const seedlm_format& f);
+int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
+                const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
+                const DeviceInfo& dev);
+int launch_decompress(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
+                      float* W, int64_t ldw, cudaStream_t stream, const DeviceInfo& dev);
+int launch_dense_gemv_f16(int rows, int cols, const uint16_t* W, int64_t ldw, const uint16_t* x,
+                          float* y, cudaStream_t stream, const DeviceInfo& dev);
+int launch_gemm_small(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
+                      const uint16_t* X, int is_bf16, int M, float* Y, cudaStream_t stream,
+                      const DeviceInfo& dev);
+
+}  // namespace seedlm

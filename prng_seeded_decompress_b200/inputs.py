@@ -45,23 +45,24 @@ def make_format(rows: int, cols: int, C: int, P: int) -> dict:
 def draw_fields(rng: np.random.Generator, rows: int, nb: int, P: int,
                 e_range=(8, 12)):
     """seeds (rows, nb) uint16, q (rows, nb, P) int8, e (rows, nb) uint8."""
-    seeds = rng.integers(1, 65536, size=(rows, nb), dtype=np.int64).astype(np.uint16)
-    q = rng.integers(-8, 8, size=(rows, nb, P), dtype=np.int64).astype(np.int8)
-    e = rng.integers(e_range[0], e_range[1] + 1, size=(rows, nb), dtype=np.int64)
-    return seeds, q, e.astype(np.uint8)
+    seeds = rng.integers(1, 65535, size=(rows, nb), dtype=np.uint16, endpoint=True)
+    q = rng.integers(-8, 7, size=(rows, nb, P), dtype=np.int8, endpoint=True)
+    e = rng.integers(e_range[0], e_range[1], size=(rows, nb), dtype=np.uint8, endpoint=True)
+    return seeds, q, e
 
 
 def pack_records(fmt: dict, seeds, q, e, rng: np.random.Generator | None = None):
     """Pack the fields into (rec, eplane) in the layout described above."""
     rows, nb, P = fmt["rows"], fmt["nb"], fmt["P"]
     seeds = np.asarray(seeds, dtype=np.uint32).reshape(rows, nb)
-    q = np.asarray(q, dtype=np.int64).reshape(rows, nb, P)
+    q = np.asarray(q).reshape(rows, nb, P)
     e = np.asarray(e, dtype=np.uint32).reshape(rows, nb)
     if np.any((q < -8) | (q > 7)) or np.any(e > 15):
         raise ValueError("fields out of range")
     word = seeds << np.uint32(16)
     for p in range(P):
-        word |= (q[:, :, p].astype(np.uint32) & np.uint32(15)) << np.uint32(4 * p)
+        word |= (q[:, :, p].astype(np.int32).astype(np.uint32) & np.uint32(15)) << \
+            np.uint32(4 * p)
     rec = np.zeros((rows, fmt["rec_pitch"]), np.uint32)
     if rng is not None and fmt["rec_pitch"] > nb:
         rec[:, nb:] = rng.integers(0, 2 ** 32, size=(rows, fmt["rec_pitch"] - nb),

@@ -1,0 +1,166 @@
+"""ctypes binding of libseedlm.so (see include/seedlm.h for the contract).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  Tensors are passed as raw device pointers; the stream defaults
+to PyTorch's current stream on the tensors' device.  If the library has not
+been built, importing this module raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libseedlm.so")
+
+F16 = 0
+BF16 = 1
+
+#: Every symbol include/seedlm.h declares.
+EXPORTS = (
+    "seedlm_init", "seedlm_decompress", "seedlm_gemv", "seedlm_gemm_smallM",
+    "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
+    "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
+)
+
+
+class SeedLMError(RuntimeError):
+    def __init__(self, fn: str, code: int, detail: str):
+        super().__init__(f"{fn} failed with {code}: {detail}")
+        self.code = code
+
+
+class Format(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("C", "P", "K", "rows", "cols", "nb", "rec_pitch", "e_pitch")]
+
+    @classmethod
+    def from_dict(cls, d: dict) -> "Format":
+        return cls(*(int(d[k]) for k in ("C", "P", "K", "rows", "cols", "nb", "rec_pitch",
+                                         "e_pitch")))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m prng_seeded_decompress_b200.build`"
+            " (the SeedLM kernels have no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    fmtp = ctypes.POINTER(Format)
+    sig = {
+        "seedlm_init": (ctypes.c_int, []),
+        "seedlm_decompress": (ctypes.c_int, [fmtp, vp, vp, vp, i64, vp]),
+        "seedlm_gemv": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, vp, vp]),
+        "seedlm_gemm_smallM": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp,
+                                              vp]),
+        "seedlm_dense_gemv_f16": (ctypes.c_int, [i32, i32, vp, i64, vp, vp, vp]),
+        "seedlm_row_bytes_ideal": (i64, [fmtp]),
+        "seedlm_row_bytes_stored": (i64, [fmtp]),
+        "seedlm_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+        "seedlm_last_cuda_error": (ctypes.c_int, []),
+        "seedlm_launch_count": (i64, []),
+        "seedlm_shutdown": (None, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def strerror(code: int) -> str:
+    return lib.seedlm_strerror(code).decode()
+
+
+def last_cuda_error() -> int:
+    return int(lib.seedlm_last_cuda_error())
+
+
+def launch_count() -> int:
+    return int(lib.seedlm_launch_count())
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        detail = strerror(rc)
+        if rc == -3:
+            detail += f" (cudaError {last_cuda_error()})"
+        raise SeedLMError(fn, rc, detail)
+
+
+def _ptr(t) -> int | None:
+    """Device (or host) address of a tensor, an int address, or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream, like=None):
+    if stream is None:
+        import torch
+        dev = like.device if (like is not None and hasattr(like, "device")) else None
+        return torch.cuda.current_stream(dev).cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _act_dtype(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return F16
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"activations must be float16 or bfloat16, got {t.dtype}")
+
+
+def _fmt(fmt) -> Format:
+    return fmt if isinstance(fmt, Format) else Format.from_dict(fmt)
+
+
+def init():
+    _check("seedlm_init", lib.seedlm_init())
+
+
+def decompress(fmt, rec, eplane, W, ldw: int | None = None, stream=None):
+    """W[:rows, :cols] = the rebuilt weights (fp32)."""
+    f = _fmt(fmt)
+    ld = ldw if ldw is not None else (W.stride(0) if W.dim() == 2 else f.cols)
+    _check("seedlm_decompress", lib.seedlm_decompress(
+        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(W), ld, _stream(stream, W)))
+
+
+def gemv(fmt, rec, eplane, x, y, stream=None):
+    """y = W x; x float16/bfloat16 (cols), y float32 (rows)."""
+    f = _fmt(fmt)
+    _check("seedlm_gemv", lib.seedlm_gemv(
+        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(x), _act_dtype(x), _ptr(y),
+        _stream(stream, y)))
+
+
+def gemm_smallM(fmt, rec, eplane, X, Y, stream=None):
+    """Y = X W^T; X float16/bfloat16 (M, cols), Y float32 (M, rows)."""
+    f = _fmt(fmt)
+    _check("seedlm_gemm_smallM", lib.seedlm_gemm_smallM(
+        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), int(X.shape[0]),
+        _ptr(Y), _stream(stream, Y)))
+
+
+def dense_gemv_f16(W, x, y, stream=None):
+    """y = W x with dense fp16 W (rows, cols) -- the reference point."""
+    _check("seedlm_dense_gemv_f16", lib.seedlm_dense_gemv_f16(
+        int(W.shape[0]), int(W.shape[1]), _ptr(W), int(W.stride(0)), _ptr(x), _ptr(y),
+        _stream(stream, y)))
+
+
+def row_bytes(fmt) -> tuple[int, int]:
+    """(ideal, stored) compressed bytes per row."""
+    f = _fmt(fmt)
+    return int(lib.seedlm_row_bytes_ideal(ctypes.byref(f))), \
+        int(lib.seedlm_row_bytes_stored(ctypes.byref(f)))

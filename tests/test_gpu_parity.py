@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA path against the CPU oracle on the same seeded inputs.
+
+Decompression must match bit for bit (every weight is a short dyadic
+rational, exact in fp32).  Products must satisfy, per output,
+|y - y_oracle| <= 1e-5 * sum_j |W_rj x_j| (the oracle accumulates in fp64).
+All calls go through the C ABI (ctypes binding).
+"""
+import numpy as np
+import pytest
+
+from prng_seeded_decompress_b200 import inputs
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-5
+C8, C12 = inputs.FORMAT_4BIT, inputs.FORMAT_3BIT
+
+
+@pytest.fixture(scope="module")
+def sl():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from prng_seeded_decompress_b200 import build
+    build.build()
+    from prng_seeded_decompress_b200 import seedlm
+    seedlm.init()
+    return seedlm
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def act_tensor(bits, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda()
+    return t.view(torch.float16 if dtype == "f16" else torch.bfloat16)
+
+
+def planes(L):
+    rec = dev(L["rec"].view(np.int32))
+    ep = dev(L["eplane"]) if L["fmt"]["P"] == 4 else None
+    return rec, ep
+
+
+def gpu_gemv(sl, L, xbits, dtype="f16"):
+    rec, ep = planes(L)
+    x = act_tensor(xbits, dtype)
+    y = torch.full((L["fmt"]["rows"],), float("nan"), device="cuda")
+    sl.gemv(L["fmt"], rec, ep, x, y)
+    torch.cuda.synchronize()
+    return y.cpu().numpy().astype(np.float64)
+
+
+def assert_within(y, ref, refabs):
+    err = np.abs(y - ref)
+    bound = TOL * refabs + 1e-30
+    bad = np.nonzero(err > bound)[0]
+    assert bad.size == 0, f"{bad.size} outputs out of tolerance, e.g. row {bad[:5]}: " \
+                          f"err {err[bad[:5]]} bound {bound[bad[:5]]}"
+
+
+# ------------------------------------------------------------- decompress
+
+DECOMP_SHAPES = [
+    (C8, 512, 512), (C8, 37, 203), (C8, 1, 1), (C8, 3, 8), (C8, 130, 2048),
+    (C12, 61, 4096), (C12, 17, 1000), (C12, 2, 12), (C12, 5, 13),
+]
+
+
+@pytest.mark.parametrize("cp,rows,cols", DECOMP_SHAPES)
+def test_decompress_bit_exact(sl, oracle_mod, cp, rows, cols):
+    L = inputs.make_layer(rows, cols, *cp, seed=1000 + rows + cols, e_range=(0, 15))
+    rec, ep = planes(L)
+    W = torch.full((rows, cols), float("nan"), device="cuda")
+    sl.decompress(L["fmt"], rec, ep, W)
+    torch.cuda.synchronize()
+    ref = oracle_mod.decompress(L["fmt"], L["rec"], L["eplane"]).astype(np.float32)
+    got = W.cpu().numpy()
+    # Bit patterns, so that -0 and +0 would differ too.
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_decompress_leading_dimension_and_seed_zero(sl, oracle_mod):
+    fmt = inputs.make_format(3, 20, 8, 3)
+    seeds = np.array([[0, 1, 65535], [0, 0, 0], [12345, 0, 7]])
+    q = np.random.default_rng(3).integers(-8, 8, size=(3, 3, 3))
+    e = np.array([[0, 15, 8], [3, 4, 5], [12, 12, 12]])
+    rec_np, ep_np = inputs.pack_records(fmt, seeds, q, e)
+    L = dict(fmt=fmt, rec=rec_np, eplane=ep_np)
+    rec, ep = planes(L)
+    W = torch.full((3, 27), -1.0, device="cuda")
+    sl.decompress(fmt, rec, ep, W, ldw=27)
+    torch.cuda.synchronize()
+    ref = oracle_mod.decompress(fmt, rec_np, ep_np)
+    got = W.cpu().numpy()
+    assert np.array_equal(got[:, :20], ref.astype(np.float32))
+    assert np.all(got[:, 20:] == -1.0)
+
+
+# ------------------------------------------------------------------- gemv
+
+GEMV_SHAPES = [
+    (C8, 512, 512), (C8, 1024, 1024), (C8, 64, 2048), (C8, 37, 203), (C8, 1, 8),
+    (C8, 5, 1), (C8, 333, 4096), (C8, 70, 9000),
+    (C12, 96, 4096), (C12, 40, 14336), (C12, 17, 1000), (C12, 3, 12), (C12, 9, 25),
+]
+
+
+@pytest.mark.parametrize("cp,rows,cols", GEMV_SHAPES)
+def test_gemv_matches_oracle(sl, oracle_mod, cp, rows, cols):
+    L = inputs.make_layer(rows, cols, *cp, seed=2000 + rows + cols)
+    xb, xv = inputs.make_activations((cols,), "f16", 3000 + cols)
+    y = gpu_gemv(sl, L, xb)
+    ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv)
+    assert_within(y, ref, refabs)
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_gemv_bf16_activations(sl, oracle_mod, cp):
+    L = inputs.make_layer(200, 3000, *cp, seed=11)
+    xb, xv = inputs.make_activations((3000,), "bf16", 12)
+    y = gpu_gemv(sl, L, xb, "bf16")
+    ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv)
+    assert_within(y, ref, refabs)
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_gemv_one_hot_is_bit_exact(sl, oracle_mod, cp):
+    # One nonzero product per row: the fused kernel must return column j of W
+    # exactly (closed-form special case).
+    rows, cols = 77, 777
+    L = inputs.make_layer(rows, cols, *cp, seed=21, e_range=(0, 15))
+    W = oracle_mod.decompress(L["fmt"], L["rec"], L["eplane"])
+    for j in (0, 5, cols - 1):
+        xv = np.zeros(cols)
+        xv[j] = 1.0
+        xb = xv.astype(np.float16).view(np.uint16)
+        y = gpu_gemv(sl, L, xb)
+        assert np.array_equal(y, W[:, j])
+
+
+def test_gemv_is_deterministic_and_needs_no_zeroed_output(sl):
+    L = inputs.make_layer(1000, 8192, *C8, seed=31)
+    xb, _ = inputs.make_activations((8192,), "f16", 32)
+    y1 = gpu_gemv(sl, L, xb)
+    y2 = gpu_gemv(sl, L, xb)
+    assert np.array_equal(y1.view(np.uint64), y2.view(np.uint64))
+
+
+def test_gemv_empty_shapes(sl):
+    for rows, cols in ((0, 64), (5, 0)):
+        L = inputs.make_layer(rows, cols, *C8, seed=1)
+        xb = np.zeros(max(cols, 1), np.uint16)
+        if rows:
+            y = gpu_gemv(sl, L, xb)
+            assert np.array_equal(y, np.zeros(rows))
+        else:
+            rec, ep = planes(L)
+            y = torch.zeros(1, device="cuda")
+            sl.gemv(L["fmt"], rec, ep, act_tensor(xb, "f16"), y)
+
+
+@pytest.mark.parametrize("cp,rows,cols", [(C8, 8192, 28672), (C8, 10240, 8192),
+                                          (C12, 28672, 4096), (C12, 4096, 14336)])
+def test_gemv_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols):
+    # The layer shapes the benchmark times, checked on a sample of rows that
+    # covers the first and last tiles.
+    L = inputs.make_layer(rows, cols, *cp, seed=rows + 7 * cols)
+    xb, xv = inputs.make_activations((cols,), "f16", 99)
+    y = gpu_gemv(sl, L, xb)
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([np.arange(8), np.arange(rows - 8, rows),
+                                       rng.integers(0, rows, 48)]))
+    ref, refabs = oracle_mod.gemv_rows(L["fmt"], L["rec"], L["eplane"], xv, sample)
+    assert_within(y[sample], ref, refabs)
+
+
+def test_decompress_then_dense_equals_fused(sl, oracle_mod):
+    L = inputs.make_layer(300, 5000, *C8, seed=41)
+    xb, xv = inputs.make_activations((5000,), "f16", 42)
+    rec, ep = planes(L)
+    W = torch.empty((300, 5000), device="cuda")
+    sl.decompress(L["fmt"], rec, ep, W)
+    y = gpu_gemv(sl, L, xb)
+    Wd = W.cpu().numpy().astype(np.float64)
+    ref = Wd @ xv
+    assert_within(y, ref, np.abs(Wd) @ np.abs(xv))
+
+
+# ------------------------------------------------------------ small-M GEMM
+
+@pytest.mark.parametrize("cp", [C8, C12])
+@pytest.mark.parametrize("M", [1, 3, 8, 16, 64])
+def test_gemm_small_matches_oracle(sl, oracle_mod, cp, M):
+    rows, cols = 150, 2000
+    L = inputs.make_layer(rows, cols, *cp, seed=50 + M)
+    Xb, Xv = inputs.make_activations((M, cols), "bf16", 60 + M)
+    rec, ep = planes(L)
+    X = act_tensor(Xb, "bf16")
+    Y = torch.full((M, rows), float("nan"), device="cuda")
+    sl.gemm_smallM(L["fmt"], rec, ep, X, Y)
+    torch.cuda.synchronize()
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv)
+    got = Y.cpu().numpy().astype(np.float64)
+    for m in range(M):
+        assert_within(got[m], ref[m], refabs[m])
+
+
+def test_gemm_m1_equals_gemv_within_tolerance(sl, oracle_mod):
+    L = inputs.make_layer(256, 4096, *C8, seed=71)
+    xb, xv = inputs.make_activations((1, 4096), "bf16", 72)
+    rec, ep = planes(L)
+    Y = torch.empty((1, 256), device="cuda")
+    sl.gemm_smallM(L["fmt"], rec, ep, act_tensor(xb, "bf16"), Y)
+    y = gpu_gemv(sl, L, xb[0], "bf16")
+    _, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv[0])
+    assert np.all(np.abs(Y.cpu().numpy()[0] - y) <= 2 * TOL * refabs + 1e-30)
+
+
+# --------------------------------------------------------- dense reference
+
+def test_dense_f16_gemv(sl):
+    rng = np.random.default_rng(5)
+    rows, cols = 1001, 4104
+    Wh = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float16)
+    xh = rng.standard_normal(cols).astype(np.float16)
+    y = torch.empty(rows, device="cuda")
+    sl.dense_gemv_f16(dev(Wh.view(np.int16)), dev(xh.view(np.int16)), y)
+    torch.cuda.synchronize()
+    Wd, xd = Wh.astype(np.float64), xh.astype(np.float64)
+    assert_within(y.cpu().numpy().astype(np.float64), Wd @ xd, np.abs(Wd) @ np.abs(xd))
+
+
+def test_misaligned_record_pointer_is_rejected(sl):
+    L = inputs.make_layer(8, 64, *C8, seed=1)
+    rec, _ = planes(L)
+    x = torch.zeros(64, dtype=torch.float16, device="cuda")
+    y = torch.zeros(8, device="cuda")
+    with pytest.raises(sl.SeedLMError):
+        sl.gemv(L["fmt"], rec.data_ptr() + 4, None, x, y)
