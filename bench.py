@@ -328,12 +328,15 @@ def extras(torch, sl, args):
                 Xb, _ = inputs.make_activations((M, N), "bf16", 950 + M)
                 X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
                 Y = torch.empty((M, R), device="cuda")
-                fn = lambda i: sl.gemm_smallM(f, mats[i % 2]["rec"], mats[i % 2]["ep"], X, Y)  # noqa
+                ws = sl.gemm_workspace(f, M)
+                fn = lambda i: sl.gemm_smallM(f, mats[i % 2]["rec"], mats[i % 2]["ep"], X, Y,  # noqa
+                                              workspace=ws)
                 fn(0)
-                reps = 20 if M > 1 else 50
+                reps = 50
                 us = time_region(torch, fn, reps) / reps * 1e3
-                gemm[f"{tag}/{name}/M={M}"] = {"us_per_call": round(us, 2),
-                                               "weights_per_s_e9": round(R * N / us / 1e3, 2)}
+                gemm[f"{tag}/{name}/M={M}"] = {
+                    "us_per_call": round(us, 2), "weights_per_s_e9": round(R * N / us / 1e3, 2),
+                    "tflops_useful": round(2 * M * R * N / us / 1e6, 2)}
             xb, _ = inputs.make_activations((N,), "bf16", 990)
             x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
             y = torch.empty(R, device="cuda")
@@ -395,7 +398,7 @@ def seedlm_arm(args):
         build.build()
     if world > 1:
         torch.distributed.barrier()
-    from prng_seeded_decompress_b200 import inputs, seedlm as sl
+    from prng_seeded_decompress_b200 import dist_util, inputs, seedlm as sl
     sl.init()
     hbm_peak, peak_kind = load_peaks()
 
@@ -429,10 +432,7 @@ def seedlm_arm(args):
     with ClockSampler(local_rank) as clk:
         ms = time_region(torch, step, args.steps)
     launches = sl.launch_count() - n0
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = dist_util.max_over_ranks(ms, device="cuda")
     w, comp, alg = layer_bytes(shapes, cp)
     secs = ms / 1e3
     value = 2 * w * args.steps * world / secs / 1e9
@@ -460,13 +460,24 @@ def seedlm_arm(args):
     if world > 1:
         torch.distributed.barrier()
     e2e_ms = time_region(torch, e2e_step, args.steps)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = dist_util.max_over_ranks(e2e_ms, device="cuda")
     e2e_value = 2 * w * args.steps * world / (e2e_ms / 1e3) / 1e9
 
-    traffic = profile_traffic("gemv_c8_kernel")
+    # Per-shape times (same rotation over the resident copies).
+    per_shape = {}
+    for i, (name, R, N) in enumerate(shapes):
+        f, y = fmts[i], ys[i]
+        fn = lambda k, i=i, f=f, y=y: sl.gemv(f, layers[k % args.layers][i]["rec"], None,  # noqa
+                                             xs[layers[0][i]["N"]], y)
+        reps = min(args.steps, 400)
+        us = time_region(torch, fn, reps) / reps * 1e3
+        C, P = cp
+        nb = (N + C - 1) // C
+        per_shape[name] = {"us": round(us, 2),
+                           "compressed_gbs": round(R * nb * 4 / us / 1e3, 1),
+                           "fp16_equiv_gbs": round(2 * R * N / us / 1e3, 1)}
+
+    traffic = profile_traffic("gemv_kernel<8>")
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
@@ -481,12 +492,13 @@ def seedlm_arm(args):
                          f"({comp / 1e6:.0f} MB) of {args.layers} resident",
                    "parallelism": f"replicas x{world} (independent layer stacks per GPU)"},
         "us_per_gemv": round(ms * 1e3 / (args.steps * len(shapes)), 3),
+        "per_shape": per_shape,
         "compressed_gbs": round(comp_gbs, 1),
         "hbm_roofline_pct": round(100 * comp_gbs / hbm_peak, 2),
         "hbm_roofline_pct_of_8tbs_spec": round(100 * comp_gbs / 8000, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "kernel": "gemv_c8_kernel",
+                     "kernel": "gemv_kernel<8>",
                      "traffic": None if traffic is None else traffic["bytes_per_launch"],
                      "algorithmic_bytes_per_launch": round(alg / len(shapes))},
         "clocks": clk.result(),

@@ -108,9 +108,26 @@ SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const 
                 const void* x, int x_dtype, float* y, seedlm_stream stream);
 
 /* Y = X W^T for a small batch: X is M x cols (row-major, type x_dtype), Y is
- * M x rows fp32 (row-major).  1 <= M <= 64. */
+ * M x rows fp32 (row-major), 1 <= M <= 64.  M = 1 runs the GEMV kernel; for
+ * M >= 2 the rebuilt weight tiles feed the tcgen05 tensor cores (tf32 hi/lo
+ * pieces, exact products, fp32 accumulation in TMEM).  `workspace` is device
+ * memory of at least seedlm_gemm_smallM_workspace_bytes(fmt, M) bytes,
+ * 256-byte aligned (may be NULL when that size is 0).  It holds split-K
+ * partial sums and per-tile counters: it must be zero-filled before its first
+ * use, every call leaves it ready for the next, and calls sharing one
+ * workspace must not run concurrently (calls on one stream never do). */
 SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
-                       const void* X, int x_dtype, int M, float* Y, seedlm_stream stream);
+                       const void* X, int x_dtype, int M, float* Y, void* workspace,
+                       int64_t workspace_bytes, seedlm_stream stream);
+
+/* Workspace bytes seedlm_gemm_smallM needs for this format and M on the
+ * current device (HOST function; 0 if none, negative on error). */
+SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M);
+
+/* Reads and clears the device-side error flag of the current device: 1 if a
+ * kernel gave up waiting on one of its own barriers (the outputs of that call
+ * are then undefined), else 0.  HOST function; synchronous. */
+SEEDLM_API int seedlm_device_error(int* flag);
 
 /* Reference point, not part of the method: y = W x with W dense fp16
  * (rows x cols, row-major, leading dimension ldw halves, 16-byte aligned with

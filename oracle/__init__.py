@@ -193,3 +193,15 @@ def gemv_rows(fmt, rec, eplane, x, rows):
     if fmt["P"] == 4:
         ep = np.asarray(eplane).reshape(fmt["rows"], fmt["e_pitch"])[rows]
     return gemv(sub, rec, ep, x)
+
+
+def gemm_rows(fmt, rec, eplane, X, rows):
+    """Y and Yabs (M, len(rows)) for a subset of rows only."""
+    rows = np.asarray(rows, dtype=np.int64)
+    sub = dict(fmt)
+    sub["rows"] = len(rows)
+    rec = np.asarray(rec).reshape(fmt["rows"], fmt["rec_pitch"])[rows]
+    ep = None
+    if fmt["P"] == 4:
+        ep = np.asarray(eplane).reshape(fmt["rows"], fmt["e_pitch"])[rows]
+    return gemm(sub, rec, ep, X)

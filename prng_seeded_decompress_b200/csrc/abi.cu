@@ -134,12 +134,13 @@ int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* ep
 }
 
 int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
-                       const void* X, int x_dtype, int M, float* Y, seedlm_stream stream) {
+                       const void* X, int x_dtype, int M, float* Y, void* workspace,
+                       int64_t workspace_bytes, seedlm_stream stream) {
   int rc = check_format(fmt);
   if (rc) return rc;
   if ((rc = check_planes(fmt, rec, eplane))) return rc;
   if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
-  if (M < 1 || M > 64) return SEEDLM_EINVAL;
+  if (M < 1 || M > 64 || workspace_bytes < 0) return SEEDLM_EINVAL;
   if (fmt->rows == 0) return SEEDLM_OK;
   if (!Y || !aligned(Y, 4)) return SEEDLM_EINVAL;
   if (fmt->cols > 0 && (!X || !aligned(X, 2))) return SEEDLM_EINVAL;
@@ -148,8 +149,32 @@ int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint
   if (fmt->cols == 0)
     return record_cuda_error(
         cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), (cudaStream_t)stream));
-  return launch_gemm_small(*fmt, rec, eplane, static_cast<const uint16_t*>(X),
-                           x_dtype == SEEDLM_BF16, M, Y, (cudaStream_t)stream, dev);
+  const uint16_t* Xh = static_cast<const uint16_t*>(X);
+  if (M == 1)
+    return launch_gemv(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, Y, (cudaStream_t)stream,
+                       dev);
+  return launch_gemm_tc(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, M, Y, workspace,
+                        workspace_bytes, (cudaStream_t)stream, dev);
+}
+
+int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M) {
+  if (check_format(fmt) || M < 1 || M > 64) return SEEDLM_EINVAL;
+  if (M == 1 || fmt->rows == 0 || fmt->cols == 0) return 0;
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  return gemm_tc_workspace_bytes(*fmt, M, dev);
+}
+
+int seedlm_device_error(int* flag) {
+  if (!flag) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  unsigned int v = 0;
+  if ((rc = read_and_clear_tc_error(&v))) return rc;
+  *flag = v ? 1 : 0;
+  return SEEDLM_OK;
 }
 
 int seedlm_dense_gemv_f16(int32_t rows, int32_t cols, const uint16_t* W, int64_t ldw,

@@ -154,7 +154,7 @@ __device__ __forceinline__ BlockC8 decode_c8(uint32_t rec, const uint32_t* __res
                                              const uint32_t* __restrict__ t_hi) {
   BlockC8 b;
   b.lo = rec;
-  b.hi = t_lo[(rec >> 16) & 0xffu] ^ t_hi[rec >> 24];
+  b.hi = t_lo[prmt<0x4442u>(rec, 0u)] ^ t_hi[rec >> 24];  // seed bytes 0 and 1
   // (q0, q1, q1, q2) as nibbles, one per byte, then sign-extended.
   uint32_t v = prmt<0x1440u>(rec, rec >> 4) & 0x0f0f0f0fu;
   uint32_t s = sext_nibble_bytes(v);

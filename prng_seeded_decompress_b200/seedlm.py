@@ -19,6 +19,7 @@ BF16 = 1
 #: Every symbol include/seedlm.h declares.
 EXPORTS = (
     "seedlm_init", "seedlm_decompress", "seedlm_gemv", "seedlm_gemm_smallM",
+    "seedlm_gemm_smallM_workspace_bytes", "seedlm_device_error",
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
 )
@@ -53,7 +54,9 @@ def _load():
         "seedlm_decompress": (ctypes.c_int, [fmtp, vp, vp, vp, i64, vp]),
         "seedlm_gemv": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, vp, vp]),
         "seedlm_gemm_smallM": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp,
-                                              vp]),
+                                              vp, i64, vp]),
+        "seedlm_gemm_smallM_workspace_bytes": (i64, [fmtp, ctypes.c_int]),
+        "seedlm_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
         "seedlm_dense_gemv_f16": (ctypes.c_int, [i32, i32, vp, i64, vp, vp, vp]),
         "seedlm_row_bytes_ideal": (i64, [fmtp]),
         "seedlm_row_bytes_stored": (i64, [fmtp]),
@@ -144,12 +147,43 @@ def gemv(fmt, rec, eplane, x, y, stream=None):
         _stream(stream, y)))
 
 
-def gemm_smallM(fmt, rec, eplane, X, Y, stream=None):
-    """Y = X W^T; X float16/bfloat16 (M, cols), Y float32 (M, rows)."""
+def gemm_workspace_bytes(fmt, M: int) -> int:
+    n = int(lib.seedlm_gemm_smallM_workspace_bytes(ctypes.byref(_fmt(fmt)), int(M)))
+    if n < 0:
+        _check("seedlm_gemm_smallM_workspace_bytes", n)
+    return n
+
+
+def gemm_workspace(fmt, M: int, device=None):
+    """A zero-filled device workspace for seedlm_gemm_smallM (torch uint8 tensor).
+
+    It can be reused by every later call with the same or a smaller need;
+    calls that share it must not run concurrently."""
+    import torch
+    n = gemm_workspace_bytes(fmt, M)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def gemm_smallM(fmt, rec, eplane, X, Y, workspace=None, stream=None):
+    """Y = X W^T; X float16/bfloat16 (M, cols), Y float32 (M, rows).
+
+    `workspace` comes from gemm_workspace(); if omitted a fresh one is made."""
     f = _fmt(fmt)
+    M = int(X.shape[0])
+    if workspace is None:
+        workspace = gemm_workspace(f, M, device=Y.device)
+    nbytes = workspace.numel() * workspace.element_size()
     _check("seedlm_gemm_smallM", lib.seedlm_gemm_smallM(
-        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), int(X.shape[0]),
-        _ptr(Y), _stream(stream, Y)))
+        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), M, _ptr(Y),
+        _ptr(workspace), nbytes, _stream(stream, Y)))
+
+
+def device_error() -> int:
+    """1 if a kernel gave up on one of its own bounded waits since the last
+    check (and clears the flag), else 0.  Synchronous."""
+    flag = ctypes.c_int(0)
+    _check("seedlm_device_error", lib.seedlm_device_error(ctypes.byref(flag)))
+    return int(flag.value)
 
 
 def dense_gemv_f16(W, x, y, stream=None):

@@ -190,32 +190,71 @@ def test_decompress_then_dense_equals_fused(sl, oracle_mod):
 
 # ------------------------------------------------------------ small-M GEMM
 
+def gpu_gemm(sl, L, Xb, dtype="bf16", workspace=None):
+    rec, ep = planes(L)
+    M = Xb.shape[0]
+    X = act_tensor(Xb, dtype)
+    Y = torch.full((M, L["fmt"]["rows"]), float("nan"), device="cuda")
+    sl.gemm_smallM(L["fmt"], rec, ep, X, Y, workspace=workspace)
+    torch.cuda.synchronize()
+    assert sl.device_error() == 0
+    return Y.cpu().numpy().astype(np.float64)
+
+
 @pytest.mark.parametrize("cp", [C8, C12])
-@pytest.mark.parametrize("M", [1, 3, 8, 16, 64])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 17, 33, 64])
 def test_gemm_small_matches_oracle(sl, oracle_mod, cp, M):
-    rows, cols = 150, 2000
+    rows, cols = 300, 3000  # 3 row tiles (one ragged), ragged last stage, split-K
     L = inputs.make_layer(rows, cols, *cp, seed=50 + M)
     Xb, Xv = inputs.make_activations((M, cols), "bf16", 60 + M)
-    rec, ep = planes(L)
-    X = act_tensor(Xb, "bf16")
-    Y = torch.full((M, rows), float("nan"), device="cuda")
-    sl.gemm_smallM(L["fmt"], rec, ep, X, Y)
-    torch.cuda.synchronize()
+    got = gpu_gemm(sl, L, Xb)
     ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv)
-    got = Y.cpu().numpy().astype(np.float64)
     for m in range(M):
         assert_within(got[m], ref[m], refabs[m])
 
 
-def test_gemm_m1_equals_gemv_within_tolerance(sl, oracle_mod):
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_gemm_small_fp16_and_odd_shapes(sl, oracle_mod, cp):
+    for rows, cols, M in ((1, 12, 5), (129, 100, 16), (70, 1000, 40)):
+        L = inputs.make_layer(rows, cols, *cp, seed=rows + cols + M)
+        Xb, Xv = inputs.make_activations((M, cols), "f16", 5)
+        got = gpu_gemm(sl, L, Xb, "f16")
+        ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv)
+        for m in range(M):
+            assert_within(got[m], ref[m], refabs[m])
+
+
+def test_gemm_workspace_reuse_is_deterministic(sl):
+    # The same workspace across calls (counters must be left at zero) and
+    # bit-identical results (split-K partials are added in a fixed order).
+    L = inputs.make_layer(1000, 8192, *C8, seed=81)
+    Xb, _ = inputs.make_activations((64, 8192), "bf16", 82)
+    ws = sl.gemm_workspace(L["fmt"], 64)
+    a = gpu_gemm(sl, L, Xb, workspace=ws)
+    b = gpu_gemm(sl, L, Xb, workspace=ws)
+    assert np.array_equal(a.view(np.uint64), b.view(np.uint64))
+
+
+@pytest.mark.parametrize("cp,rows,cols,M", [(C8, 8192, 28672, 64), (C8, 28672, 8192, 16),
+                                            (C12, 8192, 28672, 16), (C12, 28672, 8192, 64)])
+def test_gemm_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols, M):
+    L = inputs.make_layer(rows, cols, *cp, seed=rows + cols + M)
+    Xb, Xv = inputs.make_activations((M, cols), "bf16", 91)
+    got = gpu_gemm(sl, L, Xb)
+    rng = np.random.default_rng(1)
+    sample = np.unique(np.concatenate([np.arange(4), np.arange(rows - 4, rows),
+                                       rng.integers(0, rows, 12)]))
+    ref, refabs = oracle_mod.gemm_rows(L["fmt"], L["rec"], L["eplane"], Xv, sample)
+    for m in range(M):
+        assert_within(got[m, sample], ref[m], refabs[m])
+
+
+def test_gemm_m1_equals_gemv_bitwise(sl):
     L = inputs.make_layer(256, 4096, *C8, seed=71)
-    xb, xv = inputs.make_activations((1, 4096), "bf16", 72)
-    rec, ep = planes(L)
-    Y = torch.empty((1, 256), device="cuda")
-    sl.gemm_smallM(L["fmt"], rec, ep, act_tensor(xb, "bf16"), Y)
+    xb, _ = inputs.make_activations((1, 4096), "bf16", 72)
+    got = gpu_gemm(sl, L, xb)
     y = gpu_gemv(sl, L, xb[0], "bf16")
-    _, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv[0])
-    assert np.all(np.abs(Y.cpu().numpy()[0] - y) <= 2 * TOL * refabs + 1e-30)
+    assert np.array_equal(got[0], y)
 
 
 # --------------------------------------------------------- dense reference
