@@ -555,6 +555,43 @@ def reference_arm(args):
     }), flush=True)
 
 
+def profile_case(name: str):
+    """One small single-kernel workload for an ncu capture (inputs > L2)."""
+    import numpy as np
+    import torch
+
+    from prng_seeded_decompress_b200 import build, inputs
+    build.build()
+    from prng_seeded_decompress_b200 import seedlm as sl
+    sl.init()
+    if name == "decompress":
+        L = inputs.make_layer(8192, 28672, 8, 3, seed=1)
+        rec = torch.from_numpy(L["rec"].view(np.int32)).cuda()
+        W = torch.empty((8192, 28672), device="cuda")
+        for _ in range(3):
+            sl.decompress(L["fmt"], rec, None, W)
+    elif name in ("gemm64", "gemm16"):
+        M = 64 if name == "gemm64" else 16
+        L = inputs.make_layer(28672, 8192, 8, 3, seed=2)
+        rec = torch.from_numpy(L["rec"].view(np.int32)).cuda()
+        Xb, _ = inputs.make_activations((M, 8192), "bf16", 3)
+        X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+        Y = torch.empty((M, 28672), device="cuda")
+        ws = sl.gemm_workspace(L["fmt"], M)
+        for _ in range(3):
+            sl.gemm_smallM(L["fmt"], rec, None, X, Y, workspace=ws)
+    elif name == "dense":
+        W = torch.randn((57344, 8192), device="cuda").half()
+        x = torch.randn(8192, device="cuda").half()
+        y = torch.empty(57344, device="cuda")
+        for _ in range(3):
+            sl.dense_gemv_f16(W, x, y)
+    torch.cuda.synchronize()
+    if sl.device_error():
+        raise SystemExit("device error flag raised")
+    print(f"case {name} ok", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -566,7 +603,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
+    ap.add_argument("--case", choices=("decompress", "gemm64", "gemm16", "dense"),
+                    help="run one small single-kernel workload (for ncu) and exit")
     args = ap.parse_args()
+    if args.case:
+        profile_case(args.case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -1,11 +1,12 @@
 // decompress.cu -- W = the rebuilt weights, written out in fp32.
 //
 // Eq (1) of the paperhub.cn review thread, W_blk = U t, applied to every
-// block.  A thread takes 4 consecutive blocks of a row (one 16-byte record
-// load), rebuilds their weights exactly (see seedlm_device.cuh) and stores
-// them with 16-byte streaming stores when the destination allows.  The kernel
-// is bound by the 4 bytes per weight it writes, eight times the 0.5 bytes per
-// weight it reads.
+// block.  A lane takes 4 consecutive blocks of a row (one 16-byte record
+// load) and rebuilds their weights exactly (see seedlm_device.cuh); a warp's
+// 32 lanes cover 128 consecutive blocks, staged in shared memory and written
+// out with fully coalesced 16-byte streaming stores.  The kernel is bound by
+// the 4 bytes per weight it writes, eight times the 0.5 bytes per weight it
+// reads.
 #include <cuda_runtime.h>
 
 #include "seedlm_device.cuh"
@@ -72,19 +73,21 @@ __device__ __forceinline__ void rebuild_block(uint32_t word, uint32_t e4, const 
   }
 }
 
-// One thread per chunk of 4 blocks (grid-stride, next chunk loaded before
-// the current one is rebuilt).  Chunks never straddle rows; blocks of a
-// chunk at or past nb are skipped (rec_pitch covers the 16-byte load).
+// A warp item is 32 consecutive chunks (4 blocks each) of one row: lane l
+// rebuilds chunk 32j + l into its slice of a per-warp staging buffer (one
+// padding float4 per lane keeps the writes conflict-free).  Float4 f of the
+// item belongs to column 128 j C + 4 f, so the warp then writes the item
+// back with store instructions that each cover 512 contiguous bytes.  The
+// next item's records are loaded before the current one is rebuilt.
 template <int C>
 __global__ void __launch_bounds__(kThreads)
 decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane, int rows,
                   int cols, int nb, int rec_pitch, int e_pitch, float* __restrict__ W, int64_t ldw,
                   int vec) {
-  // Jump tables: 32-bit words for C = 8 (stream bits 16..47 suffice), 64-bit
-  // for C = 12 (bits 16..79).
-  __shared__ __align__(16) unsigned char tab[512 * 8];
-  uint32_t* t32 = reinterpret_cast<uint32_t*>(tab);
-  uint2* t64 = reinterpret_cast<uint2*>(tab);
+  constexpr int F = C;  // float4 per chunk (4 blocks x C floats / 4)
+  extern __shared__ __align__(16) unsigned char dsm[];
+  uint32_t* t32 = reinterpret_cast<uint32_t*>(dsm);
+  uint2* t64 = reinterpret_cast<uint2*>(dsm);
   for (int i = threadIdx.x; i < 512; i += kThreads) {
     uint64_t v = i < 256 ? kStreamTables.lo[i] : kStreamTables.hi[i - 256];
     if constexpr (C == 8)
@@ -93,45 +96,61 @@ decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ 
       t64[i] = make_uint2((uint32_t)v, (uint32_t)(v >> 32));
   }
   __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* stage = reinterpret_cast<float4*>(dsm + 512 * 8) + warp * 32 * (F + 1);
   const int cpr = (nb + kRecs - 1) / kRecs;  // chunks per row
-  const int64_t total = (int64_t)rows * cpr;
-  const int64_t step = (int64_t)gridDim.x * kThreads;
-  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (i >= total) return;
-  int r = (int)(i / cpr), k = (int)(i - (int64_t)r * cpr);
-  Chunk cur = load_chunk<C>(rec, eplane, rec_pitch, e_pitch, r, k);
+  const int ipr = (cpr + 31) / 32;           // warp items per row
+  const int64_t items = (int64_t)rows * ipr;
+  const int64_t wstep = (int64_t)gridDim.x * (kThreads / 32);
+  int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + warp;
+  if (it >= items) return;
+  auto locate = [&](int64_t item, int& r, int& k) {
+    r = (int)(item / ipr);
+    k = (int)(item - (int64_t)r * ipr) * 32 + lane;
+  };
+  int r, k;
+  locate(it, r, k);
+  Chunk cur = k < cpr ? load_chunk<C>(rec, eplane, rec_pitch, e_pitch, r, k) : Chunk{};
   while (true) {
-    const int64_t inext = i + step;
+    const int64_t inext = it + wstep;
     int rn = 0, kn = 0;
-    Chunk nxt;
-    if (inext < total) {
-      rn = (int)(inext / cpr);
-      kn = (int)(inext - (int64_t)rn * cpr);
-      nxt = load_chunk<C>(rec, eplane, rec_pitch, e_pitch, rn, kn);
+    Chunk nxt{};
+    if (inext < items) {
+      locate(inext, rn, kn);
+      if (kn < cpr) nxt = load_chunk<C>(rec, eplane, rec_pitch, e_pitch, rn, kn);
     }
     const uint32_t words[kRecs] = {cur.rec.x, cur.rec.y, cur.rec.z, cur.rec.w};
 #pragma unroll
     for (int q = 0; q < kRecs; ++q) {
-      const int b = kRecs * k + q;
-      if (b < nb) {
-        float w[C];
-        rebuild_block<C>(words[q], (cur.e >> (4 * q)) & 15u, t32, t64, w);
-        float* dst = W + (size_t)r * (size_t)ldw + (size_t)b * C;
-        const int j0 = b * C;
-        if (vec && j0 + C <= cols) {
+      float w[C];
+      rebuild_block<C>(words[q], (cur.e >> (4 * q)) & 15u, t32, t64, w);
 #pragma unroll
-          for (int v = 0; v < C / 4; ++v)
-            __stcs(reinterpret_cast<float4*>(dst) + v,
-                   make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
-        } else {
+      for (int v = 0; v < C / 4; ++v)
+        stage[lane * (F + 1) + q * (C / 4) + v] =
+            make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    }
+    __syncwarp();
+    const int j = (k - lane) / 32;  // item index within the row
+    float* dst_row = W + (size_t)r * (size_t)ldw + (size_t)128 * j * C;
+    const int col0 = 128 * j * C;
 #pragma unroll
-          for (int c = 0; c < C; ++c)
-            if (j0 + c < cols) dst[c] = w[c];
-        }
+    for (int q = 0; q < F; ++q) {
+      const int ff = q * 32 + lane;
+      const int c = ff / F, v = ff - c * F;
+      const float4 val = stage[c * (F + 1) + v];
+      const int j0 = col0 + 4 * ff;
+      if (vec && j0 + 4 <= cols) {
+        __stcs(reinterpret_cast<float4*>(dst_row + 4 * ff), val);
+      } else if (j0 < cols) {
+        const float e4[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (j0 + u < cols) dst_row[4 * ff + u] = e4[u];
       }
     }
-    if (inext >= total) return;
-    i = inext;
+    __syncwarp();
+    if (inext >= items) return;
+    it = inext;
     r = rn;
     k = kn;
     cur = nxt;
@@ -142,18 +161,26 @@ decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ 
 
 int launch_decompress(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane, float* W,
                       int64_t ldw, cudaStream_t stream, const DeviceInfo& dev) {
-  const int64_t total = (int64_t)f.rows * ((f.nb + kRecs - 1) / kRecs);
-  if (total == 0) return SEEDLM_OK;
+  const int cpr = (f.nb + kRecs - 1) / kRecs;
+  const int64_t items = (int64_t)f.rows * ((cpr + 31) / 32);
+  if (items == 0) return SEEDLM_OK;
   const int vec = ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && (ldw % 4) == 0) ? 1 : 0;
-  int64_t want = (total + kThreads - 1) / kThreads;
-  int64_t cap = (int64_t)dev.num_sms * 16;
+  const int warps = kThreads / 32;
+  int64_t want = (items + warps - 1) / warps;
+  int64_t cap = (int64_t)dev.num_sms * 4;
   int grid = (int)(want < cap ? want : cap);
-  if (f.C == 8)
-    decompress_kernel<8><<<grid, kThreads, 0, stream>>>(rec, eplane, f.rows, f.cols, f.nb,
-                                                        f.rec_pitch, f.e_pitch, W, ldw, vec);
-  else
-    decompress_kernel<12><<<grid, kThreads, 0, stream>>>(rec, eplane, f.rows, f.cols, f.nb,
-                                                         f.rec_pitch, f.e_pitch, W, ldw, vec);
+  const size_t smem = 512 * 8 + (size_t)warps * 32 * (f.C + 1) * 16;
+  if (f.C == 8) {
+    int rc = allow_max_smem((const void*)decompress_kernel<8>, dev);
+    if (rc) return rc;
+    decompress_kernel<8><<<grid, kThreads, smem, stream>>>(rec, eplane, f.rows, f.cols, f.nb,
+                                                           f.rec_pitch, f.e_pitch, W, ldw, vec);
+  } else {
+    int rc = allow_max_smem((const void*)decompress_kernel<12>, dev);
+    if (rc) return rc;
+    decompress_kernel<12><<<grid, kThreads, smem, stream>>>(rec, eplane, f.rows, f.cols, f.nb,
+                                                            f.rec_pitch, f.e_pitch, W, ldw, vec);
+  }
   count_launch();
   return record_cuda_error(cudaGetLastError());
 }

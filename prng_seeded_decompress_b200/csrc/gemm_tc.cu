@@ -9,8 +9,9 @@
 //   * D = W_tile (128 rows) x X^T (NB columns, NB = batch rounded up to 16)
 //     accumulates in TMEM in fp32 (128 lanes x NB columns).
 //   * Each K stage (64 columns for C = 8, 48 for C = 12, i.e. a whole number
-//     of blocks) is built by all 256 threads: two threads per W row load the
-//     row's records for the stage, rebuild the weights exactly in fp32 (see
+//     of blocks) is built by all 512 threads: four threads per W row load the
+//     row's records for the stage (one stage ahead, into registers), rebuild
+//     the weights exactly in fp32 (see
 //     seedlm_device.cuh) and split each into tf32 pieces hi + lo, both exact
 //     (a weight has at most 21 significant bits; tf32 keeps 11).  X is
 //     converted to fp32, which tf32 holds exactly for fp16 or bf16 inputs.
@@ -40,7 +41,7 @@ __device__ unsigned int g_tc_error = 0;
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
 template <int C>
@@ -59,6 +60,7 @@ struct TcCfg<12> {
 struct TcGeom {
   int rows, cols, nb, rec_pitch, e_pitch, M;
   int splits, chunks_per_split, nchunks, tiles;
+  int x_vec;  // X rows are 8-byte aligned and cols % 4 == 0: load X 4 elements at a time
 };
 
 template <int C, int NB>
@@ -126,37 +128,74 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   const uint32_t idesc = tc::idesc_tf32(NB);
   bool ok = true;
 
-  // Producer roles: thread t rebuilds half of the stage's blocks of W row t/2.
-  const int prow = tid >> 1, phalf = tid & 1;
+  // Producer roles: four threads per W row, each rebuilding a quarter of the
+  // row's blocks of the stage; the X slice is split over all threads.  The
+  // next stage's records and X values are loaded before the current stage is
+  // built.
+  constexpr int BPT = BLK / 4;                                // blocks per thread
+  constexpr int XCH = NB * (KC / 4);                          // 4-element X chunks per stage
+  constexpr int XPT = (XCH + kThreads - 1) / kThreads;        // X chunks per thread
+  // Warp w owns rows 8w..8w+7; lane l takes row 8w + (l & 7) and quarter
+  // l >> 3, so the 8 lanes of a quarter-warp store to 8 different rows of a
+  // core matrix (distinct banks).
+  const int prow = 8 * warp + (lane & 7), pq = lane >> 3;
   const int gr = r0 + prow;
   const bool row_ok = gr < g.rows;
 
+  struct Pref {
+    uint32_t w[BPT];
+    uint32_t e;
+    uint2 x[XPT];
+  };
+  auto load_pref = [&](int chunk, Pref& p) {
+    const int b_first = chunk * BLK + pq * BPT;
+    const bool blk_ok = row_ok && b_first < g.nb;
+    if constexpr (BPT == 2) {
+      uint2 v = blk_ok ? ld_stream_u2(rec + (size_t)gr * g.rec_pitch + b_first) : make_uint2(0u, 0u);
+      p.w[0] = v.x;
+      p.w[1] = v.y;
+    } else {
+      p.w[0] = blk_ok ? __ldg(rec + (size_t)gr * g.rec_pitch + b_first) : 0u;
+    }
+    p.e = 0;
+    if constexpr (C == 12)
+      p.e = blk_ok ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b_first >> 1)) : 0u;
+#pragma unroll
+    for (int k = 0; k < XPT; ++k) {
+      const int i = tid + k * kThreads;
+      const int k4 = i / NB, n = i - k4 * NB;  // n fastest: distinct banks when stored
+      const int col = chunk * KC + 4 * k4;
+      uint2 v = make_uint2(0u, 0u);
+      if (i < XCH && n < g.M) {
+        const uint16_t* src = X + (size_t)n * g.cols + col;
+        if (g.x_vec) {
+          if (col < g.cols) v = __ldg(reinterpret_cast<const uint2*>(src));
+        } else {
+          uint32_t h[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) h[u] = col + u < g.cols ? (uint32_t)__ldg(src + u) : 0u;
+          v = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+        }
+      }
+      p.x[k] = v;
+    }
+  };
+
+  Pref cur, nxt;
+  if (n_iter > 0) load_pref(c_begin, cur);
   for (int it = 0; it < n_iter; ++it) {
     const int s = it % STAGES;
     const int use = it / STAGES;
     unsigned char* st = smem + s * L::STAGE_BYTES;
+    if (it + 1 < n_iter) load_pref(c_begin + it + 1, nxt);
     if (use > 0) ok = tc::mbar_wait(bar0 + 8 * s, (use - 1) & 1, kWaitLimit) && ok;
-    const int chunk = c_begin + it;
 
     // ---- A: rebuilt weights, hi and lo tf32 pieces
-    const int b_first = chunk * BLK + phalf * (BLK / 2);
-    uint32_t words[BLK / 2];
-    uint32_t ebyte = 0;
-    const bool blk_ok = row_ok && b_first < g.nb;
-    if constexpr (C == 8) {
-      uint4 v = blk_ok ? ld_stream_u4(rec + (size_t)gr * g.rec_pitch + b_first)
-                       : make_uint4(0u, 0u, 0u, 0u);
-      words[0] = v.x; words[1] = v.y; words[2] = v.z; words[3] = v.w;
-    } else {
-      uint2 v = blk_ok ? ld_stream_u2(rec + (size_t)gr * g.rec_pitch + b_first) : make_uint2(0u, 0u);
-      words[0] = v.x; words[1] = v.y;
-      ebyte = blk_ok ? ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b_first >> 1)) : 0u;
-    }
 #pragma unroll
-    for (int i = 0; i < BLK / 2; ++i) {
+    for (int i = 0; i < BPT; ++i) {
       float w[C];
       if constexpr (C == 8) {
-        const BlockC8 blk = decode_c8(words[i], t32, t32 + 256);
+        const BlockC8 blk = decode_c8(cur.w[i], t32, t32 + 256);
         const float nm = __uint_as_float(blk.negm);
         w[0] = __int_as_float(weight_bits_c8<0>(blk)) + nm;
         w[1] = __int_as_float(weight_bits_c8<1>(blk)) + nm;
@@ -167,7 +206,9 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         w[6] = __int_as_float(weight_bits_c8<6>(blk)) + nm;
         w[7] = __int_as_float(weight_bits_c8<7>(blk)) + nm;
       } else {
-        const BlockC12 blk = decode_c12(words[i], (ebyte >> (4 * i)) & 15u, t64, t64 + 256);
+        const int b_first = (c_begin + it) * BLK + pq * BPT;
+        const uint32_t e4 = (b_first & 1) ? (cur.e >> 4) : cur.e;
+        const BlockC12 blk = decode_c12(cur.w[i], e4 & 15u, t64, t64 + 256);
         const float nm = __uint_as_float(blk.negm);
         w[0] = __int_as_float(weight_bits_c12<0>(blk)) + nm;
         w[1] = __int_as_float(weight_bits_c12<1>(blk)) + nm;
@@ -182,7 +223,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         w[10] = __int_as_float(weight_bits_c12<10>(blk)) + nm;
         w[11] = __int_as_float(weight_bits_c12<11>(blk)) + nm;
       }
-      const int k4_0 = (phalf * (BLK / 2) + i) * (C / 4);
+      const int k4_0 = (pq * BPT + i) * (C / 4);
 #pragma unroll
       for (int q = 0; q < C / 4; ++q) {
         float h[4], l[4];
@@ -195,16 +236,18 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     }
 
     // ---- B: X[:, stage columns] as fp32 (exact in tf32), zero-padded
-    for (int i = tid; i < NB * (KC / 4); i += kThreads) {
-      const int n = i / (KC / 4), k4 = i - n * (KC / 4);
-      const int col = chunk * KC + 4 * k4;
-      float v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = (n < g.M && col + u < g.cols) ? act_to_float(X[(size_t)n * g.cols + col + u], is_bf16)
-                                             : 0.f;
-      *reinterpret_cast<float4*>(st + 2 * L::A_BYTES + core_off<L::SBO>(n, k4)) =
-          make_float4(v[0], v[1], v[2], v[3]);
+    for (int k = 0; k < XPT; ++k) {
+      const int i = tid + k * kThreads;
+      if (i < XCH) {
+        const int k4 = i / NB, n = i - k4 * NB;
+        const uint2 v = cur.x[k];
+        const float4 f = make_float4(act_to_float((uint16_t)(v.x & 0xffffu), is_bf16),
+                                     act_to_float((uint16_t)(v.x >> 16), is_bf16),
+                                     act_to_float((uint16_t)(v.y & 0xffffu), is_bf16),
+                                     act_to_float((uint16_t)(v.y >> 16), is_bf16));
+        *reinterpret_cast<float4*>(st + 2 * L::A_BYTES + core_off<L::SBO>(n, k4)) = f;
+      }
     }
 
     tc::fence_proxy_async_smem();
@@ -222,6 +265,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       }
       tc::mma_commit(bar0 + 8 * s);
     }
+    cur = nxt;
   }
 
   // ---- epilogue: wait for the last MMAs, read D, write Y or a partial
@@ -301,6 +345,7 @@ TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev) {
   g.splits = want < 1 ? 1 : (want > cap ? cap : want);
   g.chunks_per_split = (g.nchunks + g.splits - 1) / g.splits;
   g.splits = (g.nchunks + g.chunks_per_split - 1) / g.chunks_per_split;
+  g.x_vec = 0;
   return g;
 }
 
@@ -332,7 +377,8 @@ int64_t gemm_tc_workspace_bytes(const seedlm_format& f, int M, const DeviceInfo&
 int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                    const uint16_t* X, int is_bf16, int M, float* Y, void* workspace,
                    int64_t workspace_bytes, cudaStream_t stream, const DeviceInfo& dev) {
-  const TcGeom g = make_tc_geom(f, M, dev);
+  TcGeom g = make_tc_geom(f, M, dev);
+  g.x_vec = (f.cols % 4 == 0 && (reinterpret_cast<uintptr_t>(X) & 7u) == 0) ? 1 : 0;
   const int64_t need = gemm_tc_workspace_bytes(f, M, dev);
   if (workspace_bytes < need) return SEEDLM_EINVAL;
   float* partial = nullptr;

@@ -20,6 +20,10 @@
 //     to within one item.  Row sums are reduced with warp shuffles and then
 //     across warps in shared memory, in a fixed order, so every call gives
 //     the same bits.
+//   * Launched with programmatic stream serialization: the first record
+//     loads are issued before griddepcontrol.wait, so back-to-back GEMVs
+//     overlap one kernel's tail with the next one's prologue; x is read only
+//     after the wait.
 #include <cuda_runtime.h>
 
 #include "seedlm_device.cuh"
@@ -185,7 +189,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
             const uint16_t* __restrict__ x, int is_bf16, float* __restrict__ y, GemvGeom g) {
   extern __shared__ __align__(16) unsigned char smem[];
-  stage_x_and_tables<C>(smem, x, is_bf16, g);
   const void* t_lo = smem;
   const void* t_hi = smem + Smem<C>::kTableBytes / 2;
   float* part = reinterpret_cast<float*>(smem + Smem<C>::kTableBytes);
@@ -197,22 +200,32 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
   const int g0 = (int)((int64_t)blockIdx.x * g.groups / gridDim.x);
   const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
 
+  bool first_pass = true;
   for (int p0 = g0; p0 < g1; p0 += kMaxGroups) {
     const int p1 = min(p0 + kMaxGroups, g1);
-    for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x) part[i] = 0.f;
-    __syncthreads();  // x, tables and zeroed partials ready
     const int items = (p1 - p0) * g.n_spans;
     const int i0 = (int)((int64_t)warp * items / nw), i1 = (int)((int64_t)(warp + 1) * items / nw);
-    if (i0 < i1) {
-      int grp = p0 + i0 / g.n_spans, span = i0 % g.n_spans;  // item being rebuilt
-      int lgrp = grp, lspan = span, li = i0;                   // next item to load
-      RecSet<C> buf[kPrefetch + 1];
+    // The first record sets are requested before anything else: they do not
+    // depend on x, so their latency overlaps the staging of x (and, with
+    // programmatic dependent launch, the tail of the previous kernel).
+    int grp = p0 + (i0 < i1 ? i0 / g.n_spans : 0), span = i0 < i1 ? i0 % g.n_spans : 0;
+    int lgrp = grp, lspan = span, li = i0;
+    RecSet<C> buf[kPrefetch + 1];
 #pragma unroll
-      for (int k = 0; k <= kPrefetch; ++k) {
-        if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
-        ++li;
-        if (++lspan == g.n_spans) { lspan = 0; ++lgrp; }
-      }
+    for (int k = 0; k <= kPrefetch; ++k) {
+      if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
+      ++li;
+      if (++lspan == g.n_spans) { lspan = 0; ++lgrp; }
+    }
+    if (first_pass) {
+      // x may be the previous kernel's output: wait for it only now.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      stage_x_and_tables<C>(smem, x, is_bf16, g);
+      first_pass = false;
+    }
+    for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x) part[i] = 0.f;
+    __syncthreads();  // x, tables and zeroed partials ready
+    if (i0 < i1) {
       float2 acc[kRowsPerTask];
 #pragma unroll
       for (int j = 0; j < kRowsPerTask; ++j) acc[j] = make_float2(0.f, 0.f);
@@ -243,6 +256,10 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
       }
     }
     __syncthreads();
+    if (p1 == g1) {
+      // The next kernel in the stream may start its prologue now.
+      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     for (int t = threadIdx.x; t < (p1 - p0) * kRowsPerTask; t += blockDim.x) {
       const int r = p0 * kRowsPerTask + t;
       if (r < g.rows) {
@@ -293,10 +310,20 @@ int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* epla
   const void* kern = (f.C == 8) ? (const void*)gemv_kernel<8> : (const void*)gemv_kernel<12>;
   int rc = allow_max_smem(kern, dev);
   if (rc) return rc;
-  if (f.C == 8)
-    gemv_kernel<8><<<grid, wpc * 32, smem, stream>>>(rec, eplane, x, is_bf16, y, g);
-  else
-    gemv_kernel<12><<<grid, wpc * 32, smem, stream>>>(rec, eplane, x, is_bf16, y, g);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(wpc * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = (f.C == 8)
+                        ? cudaLaunchKernelEx(&cfg, gemv_kernel<8>, rec, eplane, x, is_bf16, y, g)
+                        : cudaLaunchKernelEx(&cfg, gemv_kernel<12>, rec, eplane, x, is_bf16, y, g);
+  if (err != cudaSuccess) return record_cuda_error(err);
   count_launch();
   return record_cuda_error(cudaGetLastError());
 }
