@@ -124,6 +124,26 @@ SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec,
  * current device (HOST function; 0 if none, negative on error). */
 SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M);
 
+/* Same result as seedlm_gemm_smallM, for callers that cannot allocate device
+ * memory -- e.g. code embedded in a host program that owns all of the GPU's
+ * memory through its own pool, or a path where cudaMalloc's implicit device
+ * synchronisation is not acceptable -- and so cannot provide a workspace.
+ * It has no counterpart in the SeedLM pages; it only changes where the
+ * split-K scratch lives.  The scratch is one array inside libseedlm.so
+ * (16 MiB of partial tiles + 64 KiB of counters) that every GPU which loads
+ * the library holds until the process exits; no call allocates or frees
+ * anything.  Calls whose partial tiles would not fit (128-row tiles x splits
+ * x M rounded up to 16 x 512 bytes > 16 MiB) return SEEDLM_EUNSUPPORTED; use
+ * seedlm_gemm_smallM with a workspace for those.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) -- make that
+ * first call before any stream capture on that device.  Every call clears
+ * the counters and then reuses the same array, so calls that overlap on the
+ * GPU (two streams, or unordered host threads) race and give wrong results:
+ * order them, for example on one stream. */
+SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt, const uint32_t* rec,
+                                          const uint8_t* eplane, const void* X, int x_dtype,
+                                          int M, float* Y, seedlm_stream stream);
+
 /* Reads and clears the device-side error flag of the current device: 1 if a
  * kernel gave up waiting on one of its own barriers (the outputs of that call
  * are then undefined), else 0.  HOST function; synchronous. */

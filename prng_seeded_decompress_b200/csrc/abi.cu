@@ -80,6 +80,8 @@ int record_cuda_error(cudaError_t err) {
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int current_device_info(DeviceInfo* out) { return device_info(out); }
+
 int allow_max_smem(const void* kernel, const DeviceInfo& dev) {
   static std::mutex m;
   static std::set<std::pair<const void*, int>> done;

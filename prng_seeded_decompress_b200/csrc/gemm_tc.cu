@@ -30,6 +30,8 @@
 //     library's device error flag, and TMEM is always released.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
 #include "tcgen05.cuh"
@@ -419,4 +421,104 @@ int read_and_clear_tc_error(unsigned int* out) {
   return SEEDLM_OK;
 }
 
+// ------------------------------------------------ allocation-free variant
+//
+// For callers that cannot allocate device memory themselves, the split-K
+// partial tiles and the per-tile counters of the tensor-core GEMM live in one
+// array that the library owns for the life of the process.
+
+constexpr int64_t kNoAllocPartialBytes = 16ll << 20;  // split-K partial tiles
+constexpr int64_t kNoAllocCounterBytes = 64ll << 10;  // one uint32 per 128-row tile
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[kNoAllocPartialBytes + kNoAllocCounterBytes];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the name is only a host-side stand-in for it).
+int noalloc_scratch(const DeviceInfo& dev, unsigned char** out) {
+  if (dev.device < 0 || dev.device >= 64) return SEEDLM_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev.device]) {
+    void* p = nullptr;
+    cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess) return record_cuda_error(err);
+    if (!p) return SEEDLM_ECUDA;
+    g_noalloc_addr[dev.device] = p;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_addr[dev.device]);
+  return SEEDLM_OK;
+}
+
+}  // namespace
+
 }  // namespace seedlm
+
+using namespace seedlm;
+
+extern "C" SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt,
+                                                     const uint32_t* rec, const uint8_t* eplane,
+                                                     const void* X, int x_dtype, int M, float* Y,
+                                                     seedlm_stream stream) {
+  if (!fmt) return SEEDLM_EINVAL;
+  const bool c8 = fmt->C == 8 && fmt->P == 3 && fmt->K == 16;
+  const bool c12 = fmt->C == 12 && fmt->P == 4 && fmt->K == 16;
+  if (!c8 && !c12) return SEEDLM_EUNSUPPORTED;
+  if (fmt->rows < 0 || fmt->cols < 0 || fmt->nb != (fmt->cols + fmt->C - 1) / fmt->C ||
+      fmt->rec_pitch < fmt->nb || fmt->rec_pitch % 4 != 0 ||
+      (c12 && fmt->e_pitch < (fmt->nb + 1) / 2))
+    return SEEDLM_EINVAL;
+  if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
+  if (M < 1 || M > 64) return SEEDLM_EINVAL;
+  if (fmt->rows == 0) return SEEDLM_OK;
+  if (fmt->nb > 0 && (!rec || (reinterpret_cast<uintptr_t>(rec) & 15u))) return SEEDLM_EINVAL;
+  if (fmt->nb > 0 && c12 && !eplane) return SEEDLM_EINVAL;
+  if (!Y || (reinterpret_cast<uintptr_t>(Y) & 3u)) return SEEDLM_EINVAL;
+  if (fmt->cols > 0 && (!X || (reinterpret_cast<uintptr_t>(X) & 1u))) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (fmt->cols == 0)
+    return record_cuda_error(cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), st));
+  const uint16_t* Xh = static_cast<const uint16_t*>(X);
+  const int is_bf16 = x_dtype == SEEDLM_BF16;
+  if (M == 1) return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
+
+  TcGeom g = make_tc_geom(*fmt, M, dev);
+  g.x_vec = (fmt->cols % 4 == 0 && (reinterpret_cast<uintptr_t>(X) & 7u) == 0) ? 1 : 0;
+  const int NB = (M + 15) / 16 * 16;
+  const int64_t part_bytes =
+      g.splits > 1 ? (int64_t)g.tiles * g.splits * NB * kTileM * (int64_t)sizeof(float) : 0;
+  const int64_t cnt_bytes = g.splits > 1 ? (int64_t)g.tiles * 4 : 0;
+  if (part_bytes > kNoAllocPartialBytes || cnt_bytes > kNoAllocCounterBytes)
+    return SEEDLM_EUNSUPPORTED;  // needs more scratch than the library holds
+  float* partial = nullptr;
+  unsigned int* counters = nullptr;
+  if (g.splits > 1) {
+    unsigned char* base = nullptr;
+    if ((rc = noalloc_scratch(dev, &base))) return rc;
+    partial = reinterpret_cast<float*>(base);
+    counters = reinterpret_cast<unsigned int*>(base + kNoAllocPartialBytes);
+    // The counters must start at zero; the last call may have left them in
+    // any state if it failed part-way.
+    if ((rc = record_cuda_error(cudaMemsetAsync(counters, 0, (size_t)cnt_bytes, st)))) return rc;
+  }
+  if (fmt->C == 8) {
+    switch (NB) {
+      case 16: return launch_tc<8, 16>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+      case 32: return launch_tc<8, 32>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+      case 48: return launch_tc<8, 48>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+      default: return launch_tc<8, 64>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+    }
+  }
+  switch (NB) {
+    case 16: return launch_tc<12, 16>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+    case 32: return launch_tc<12, 32>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+    case 48: return launch_tc<12, 48>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+    default: return launch_tc<12, 64>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
+  }
+}

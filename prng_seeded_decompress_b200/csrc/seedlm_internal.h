@@ -16,6 +16,9 @@ struct DeviceInfo {
   int cc_major, cc_minor;
 };
 
+// Properties of the current device (cached per device); SEEDLM_OK or an error.
+int current_device_info(DeviceInfo* out);
+
 // Records err as this thread's last CUDA error; SEEDLM_OK or SEEDLM_ECUDA.
 int record_cuda_error(cudaError_t err);
 // Counts one kernel launch (process-wide).

@@ -19,7 +19,7 @@ BF16 = 1
 #: Every symbol include/seedlm.h declares.
 EXPORTS = (
     "seedlm_init", "seedlm_decompress", "seedlm_gemv", "seedlm_gemm_smallM",
-    "seedlm_gemm_smallM_workspace_bytes", "seedlm_device_error",
+    "seedlm_gemm_smallM_workspace_bytes", "seedlm_gemm_smallM_noalloc", "seedlm_device_error",
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
 )
@@ -56,6 +56,8 @@ def _load():
         "seedlm_gemm_smallM": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp,
                                               vp, i64, vp]),
         "seedlm_gemm_smallM_workspace_bytes": (i64, [fmtp, ctypes.c_int]),
+        "seedlm_gemm_smallM_noalloc": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int,
+                                                      ctypes.c_int, vp, vp]),
         "seedlm_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
         "seedlm_dense_gemv_f16": (ctypes.c_int, [i32, i32, vp, i64, vp, vp, vp]),
         "seedlm_row_bytes_ideal": (i64, [fmtp]),
@@ -176,6 +178,15 @@ def gemm_smallM(fmt, rec, eplane, X, Y, workspace=None, stream=None):
     _check("seedlm_gemm_smallM", lib.seedlm_gemm_smallM(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), M, _ptr(Y),
         _ptr(workspace), nbytes, _stream(stream, Y)))
+
+
+def gemm_smallM_noalloc(fmt, rec, eplane, X, Y, stream=None):
+    """Y = X W^T without a workspace: the split-K scratch is an array inside
+    the library (16 MiB of partials); calls sharing it must not overlap."""
+    f = _fmt(fmt)
+    _check("seedlm_gemm_smallM_noalloc", lib.seedlm_gemm_smallM_noalloc(
+        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), int(X.shape[0]),
+        _ptr(Y), _stream(stream, Y)))
 
 
 def device_error() -> int:
