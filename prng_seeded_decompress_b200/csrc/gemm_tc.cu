@@ -183,13 +183,11 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     }
   };
 
-  Pref cur, nxt;
-  if (n_iter > 0) load_pref(c_begin, cur);
-  for (int it = 0; it < n_iter; ++it) {
+  // Build one stage from its prefetched records and X values.
+  auto build_stage = [&](int it, const Pref& cur) {
     const int s = it % STAGES;
     const int use = it / STAGES;
     unsigned char* st = smem + s * L::STAGE_BYTES;
-    if (it + 1 < n_iter) load_pref(c_begin + it + 1, nxt);
     if (use > 0) ok = tc::mbar_wait(bar0 + 8 * s, (use - 1) & 1, kWaitLimit) && ok;
 
     // ---- A: rebuilt weights, hi and lo tf32 pieces
@@ -267,7 +265,23 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       }
       tc::mma_commit(bar0 + 8 * s);
     }
-    cur = nxt;
+  };
+
+  // Record sets and X values are loaded two stages ahead of the one being
+  // built (a ring of three register buffers, unrolled so they stay in
+  // registers).
+  Pref pf[3];
+  if (n_iter > 0) load_pref(c_begin, pf[0]);
+  if (n_iter > 1) load_pref(c_begin + 1, pf[1]);
+  for (int it0 = 0; it0 < n_iter; it0 += 3) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int it = it0 + k;
+      if (it < n_iter) {
+        if (it + 2 < n_iter) load_pref(c_begin + it + 2, pf[(k + 2) % 3]);
+        build_stage(it, pf[k]);
+      }
+    }
   }
 
   // ---- epilogue: wait for the last MMAs, read D, write Y or a partial
