@@ -52,7 +52,9 @@ def up_to_date() -> bool:
 
 def _compile(src: str, verbose: bool) -> str:
     obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+    # SEEDLM_NVCC_FLAGS: extra flags for experiments (e.g. -DNAME=VALUE).
+    extra = os.environ.get("SEEDLM_NVCC_FLAGS", "").split()
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)

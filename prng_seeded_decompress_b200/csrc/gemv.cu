@@ -29,13 +29,26 @@
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
 
+// 1: take the C = 8 coefficient decode from two 256-entry shared tables;
+// 0: compute it with byte arithmetic and dp2a.
+#ifndef SEEDLM_GEMV_COEF_TABLES
+#define SEEDLM_GEMV_COEF_TABLES 1
+#endif
+
 namespace seedlm {
 
 namespace {
 
-constexpr int kMaxWarps = 16;
+// Warps per CTA (one CTA per SM) and record sets in flight ahead of the one
+// being rebuilt.  C = 8 runs 24 warps with one set ahead; C = 12 needs more
+// registers per lane (four dp2a windows per weight) and spills at 24 warps, so
+// it keeps 16 warps with two sets ahead.
+template <int C>
+struct Tune {
+  static constexpr int kWarps = (C == 8) ? 24 : 16;
+  static constexpr int kPrefetch = (C == 8) ? 1 : 2;
+};
 constexpr int kRowsPerTask = 4;
-constexpr int kPrefetch = 2;     // record sets in flight ahead of the one being rebuilt
 constexpr int kMaxGroups = 128;  // row groups per partial-sum pass
 
 struct GemvGeom {
@@ -53,8 +66,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Shared-memory map: [jump tables][partial sums][x slots].
 template <int C>
 struct Smem {
-  static constexpr int kTableBytes = (C == 8) ? 2 * 256 * 4 : 2 * 256 * 8;
-  static constexpr int kPartBytes = kMaxGroups * kRowsPerTask * kMaxWarps * 4;
+  // C = 8: jump tables (2 KB) + coefficient tables (4 KB); C = 12: jump tables.
+  static constexpr int kJumpBytes = (C == 8) ? 2 * 256 * 4 : 2 * 256 * 8;
+  static constexpr int kTableBytes = (C == 8) ? kJumpBytes + 2 * 256 * 8 : kJumpBytes;
+  static constexpr int kPartBytes = kMaxGroups * kRowsPerTask * Tune<C>::kWarps * 4;
   static constexpr int kHead = kTableBytes + kPartBytes;
   static constexpr int kSlotFloats = (C == 8) ? 16 : 32;  // per record pair
 };
@@ -76,6 +91,8 @@ __device__ void stage_x_and_tables(unsigned char* smem, const uint16_t* __restri
     uint32_t* t = reinterpret_cast<uint32_t*>(smem);
     for (int i = threadIdx.x; i < 512; i += blockDim.x)
       t[i] = (uint32_t)(i < 256 ? kStreamTables.lo[i] : kStreamTables.hi[i - 256]);
+    uint2* tq = reinterpret_cast<uint2*>(smem + Smem<8>::kJumpBytes);
+    fill_coef_tables_c8(tq, tq + 256, threadIdx.x, blockDim.x);
   } else {
     uint2* t = reinterpret_cast<uint2*>(smem);
     for (int i = threadIdx.x; i < 512; i += blockDim.x) {
@@ -143,8 +160,14 @@ __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const floa
     if constexpr (C == 8) {
       const uint32_t* tl = static_cast<const uint32_t*>(t_lo);
       const uint32_t* th = static_cast<const uint32_t*>(t_hi);
+#if SEEDLM_GEMV_COEF_TABLES
+      const uint2* tq1 = reinterpret_cast<const uint2*>(th + 256);
+      const BlockC8 A = decode_c8_tab(cur.r[j].x, tl, th, tq1, tq1 + 256);
+      const BlockC8 B = decode_c8_tab(cur.r[j].y, tl, th, tq1, tq1 + 256);
+#else
       const BlockC8 A = decode_c8(cur.r[j].x, tl, th);
       const BlockC8 B = decode_c8(cur.r[j].y, tl, th);
+#endif
       const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
 #define SEEDLM_C8_STEP(c)                                                        \
   {                                                                              \
@@ -178,19 +201,19 @@ __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const floa
 
 // CTA b owns the contiguous row groups [g0, g1) (sizes differ by at most
 // one group); its (group, span) items are split into equal contiguous ranges,
-// one per warp.  A warp walks its range with record sets loaded kPrefetch
+// one per warp.  A warp walks its range with record sets loaded Tune<C>::kPrefetch
 // items ahead (across group boundaries), and whenever it leaves a group it
 // reduces its 4 row sums with shuffles into shared memory.  After a barrier
 // the partial sums of each row are added in warp order -- the same order on
 // every call -- and written.  Groups are processed in passes of at most
 // kMaxGroups so the partial-sum buffer stays small.
 template <int C>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+__global__ void __launch_bounds__(Tune<C>::kWarps * 32, 1)
 gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
             const uint16_t* __restrict__ x, int is_bf16, float* __restrict__ y, GemvGeom g) {
   extern __shared__ __align__(16) unsigned char smem[];
   const void* t_lo = smem;
-  const void* t_hi = smem + Smem<C>::kTableBytes / 2;
+  const void* t_hi = smem + Smem<C>::kJumpBytes / 2;
   float* part = reinterpret_cast<float*>(smem + Smem<C>::kTableBytes);
   const float* xs = reinterpret_cast<const float*>(smem + Smem<C>::kHead);
 
@@ -210,9 +233,9 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
     // programmatic dependent launch, the tail of the previous kernel).
     int grp = p0 + (i0 < i1 ? i0 / g.n_spans : 0), span = i0 < i1 ? i0 % g.n_spans : 0;
     int lgrp = grp, lspan = span, li = i0;
-    RecSet<C> buf[kPrefetch + 1];
+    RecSet<C> buf[Tune<C>::kPrefetch + 1];
 #pragma unroll
-    for (int k = 0; k <= kPrefetch; ++k) {
+    for (int k = 0; k <= Tune<C>::kPrefetch; ++k) {
       if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
       ++li;
       if (++lspan == g.n_spans) { lspan = 0; ++lgrp; }
@@ -233,7 +256,7 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
       bool done = false;
       while (!done) {
 #pragma unroll
-        for (int k = 0; k <= kPrefetch; ++k) {
+        for (int k = 0; k <= Tune<C>::kPrefetch; ++k) {
           if (!done) {
             rebuild_and_dot<C>(buf[k], xs, span * 32 + lane, swz, t_lo, t_hi, acc);
             if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
@@ -306,7 +329,8 @@ int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* epla
   // spread over all SMs.
   int grid = g.groups < dev.num_sms ? g.groups : dev.num_sms;
   int items_per_cta = (g.groups + grid - 1) / grid * g.n_spans;
-  int wpc = items_per_cta < kMaxWarps ? items_per_cta : kMaxWarps;
+  const int max_warps = (f.C == 8) ? Tune<8>::kWarps : Tune<12>::kWarps;
+  int wpc = items_per_cta < max_warps ? items_per_cta : max_warps;
   const void* kern = (f.C == 8) ? (const void*)gemv_kernel<8> : (const void*)gemv_kernel<12>;
   int rc = allow_max_smem(kern, dev);
   if (rc) return rc;

@@ -169,6 +169,42 @@ __device__ __forceinline__ BlockC8 decode_c8(uint32_t rec, const uint32_t* __res
   return b;
 }
 
+// Coefficient tables for C = 8 (built per CTA by fill_coef_tables_c8):
+//   tq1[v], v = q0 | q1 << 4 (record byte 0):  (A01 = (q0, 256 q0 + q1), -32768 (q0 + q1))
+//   tq2[v], v = q1 | q2 << 4 (record bits 4..11): (A23 = (256 q1 + q2, 256 q2), -32768 q2)
+// with q the signed values of the nibbles.
+__device__ __forceinline__ int32_t nibble_value(uint32_t n) { return (int32_t)(n & 15u) - (int32_t)((n & 8u) << 1); }
+
+__device__ __forceinline__ uint32_t pack_s16(int32_t lo, int32_t hi) {
+  return ((uint32_t)lo & 0xffffu) | ((uint32_t)hi << 16);
+}
+
+__device__ __forceinline__ void fill_coef_tables_c8(uint2* tq1, uint2* tq2, int tid, int nthreads) {
+  for (int v = tid; v < 256; v += nthreads) {
+    const int32_t a = nibble_value(v), b = nibble_value(v >> 4);
+    tq1[v] = make_uint2(pack_s16(a, 256 * a + b), (uint32_t)(-32768 * (a + b)));
+    tq2[v] = make_uint2(pack_s16(256 * a + b, 256 * b), (uint32_t)(-32768 * b));
+  }
+}
+
+// decode_c8 with the coefficient part taken from the two tables above.
+__device__ __forceinline__ BlockC8 decode_c8_tab(uint32_t rec, const uint32_t* __restrict__ t_lo,
+                                                 const uint32_t* __restrict__ t_hi,
+                                                 const uint2* __restrict__ tq1,
+                                                 const uint2* __restrict__ tq2) {
+  BlockC8 b;
+  b.lo = rec;
+  b.hi = t_lo[prmt<0x4442u>(rec, 0u)] ^ t_hi[rec >> 24];
+  const uint2 c1 = tq1[rec & 0xffu];
+  const uint2 c2 = tq2[(rec >> 4) & 0xffu];
+  b.a01 = c1.x;
+  b.a23 = c2.x;
+  const uint32_t e23 = (rec << 11) & 0x07800000u;
+  b.init = (int32_t)(kMagicBits - e23 + c1.y + c2.y);
+  b.negm = kNegMagicBits - e23;
+  return b;
+}
+
 // Integer weight c of a C = 8 block, biased by bits(M_e) (see 3. above).
 template <int c>
 __device__ __forceinline__ int32_t weight_bits_c8(const BlockC8& b) {
