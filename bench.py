@@ -588,6 +588,19 @@ def profile_case(name: str):
         ws = sl.gemm_workspace(L["fmt"], M)
         for _ in range(3):
             sl.gemm_smallM(L["fmt"], rec, None, X, Y, workspace=ws)
+    elif name == "gemv":
+        # The four GEMVs of one 4-bit Llama-3-70B layer, twice (the first
+        # round warms up; capture with -s 4 -c 4).
+        lay = []
+        for i, (_, R, N) in enumerate(LAYER_70B):
+            L = inputs.make_layer(R, N, 8, 3, seed=10 + i)
+            xb, _ = inputs.make_activations((N,), "f16", 20 + i)
+            lay.append((L["fmt"], torch.from_numpy(L["rec"].view(np.int32)).cuda(),
+                        torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16),
+                        torch.empty(R, device="cuda")))
+        for _ in range(2):
+            for f, rec, x, y in lay:
+                sl.gemv(f, rec, None, x, y)
     elif name == "dense":
         W = torch.randn((57344, 8192), device="cuda").half()
         x = torch.randn(8192, device="cuda").half()
@@ -611,7 +624,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
-    ap.add_argument("--case", choices=("decompress", "gemm64", "gemm16", "dense"),
+    ap.add_argument("--case", choices=("gemv", "decompress", "gemm64", "gemm16", "dense"),
                     help="run one small single-kernel workload (for ncu) and exit")
     args = ap.parse_args()
     if args.case:

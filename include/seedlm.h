@@ -110,18 +110,21 @@ SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const 
 /* Y = X W^T for a small batch: X is M x cols (row-major, type x_dtype), Y is
  * M x rows fp32 (row-major), 1 <= M <= 64.  M = 1 runs the GEMV kernel; for
  * M >= 2 the rebuilt weight tiles feed the tcgen05 tensor cores (tf32 hi/lo
- * pieces, exact products, fp32 accumulation in TMEM).  `workspace` is device
- * memory of at least seedlm_gemm_smallM_workspace_bytes(fmt, M) bytes,
- * 256-byte aligned (may be NULL when that size is 0).  It holds split-K
- * partial sums and per-tile counters: it must be zero-filled before its first
- * use, every call leaves it ready for the next, and calls sharing one
- * workspace must not run concurrently (calls on one stream never do). */
+ * pieces, exact products, fp32 accumulation in TMEM) -- two launches: X is
+ * first converted into the operand layout, then one CTA per SM runs the GEMM.
+ * `workspace` is device memory of at least
+ * seedlm_gemm_smallM_workspace_bytes(fmt, M) bytes, 256-byte aligned.  It
+ * holds per-tile counters, X in the operand layout and the partial tiles of
+ * row tiles shared by several CTAs: it must be zero-filled before its first
+ * use, every call leaves the counters at zero for the next, and calls sharing
+ * one workspace must not run concurrently (calls on one stream never do). */
 SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
                        const void* X, int x_dtype, int M, float* Y, void* workspace,
                        int64_t workspace_bytes, seedlm_stream stream);
 
 /* Workspace bytes seedlm_gemm_smallM needs for this format and M on the
- * current device (HOST function; 0 if none, negative on error). */
+ * current device (HOST function; 0 for M = 1 or an empty matrix, negative on
+ * error). */
 SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M);
 
 /* Same result as seedlm_gemm_smallM, for callers that cannot allocate device
@@ -129,17 +132,17 @@ SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, 
  * memory through its own pool, or a path where cudaMalloc's implicit device
  * synchronisation is not acceptable -- and so cannot provide a workspace.
  * It has no counterpart in the SeedLM pages; it only changes where the
- * split-K scratch lives.  The scratch is one array inside libseedlm.so
- * (16 MiB of partial tiles + 64 KiB of counters) that every GPU which loads
- * the library holds until the process exits; no call allocates or frees
- * anything.  Calls whose partial tiles would not fit (128-row tiles x splits
- * x M rounded up to 16 x 512 bytes > 16 MiB) return SEEDLM_EUNSUPPORTED; use
- * seedlm_gemm_smallM with a workspace for those.  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress) -- make that
- * first call before any stream capture on that device.  Every call clears
- * the counters and then reuses the same array, so calls that overlap on the
- * GPU (two streams, or unordered host threads) race and give wrong results:
- * order them, for example on one stream. */
+ * workspace lives.  It is one array inside libseedlm.so (16 MiB + 64 KiB)
+ * that every GPU which loads the library holds until the process exits; no
+ * call allocates or frees anything.  Calls whose workspace would not fit
+ * (seedlm_gemm_smallM_workspace_bytes(fmt, M) > 16 MiB + 64 KiB) return
+ * SEEDLM_EUNSUPPORTED; use seedlm_gemm_smallM with a workspace for those.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) -- make that first call before any stream capture on
+ * that device.  Every call clears the counters and then reuses the same
+ * array, so calls that overlap on the GPU (two streams, or unordered host
+ * threads) race and give wrong results: order them, for example on one
+ * stream. */
 SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt, const uint32_t* rec,
                                           const uint8_t* eplane, const void* X, int x_dtype,
                                           int M, float* Y, seedlm_stream stream);

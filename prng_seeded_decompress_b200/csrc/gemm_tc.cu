@@ -4,30 +4,38 @@
 // Where the batch makes the product a real contraction (several rows of X
 // share every rebuilt weight), the reconstructed tiles feed tcgen05.mma
 // (paperhub.cn review thread: the weights are rebuilt from s and t and then
-// used to compute the activations).  The layout per CTA:
+// used to compute the activations).  One call is two launches:
 //
-//   * D = W_tile (128 rows) x X^T (NB columns, NB = batch rounded up to 16)
-//     accumulates in TMEM in fp32 (128 lanes x NB columns).
-//   * Each K stage (64 columns for C = 8, 48 for C = 12, i.e. a whole number
-//     of blocks) is built by all 512 threads: four threads per W row load the
-//     row's records for the stage (one stage ahead, into registers), rebuild
-//     the weights exactly in fp32 (see
-//     seedlm_device.cuh) and split each into tf32 pieces hi + lo, both exact
-//     (a weight has at most 21 significant bits; tf32 keeps 11).  X is
-//     converted to fp32, which tf32 holds exactly for fp16 or bf16 inputs.
-//     The operands are written in the K-major core-matrix layout (8 rows x
-//     16 bytes per core matrix, no swizzle).
-//   * One thread issues 2 x (stage K / 8) MMAs per stage (kind::tf32,
-//     M = 128, N = NB) -- hi and lo pieces into the same accumulator -- and
-//     commits them to the stage's mbarrier; the other threads go on building
-//     the next stage.  A stage is rebuilt only after its MMAs have completed.
-//   * Split-K: the columns are divided into `splits` ranges so that there are
-//     about three CTAs per SM.  Each CTA writes its fp32 partial tile to the
-//     caller's workspace; the last CTA of a row tile to arrive (atomic
-//     counter) adds the partials in split order -- a fixed order, so every
-//     call gives the same bits -- writes Y and resets the counter to zero.
-//   * Every mbarrier wait is bounded; a wait that gives up raises the
-//     library's device error flag, and TMEM is always released.
+//   1. stage_x_kernel writes X (fp16 or bf16, M x cols) into the workspace as
+//      fp32 -- exact in tf32 for either input type -- already in the
+//      tensor-core operand layout, one contiguous slab per K chunk (NB x KC,
+//      NB = M rounded up to 16, zero-padded), so the GEMM copies a chunk of X
+//      into shared memory with a single bulk copy.
+//   2. gemm_tc_kernel, one CTA per SM.  The work is the list of
+//      (128-row tile, K chunk) units in tile-major order, cut into equal
+//      contiguous ranges, one per CTA ("stream-K"), so every SM gets the same
+//      number of units whatever the shape.  Inside a CTA:
+//        * 16 producer warps rebuild the unit's 128 x KC weights exactly in
+//          fp32 (seedlm_device.cuh), split each into tf32 pieces hi + lo (both
+//          exact: a weight has at most 21 significant bits, tf32 keeps 11)
+//          and store them straight into tensor memory with tcgen05.st -- A
+//          operand stages, 128 lanes = rows, one column per K element.  Warp w
+//          owns TMEM lanes 32(w%4).. and a quarter (w/4) of the chunk's blocks.
+//        * one warp issues the MMAs (kind::tf32, M = 128, N = NB, A from TMEM,
+//          B = X chunk from shared memory): hi and lo pieces into the same
+//          fp32 accumulator in TMEM.  It also keeps the X slabs coming, a few
+//          chunks ahead, with bulk copies.
+//        * stages are handed over with mbarriers only (A stage full: all 16
+//          producer warps arrived; A stage / X slab free: tcgen05.commit of the
+//          MMAs that read it), so no warp waits for the whole CTA.
+//        * the accumulator is double-buffered in TMEM.  At the end of each
+//          tile segment warps 0-3 read it out: a tile owned by one CTA goes
+//          straight to Y; otherwise each CTA writes a partial tile to the
+//          workspace and the last of the tile's CTAs to arrive (atomic
+//          counter) adds the partials in CTA order -- a fixed order, so every
+//          call gives the same bits -- writes Y and resets the counter.
+//   Every mbarrier wait is bounded; a wait that gives up raises the library's
+//   device error flag, and TMEM is always released.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -43,69 +51,129 @@ __device__ unsigned int g_tc_error = 0;
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 512;
+constexpr int kProdWarps = 16;
+constexpr int kThreads = (kProdWarps + 1) * 32;  // + the MMA / X-loader warp
+constexpr int kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
+// Per format: K columns per unit (8 blocks), blocks per producer thread, A
+// stages in TMEM, X slabs in shared memory, record sets a thread loads ahead.
 template <int C>
 struct TcCfg;
 template <>
 struct TcCfg<8> {
-  static constexpr int KC = 64;  // columns per stage = 8 blocks
-  static constexpr int STAGES = 2;
+  static constexpr int KC = 64;
+  static constexpr int AS = 3;  // 3 x 128 TMEM columns + 2 accumulators of 64
+  static constexpr int XS = 5;
 };
 template <>
 struct TcCfg<12> {
-  static constexpr int KC = 48;  // 4 blocks
-  static constexpr int STAGES = 3;
+  static constexpr int KC = 96;
+  static constexpr int AS = 2;  // 2 x 192 TMEM columns + 2 accumulators of 64
+  static constexpr int XS = 4;
 };
+constexpr int kBpt = 2;        // blocks per producer thread and unit
+constexpr int kRecAhead = 4;   // units of records a producer thread has in flight
 
 struct TcGeom {
   int rows, cols, nb, rec_pitch, e_pitch, M;
-  int splits, chunks_per_split, nchunks, tiles;
-  int x_vec;  // X rows are 8-byte aligned and cols % 4 == 0: load X 4 elements at a time
+  int nchunks, tiles;
+  long long units;  // tiles * nchunks
+  int segs_max;     // most tiles any one CTA touches
 };
 
 template <int C, int NB>
 struct TcSmem {
   static constexpr int KC = TcCfg<C>::KC;
-  static constexpr int STAGES = TcCfg<C>::STAGES;
-  static constexpr int SBO = KC * 32;  // bytes between 8-row groups (KC/4 core matrices of 128 B)
-  static constexpr int A_BYTES = kTileM * KC * 4;
-  static constexpr int B_BYTES = NB * KC * 4;
-  static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
-  static constexpr int TABLE_OFF = STAGES * STAGE_BYTES;
+  static constexpr int AS = TcCfg<C>::AS;
+  static constexpr int XS = TcCfg<C>::XS;
+  static constexpr int SBO = KC * 32;  // bytes between 8-row groups of X (KC/4 core matrices)
+  static constexpr int XB = NB * KC * 4;  // one X slab
+  static constexpr int TABLE_OFF = XS * XB;
   static constexpr int TABLE_BYTES = (C == 8) ? 512 * 4 : 512 * 8;
-  static constexpr int BAR_OFF = TABLE_OFF + TABLE_BYTES;  // STAGES mbarriers (8 B each)
-  static constexpr int SLOT_OFF = BAR_OFF + 8 * STAGES;    // TMEM address, last-CTA flag
+  static constexpr int BAR_OFF = TABLE_OFF + TABLE_BYTES;
+  // mbarriers: xfull[XS] xfree[XS] afull[AS] afree[AS] dfull[2] dfree[2]
+  static constexpr int NBAR = 2 * XS + 2 * AS + 4;
+  static constexpr int SLOT_OFF = BAR_OFF + 8 * NBAR;  // TMEM base, last-CTA flag, give-up flag
   static constexpr int TOTAL = SLOT_OFF + 16;
-  static constexpr uint32_t TMEM_COLS = NB <= 32 ? 32 : 64;
+  static constexpr int D_COL = AS * 2 * KC;  // first accumulator column
+  static_assert(D_COL + 2 * 64 <= kTmemCols, "TMEM budget");
+  static_assert(KC == 4 * kBpt * C, "four producer quarters of kBpt blocks per unit");
 };
 
-// Byte offset of element (row, k) in a K-major core-matrix operand.
-template <int SBO>
-__device__ __forceinline__ uint32_t core_off(int row, int k4) {
-  return (uint32_t)(row >> 3) * SBO + (uint32_t)k4 * 128u + (uint32_t)(row & 7) * 16u;
+// Float offset of X element (n, k) inside a slab (K-major core matrices:
+// 8 rows x 16 bytes, adjacent along K at 128 B, 8-row groups at SBO).
+template <int KC>
+__host__ __device__ constexpr int slab_index(int n, int k) {
+  return ((n >> 3) * (KC * 32) + (k >> 2) * 128 + (n & 7) * 16) / 4 + (k & 3);
 }
 
-__device__ __forceinline__ void split_tf32(float w, float& hi, float& lo) {
-  hi = __uint_as_float(__float_as_uint(w) & 0xFFFFE000u);
-  lo = w - hi;  // exact; at most 10 significant bits, so exact in tf32 too
+template <int C, int NB>
+__global__ void __launch_bounds__(256)
+stage_x_kernel(const uint16_t* __restrict__ X, int is_bf16, int M, int cols, int nchunks,
+               float* __restrict__ Xs) {
+  constexpr int KC = TcCfg<C>::KC;
+  constexpr int PER_CHUNK = NB * (KC / 4);  // float4 groups per slab
+  // The GEMM may start its prologue at once; it reads Xs only after
+  // griddepcontrol.wait, i.e. after this grid has finished.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const long long total = (long long)nchunks * PER_CHUNK;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int chunk = (int)(i / PER_CHUNK);
+    const int rem = (int)(i - (long long)chunk * PER_CHUNK);
+    const int n = rem / (KC / 4), k4 = rem - n * (KC / 4);  // k fastest: coalesced reads
+    const int col = chunk * KC + 4 * k4;
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      v[u] = (n < M && col + u < cols) ? act_to_float(X[(size_t)n * cols + col + u], is_bf16)
+                                       : 0.f;
+    *reinterpret_cast<float4*>(Xs + (size_t)chunk * (NB * KC) + slab_index<KC>(n, 4 * k4)) =
+        make_float4(v[0], v[1], v[2], v[3]);
+  }
 }
+
+__device__ __forceinline__ long long unit_begin(int cta, long long units, int ctas) {
+  return (long long)cta * units / ctas;
+}
+// The CTA whose range holds unit u.
+__device__ __forceinline__ int unit_owner(long long u, long long units, int ctas) {
+  return (int)(((u + 1) * ctas + units - 1) / units) - 1;
+}
+
+// Exact tf32 pieces of two rebuilt weights given as magic-biased floats b
+// (weight = b + nm): hi keeps the top 11 significant bits, lo = w - hi.
+__device__ __forceinline__ void split_pair(float b0, float b1, float nm, uint32_t& h0,
+                                           uint32_t& h1, uint32_t& l0, uint32_t& l1) {
+  const float2 w = __fadd2_rn(make_float2(b0, b1), make_float2(nm, nm));  // exact
+  h0 = __float_as_uint(w.x) & 0xFFFFE000u;
+  h1 = __float_as_uint(w.y) & 0xFFFFE000u;
+  const float2 l = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)),
+                              make_float2(-1.f, -1.f), w);  // exact
+  l0 = __float_as_uint(l.x);
+  l1 = __float_as_uint(l.y);
+}
+
+template <int C>
+struct RecUnit {
+  uint2 r;     // the thread's two records of this unit
+  uint32_t e;  // C = 12: their exponent byte
+};
 
 template <int C, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
-               const uint16_t* __restrict__ X, int is_bf16, float* __restrict__ Y,
-               float* __restrict__ partial, unsigned int* __restrict__ counters, TcGeom g) {
+               const float* __restrict__ Xs, float* __restrict__ Y, float* __restrict__ partial,
+               unsigned int* __restrict__ counters, TcGeom g) {
   using L = TcSmem<C, NB>;
-  constexpr int KC = L::KC, STAGES = L::STAGES, BLK = KC / C;
+  constexpr int KC = L::KC, AS = L::AS, XS = L::XS;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x / g.splits, split = blockIdx.x - tile * g.splits;
-  const int r0 = tile * kTileM;
-  const int c_begin = split * g.chunks_per_split;
-  const int c_end = min(c_begin + g.chunks_per_split, g.nchunks);
-  const int n_iter = c_end > c_begin ? c_end - c_begin : 0;
+  const int ctas = gridDim.x;
+  const long long u_begin = unit_begin(blockIdx.x, g.units, ctas);
+  const int n_units = (int)(unit_begin(blockIdx.x + 1, g.units, ctas) - u_begin);
+  const int t_first = (int)(u_begin / g.nchunks);
 
   uint32_t* t32 = reinterpret_cast<uint32_t*>(smem + L::TABLE_OFF);
   uint2* t64 = reinterpret_cast<uint2*>(smem + L::TABLE_OFF);
@@ -116,235 +184,263 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     else
       t64[i] = make_uint2((uint32_t)v, (uint32_t)(v >> 32));
   }
-  const uint32_t bar0 = tc::smem_u32(smem + L::BAR_OFF);
+  const uint32_t bar = tc::smem_u32(smem + L::BAR_OFF);
+  auto xfull = [&](int s) { return bar + 8 * s; };
+  auto xfree = [&](int s) { return bar + 8 * (XS + s); };
+  auto afull = [&](int s) { return bar + 8 * (2 * XS + s); };
+  auto afree = [&](int s) { return bar + 8 * (2 * XS + AS + s); };
+  auto dfull = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + b); };
+  auto dfree = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + 2 + b); };
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) tc::mbar_init(bar0 + 8 * s, 1);
+    for (int s = 0; s < XS; ++s) {
+      tc::mbar_init(xfull(s), 1);
+      tc::mbar_init(xfree(s), 1);
+    }
+    for (int s = 0; s < AS; ++s) {
+      tc::mbar_init(afull(s), kProdWarps);
+      tc::mbar_init(afree(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(dfull(b), 1);
+      tc::mbar_init(dfree(b), 4);
+    }
     tc::fence_mbar_init();
+    slot[2] = 0u;  // give-up flag shared by all bounded waits
   }
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(slot), L::TMEM_COLS);
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(slot), kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = slot[0];
-  const uint32_t idesc = tc::idesc_tf32(NB);
+  volatile uint32_t* abort_flag = slot + 2;
   bool ok = true;
 
-  // Producer roles: four threads per W row, each rebuilding a quarter of the
-  // row's blocks of the stage; the X slice is split over all threads.  The
-  // next stage's records and X values are loaded before the current stage is
-  // built.
-  constexpr int BPT = BLK / 4;                                // blocks per thread
-  constexpr int XCH = NB * (KC / 4);                          // 4-element X chunks per stage
-  constexpr int XPT = (XCH + kThreads - 1) / kThreads;        // X chunks per thread
-  // Warp w owns rows 8w..8w+7; lane l takes row 8w + (l & 7) and quarter
-  // l >> 3, so the 8 lanes of a quarter-warp store to 8 different rows of a
-  // core matrix (distinct banks).
-  const int prow = 8 * warp + (lane & 7), pq = lane >> 3;
-  const int gr = r0 + prow;
-  const bool row_ok = gr < g.rows;
-
-  struct Pref {
-    uint32_t w[BPT];
-    uint32_t e;
-    uint2 x[XPT];
+  auto seg_first = [&](int i) { return i == 0 || (u_begin + i) % g.nchunks == 0; };
+  auto seg_last = [&](int i) {
+    return i == n_units - 1 || (u_begin + i) % g.nchunks == g.nchunks - 1;
   };
-  auto load_pref = [&](int chunk, Pref& p) {
-    const int b_first = chunk * BLK + pq * BPT;
-    const bool blk_ok = row_ok && b_first < g.nb;
-    if constexpr (BPT == 2) {
-      uint2 v = blk_ok ? ld_stream_u2(rec + (size_t)gr * g.rec_pitch + b_first) : make_uint2(0u, 0u);
-      p.w[0] = v.x;
-      p.w[1] = v.y;
-    } else {
-      p.w[0] = blk_ok ? __ldg(rec + (size_t)gr * g.rec_pitch + b_first) : 0u;
-    }
-    p.e = 0;
-    if constexpr (C == 12)
-      p.e = blk_ok ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b_first >> 1)) : 0u;
+
+  if (warp == kProdWarps) {
+    // ------------------------------------------------ MMA issue + X slabs
+    if (lane == 0) {
+      const uint32_t xs0 = tc::smem_u32(smem);
+      auto load_x = [&](int i) {
+        const int s = i % XS;
+        const int chunk = (int)((u_begin + i) % g.nchunks);
+        tc::mbar_arrive_expect_tx(xfull(s), L::XB);
+        tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)chunk * (NB * KC), L::XB, xfull(s));
+      };
+      // Xs is written by the previous kernel on the stream.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int i = 0; i < XS && i < n_units; ++i) load_x(i);
+      const uint32_t idesc = tc::idesc_tf32(NB);
+      int seg = 0;
+      for (int i = 0; i < n_units; ++i) {
+        const bool first = seg_first(i);
+        if (first && i > 0) ++seg;
+        const int db = seg & 1;
+        if (first && seg >= 2)  // accumulator db was last used by segment seg - 2
+          ok = tc::mbar_wait_or_abort(dfree(db), ((seg >> 1) - 1) & 1, kWaitLimit, abort_flag) && ok;
+        const int xs = i % XS, as = i % AS;
+        ok = tc::mbar_wait_or_abort(xfull(xs), (i / XS) & 1, kWaitLimit, abort_flag) && ok;
+        ok = tc::mbar_wait_or_abort(afull(as), (i / AS) & 1, kWaitLimit, abort_flag) && ok;
+        tc::fence_after_sync();
+        const uint32_t a_hi = tmem + as * 2 * KC, a_lo = a_hi + KC;
+        const uint32_t d = tmem + L::D_COL + 64 * db;
+        const uint32_t xb = xs0 + xs * L::XB;
 #pragma unroll
-    for (int k = 0; k < XPT; ++k) {
-      const int i = tid + k * kThreads;
-      const int k4 = i / NB, n = i - k4 * NB;  // n fastest: distinct banks when stored
-      const int col = chunk * KC + 4 * k4;
-      uint2 v = make_uint2(0u, 0u);
-      if (i < XCH && n < g.M) {
-        const uint16_t* src = X + (size_t)n * g.cols + col;
-        if (g.x_vec) {
-          if (col < g.cols) v = __ldg(reinterpret_cast<const uint2*>(src));
-        } else {
-          uint32_t h[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) h[u] = col + u < g.cols ? (uint32_t)__ldg(src + u) : 0u;
-          v = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+        for (int kk = 0; kk < KC / 8; ++kk) {
+          const uint64_t bd = tc::smem_desc(xb + 256 * kk, 128, L::SBO);
+          tc::mma_tf32_ts(d, a_hi + 8 * kk, bd, idesc, (first && kk == 0) ? 0u : 1u);
+          tc::mma_tf32_ts(d, a_lo + 8 * kk, bd, idesc, 1u);
+        }
+        tc::mma_commit(afree(as));
+        tc::mma_commit(xfree(xs));
+        if (seg_last(i)) tc::mma_commit(dfull(db));
+        // Refill the slab of unit i - 2 (its MMAs were queued two units ago).
+        if (i >= 2 && i - 2 + XS < n_units) {
+          ok = tc::mbar_wait_or_abort(xfree((i - 2) % XS), ((i - 2) / XS) & 1, kWaitLimit, abort_flag) && ok;
+          load_x(i - 2 + XS);
         }
       }
-      p.x[k] = v;
-    }
-  };
-
-  // Build one stage from its prefetched records and X values.
-  auto build_stage = [&](int it, const Pref& cur) {
-    const int s = it % STAGES;
-    const int use = it / STAGES;
-    unsigned char* st = smem + s * L::STAGE_BYTES;
-    if (use > 0) ok = tc::mbar_wait(bar0 + 8 * s, (use - 1) & 1, kWaitLimit) && ok;
-
-    // ---- A: rebuilt weights, hi and lo tf32 pieces
-#pragma unroll
-    for (int i = 0; i < BPT; ++i) {
-      float w[C];
-      if constexpr (C == 8) {
-        const BlockC8 blk = decode_c8(cur.w[i], t32, t32 + 256);
-        const float nm = __uint_as_float(blk.negm);
-        w[0] = __int_as_float(weight_bits_c8<0>(blk)) + nm;
-        w[1] = __int_as_float(weight_bits_c8<1>(blk)) + nm;
-        w[2] = __int_as_float(weight_bits_c8<2>(blk)) + nm;
-        w[3] = __int_as_float(weight_bits_c8<3>(blk)) + nm;
-        w[4] = __int_as_float(weight_bits_c8<4>(blk)) + nm;
-        w[5] = __int_as_float(weight_bits_c8<5>(blk)) + nm;
-        w[6] = __int_as_float(weight_bits_c8<6>(blk)) + nm;
-        w[7] = __int_as_float(weight_bits_c8<7>(blk)) + nm;
-      } else {
-        const int b_first = (c_begin + it) * BLK + pq * BPT;
-        const uint32_t e4 = (b_first & 1) ? (cur.e >> 4) : cur.e;
-        const BlockC12 blk = decode_c12(cur.w[i], e4 & 15u, t64, t64 + 256);
-        const float nm = __uint_as_float(blk.negm);
-        w[0] = __int_as_float(weight_bits_c12<0>(blk)) + nm;
-        w[1] = __int_as_float(weight_bits_c12<1>(blk)) + nm;
-        w[2] = __int_as_float(weight_bits_c12<2>(blk)) + nm;
-        w[3] = __int_as_float(weight_bits_c12<3>(blk)) + nm;
-        w[4] = __int_as_float(weight_bits_c12<4>(blk)) + nm;
-        w[5] = __int_as_float(weight_bits_c12<5>(blk)) + nm;
-        w[6] = __int_as_float(weight_bits_c12<6>(blk)) + nm;
-        w[7] = __int_as_float(weight_bits_c12<7>(blk)) + nm;
-        w[8] = __int_as_float(weight_bits_c12<8>(blk)) + nm;
-        w[9] = __int_as_float(weight_bits_c12<9>(blk)) + nm;
-        w[10] = __int_as_float(weight_bits_c12<10>(blk)) + nm;
-        w[11] = __int_as_float(weight_bits_c12<11>(blk)) + nm;
+      // Before the CTA can exit and release TMEM: every bulk copy it issued
+      // has landed and its last MMAs have completed.  These waits are bounded
+      // but not cut short by the give-up flag.
+      for (int s = 0; s < XS && s < n_units; ++s) {
+        const int k = (n_units - 1 - s) / XS;  // last load into slab s
+        ok = tc::mbar_wait(xfull(s), k & 1, kWaitLimit) && ok;
       }
-      const int k4_0 = (pq * BPT + i) * (C / 4);
-#pragma unroll
-      for (int q = 0; q < C / 4; ++q) {
-        float h[4], l[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) split_tf32(w[4 * q + u], h[u], l[u]);
-        const uint32_t off = core_off<L::SBO>(prow, k4_0 + q);
-        *reinterpret_cast<float4*>(st + off) = make_float4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<float4*>(st + L::A_BYTES + off) = make_float4(l[0], l[1], l[2], l[3]);
+      if (n_units > 0) {
+        const int last = n_units - 1;
+        ok = tc::mbar_wait(afree(last % AS), (last / AS) & 1, kWaitLimit) && ok;
       }
     }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ producers (+ epilogue)
+    const int lq = warp & 3, kq = warp >> 2;
+    const int prow = 32 * lq + lane;  // TMEM lane = row in the tile
+    auto load_rec = [&](int i, RecUnit<C>& p) {
+      const long long u = u_begin + i;
+      const int tile = (int)(u / g.nchunks), chunk = (int)(u - (long long)tile * g.nchunks);
+      const int gr = tile * kTileM + prow;
+      const int b0 = chunk * (KC / C) + kq * kBpt;  // even
+      const bool ok_ = gr < g.rows && b0 < g.nb;
+      p.r = ok_ ? ld_stream_u2(rec + (size_t)gr * g.rec_pitch + b0) : make_uint2(0u, 0u);
+      p.e = 0;
+      if constexpr (C == 12)
+        p.e = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
+    };
 
-    // ---- B: X[:, stage columns] as fp32 (exact in tf32), zero-padded
-#pragma unroll
-    for (int k = 0; k < XPT; ++k) {
-      const int i = tid + k * kThreads;
-      if (i < XCH) {
-        const int k4 = i / NB, n = i - k4 * NB;
-        const uint2 v = cur.x[k];
-        const float4 f = make_float4(act_to_float((uint16_t)(v.x & 0xffffu), is_bf16),
-                                     act_to_float((uint16_t)(v.x >> 16), is_bf16),
-                                     act_to_float((uint16_t)(v.y & 0xffffu), is_bf16),
-                                     act_to_float((uint16_t)(v.y >> 16), is_bf16));
-        *reinterpret_cast<float4*>(st + 2 * L::A_BYTES + core_off<L::SBO>(n, k4)) = f;
-      }
-    }
-
-    tc::fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
+    auto produce = [&](int i, const RecUnit<C>& cur) {
+      const int as = i % AS;
+      if (i >= AS) ok = tc::mbar_wait_or_abort(afree(as), ((i / AS) - 1) & 1, kWaitLimit, abort_flag) && ok;
       tc::fence_after_sync();
-      const uint32_t a_hi = tc::smem_u32(st), a_lo = a_hi + L::A_BYTES, bb = a_hi + 2 * L::A_BYTES;
+      const uint32_t col0 = tmem + ((uint32_t)(32 * lq) << 16) + as * 2 * KC + kq * kBpt * C;
+      uint32_t hi[kBpt * C], lo[kBpt * C];
 #pragma unroll
-      for (int kk = 0; kk < KC / 8; ++kk) {
-        const uint64_t db = tc::smem_desc(bb + 256 * kk, 128, L::SBO);
-        tc::mma_tf32(tmem, tc::smem_desc(a_hi + 256 * kk, 128, L::SBO), db, idesc,
-                     (it > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_tf32(tmem, tc::smem_desc(a_lo + 256 * kk, 128, L::SBO), db, idesc, 1u);
+      for (int j = 0; j < kBpt; ++j) {
+        const uint32_t r = j ? cur.r.y : cur.r.x;
+        float b[C];
+        float nm;
+        if constexpr (C == 8) {
+          const BlockC8 blk = decode_c8(r, t32, t32 + 256);
+          nm = __uint_as_float(blk.negm);
+          b[0] = __int_as_float(weight_bits_c8<0>(blk));
+          b[1] = __int_as_float(weight_bits_c8<1>(blk));
+          b[2] = __int_as_float(weight_bits_c8<2>(blk));
+          b[3] = __int_as_float(weight_bits_c8<3>(blk));
+          b[4] = __int_as_float(weight_bits_c8<4>(blk));
+          b[5] = __int_as_float(weight_bits_c8<5>(blk));
+          b[6] = __int_as_float(weight_bits_c8<6>(blk));
+          b[7] = __int_as_float(weight_bits_c8<7>(blk));
+        } else {
+          const BlockC12 blk = decode_c12(r, (j ? cur.e >> 4 : cur.e) & 15u, t64, t64 + 256);
+          nm = __uint_as_float(blk.negm);
+          b[0] = __int_as_float(weight_bits_c12<0>(blk));
+          b[1] = __int_as_float(weight_bits_c12<1>(blk));
+          b[2] = __int_as_float(weight_bits_c12<2>(blk));
+          b[3] = __int_as_float(weight_bits_c12<3>(blk));
+          b[4] = __int_as_float(weight_bits_c12<4>(blk));
+          b[5] = __int_as_float(weight_bits_c12<5>(blk));
+          b[6] = __int_as_float(weight_bits_c12<6>(blk));
+          b[7] = __int_as_float(weight_bits_c12<7>(blk));
+          b[8] = __int_as_float(weight_bits_c12<8>(blk));
+          b[9] = __int_as_float(weight_bits_c12<9>(blk));
+          b[10] = __int_as_float(weight_bits_c12<10>(blk));
+          b[11] = __int_as_float(weight_bits_c12<11>(blk));
+        }
+#pragma unroll
+        for (int c = 0; c < C; c += 2)
+          split_pair(b[c], b[c + 1], nm, hi[j * C + c], hi[j * C + c + 1], lo[j * C + c],
+                     lo[j * C + c + 1]);
       }
-      tc::mma_commit(bar0 + 8 * s);
-    }
-  };
-
-  // Record sets and X values are loaded two stages ahead of the one being
-  // built (a ring of three register buffers, unrolled so they stay in
-  // registers).
-  Pref pf[3];
-  if (n_iter > 0) load_pref(c_begin, pf[0]);
-  if (n_iter > 1) load_pref(c_begin + 1, pf[1]);
-  for (int it0 = 0; it0 < n_iter; it0 += 3) {
+      if constexpr (C == 8) {
+        tc::tmem_st16(col0, hi);
+        tc::tmem_st16(col0 + KC, lo);
+      } else {
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      const int it = it0 + k;
-      if (it < n_iter) {
-        if (it + 2 < n_iter) load_pref(c_begin + it + 2, pf[(k + 2) % 3]);
-        build_stage(it, pf[k]);
+        for (int q = 0; q < 3; ++q) {
+          tc::tmem_st8(col0 + 8 * q, hi + 8 * q);
+          tc::tmem_st8(col0 + KC + 8 * q, lo + 8 * q);
+        }
       }
-    }
-  }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(afull(as));
+    };
 
-  // ---- epilogue: wait for the last MMAs, read D, write Y or a partial
-  float d[NB];
-#pragma unroll
-  for (int n = 0; n < NB; ++n) d[n] = 0.f;
-  if (n_iter > 0) {
-    const int s_last = (n_iter - 1) % STAGES, use_last = (n_iter - 1) / STAGES;
-    ok = tc::mbar_wait(bar0 + 8 * s_last, use_last & 1, kWaitLimit) && ok;
-    tc::fence_after_sync();
-    if (warp < 4) {
+    // Warps 0-3 (all 128 TMEM lanes) drain the accumulator of a segment, 16
+    // columns at a time.
+    auto epilogue = [&](int seg, int tile) {
+      const int db = seg & 1;
+      ok = tc::mbar_wait_or_abort(dfull(db), (seg >> 1) & 1, kWaitLimit, abort_flag) && ok;
+      tc::fence_after_sync();
+      const int row = 32 * warp + lane;
+      const int gr = tile * kTileM + row;
+      const int first = unit_owner((long long)tile * g.nchunks, g.units, ctas);
+      const int last = unit_owner((long long)(tile + 1) * g.nchunks - 1, g.units, ctas);
+      float* mine = partial + ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);
 #pragma unroll
       for (int n16 = 0; n16 < NB / 16; ++n16) {
         float v[16];
-        tc::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + 16 * n16, v);
+        tc::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + L::D_COL + 64 * db + 16 * n16, v);
+        if (first == last) {
+          if (gr < g.rows) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) d[16 * n16 + i] = v[i];
-      }
-    }
-  }
-  if (!ok) atomicOr(&g_tc_error, 1u);
-  const int row = 32 * warp + lane;  // valid for warp < 4
-  if (g.splits == 1) {
-    if (warp < 4 && r0 + row < g.rows) {
+            for (int q = 0; q < 16; ++q)
+              if (16 * n16 + q < g.M) Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q];
+          }
+        } else {
 #pragma unroll
-      for (int n = 0; n < NB; ++n)
-        if (n < g.M) Y[(size_t)n * g.rows + r0 + row] = d[n];
-    }
-  } else {
-    float* mine = partial + ((size_t)(tile * g.splits + split) * NB) * kTileM;
-    if (warp < 4) {
-#pragma unroll
-      for (int n = 0; n < NB; ++n) mine[n * kTileM + row] = d[n];
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) slot[1] = (atomicAdd(&counters[tile], 1u) == (unsigned)(g.splits - 1)) ? 1u : 0u;
-    __syncthreads();
-    if (slot[1]) {
-      __threadfence();
-      const float* base = partial + ((size_t)tile * g.splits * NB) * kTileM;
-      for (int i = tid; i < g.M * kTileM; i += kThreads) {
-        const int n = i / kTileM, rr = i - n * kTileM;
-        if (r0 + rr < g.rows) {
-          float acc = 0.f;
-          for (int sp = 0; sp < g.splits; ++sp) acc += base[((size_t)sp * NB + n) * kTileM + rr];
-          Y[(size_t)n * g.rows + r0 + rr] = acc;
+          for (int q = 0; q < 16; ++q) mine[(16 * n16 + q) * kTileM + row] = v[q];
         }
       }
-      if (tid == 0) counters[tile] = 0u;
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(dfree(db));
+      if (first == last) return;
+      __threadfence();
+      tc::named_sync(128);
+      if (tid == 0)
+        slot[1] = (atomicAdd(&counters[tile], 1u) == (unsigned)(last - first)) ? 1u : 0u;
+      tc::named_sync(128);
+      if (slot[1]) {
+        __threadfence();
+        if (gr < g.rows) {
+          for (int n = 0; n < g.M; ++n) {
+            float acc = 0.f;
+            for (int c = first; c <= last; ++c) {
+              const int cseg = tile - (int)(unit_begin(c, g.units, ctas) / g.nchunks);
+              acc += partial[((size_t)c * g.segs_max + cseg) * (NB * kTileM) + n * kTileM + row];
+            }
+            Y[(size_t)n * g.rows + gr] = acc;
+          }
+        }
+        if (tid == 0) counters[tile] = 0u;
+      }
+      tc::named_sync(128);  // slot[1] is rewritten by the next segment
+    };
+
+    RecUnit<C> ring[kRecAhead];
+#pragma unroll
+    for (int k = 0; k < kRecAhead; ++k)
+      if (k < n_units) load_rec(k, ring[k]);
+    int seg = 0;
+    for (int i0 = 0; i0 < n_units; i0 += kRecAhead) {
+#pragma unroll
+      for (int k = 0; k < kRecAhead; ++k) {
+        const int i = i0 + k;
+        if (i < n_units) {
+          const RecUnit<C> cur = ring[k];
+          if (i + kRecAhead < n_units) load_rec(i + kRecAhead, ring[k]);
+          if (seg_first(i) && i > 0) ++seg;
+          produce(i, cur);
+          if (warp < 4 && seg_last(i)) epilogue(seg, t_first + seg);
+        }
+      }
     }
   }
+
+  if (!ok) atomicOr(&g_tc_error, 1u);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, L::TMEM_COLS);
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 template <int C>
-int tc_kc() {
+constexpr int tc_kc() {
   return TcCfg<C>::KC;
 }
 
-TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev) {
+int kc_of(int C) { return C == 8 ? tc_kc<8>() : tc_kc<12>(); }
+
+TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev, int* ctas) {
   TcGeom g;
   g.rows = f.rows;
   g.cols = f.cols;
@@ -352,75 +448,114 @@ TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev) {
   g.rec_pitch = f.rec_pitch;
   g.e_pitch = f.e_pitch;
   g.M = M;
-  const int KC = f.C == 8 ? tc_kc<8>() : tc_kc<12>();
+  const int KC = kc_of(f.C);
   g.nchunks = (f.cols + KC - 1) / KC;
   g.tiles = (f.rows + kTileM - 1) / kTileM;
-  // About three CTAs per SM, each with at least 4 stages of work.
-  int want = (3 * dev.num_sms + g.tiles - 1) / g.tiles;
-  int cap = g.nchunks / 4 > 1 ? g.nchunks / 4 : 1;
-  g.splits = want < 1 ? 1 : (want > cap ? cap : want);
-  g.chunks_per_split = (g.nchunks + g.splits - 1) / g.splits;
-  g.splits = (g.nchunks + g.chunks_per_split - 1) / g.chunks_per_split;
-  g.x_vec = 0;
+  g.units = (long long)g.tiles * g.nchunks;
+  const int G = g.units < dev.num_sms ? (int)g.units : dev.num_sms;
+  int segs = 1;
+  for (int b = 0; b < G; ++b) {
+    const long long a = (long long)b * g.units / G, e = (long long)(b + 1) * g.units / G;
+    const int s = (int)((e - 1) / g.nchunks - a / g.nchunks) + 1;
+    if (s > segs) segs = s;
+  }
+  g.segs_max = segs;
+  *ctas = G < 1 ? 1 : G;
   return g;
 }
 
+// Workspace: [tile counters][X slabs][partial tiles], each part 256-aligned.
+struct TcWorkspace {
+  int64_t cnt_bytes, xs_bytes, part_bytes;
+  int64_t total() const { return cnt_bytes + xs_bytes + part_bytes; }
+};
+
+int64_t round256(int64_t v) { return (v + 255) / 256 * 256; }
+
+TcWorkspace tc_workspace(const TcGeom& g, int C, int ctas) {
+  const int NB = (g.M + 15) / 16 * 16;
+  TcWorkspace w;
+  w.cnt_bytes = round256((int64_t)g.tiles * 4);
+  w.xs_bytes = round256((int64_t)g.nchunks * NB * kc_of(C) * 4);
+  w.part_bytes = round256((int64_t)ctas * g.segs_max * NB * kTileM * 4);
+  return w;
+}
+
 template <int C, int NB>
-int launch_tc(const TcGeom& g, const uint32_t* rec, const uint8_t* eplane, const uint16_t* X,
-              int is_bf16, float* Y, float* partial, unsigned int* counters, cudaStream_t stream,
-              const DeviceInfo& dev) {
+int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* eplane,
+              const uint16_t* X, int is_bf16, float* Y, unsigned char* ws, const TcWorkspace& w,
+              cudaStream_t stream, const DeviceInfo& dev) {
   using L = TcSmem<C, NB>;
   if ((size_t)L::TOTAL > (size_t)dev.max_smem_optin) return SEEDLM_EUNSUPPORTED;
   int rc = allow_max_smem((const void*)gemm_tc_kernel<C, NB>, dev);
   if (rc) return rc;
-  gemm_tc_kernel<C, NB><<<g.tiles * g.splits, kThreads, L::TOTAL, stream>>>(
-      rec, eplane, X, is_bf16, Y, partial, counters, g);
+  unsigned int* counters = reinterpret_cast<unsigned int*>(ws);
+  float* xs = reinterpret_cast<float*>(ws + w.cnt_bytes);
+  float* partial = reinterpret_cast<float*>(ws + w.cnt_bytes + w.xs_bytes);
+
+  const long long groups = (long long)g.nchunks * NB * (TcCfg<C>::KC / 4);
+  long long want = (groups + 255) / 256;
+  const long long cap = 8ll * dev.num_sms;
+  const int sgrid = (int)(want < cap ? (want < 1 ? 1 : want) : cap);
+  stage_x_kernel<C, NB><<<sgrid, 256, 0, stream>>>(X, is_bf16, g.M, g.cols, g.nchunks, xs);
+  count_launch();
+  if ((rc = record_cuda_error(cudaGetLastError()))) return rc;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::TOTAL;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<C, NB>, rec, eplane,
+                                       (const float*)xs, Y, partial, counters, g);
+  if (err != cudaSuccess) return record_cuda_error(err);
   count_launch();
   return record_cuda_error(cudaGetLastError());
+}
+
+int dispatch_tc(const seedlm_format& f, const TcGeom& g, int ctas, const uint32_t* rec,
+                const uint8_t* eplane, const uint16_t* X, int is_bf16, float* Y,
+                unsigned char* ws, const TcWorkspace& w, cudaStream_t st, const DeviceInfo& dev) {
+  const int NB = (g.M + 15) / 16 * 16;
+  if (f.C == 8) {
+    switch (NB) {
+      case 16: return launch_tc<8, 16>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+      case 32: return launch_tc<8, 32>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+      case 48: return launch_tc<8, 48>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+      default: return launch_tc<8, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    }
+  }
+  switch (NB) {
+    case 16: return launch_tc<12, 16>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    case 32: return launch_tc<12, 32>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    case 48: return launch_tc<12, 48>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    default: return launch_tc<12, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+  }
 }
 
 }  // namespace
 
 int64_t gemm_tc_workspace_bytes(const seedlm_format& f, int M, const DeviceInfo& dev) {
-  const TcGeom g = make_tc_geom(f, M, dev);
-  if (g.splits <= 1) return 0;
-  const int NB = (M + 15) / 16 * 16;
-  const int64_t part = (int64_t)g.tiles * g.splits * NB * kTileM * 4;
-  const int64_t cnt = ((int64_t)g.tiles * 4 + 255) / 256 * 256;
-  return (part + 255) / 256 * 256 + cnt;
+  int ctas = 1;
+  const TcGeom g = make_tc_geom(f, M, dev, &ctas);
+  return tc_workspace(g, f.C, ctas).total();
 }
 
 int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                    const uint16_t* X, int is_bf16, int M, float* Y, void* workspace,
                    int64_t workspace_bytes, cudaStream_t stream, const DeviceInfo& dev) {
-  TcGeom g = make_tc_geom(f, M, dev);
-  g.x_vec = (f.cols % 4 == 0 && (reinterpret_cast<uintptr_t>(X) & 7u) == 0) ? 1 : 0;
-  const int64_t need = gemm_tc_workspace_bytes(f, M, dev);
-  if (workspace_bytes < need) return SEEDLM_EINVAL;
-  float* partial = nullptr;
-  unsigned int* counters = nullptr;
-  if (need > 0) {
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SEEDLM_EINVAL;
-    const int NB = (M + 15) / 16 * 16;
-    const int64_t part = ((int64_t)g.tiles * g.splits * NB * kTileM * 4 + 255) / 256 * 256;
-    partial = static_cast<float*>(workspace);
-    counters = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + part);
-  }
-  const int NB = (M + 15) / 16 * 16;
-  if (f.C == 8) {
-    switch (NB) {
-      case 16: return launch_tc<8, 16>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-      case 32: return launch_tc<8, 32>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-      case 48: return launch_tc<8, 48>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-      default: return launch_tc<8, 64>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-    }
-  }
-  switch (NB) {
-    case 16: return launch_tc<12, 16>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-    case 32: return launch_tc<12, 32>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-    case 48: return launch_tc<12, 48>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-    default: return launch_tc<12, 64>(g, rec, eplane, X, is_bf16, Y, partial, counters, stream, dev);
-  }
+  int ctas = 1;
+  const TcGeom g = make_tc_geom(f, M, dev, &ctas);
+  const TcWorkspace w = tc_workspace(g, f.C, ctas);
+  if (workspace_bytes < w.total()) return SEEDLM_EINVAL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SEEDLM_EINVAL;
+  return dispatch_tc(f, g, ctas, rec, eplane, X, is_bf16, Y,
+                     static_cast<unsigned char*>(workspace), w, stream, dev);
 }
 
 int read_and_clear_tc_error(unsigned int* out) {
@@ -437,14 +572,12 @@ int read_and_clear_tc_error(unsigned int* out) {
 
 // ------------------------------------------------ allocation-free variant
 //
-// For callers that cannot allocate device memory themselves, the split-K
-// partial tiles and the per-tile counters of the tensor-core GEMM live in one
+// For callers that cannot allocate device memory themselves, the workspace of
+// the tensor-core GEMM (tile counters, X slabs, partial tiles) lives in one
 // array that the library owns for the life of the process.
 
-constexpr int64_t kNoAllocPartialBytes = 16ll << 20;  // split-K partial tiles
-constexpr int64_t kNoAllocCounterBytes = 64ll << 10;  // one uint32 per 128-row tile
-static __device__ __align__(256) unsigned char
-    g_noalloc_scratch[kNoAllocPartialBytes + kNoAllocCounterBytes];
+constexpr int64_t kNoAllocBytes = (16ll << 20) + (64ll << 10);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 namespace {
 
@@ -502,37 +635,14 @@ extern "C" SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt,
   const int is_bf16 = x_dtype == SEEDLM_BF16;
   if (M == 1) return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
 
-  TcGeom g = make_tc_geom(*fmt, M, dev);
-  g.x_vec = (fmt->cols % 4 == 0 && (reinterpret_cast<uintptr_t>(X) & 7u) == 0) ? 1 : 0;
-  const int NB = (M + 15) / 16 * 16;
-  const int64_t part_bytes =
-      g.splits > 1 ? (int64_t)g.tiles * g.splits * NB * kTileM * (int64_t)sizeof(float) : 0;
-  const int64_t cnt_bytes = g.splits > 1 ? (int64_t)g.tiles * 4 : 0;
-  if (part_bytes > kNoAllocPartialBytes || cnt_bytes > kNoAllocCounterBytes)
-    return SEEDLM_EUNSUPPORTED;  // needs more scratch than the library holds
-  float* partial = nullptr;
-  unsigned int* counters = nullptr;
-  if (g.splits > 1) {
-    unsigned char* base = nullptr;
-    if ((rc = noalloc_scratch(dev, &base))) return rc;
-    partial = reinterpret_cast<float*>(base);
-    counters = reinterpret_cast<unsigned int*>(base + kNoAllocPartialBytes);
-    // The counters must start at zero; the last call may have left them in
-    // any state if it failed part-way.
-    if ((rc = record_cuda_error(cudaMemsetAsync(counters, 0, (size_t)cnt_bytes, st)))) return rc;
-  }
-  if (fmt->C == 8) {
-    switch (NB) {
-      case 16: return launch_tc<8, 16>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-      case 32: return launch_tc<8, 32>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-      case 48: return launch_tc<8, 48>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-      default: return launch_tc<8, 64>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-    }
-  }
-  switch (NB) {
-    case 16: return launch_tc<12, 16>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-    case 32: return launch_tc<12, 32>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-    case 48: return launch_tc<12, 48>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-    default: return launch_tc<12, 64>(g, rec, eplane, Xh, is_bf16, Y, partial, counters, st, dev);
-  }
+  int ctas = 1;
+  const TcGeom g = make_tc_geom(*fmt, M, dev, &ctas);
+  const TcWorkspace w = tc_workspace(g, fmt->C, ctas);
+  if (w.total() > kNoAllocBytes) return SEEDLM_EUNSUPPORTED;  // needs more than the library holds
+  unsigned char* base = nullptr;
+  if ((rc = noalloc_scratch(dev, &base))) return rc;
+  // The counters must start at zero; the last call may have left them in any
+  // state if it failed part-way.
+  if ((rc = record_cuda_error(cudaMemsetAsync(base, 0, (size_t)w.cnt_bytes, st)))) return rc;
+  return dispatch_tc(*fmt, g, ctas, rec, eplane, Xh, is_bf16, Y, base, w, st, dev);
 }

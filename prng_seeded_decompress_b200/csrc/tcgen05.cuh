@@ -1,6 +1,7 @@
 // tcgen05.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core path:
-// shared-memory matrix descriptors, tcgen05.mma (kind::tf32), TMEM
-// allocation and loads, and mbarriers with bounded waits.
+// shared-memory matrix descriptors, tcgen05.mma (kind::tf32, A from shared
+// or tensor memory), TMEM allocation, loads and stores, bulk copies and
+// mbarriers with bounded waits.
 #pragma once
 
 #include <stdint.h>
@@ -45,6 +46,19 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
       :
       : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
+        "r"(0u), "r"(0u));
+}
+
+// Same with A taken from tensor memory: A is 128 lanes (rows) x 8 columns
+// (one tf32 per column) starting at TMEM address `a_tmem`.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
         "r"(0u), "r"(0u));
 }
 
@@ -99,11 +113,62 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 16 (or 8) 32-bit columns into TMEM; warp w writes lanes
+// 32(w%4)..32(w%4)+31, thread i its own lane.  Complete with tmem_wait_st.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" : : "r"(mbar), "r"(count) : "memory");
 }
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Plain arrival (release, CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" : : "r"(mbar) : "memory");
+}
+// Arrival that also expects `bytes` of asynchronous copies on this phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               :
+               : "r"(mbar), "r"(bytes)
+               : "memory");
+}
+// Plain (untiled, single-CTA) bulk copy of `bytes` from global memory to this
+// CTA's shared memory; completion is counted on `mbar`.  Both addresses
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :
+      : "r"(dst), "l"(src), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+// Barrier 1 over the first `n` threads of the CTA (n a multiple of 32).
+__device__ __forceinline__ void named_sync(uint32_t n) {
+  asm volatile("bar.sync 1, %0;" : : "r"(n) : "memory");
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -127,6 +192,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64
         : "memory");
     if (done) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// As mbar_wait, sharing one give-up flag across the CTA: once any wait has
+// given up (and set *abort), every later wait returns false at once, so a
+// broken hand-over costs one time-out, not one per wait.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t mbar, uint32_t parity,
+                                                   uint64_t limit_ns, volatile uint32_t* abort) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1u;
+      return false;
+    }
   }
 }
 

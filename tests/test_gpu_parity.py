@@ -5,6 +5,8 @@ rational, exact in fp32).  Products must satisfy, per output,
 |y - y_oracle| <= 1e-5 * sum_j |W_rj x_j| (the oracle accumulates in fp64).
 All calls go through the C ABI (ctypes binding).
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -222,6 +224,19 @@ def test_gemm_small_fp16_and_odd_shapes(sl, oracle_mod, cp):
         ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv)
         for m in range(M):
             assert_within(got[m], ref[m], refabs[m])
+
+
+@pytest.mark.parametrize("cp,rows,cols,M", [(C8, 57344, 128, 16), (C12, 20000, 200, 33)])
+def test_gemm_many_short_tiles_per_cta(sl, oracle_mod, cp, rows, cols, M):
+    # Few K chunks per row tile and many tiles: each CTA's range covers several
+    # whole tiles (written straight to Y) plus shared ones at its ends, and
+    # reuses both TMEM accumulators more than once.
+    L = inputs.make_layer(rows, cols, *cp, seed=rows + M)
+    Xb, Xv = inputs.make_activations((M, cols), "bf16", 17)
+    got = gpu_gemm(sl, L, Xb)
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv, threads=os.cpu_count() or 1)
+    for m in range(M):
+        assert_within(got[m], ref[m], refabs[m])
 
 
 def test_gemm_workspace_reuse_is_deterministic(sl):

@@ -1,8 +1,8 @@
 """seedlm_gemm_smallM_noalloc: the small-M GEMM for callers that cannot
 allocate device memory (a library embedded in a host program that owns the
 GPU's memory pool, or a path that must not pay cudaMalloc's implicit device
-synchronisation), so cannot hand in a workspace.  Its split-K scratch is an
-array inside libseedlm.so.
+synchronisation), so cannot hand in a workspace.  Its workspace is an array
+inside libseedlm.so.
 
 These tests call the entry point through the C ABI (ctypes) and compare it
 with seedlm_gemm_smallM (caller workspace) on the same inputs, within the
@@ -95,14 +95,15 @@ def test_noalloc_matches_workspace_entry_on_two_calls(sl, oracle_mod, cp, rows, 
 
 @pytest.mark.gpu
 def test_noalloc_rejects_problems_beyond_its_scratch(sl):
-    # 38400 rows = 300 tiles, split in two over 8192 columns at M = 64:
-    # 600 partial tiles x 32 KiB = 19.7 MB > 16 MiB of scratch.
+    # 38400 rows = 300 tiles over 8192 columns at M = 64: one CTA per SM
+    # covers about two tiles, touches up to four, and keeps a 32 KiB partial
+    # tile for each -- more than the 16 MiB + 64 KiB the library holds.
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     rows, cols, M = 38400, 8192, 64
     fmt = inputs.make_format(rows, cols, *C8)
     need = sl.gemm_workspace_bytes(fmt, M)
-    if need <= 16 << 20:
+    if need <= (16 << 20) + (64 << 10):
         pytest.skip("this device splits the problem so that it fits")
     rec = torch.zeros((rows, fmt["rec_pitch"]), dtype=torch.int32, device="cuda")
     X = torch.zeros((M, cols), dtype=torch.bfloat16, device="cuda")
