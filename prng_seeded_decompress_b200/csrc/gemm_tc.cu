@@ -52,7 +52,9 @@ namespace {
 
 constexpr int kTileM = 128;
 constexpr int kProdWarps = 16;
-constexpr int kThreads = (kProdWarps + 1) * 32;  // + the MMA / X-loader warp
+constexpr int kMmaWarp = kProdWarps;         // issues the MMAs (one thread)
+constexpr int kLoaderWarp = kProdWarps + 1;  // copies the X slabs (one thread)
+constexpr int kThreads = (kProdWarps + 2) * 32;
 constexpr int kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
@@ -92,8 +94,8 @@ struct TcSmem {
   static constexpr int TABLE_OFF = XS * XB;
   static constexpr int TABLE_BYTES = (C == 8) ? 512 * 4 : 512 * 8;
   static constexpr int BAR_OFF = TABLE_OFF + TABLE_BYTES;
-  // mbarriers: xfull[XS] xfree[XS] afull[AS] afree[AS] dfull[2] dfree[2]
-  static constexpr int NBAR = 2 * XS + 2 * AS + 4;
+  // mbarriers: xfull[XS] xfree[XS] afull[AS] afree[AS] dfree[2]
+  static constexpr int NBAR = 2 * XS + 2 * AS + 2;
   static constexpr int SLOT_OFF = BAR_OFF + 8 * NBAR;  // TMEM base, last-CTA flag, give-up flag
   static constexpr int TOTAL = SLOT_OFF + 16;
   static constexpr int D_COL = AS * 2 * KC;  // first accumulator column
@@ -155,6 +157,18 @@ __device__ __forceinline__ void split_pair(float b0, float b1, float nm, uint32_
   l1 = __float_as_uint(l.y);
 }
 
+// (tile, chunk) of consecutive units, advanced without dividing: a 64-bit
+// division costs hundreds of instructions, more than rebuilding a unit.
+struct UnitCursor {
+  int tile, chunk;
+  __device__ __forceinline__ void next(int nchunks) {
+    if (++chunk == nchunks) {
+      chunk = 0;
+      ++tile;
+    }
+  }
+};
+
 template <int C>
 struct RecUnit {
   uint2 r;     // the thread's two records of this unit
@@ -174,6 +188,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   const long long u_begin = unit_begin(blockIdx.x, g.units, ctas);
   const int n_units = (int)(unit_begin(blockIdx.x + 1, g.units, ctas) - u_begin);
   const int t_first = (int)(u_begin / g.nchunks);
+  const UnitCursor c0{t_first, (int)(u_begin - (long long)t_first * g.nchunks)};
 
   uint32_t* t32 = reinterpret_cast<uint32_t*>(smem + L::TABLE_OFF);
   uint2* t64 = reinterpret_cast<uint2*>(smem + L::TABLE_OFF);
@@ -185,12 +200,15 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       t64[i] = make_uint2((uint32_t)v, (uint32_t)(v >> 32));
   }
   const uint32_t bar = tc::smem_u32(smem + L::BAR_OFF);
+  // xfull: X slab landed.  xfree: the MMAs that read the slab completed.
+  // afull: all producer warps stored the A stage.  afree: the unit's MMAs
+  // completed: its A stage may be reused and, at a segment's end, the
+  // accumulator is final.  dfree: warps 0-3 have read an accumulator out.
   auto xfull = [&](int s) { return bar + 8 * s; };
   auto xfree = [&](int s) { return bar + 8 * (XS + s); };
   auto afull = [&](int s) { return bar + 8 * (2 * XS + s); };
   auto afree = [&](int s) { return bar + 8 * (2 * XS + AS + s); };
-  auto dfull = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + b); };
-  auto dfree = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + 2 + b); };
+  auto dfree = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + b); };
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
   if (tid == 0) {
     for (int s = 0; s < XS; ++s) {
@@ -201,10 +219,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       tc::mbar_init(afull(s), kProdWarps);
       tc::mbar_init(afree(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(dfull(b), 1);
-      tc::mbar_init(dfree(b), 4);
-    }
+    for (int b = 0; b < 2; ++b) tc::mbar_init(dfree(b), 4);
     tc::fence_mbar_init();
     slot[2] = 0u;  // give-up flag shared by all bounded waits
   }
@@ -216,61 +231,64 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   volatile uint32_t* abort_flag = slot + 2;
   bool ok = true;
 
-  auto seg_first = [&](int i) { return i == 0 || (u_begin + i) % g.nchunks == 0; };
-  auto seg_last = [&](int i) {
-    return i == n_units - 1 || (u_begin + i) % g.nchunks == g.nchunks - 1;
-  };
-
-  if (warp == kProdWarps) {
-    // ------------------------------------------------ MMA issue + X slabs
+  if (warp == kLoaderWarp) {
+    // ------------------------------------------------ X slabs
     if (lane == 0) {
       const uint32_t xs0 = tc::smem_u32(smem);
-      auto load_x = [&](int i) {
-        const int s = i % XS;
-        const int chunk = (int)((u_begin + i) % g.nchunks);
-        tc::mbar_arrive_expect_tx(xfull(s), L::XB);
-        tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)chunk * (NB * KC), L::XB, xfull(s));
-      };
+      UnitCursor xc = c0;
       // Xs is written by the previous kernel on the stream.
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int i = 0; i < XS && i < n_units; ++i) load_x(i);
+      for (int j = 0; j < n_units; ++j, xc.next(g.nchunks)) {
+        const int s = j % XS;
+        if (j >= XS)  // the slab's previous unit (j - XS) has finished its MMAs
+          ok = tc::mbar_wait_or_abort(xfree(s), ((j / XS) - 1) & 1, kWaitLimit, abort_flag) && ok;
+        tc::mbar_arrive_expect_tx(xfull(s), L::XB);
+        tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)xc.chunk * (NB * KC), L::XB, xfull(s));
+      }
+      // Every copy this thread issued has landed before the CTA may exit
+      // (bounded, and not cut short by the give-up flag).
+      for (int s = 0; s < XS && s < n_units; ++s) {
+        const int k = (n_units - 1 - s) / XS;  // last load into slab s
+        ok = tc::mbar_wait(xfull(s), k & 1, kWaitLimit) && ok;
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issue
+    if (lane == 0) {
       const uint32_t idesc = tc::idesc_tf32(NB);
+      const uint64_t bdesc0 = tc::smem_desc(tc::smem_u32(smem), 128, L::SBO);  // slab 0, K slice 0
       int seg = 0;
-      for (int i = 0; i < n_units; ++i) {
-        const bool first = seg_first(i);
+      UnitCursor mc = c0;
+      for (int i = 0; i < n_units; ++i, mc.next(g.nchunks)) {
+        const bool first = i == 0 || mc.chunk == 0;
         if (first && i > 0) ++seg;
         const int db = seg & 1;
         if (first && seg >= 2)  // accumulator db was last used by segment seg - 2
           ok = tc::mbar_wait_or_abort(dfree(db), ((seg >> 1) - 1) & 1, kWaitLimit, abort_flag) && ok;
         const int xs = i % XS, as = i % AS;
-        ok = tc::mbar_wait_or_abort(xfull(xs), (i / XS) & 1, kWaitLimit, abort_flag) && ok;
-        ok = tc::mbar_wait_or_abort(afull(as), (i / AS) & 1, kWaitLimit, abort_flag) && ok;
+        if (!tc::mbar_try_wait2(xfull(xs), (i / XS) & 1, afull(as), (i / AS) & 1)) {
+          ok = tc::mbar_wait_or_abort(xfull(xs), (i / XS) & 1, kWaitLimit, abort_flag) && ok;
+          ok = tc::mbar_wait_or_abort(afull(as), (i / AS) & 1, kWaitLimit, abort_flag) && ok;
+        }
         tc::fence_after_sync();
+        // This thread's issue rate bounds the kernel (an MMA of this shape
+        // takes the tensor core about 45 cycles), so everything but the MMAs
+        // is computed up front.
         const uint32_t a_hi = tmem + as * 2 * KC, a_lo = a_hi + KC;
         const uint32_t d = tmem + L::D_COL + 64 * db;
-        const uint32_t xb = xs0 + xs * L::XB;
+        const uint64_t bd = bdesc0 + (uint64_t)((xs * L::XB) >> 4);
+        const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
         for (int kk = 0; kk < KC / 8; ++kk) {
-          const uint64_t bd = tc::smem_desc(xb + 256 * kk, 128, L::SBO);
-          tc::mma_tf32_ts(d, a_hi + 8 * kk, bd, idesc, (first && kk == 0) ? 0u : 1u);
-          tc::mma_tf32_ts(d, a_lo + 8 * kk, bd, idesc, 1u);
+          tc::mma_tf32_ts(d, a_hi + 8 * kk, bd + 16 * kk, idesc, kk == 0 ? acc0 : 1u);
+          tc::mma_tf32_ts(d, a_lo + 8 * kk, bd + 16 * kk, idesc, 1u);
         }
-        tc::mma_commit(afree(as));
-        tc::mma_commit(xfree(xs));
-        if (seg_last(i)) tc::mma_commit(dfull(db));
-        // Refill the slab of unit i - 2 (its MMAs were queued two units ago).
-        if (i >= 2 && i - 2 + XS < n_units) {
-          ok = tc::mbar_wait_or_abort(xfree((i - 2) % XS), ((i - 2) / XS) & 1, kWaitLimit, abort_flag) && ok;
-          load_x(i - 2 + XS);
-        }
+        tc::mma_commit(afree(as));  // A stage free; at a segment's end the accumulator is final
+        tc::mma_commit(xfree(xs));  // X slab free
       }
-      // Before the CTA can exit and release TMEM: every bulk copy it issued
-      // has landed and its last MMAs have completed.  These waits are bounded
-      // but not cut short by the give-up flag.
-      for (int s = 0; s < XS && s < n_units; ++s) {
-        const int k = (n_units - 1 - s) / XS;  // last load into slab s
-        ok = tc::mbar_wait(xfull(s), k & 1, kWaitLimit) && ok;
-      }
+      // The CTA releases TMEM only after its last MMAs have completed
+      // (bounded, not cut short by the give-up flag).
       if (n_units > 0) {
         const int last = n_units - 1;
         ok = tc::mbar_wait(afree(last % AS), (last / AS) & 1, kWaitLimit) && ok;
@@ -281,11 +299,9 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     // ------------------------------------------------ producers (+ epilogue)
     const int lq = warp & 3, kq = warp >> 2;
     const int prow = 32 * lq + lane;  // TMEM lane = row in the tile
-    auto load_rec = [&](int i, RecUnit<C>& p) {
-      const long long u = u_begin + i;
-      const int tile = (int)(u / g.nchunks), chunk = (int)(u - (long long)tile * g.nchunks);
-      const int gr = tile * kTileM + prow;
-      const int b0 = chunk * (KC / C) + kq * kBpt;  // even
+    auto load_rec = [&](const UnitCursor& u, RecUnit<C>& p) {
+      const int gr = u.tile * kTileM + prow;
+      const int b0 = u.chunk * (KC / C) + kq * kBpt;  // even
       const bool ok_ = gr < g.rows && b0 < g.nb;
       p.r = ok_ ? ld_stream_u2(rec + (size_t)gr * g.rec_pitch + b0) : make_uint2(0u, 0u);
       p.e = 0;
@@ -354,9 +370,10 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
 
     // Warps 0-3 (all 128 TMEM lanes) drain the accumulator of a segment, 16
     // columns at a time.
-    auto epilogue = [&](int seg, int tile) {
+    auto epilogue = [&](int seg, int tile, int i_last) {
       const int db = seg & 1;
-      ok = tc::mbar_wait_or_abort(dfull(db), (seg >> 1) & 1, kWaitLimit, abort_flag) && ok;
+      ok = tc::mbar_wait_or_abort(afree(i_last % AS), (i_last / AS) & 1, kWaitLimit, abort_flag) &&
+           ok;
       tc::fence_after_sync();
       const int row = 32 * warp + lane;
       const int gr = tile * kTileM + row;
@@ -390,13 +407,14 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       if (slot[1]) {
         __threadfence();
         if (gr < g.rows) {
-          for (int n = 0; n < g.M; ++n) {
-            float acc = 0.f;
-            for (int c = first; c <= last; ++c) {
-              const int cseg = tile - (int)(unit_begin(c, g.units, ctas) / g.nchunks);
-              acc += partial[((size_t)c * g.segs_max + cseg) * (NB * kTileM) + n * kTileM + row];
+          // Y = partial(first) + partial(first + 1) + ... in CTA order.
+          for (int c = first; c <= last; ++c) {
+            const int cseg = tile - (int)(unit_begin(c, g.units, ctas) / g.nchunks);
+            const float* p = partial + ((size_t)c * g.segs_max + cseg) * (NB * kTileM) + row;
+            for (int n = 0; n < g.M; ++n) {
+              float* y = Y + (size_t)n * g.rows + gr;
+              *y = (c == first) ? p[n * kTileM] : *y + p[n * kTileM];
             }
-            Y[(size_t)n * g.rows + gr] = acc;
           }
         }
         if (tid == 0) counters[tile] = 0u;
@@ -405,9 +423,14 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     };
 
     RecUnit<C> ring[kRecAhead];
+    UnitCursor rc = c0;  // next unit whose records are loaded
 #pragma unroll
     for (int k = 0; k < kRecAhead; ++k)
-      if (k < n_units) load_rec(k, ring[k]);
+      if (k < n_units) {
+        load_rec(rc, ring[k]);
+        rc.next(g.nchunks);
+      }
+    UnitCursor pc = c0;  // unit being rebuilt
     int seg = 0;
     for (int i0 = 0; i0 < n_units; i0 += kRecAhead) {
 #pragma unroll
@@ -415,10 +438,15 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         const int i = i0 + k;
         if (i < n_units) {
           const RecUnit<C> cur = ring[k];
-          if (i + kRecAhead < n_units) load_rec(i + kRecAhead, ring[k]);
-          if (seg_first(i) && i > 0) ++seg;
+          if (i + kRecAhead < n_units) {
+            load_rec(rc, ring[k]);
+            rc.next(g.nchunks);
+          }
+          if (i > 0 && pc.chunk == 0) ++seg;
           produce(i, cur);
-          if (warp < 4 && seg_last(i)) epilogue(seg, t_first + seg);
+          if (warp < 4 && (i == n_units - 1 || pc.chunk == g.nchunks - 1))
+            epilogue(seg, pc.tile, i);
+          pc.next(g.nchunks);
         }
       }
     }

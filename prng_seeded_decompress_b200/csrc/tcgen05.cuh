@@ -179,7 +179,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Waits until the mbarrier's phase with the given parity has completed, for
 // at most `limit_ns` nanoseconds.  Returns false if it gave up.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(done)
+      : "r"(mbar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(mbar, parity)) return true;  // fast path: no timer read
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     uint32_t done;
@@ -195,11 +208,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64
   }
 }
 
+// Both phases complete?  One round trip to the barrier unit for the two
+// checks (the fast path of waiting on two barriers at once).
+__device__ __forceinline__ bool mbar_try_wait2(uint32_t b1, uint32_t p1, uint32_t b2, uint32_t p2) {
+  uint32_t d1, d2;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%2], %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 q, [%4], %5;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "selp.u32 %1, 1, 0, q;\n\t}\n"
+      : "=r"(d1), "=r"(d2)
+      : "r"(b1), "r"(p1), "r"(b2), "r"(p2)
+      : "memory");
+  return (d1 & d2) != 0;
+}
+
 // As mbar_wait, sharing one give-up flag across the CTA: once any wait has
 // given up (and set *abort), every later wait returns false at once, so a
 // broken hand-over costs one time-out, not one per wait.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint32_t mbar, uint32_t parity,
                                                    uint64_t limit_ns, volatile uint32_t* abort) {
+  if (mbar_try_wait(mbar, parity)) return true;  // fast path: no timer read
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     uint32_t done;
