@@ -208,6 +208,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64
   }
 }
 
+// try_wait that lets the hardware park the thread for up to `hint_ns`
+// (woken early when the phase completes), so waiting warps do not take
+// issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t mbar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(done)
+      : "r"(mbar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
 // Both phases complete?  One round trip to the barrier unit for the two
 // checks (the fast path of waiting on two barriers at once).
 __device__ __forceinline__ bool mbar_try_wait2(uint32_t b1, uint32_t p1, uint32_t b2, uint32_t p2) {
@@ -232,15 +247,7 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint32_t mbar, uint32_t parit
   if (mbar_try_wait(mbar, parity)) return true;  // fast path: no timer read
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(mbar), "r"(parity)
-        : "memory");
-    if (done) return true;
+    if (mbar_try_wait_sleep(mbar, parity, 20000u)) return true;
     if (*abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1u;
