@@ -196,7 +196,27 @@ def cpu_baseline(shapes, fmt_cp, target_s=12.0):
     return {"value": round(2 * w / s / 1e9, 6), "unit": UNIT, "cores": threads,
             "kind": "oracle",
             "sample": f"first {rows} rows of each of the 4 layer shapes, {passes} pass(es): "
-                      f"{w / 1e6:.1f} M weights in {s:.1f} s, fp64, {threads} host threads"}
+                      f"{w / 1e6:.1f} M weights in {s:.1f} s, fp64, {threads} host threads",
+            "encode": cpu_encode_baseline()}
+
+
+def cpu_encode_baseline(blocks: int = 24):
+    """The oracle's seed search (NumPy, vectorised over seeds) on Gaussian
+    4-bit blocks, for comparison with the GPU encoder in `extras`."""
+    import numpy as np
+
+    from oracle.search import _tables, seed_search
+    t0 = time.perf_counter()
+    _tables(8, 3)                                   # pinv of all 65,535 seeds, once
+    setup = time.perf_counter() - t0
+    rng = np.random.default_rng(11)
+    W = rng.standard_normal((blocks, 8)) * 0.02
+    t0 = time.perf_counter()
+    for b in range(blocks):
+        seed_search(W[b], 8, 3)
+    s = time.perf_counter() - t0
+    return {"blocks_per_s": round(blocks / s, 2), "sample": f"{blocks} Gaussian 4-bit blocks "
+            f"in {s:.1f} s after {setup:.1f} s of pseudo-inverse tables (NumPy, fp64)"}
 
 
 # --------------------------------------------------------------- GPU arm
@@ -253,7 +273,7 @@ def layer_bytes(shapes, cp):
 
 def extras(torch, sl, args):
     """The other workloads, one GPU: square sweep, 3-bit 8B layer, small-M
-    GEMM, decompression, dense fp16 GEMV reference point."""
+    GEMM, decompression, the encoder, dense fp16 GEMV reference point."""
     import numpy as np
 
     from prng_seeded_decompress_b200 import inputs
@@ -365,6 +385,21 @@ def extras(torch, sl, args):
     out["decompress_4bit_8192x28672"] = {"us_per_call": round(us, 1),
                                         "hbm_gbs_read_plus_write": round(moved / us / 1e3, 1)}
     del W, m
+
+    # Encoder (offline): full seed / coefficient / exponent search of a
+    # Gaussian 1024 x 1024 matrix at 4 bits (131,072 blocks x 65,535 seeds x
+    # 16 exponents), one call after a warm-up call.
+    rng = np.random.default_rng(11)
+    We = torch.from_numpy((rng.standard_normal((1024, 1024)) * 0.02).astype(np.float32)).cuda()
+    fe = inputs.make_format(1024, 1024, 8, 3)
+    rec_e = torch.empty((1024, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
+    sl.encode(fe, We, rec_e)
+    ms = time_region(torch, lambda i: sl.encode(fe, We, rec_e), 1)
+    blocks = 1024 * fe["nb"]
+    out["encode_4bit_1024x1024"] = {
+        "ms_per_call": round(ms, 1), "blocks_per_s": round(blocks / (ms / 1e3)),
+        "candidates_per_s_e9": round(blocks * 65535 * 16 / (ms / 1e3) / 1e9, 2)}
+    del We, rec_e
 
     # Dense fp16 GEMV (in-house) on the 70B layer shapes, 4 rotating copies.
     rng = np.random.default_rng(3)

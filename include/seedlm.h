@@ -147,6 +147,23 @@ SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt, const uint32
                                           const uint8_t* eplane, const void* X, int x_dtype,
                                           int M, float* Y, seedlm_stream stream);
 
+/* The encoder: writes the records (and, for (12,4), the exponent plane) that
+ * represent W (rows x cols fp32, row-major, leading dimension ldw >= cols,
+ * device memory).  For every C-weight block w the seed s, coefficients q and
+ * exponent e minimise ||w - U(s) q 2^-e||^2 over all 65,535 seeds and
+ * e = 0..15, with q = clamp(round-half-even(pinv(U(s)) w 2^e), -8, 7); ties go
+ * to the smallest seed, then the largest e (paperhub.cn thread, authors'
+ * replies on parameter optimisation: a search over seeds, parallel over
+ * blocks; the rounding and exponent rules are this library's reading).  A
+ * tail block is fitted with its missing weights taken as zero.  rec/eplane
+ * use the layout of seedlm_format; record slots past nb and exponent-plane
+ * bytes past ceil(nb / 2) are left untouched.  err (optional, NULL or device
+ * memory of rows x nb doubles, 8-byte aligned) receives each block's squared
+ * error.  A full search costs ~37 M fp64 operations per 8-weight block, so
+ * this is an offline (model-load) step, not part of the hot path. */
+SEEDLM_API int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_t* rec,
+                             uint8_t* eplane, double* err, seedlm_stream stream);
+
 /* Reads and clears the device-side error flag of the current device: 1 if a
  * kernel gave up waiting on one of its own barriers (the outputs of that call
  * are then undefined), else 0.  HOST function; synchronous. */

@@ -168,6 +168,19 @@ int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M) {
   return gemm_tc_workspace_bytes(*fmt, M, dev);
 }
 
+int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_t* rec,
+                  uint8_t* eplane, double* err, seedlm_stream stream) {
+  int rc = check_format(fmt);
+  if (rc) return rc;
+  if ((rc = check_planes(fmt, rec, eplane))) return rc;
+  if (fmt->rows == 0 || fmt->cols == 0) return SEEDLM_OK;
+  if (!W || !aligned(W, 4) || ldw < fmt->cols) return SEEDLM_EINVAL;
+  if (err && !aligned(err, 8)) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  return launch_encode(*fmt, W, ldw, rec, eplane, err, (cudaStream_t)stream);
+}
+
 int seedlm_device_error(int* flag) {
   if (!flag) return SEEDLM_EINVAL;
   DeviceInfo dev;

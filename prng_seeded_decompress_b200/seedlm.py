@@ -22,6 +22,7 @@ EXPORTS = (
     "seedlm_gemm_smallM_workspace_bytes", "seedlm_gemm_smallM_noalloc", "seedlm_device_error",
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
+    "seedlm_encode",
 )
 
 
@@ -59,6 +60,7 @@ def _load():
         "seedlm_gemm_smallM_noalloc": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int,
                                                       ctypes.c_int, vp, vp]),
         "seedlm_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
+        "seedlm_encode": (ctypes.c_int, [fmtp, vp, i64, vp, vp, vp, vp]),
         "seedlm_dense_gemv_f16": (ctypes.c_int, [i32, i32, vp, i64, vp, vp, vp]),
         "seedlm_row_bytes_ideal": (i64, [fmtp]),
         "seedlm_row_bytes_stored": (i64, [fmtp]),
@@ -139,6 +141,18 @@ def decompress(fmt, rec, eplane, W, ldw: int | None = None, stream=None):
     ld = ldw if ldw is not None else (W.stride(0) if W.dim() == 2 else f.cols)
     _check("seedlm_decompress", lib.seedlm_decompress(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(W), ld, _stream(stream, W)))
+
+
+def encode(fmt, W, rec, eplane=None, err=None, ldw: int | None = None, stream=None):
+    """Search seeds, coefficients and exponents for every block of W (fp32,
+    rows x cols, device) and write them into rec (int32/uint32, rows x
+    rec_pitch) and, for C = 12, eplane (uint8, rows x e_pitch).  err, if
+    given, is a float64 (rows x nb) tensor that receives each block's squared
+    reconstruction error."""
+    f = _fmt(fmt)
+    ld = ldw if ldw is not None else (W.stride(0) if W.dim() == 2 else f.cols)
+    _check("seedlm_encode", lib.seedlm_encode(
+        ctypes.byref(f), _ptr(W), ld, _ptr(rec), _ptr(eplane), _ptr(err), _stream(stream, W)))
 
 
 def gemv(fmt, rec, eplane, x, y, stream=None):

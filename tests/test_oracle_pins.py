@@ -289,3 +289,19 @@ def test_search_prefers_the_better_seed(oracle_mod):
         for ee in range(16):
             qq = np.clip(np.rint(t * 2.0 ** ee), -8, 7)
             assert ((w - U @ qq * 2.0 ** -ee) ** 2).sum() >= err
+
+
+# ------------------------------------------------- shifted bit streams
+
+@pytest.mark.parametrize("C,P", [(8, 3), (12, 4)])
+def test_basis_of_the_state_C_steps_on_is_the_shifted_basis(oracle_mod, C, P):
+    # Column p of U(s) is built from states pC..pC+C-1 of the register started
+    # at s.  Started instead at the state C steps on, s', the register runs
+    # through the same states C later, so U(s')[:, p] = U(s)[:, p + 1].  (This
+    # is why an encoder can meet exact ties between seeds.)
+    rng = np.random.default_rng(5)
+    for s in rng.integers(1, 65536, 20):
+        states = oracle_mod.lfsr_states(int(s), C + 1)
+        s2 = int(states[C])
+        U, U2 = oracle_mod.block_basis(int(s), C, P), oracle_mod.block_basis(s2, C, P)
+        assert np.array_equal(U2[:, :P - 1], U[:, 1:])
