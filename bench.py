@@ -352,9 +352,13 @@ def extras(torch, sl, args):
             mats = [mats[0], dict(mats[0], rec=mats[0]["rec"].clone(),
                                   ep=None if mats[0]["ep"] is None else mats[0]["ep"].clone())]
             f = sl.Format.from_dict(mats[0]["fmt"])
-            for M in (1, 8, 16, 64):
-                Xb, _ = inputs.make_activations((M, N), "bf16", 950 + M)
-                X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+            # bf16 activations (three bf16 pieces of W) at every M, fp16 (two
+            # fp16 pieces) at M = 16 and 64.
+            for M, dt in ((1, "bf16"), (8, "bf16"), (16, "bf16"), (64, "bf16"), (16, "f16"),
+                          (64, "f16")):
+                Xb, _ = inputs.make_activations((M, N), dt, 950 + M)
+                X = torch.from_numpy(Xb.view(np.int16)).cuda().view(
+                    torch.bfloat16 if dt == "bf16" else torch.float16)
                 Y = torch.empty((M, R), device="cuda")
                 ws = sl.gemm_workspace(f, M)
                 fn = lambda i: sl.gemm_smallM(f, mats[i % 2]["rec"], mats[i % 2]["ep"], X, Y,  # noqa
@@ -362,7 +366,8 @@ def extras(torch, sl, args):
                 fn(0)
                 reps = 50
                 us = time_region(torch, fn, reps) / reps * 1e3
-                gemm[f"{tag}/{name}/M={M}"] = {
+                key = f"{tag}/{name}/M={M}" + ("" if dt == "bf16" else "/f16")
+                gemm[key] = {
                     "us_per_call": round(us, 2), "weights_per_s_e9": round(R * N / us / 1e3, 2),
                     "tflops_useful": round(2 * M * R * N / us / 1e6, 2)}
             xb, _ = inputs.make_activations((N,), "bf16", 990)

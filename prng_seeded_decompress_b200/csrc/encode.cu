@@ -182,23 +182,30 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
           t[p] = acc;
         }
         // Exponents in descending order: on an exact tie the larger e, met
-        // first, stays.
+        // first, stays.  |t* 2^e| shrinks with e, so once every q rounds to
+        // 0 all smaller exponents give that same candidate (error ||w||^2,
+        // met later): the loop ends there.
 #pragma unroll 4
         for (int e = 15; e >= 0; --e) {
           const double sc = (double)(1 << e), inv = 1.0 / (double)(1 << e);
           double q[P];
+          bool zero = true;
 #pragma unroll
-          for (int p = 0; p < P; ++p) q[p] = fmin(fmax(rint(t[p] * sc), -8.0), 7.0);
+          for (int p = 0; p < P; ++p) {
+            q[p] = fmin(fmax(rint(t[p] * sc), -8.0), 7.0);
+            zero = zero && q[p] == 0.0;
+          }
+          // q.b and q^T G q (G symmetric: diagonal once, off-diagonal twice).
           double qb = 0.0, qgq = 0.0;
 #pragma unroll
           for (int p = 0; p < P; ++p) {
             qb = fma(q[p], b[p], qb);
-            double gq = 0.0;
+            double row = 0.5 * ch.G[j][p * P + p] * q[p];
 #pragma unroll
-            for (int r = 0; r < P; ++r) gq = fma(ch.G[j][p * P + r], q[r], gq);
-            qgq = fma(q[p], gq, qgq);
+            for (int r = p + 1; r < P; ++r) row = fma(ch.G[j][p * P + r], q[r], row);
+            qgq = fma(q[p], row, qgq);
           }
-          const double err = fma(inv * inv, qgq, fma(-2.0 * inv, qb, ww[k]));
+          const double err = fma(2.0 * inv * inv, qgq, fma(-2.0 * inv, qb, ww[k]));
           if (err < best[k].err) {
             best[k].err = err;
             best[k].seed = seed;
@@ -206,6 +213,7 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
 #pragma unroll
             for (int p = 0; p < P; ++p) best[k].q[p] = (int)q[p];
           }
+          if (zero) break;
         }
       }
     }

@@ -4,27 +4,39 @@
 // Where the batch makes the product a real contraction (several rows of X
 // share every rebuilt weight), the reconstructed tiles feed tcgen05.mma
 // (paperhub.cn review thread: the weights are rebuilt from s and t and then
-// used to compute the activations).  One call is two launches:
+// used to compute the activations).  The MMAs are kind::f16 (K = 16) in the
+// activations' own type, with W split exactly into pieces of that type:
 //
-//   1. stage_x_kernel writes X (fp16 or bf16, M x cols) into the workspace as
-//      fp32 -- exact in tf32 for either input type -- already in the
-//      tensor-core operand layout, one contiguous slab per K chunk (NB x KC,
-//      NB = M rounded up to 16, zero-padded), so the GEMM copies a chunk of X
-//      into shared memory with a single bulk copy.
+//   * bf16 X: W = p1 + p2 + p3, three bf16 pieces (8 significant bits each;
+//     a rebuilt weight has at most 20);
+//   * fp16 X: 2^6 W = p1 + p2, two fp16 pieces (11 significant bits each; the
+//     2^6 keeps the smallest weight quantum, 2^-30, at or above fp16's 2^-24)
+//     and Y is scaled back by 2^-6.
+//
+// Every product of a piece and an activation is exact in the fp32 accumulator.
+// One call is two launches:
+//
+//   1. stage_x_kernel copies X (M x cols) into the workspace in the
+//      tensor-core operand layout, one contiguous slab per K chunk (NB x KC
+//      16-bit elements, NB = M rounded up to 16, zero-padded), so the GEMM
+//      copies a chunk of X into shared memory with a single bulk copy.
 //   2. gemm_tc_kernel, one CTA per SM.  The work is the list of
 //      (128-row tile, K chunk) units in tile-major order, cut into equal
 //      contiguous ranges, one per CTA ("stream-K"), so every SM gets the same
 //      number of units whatever the shape.  Inside a CTA:
 //        * 16 producer warps rebuild the unit's 128 x KC weights exactly in
-//          fp32 (seedlm_device.cuh), split each into tf32 pieces hi + lo (both
-//          exact: a weight has at most 21 significant bits, tf32 keeps 11)
-//          and store them straight into tensor memory with tcgen05.st -- A
-//          operand stages, 128 lanes = rows, one column per K element.  Warp w
-//          owns TMEM lanes 32(w%4).. and a quarter (w/4) of the chunk's blocks.
-//        * one warp issues the MMAs (kind::tf32, M = 128, N = NB, A from TMEM,
-//          B = X chunk from shared memory): hi and lo pieces into the same
-//          fp32 accumulator in TMEM.  It also keeps the X slabs coming, a few
-//          chunks ahead, with bulk copies.
+//          fp32 (seedlm_device.cuh), split them into pieces, pack two K
+//          neighbours per 32-bit word and store them straight into tensor
+//          memory with tcgen05.st -- A operand stages, 128 lanes = rows.  Warp
+//          w owns TMEM lanes 32(w%4).. and a quarter (w/4) of the chunk's
+//          blocks.
+//        * one thread issues the MMAs (M = 128, N = NB, A from TMEM, B = X
+//          slab from shared memory), all pieces into the same fp32
+//          accumulator in TMEM.  An MMA of this shape costs the tensor core
+//          about 45 cycles whatever N (<= 64) and K (8 for tf32, 16 here), so
+//          K = 16 halves the MMA count of a tf32 hi/lo split for fp16 X.
+//        * one thread keeps the X slabs coming, a few chunks ahead, with bulk
+//          copies.
 //        * stages are handed over with mbarriers only (A stage full: all 16
 //          producer warps arrived; A stage / X slab free: tcgen05.commit of the
 //          MMAs that read it), so no warp waits for the whole CTA.
@@ -36,6 +48,7 @@
 //          call gives the same bits -- writes Y and resets the counter.
 //   Every mbarrier wait is bounded; a wait that gives up raises the library's
 //   device error flag, and TMEM is always released.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -58,24 +71,27 @@ constexpr int kThreads = (kProdWarps + 2) * 32;
 constexpr int kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
-// Per format: K columns per unit (8 blocks), blocks per producer thread, A
-// stages in TMEM, X slabs in shared memory, record sets a thread loads ahead.
-template <int C>
+// Per format and piece count (PC = 3: bf16 pieces, PC = 2: fp16 pieces):
+// K columns per unit, blocks per producer thread and unit, A stages in TMEM
+// (PC x KC/2 columns each, two 16-bit elements per column), X slabs in
+// shared memory.
+template <int C, int PC>
 struct TcCfg;
-template <>
-struct TcCfg<8> {
-  static constexpr int KC = 64;
-  static constexpr int AS = 3;  // 3 x 128 TMEM columns + 2 accumulators of 64
+template <int PC>
+struct TcCfg<8, PC> {
+  static constexpr int KC = 128;  // 16 blocks
+  static constexpr int BPT = 4;
+  static constexpr int AS = (PC == 3) ? 2 : 3;
   static constexpr int XS = 5;
 };
-template <>
-struct TcCfg<12> {
-  static constexpr int KC = 96;
-  static constexpr int AS = 2;  // 2 x 192 TMEM columns + 2 accumulators of 64
-  static constexpr int XS = 4;
+template <int PC>
+struct TcCfg<12, PC> {
+  static constexpr int KC = 96;  // 8 blocks
+  static constexpr int BPT = 2;
+  static constexpr int AS = (PC == 3) ? 2 : 3;
+  static constexpr int XS = 5;
 };
-constexpr int kBpt = 2;        // blocks per producer thread and unit
-constexpr int kRecAhead = 4;   // units of records a producer thread has in flight
+constexpr int kRecAhead = 2;   // units of records a producer thread has in flight
 
 struct TcGeom {
   int rows, cols, nb, rec_pitch, e_pitch, M;
@@ -84,13 +100,16 @@ struct TcGeom {
   int segs_max;     // most tiles any one CTA touches
 };
 
-template <int C, int NB>
+template <int C, int NB, int PC>
 struct TcSmem {
-  static constexpr int KC = TcCfg<C>::KC;
-  static constexpr int AS = TcCfg<C>::AS;
-  static constexpr int XS = TcCfg<C>::XS;
-  static constexpr int SBO = KC * 32;  // bytes between 8-row groups of X (KC/4 core matrices)
-  static constexpr int XB = NB * KC * 4;  // one X slab
+  static constexpr int KC = TcCfg<C, PC>::KC;
+  static constexpr int AS = TcCfg<C, PC>::AS;
+  static constexpr int XS = TcCfg<C, PC>::XS;
+  static constexpr int BPT = TcCfg<C, PC>::BPT;
+  static constexpr int SBO = KC * 16;  // bytes between 8-row groups of X (KC/8 core matrices)
+  static constexpr int XB = NB * KC * 2;  // one X slab (16-bit elements)
+  static constexpr int PIECE_COLS = KC / 2;      // TMEM columns of one piece of a stage
+  static constexpr int STAGE_COLS = PC * PIECE_COLS;
   static constexpr int TABLE_OFF = XS * XB;
   static constexpr int TABLE_BYTES = (C == 8) ? 512 * 4 : 512 * 8;
   static constexpr int BAR_OFF = TABLE_OFF + TABLE_BYTES;
@@ -98,41 +117,44 @@ struct TcSmem {
   static constexpr int NBAR = 2 * XS + 2 * AS + 2;
   static constexpr int SLOT_OFF = BAR_OFF + 8 * NBAR;  // TMEM base, last-CTA flag, give-up flag
   static constexpr int TOTAL = SLOT_OFF + 16;
-  static constexpr int D_COL = AS * 2 * KC;  // first accumulator column
+  static constexpr int D_COL = AS * STAGE_COLS;  // first accumulator column
   static_assert(D_COL + 2 * 64 <= kTmemCols, "TMEM budget");
-  static_assert(KC == 4 * kBpt * C, "four producer quarters of kBpt blocks per unit");
+  static_assert(KC == 4 * BPT * C, "four producer quarters of BPT blocks per unit");
+  static_assert(KC % 16 == 0, "whole K = 16 MMA steps");
 };
 
-// Float offset of X element (n, k) inside a slab (K-major core matrices:
-// 8 rows x 16 bytes, adjacent along K at 128 B, 8-row groups at SBO).
+// Byte offset of X element (n, k) inside a slab (K-major core matrices:
+// 8 rows x 16 bytes = 8 elements, adjacent along K at 128 B, 8-row groups at
+// SBO = KC * 16 bytes).
 template <int KC>
-__host__ __device__ constexpr int slab_index(int n, int k) {
-  return ((n >> 3) * (KC * 32) + (k >> 2) * 128 + (n & 7) * 16) / 4 + (k & 3);
+__host__ __device__ constexpr int slab_byte(int n, int k) {
+  return (n >> 3) * (KC * 16) + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
 }
 
-template <int C, int NB>
+template <int KC, int NB>
 __global__ void __launch_bounds__(256)
-stage_x_kernel(const uint16_t* __restrict__ X, int is_bf16, int M, int cols, int nchunks,
-               float* __restrict__ Xs) {
-  constexpr int KC = TcCfg<C>::KC;
-  constexpr int PER_CHUNK = NB * (KC / 4);  // float4 groups per slab
+stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks,
+               unsigned char* __restrict__ Xs) {
   // The GEMM may start its prologue at once; it reads Xs only after
   // griddepcontrol.wait, i.e. after this grid has finished.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  constexpr int PER_CHUNK = NB * (KC / 8);  // 16-byte groups per slab
   const long long total = (long long)nchunks * PER_CHUNK;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int chunk = (int)(i / PER_CHUNK);
     const int rem = (int)(i - (long long)chunk * PER_CHUNK);
-    const int n = rem / (KC / 4), k4 = rem - n * (KC / 4);  // k fastest: coalesced reads
-    const int col = chunk * KC + 4 * k4;
-    float v[4];
+    const int n = rem / (KC / 8), k8 = rem - n * (KC / 8);  // k fastest: coalesced reads
+    const int col = chunk * KC + 8 * k8;
+    uint32_t v[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      v[u] = (n < M && col + u < cols) ? act_to_float(X[(size_t)n * cols + col + u], is_bf16)
-                                       : 0.f;
-    *reinterpret_cast<float4*>(Xs + (size_t)chunk * (NB * KC) + slab_index<KC>(n, 4 * k4)) =
-        make_float4(v[0], v[1], v[2], v[3]);
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t a = (n < M && col + 2 * u < cols) ? X[(size_t)n * cols + col + 2 * u] : 0u;
+      const uint32_t b = (n < M && col + 2 * u + 1 < cols) ? X[(size_t)n * cols + col + 2 * u + 1] : 0u;
+      v[u] = a | (b << 16);
+    }
+    *reinterpret_cast<uint4*>(Xs + (size_t)chunk * (NB * KC * 2) + slab_byte<KC>(n, 8 * k8)) =
+        make_uint4(v[0], v[1], v[2], v[3]);
   }
 }
 
@@ -144,17 +166,35 @@ __device__ __forceinline__ int unit_owner(long long u, long long units, int ctas
   return (int)(((u + 1) * ctas + units - 1) / units) - 1;
 }
 
-// Exact tf32 pieces of two rebuilt weights given as magic-biased floats b
-// (weight = b + nm): hi keeps the top 11 significant bits, lo = w - hi.
-__device__ __forceinline__ void split_pair(float b0, float b1, float nm, uint32_t& h0,
-                                           uint32_t& h1, uint32_t& l0, uint32_t& l1) {
-  const float2 w = __fadd2_rn(make_float2(b0, b1), make_float2(nm, nm));  // exact
-  h0 = __float_as_uint(w.x) & 0xFFFFE000u;
-  h1 = __float_as_uint(w.y) & 0xFFFFE000u;
-  const float2 l = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)),
-                              make_float2(-1.f, -1.f), w);  // exact
-  l0 = __float_as_uint(l.x);
-  l1 = __float_as_uint(l.y);
+// Pieces of two rebuilt weights (K neighbours) given as magic-biased floats
+// b (weight = b + nm), packed two per 32-bit word, the lower K index in the
+// low half.  All splits are exact.
+template <int PC>
+__device__ __forceinline__ void split_pair(float b0, float b1, float nm, uint32_t (&out)[PC]) {
+  if constexpr (PC == 3) {
+    // bf16: each piece keeps the top 8 significant bits of what is left.
+    const float2 w = __fadd2_rn(make_float2(b0, b1), make_float2(nm, nm));
+    const uint32_t h0 = __float_as_uint(w.x) & 0xFFFF0000u, h1 = __float_as_uint(w.y) & 0xFFFF0000u;
+    const float2 r = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)),
+                                make_float2(-1.f, -1.f), w);
+    const uint32_t m0 = __float_as_uint(r.x) & 0xFFFF0000u, m1 = __float_as_uint(r.y) & 0xFFFF0000u;
+    const float2 l = __ffma2_rn(make_float2(__uint_as_float(m0), __uint_as_float(m1)),
+                                make_float2(-1.f, -1.f), r);
+    out[0] = prmt<0x7632u>(h0, h1);
+    out[1] = prmt<0x7632u>(m0, m1);
+    out[2] = prmt<0x7632u>(__float_as_uint(l.x), __float_as_uint(l.y));
+  } else {
+    // fp16 of 2^6 w: the top 11 significant bits, then the rest.
+    const float2 w = __ffma2_rn(make_float2(b0, b1), make_float2(64.f, 64.f),
+                                make_float2(64.f * nm, 64.f * nm));
+    const uint32_t h0 = __float_as_uint(w.x) & 0xFFFFE000u, h1 = __float_as_uint(w.y) & 0xFFFFE000u;
+    const float2 l = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)),
+                                make_float2(-1.f, -1.f), w);
+    const __half2 ph = __floats2half2_rn(__uint_as_float(h0), __uint_as_float(h1));
+    const __half2 pl = __floats2half2_rn(l.x, l.y);
+    out[0] = *reinterpret_cast<const uint32_t*>(&ph);
+    out[1] = *reinterpret_cast<const uint32_t*>(&pl);
+  }
 }
 
 // (tile, chunk) of consecutive units, advanced without dividing: a 64-bit
@@ -171,17 +211,18 @@ struct UnitCursor {
 
 template <int C>
 struct RecUnit {
-  uint2 r;     // the thread's two records of this unit
-  uint32_t e;  // C = 12: their exponent byte
+  uint32_t r[C == 8 ? 4 : 2];  // the thread's records of this unit
+  uint32_t e;                  // C = 12: their exponent byte
 };
 
-template <int C, int NB>
+template <int C, int NB, int PC>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
-               const float* __restrict__ Xs, float* __restrict__ Y, float* __restrict__ partial,
-               unsigned int* __restrict__ counters, TcGeom g) {
-  using L = TcSmem<C, NB>;
-  constexpr int KC = L::KC, AS = L::AS, XS = L::XS;
+               const unsigned char* __restrict__ Xs, float* __restrict__ Y,
+               float* __restrict__ partial, unsigned int* __restrict__ counters, TcGeom g) {
+  using L = TcSmem<C, NB, PC>;
+  constexpr int KC = L::KC, AS = L::AS, XS = L::XS, BPT = L::BPT;
+  constexpr float kYScale = (PC == 2) ? 1.0f / 64.0f : 1.0f;  // undo the fp16 pieces' 2^6
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ctas = gridDim.x;
@@ -243,7 +284,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         if (j >= XS)  // the slab's previous unit (j - XS) has finished its MMAs
           ok = tc::mbar_wait_or_abort(xfree(s), ((j / XS) - 1) & 1, kWaitLimit, abort_flag) && ok;
         tc::mbar_arrive_expect_tx(xfull(s), L::XB);
-        tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)xc.chunk * (NB * KC), L::XB, xfull(s));
+        tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)xc.chunk * L::XB, L::XB, xfull(s));
       }
       // Every copy this thread issued has landed before the CTA may exit
       // (bounded, and not cut short by the give-up flag).
@@ -256,7 +297,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_tf32(NB);
+      const uint32_t idesc = tc::idesc_f16(NB, PC == 3 ? 1 : 0);
       const uint64_t bdesc0 = tc::smem_desc(tc::smem_u32(smem), 128, L::SBO);  // slab 0, K slice 0
       int seg = 0;
       UnitCursor mc = c0;
@@ -275,15 +316,16 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         // This thread's issue rate bounds the kernel (an MMA of this shape
         // takes the tensor core about 45 cycles), so everything but the MMAs
         // is computed up front.
-        const uint32_t a_hi = tmem + as * 2 * KC, a_lo = a_hi + KC;
+        const uint32_t a0 = tmem + as * L::STAGE_COLS;
         const uint32_t d = tmem + L::D_COL + 64 * db;
         const uint64_t bd = bdesc0 + (uint64_t)((xs * L::XB) >> 4);
         const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
-        for (int kk = 0; kk < KC / 8; ++kk) {
-          tc::mma_tf32_ts(d, a_hi + 8 * kk, bd + 16 * kk, idesc, kk == 0 ? acc0 : 1u);
-          tc::mma_tf32_ts(d, a_lo + 8 * kk, bd + 16 * kk, idesc, 1u);
-        }
+        for (int kk = 0; kk < KC / 16; ++kk)
+#pragma unroll
+          for (int pc = 0; pc < PC; ++pc)
+            tc::mma_f16_ts(d, a0 + pc * L::PIECE_COLS + 8 * kk, bd + 16 * kk, idesc,
+                           (kk == 0 && pc == 0) ? acc0 : 1u);
         tc::mma_commit(afree(as));  // A stage free; at a segment's end the accumulator is final
         tc::mma_commit(xfree(xs));  // X slab free
       }
@@ -301,27 +343,34 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     const int prow = 32 * lq + lane;  // TMEM lane = row in the tile
     auto load_rec = [&](const UnitCursor& u, RecUnit<C>& p) {
       const int gr = u.tile * kTileM + prow;
-      const int b0 = u.chunk * (KC / C) + kq * kBpt;  // even
+      const int b0 = u.chunk * (KC / C) + kq * BPT;  // a multiple of BPT
       const bool ok_ = gr < g.rows && b0 < g.nb;
-      p.r = ok_ ? ld_stream_u2(rec + (size_t)gr * g.rec_pitch + b0) : make_uint2(0u, 0u);
-      p.e = 0;
-      if constexpr (C == 12)
+      const uint32_t* src = rec + (size_t)gr * g.rec_pitch + b0;
+      if constexpr (C == 8) {
+        const uint4 v = ok_ ? ld_stream_u4(src) : make_uint4(0u, 0u, 0u, 0u);
+        p.r[0] = v.x; p.r[1] = v.y; p.r[2] = v.z; p.r[3] = v.w;
+        p.e = 0;
+      } else {
+        const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
+        p.r[0] = v.x; p.r[1] = v.y;
         p.e = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
+      }
     };
 
     auto produce = [&](int i, const RecUnit<C>& cur) {
       const int as = i % AS;
       if (i >= AS) ok = tc::mbar_wait_or_abort(afree(as), ((i / AS) - 1) & 1, kWaitLimit, abort_flag) && ok;
       tc::fence_after_sync();
-      const uint32_t col0 = tmem + ((uint32_t)(32 * lq) << 16) + as * 2 * KC + kq * kBpt * C;
-      uint32_t hi[kBpt * C], lo[kBpt * C];
+      // Piece pc of this thread's BPT * C weights: BPT * C / 2 packed columns.
+      constexpr int NPACK = BPT * C / 2;
+      const uint32_t col0 = tmem + ((uint32_t)(32 * lq) << 16) + as * L::STAGE_COLS + kq * NPACK;
+      uint32_t pk[PC][NPACK];
 #pragma unroll
-      for (int j = 0; j < kBpt; ++j) {
-        const uint32_t r = j ? cur.r.y : cur.r.x;
+      for (int j = 0; j < BPT; ++j) {
         float b[C];
         float nm;
         if constexpr (C == 8) {
-          const BlockC8 blk = decode_c8(r, t32, t32 + 256);
+          const BlockC8 blk = decode_c8(cur.r[j], t32, t32 + 256);
           nm = __uint_as_float(blk.negm);
           b[0] = __int_as_float(weight_bits_c8<0>(blk));
           b[1] = __int_as_float(weight_bits_c8<1>(blk));
@@ -332,7 +381,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           b[6] = __int_as_float(weight_bits_c8<6>(blk));
           b[7] = __int_as_float(weight_bits_c8<7>(blk));
         } else {
-          const BlockC12 blk = decode_c12(r, (j ? cur.e >> 4 : cur.e) & 15u, t64, t64 + 256);
+          const BlockC12 blk = decode_c12(cur.r[j], (j ? cur.e >> 4 : cur.e) & 15u, t64, t64 + 256);
           nm = __uint_as_float(blk.negm);
           b[0] = __int_as_float(weight_bits_c12<0>(blk));
           b[1] = __int_as_float(weight_bits_c12<1>(blk));
@@ -348,18 +397,20 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           b[11] = __int_as_float(weight_bits_c12<11>(blk));
         }
 #pragma unroll
-        for (int c = 0; c < C; c += 2)
-          split_pair(b[c], b[c + 1], nm, hi[j * C + c], hi[j * C + c + 1], lo[j * C + c],
-                     lo[j * C + c + 1]);
-      }
-      if constexpr (C == 8) {
-        tc::tmem_st16(col0, hi);
-        tc::tmem_st16(col0 + KC, lo);
-      } else {
+        for (int c = 0; c < C; c += 2) {
+          uint32_t o[PC];
+          split_pair<PC>(b[c], b[c + 1], nm, o);
 #pragma unroll
-        for (int q = 0; q < 3; ++q) {
-          tc::tmem_st8(col0 + 8 * q, hi + 8 * q);
-          tc::tmem_st8(col0 + KC + 8 * q, lo + 8 * q);
+          for (int pc = 0; pc < PC; ++pc) pk[pc][(j * C + c) / 2] = o[pc];
+        }
+      }
+#pragma unroll
+      for (int pc = 0; pc < PC; ++pc) {
+        if constexpr (C == 8) {
+          tc::tmem_st16(col0 + pc * L::PIECE_COLS, pk[pc]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < NPACK / 4; ++q) tc::tmem_st4(col0 + pc * L::PIECE_COLS + 4 * q, pk[pc] + 4 * q);
         }
       }
       tc::tmem_wait_st();
@@ -388,11 +439,11 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           if (gr < g.rows) {
 #pragma unroll
             for (int q = 0; q < 16; ++q)
-              if (16 * n16 + q < g.M) Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q];
+              if (16 * n16 + q < g.M) Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q] * kYScale;
           }
         } else {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) mine[(16 * n16 + q) * kTileM + row] = v[q];
+          for (int q = 0; q < 16; ++q) mine[(16 * n16 + q) * kTileM + row] = v[q] * kYScale;
         }
       }
       tc::fence_before_sync();
@@ -461,12 +512,8 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   }
 }
 
-template <int C>
-constexpr int tc_kc() {
-  return TcCfg<C>::KC;
-}
-
-int kc_of(int C) { return C == 8 ? tc_kc<8>() : tc_kc<12>(); }
+// K columns per unit (the same for both piece types).
+int kc_of(int C) { return C == 8 ? TcCfg<8, 3>::KC : TcCfg<12, 3>::KC; }
 
 TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev, int* ctas) {
   TcGeom g;
@@ -504,28 +551,28 @@ TcWorkspace tc_workspace(const TcGeom& g, int C, int ctas) {
   const int NB = (g.M + 15) / 16 * 16;
   TcWorkspace w;
   w.cnt_bytes = round256((int64_t)g.tiles * 4);
-  w.xs_bytes = round256((int64_t)g.nchunks * NB * kc_of(C) * 4);
+  w.xs_bytes = round256((int64_t)g.nchunks * NB * kc_of(C) * 2);
   w.part_bytes = round256((int64_t)ctas * g.segs_max * NB * kTileM * 4);
   return w;
 }
 
-template <int C, int NB>
+template <int C, int NB, int PC>
 int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* eplane,
-              const uint16_t* X, int is_bf16, float* Y, unsigned char* ws, const TcWorkspace& w,
+              const uint16_t* X, float* Y, unsigned char* ws, const TcWorkspace& w,
               cudaStream_t stream, const DeviceInfo& dev) {
-  using L = TcSmem<C, NB>;
+  using L = TcSmem<C, NB, PC>;
   if ((size_t)L::TOTAL > (size_t)dev.max_smem_optin) return SEEDLM_EUNSUPPORTED;
-  int rc = allow_max_smem((const void*)gemm_tc_kernel<C, NB>, dev);
+  int rc = allow_max_smem((const void*)gemm_tc_kernel<C, NB, PC>, dev);
   if (rc) return rc;
   unsigned int* counters = reinterpret_cast<unsigned int*>(ws);
-  float* xs = reinterpret_cast<float*>(ws + w.cnt_bytes);
+  unsigned char* xs = ws + w.cnt_bytes;
   float* partial = reinterpret_cast<float*>(ws + w.cnt_bytes + w.xs_bytes);
 
-  const long long groups = (long long)g.nchunks * NB * (TcCfg<C>::KC / 4);
+  const long long groups = (long long)g.nchunks * NB * (L::KC / 8);
   long long want = (groups + 255) / 256;
   const long long cap = 8ll * dev.num_sms;
   const int sgrid = (int)(want < cap ? (want < 1 ? 1 : want) : cap);
-  stage_x_kernel<C, NB><<<sgrid, 256, 0, stream>>>(X, is_bf16, g.M, g.cols, g.nchunks, xs);
+  stage_x_kernel<L::KC, NB><<<sgrid, 256, 0, stream>>>(X, g.M, g.cols, g.nchunks, xs);
   count_launch();
   if ((rc = record_cuda_error(cudaGetLastError()))) return rc;
 
@@ -539,31 +586,35 @@ int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* epl
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<C, NB>, rec, eplane,
-                                       (const float*)xs, Y, partial, counters, g);
+  cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<C, NB, PC>, rec, eplane,
+                                       (const unsigned char*)xs, Y, partial, counters, g);
   if (err != cudaSuccess) return record_cuda_error(err);
   count_launch();
   return record_cuda_error(cudaGetLastError());
 }
 
+template <int C, int PC>
+int dispatch_nb(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* eplane,
+                const uint16_t* X, float* Y, unsigned char* ws, const TcWorkspace& w,
+                cudaStream_t st, const DeviceInfo& dev) {
+  switch ((g.M + 15) / 16 * 16) {
+    case 16: return launch_tc<C, 16, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+    case 32: return launch_tc<C, 32, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+    case 48: return launch_tc<C, 48, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+    default: return launch_tc<C, 64, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+  }
+}
+
+// bf16 activations take three bf16 pieces of W, fp16 activations two fp16
+// pieces (of 2^6 W): A and B of one MMA always have the same type.
 int dispatch_tc(const seedlm_format& f, const TcGeom& g, int ctas, const uint32_t* rec,
                 const uint8_t* eplane, const uint16_t* X, int is_bf16, float* Y,
                 unsigned char* ws, const TcWorkspace& w, cudaStream_t st, const DeviceInfo& dev) {
-  const int NB = (g.M + 15) / 16 * 16;
-  if (f.C == 8) {
-    switch (NB) {
-      case 16: return launch_tc<8, 16>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-      case 32: return launch_tc<8, 32>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-      case 48: return launch_tc<8, 48>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-      default: return launch_tc<8, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-    }
-  }
-  switch (NB) {
-    case 16: return launch_tc<12, 16>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-    case 32: return launch_tc<12, 32>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-    case 48: return launch_tc<12, 48>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-    default: return launch_tc<12, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-  }
+  if (f.C == 8)
+    return is_bf16 ? dispatch_nb<8, 3>(g, ctas, rec, eplane, X, Y, ws, w, st, dev)
+                   : dispatch_nb<8, 2>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+  return is_bf16 ? dispatch_nb<12, 3>(g, ctas, rec, eplane, X, Y, ws, w, st, dev)
+                 : dispatch_nb<12, 2>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
 }
 
 }  // namespace

@@ -62,6 +62,29 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "r"(0u), "r"(0u));
 }
 
+// Instruction descriptor for kind::f16: D fp32, A and B both fp16 (bf16 = 0)
+// or both bf16 (bf16 = 1), K-major, M = 128, N = n (multiple of 16, <= 256).
+__host__ __device__ constexpr uint32_t idesc_f16(int n, int bf16) {
+  return (1u << 4)                        // D format: f32
+         | ((uint32_t)bf16 << 7)          // A format: f16 / bf16
+         | ((uint32_t)bf16 << 10)         // B format: f16 / bf16
+         | ((uint32_t)(n >> 3) << 17)     // N >> 3
+         | ((uint32_t)(128 >> 4) << 24);  // M >> 4
+}
+
+// kind::f16 MMA, K = 16, A from tensor memory: 128 lanes (rows) x 8 columns,
+// each column two 16-bit elements (lower K index in the low half).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
+        "r"(0u), "r"(0u));
+}
+
 // Arrive once on `mbar` when all tcgen05.mma issued so far by this thread
 // have completed.
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
@@ -132,6 +155,12 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
       : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
         "r"(r[6]), "r"(r[7])
       : "memory");
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};"
+               :
+               : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
