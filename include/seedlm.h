@@ -164,6 +164,14 @@ SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt, const uint32
 SEEDLM_API int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_t* rec,
                              uint8_t* eplane, double* err, seedlm_stream stream);
 
+/* Failure-path self test (no counterpart in the pages): launches one small
+ * kernel whose bounded mbarrier wait -- the wait the tensor-core GEMM uses,
+ * with its TMEM allocation -- waits for an arrival that never comes and gives
+ * up after limit_ns nanoseconds (1e3 .. 1e8, else SEEDLM_EINVAL).  Afterwards
+ * seedlm_device_error reports 1 and the context stays usable: this is how a
+ * stuck hand-over surfaces to the caller, without a trap or a hang. */
+SEEDLM_API int seedlm_selftest_wait_timeout(int64_t limit_ns, seedlm_stream stream);
+
 /* Reads and clears the device-side error flag of the current device: 1 if a
  * kernel gave up waiting on one of its own barriers (the outputs of that call
  * are then undefined), else 0.  HOST function; synchronous. */

@@ -181,6 +181,14 @@ int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_
   return launch_encode(*fmt, W, ldw, rec, eplane, err, (cudaStream_t)stream);
 }
 
+int seedlm_selftest_wait_timeout(int64_t limit_ns, seedlm_stream stream) {
+  if (limit_ns < 1000 || limit_ns > 100000000) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  return launch_wait_timeout((uint64_t)limit_ns, (cudaStream_t)stream);
+}
+
 int seedlm_device_error(int* flag) {
   if (!flag) return SEEDLM_EINVAL;
   DeviceInfo dev;

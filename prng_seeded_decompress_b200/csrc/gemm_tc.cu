@@ -637,6 +637,41 @@ int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* e
                      static_cast<unsigned char*>(workspace), w, stream, dev);
 }
 
+namespace {
+
+// A bounded mbarrier wait that nothing ends: the same wait, give-up flag and
+// TMEM handling as gemm_tc_kernel, run on purpose into its time limit.
+__global__ void __launch_bounds__(64, 1) wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t slot[3];
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(tc::smem_u32(&bar), 1);  // one arrival expected, none will come
+    tc::fence_mbar_init();
+    slot[2] = 0u;
+  }
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(slot), 32);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const bool ok = tc::mbar_wait_or_abort(tc::smem_u32(&bar), 0, limit_ns, slot + 2);
+  if (!ok && threadIdx.x == 0) atomicOr(&g_tc_error, 1u);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(slot[0], 32);
+  }
+}
+
+}  // namespace
+
+int launch_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+  wait_timeout_kernel<<<1, 64, 0, stream>>>(limit_ns);
+  count_launch();
+  return record_cuda_error(cudaGetLastError());
+}
+
 int read_and_clear_tc_error(unsigned int* out) {
   unsigned int v = 0, zero = 0;
   cudaError_t err = cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(v));

@@ -22,7 +22,7 @@ EXPORTS = (
     "seedlm_gemm_smallM_workspace_bytes", "seedlm_gemm_smallM_noalloc", "seedlm_device_error",
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
-    "seedlm_encode",
+    "seedlm_encode", "seedlm_selftest_wait_timeout",
 )
 
 
@@ -61,6 +61,7 @@ def _load():
                                                       ctypes.c_int, vp, vp]),
         "seedlm_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
         "seedlm_encode": (ctypes.c_int, [fmtp, vp, i64, vp, vp, vp, vp]),
+        "seedlm_selftest_wait_timeout": (ctypes.c_int, [i64, vp]),
         "seedlm_dense_gemv_f16": (ctypes.c_int, [i32, i32, vp, i64, vp, vp, vp]),
         "seedlm_row_bytes_ideal": (i64, [fmtp]),
         "seedlm_row_bytes_stored": (i64, [fmtp]),
@@ -195,8 +196,9 @@ def gemm_smallM(fmt, rec, eplane, X, Y, workspace=None, stream=None):
 
 
 def gemm_smallM_noalloc(fmt, rec, eplane, X, Y, stream=None):
-    """Y = X W^T without a workspace: the split-K scratch is an array inside
-    the library (16 MiB of partials); calls sharing it must not overlap."""
+    """Y = X W^T without a workspace: the workspace (counters, X slabs, partial
+    tiles; 16 MiB + 64 KiB) is an array inside the library; calls sharing it
+    must not overlap."""
     f = _fmt(fmt)
     _check("seedlm_gemm_smallM_noalloc", lib.seedlm_gemm_smallM_noalloc(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), int(X.shape[0]),
@@ -209,6 +211,13 @@ def device_error() -> int:
     flag = ctypes.c_int(0)
     _check("seedlm_device_error", lib.seedlm_device_error(ctypes.byref(flag)))
     return int(flag.value)
+
+
+def selftest_wait_timeout(limit_ns: int = 2_000_000, stream=None):
+    """Launch the failure-path self test: a bounded wait that gives up after
+    limit_ns, raising the flag device_error() reads."""
+    _check("seedlm_selftest_wait_timeout",
+           lib.seedlm_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def dense_gemv_f16(W, x, y, stream=None):

@@ -101,6 +101,8 @@ def test_bad_pointers_are_rejected_before_cuda(sl):
     assert L.seedlm_gemm_smallM(ctypes.byref(f), 0x1000, None, 0x2000, 0, 4, 0x3000,
                                 None, -1, None) == -1
     assert L.seedlm_device_error(None) == -1
+    for limit in (0, 999, 100000001):
+        assert L.seedlm_selftest_wait_timeout(limit, None) == -1
     assert L.seedlm_decompress(ctypes.byref(f), 0x1000, None, 0x2000, 63, None) == -1
     assert L.seedlm_dense_gemv_f16(4, 64, 0x1008, 64, 0x2000, 0x3000, None) == -1
     assert L.seedlm_dense_gemv_f16(4, 64, 0x1000, 60, 0x2000, 0x3000, None) == -1

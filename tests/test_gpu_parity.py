@@ -293,3 +293,40 @@ def test_misaligned_record_pointer_is_rejected(sl):
     y = torch.zeros(8, device="cuda")
     with pytest.raises(sl.SeedLMError):
         sl.gemv(L["fmt"], rec.data_ptr() + 4, None, x, y)
+
+
+# ------------------------------------------------------------ CUDA graphs
+
+def test_graph_replay_matches_eager_calls(sl):
+    # GEMV and the two-launch GEMM (programmatic dependent launch between the
+    # X staging and the GEMM) captured once and replayed: bit-identical to
+    # eager calls, every replay.
+    L = inputs.make_layer(512, 2048, *C8, seed=31)
+    rec, _ = planes(L)
+    xb, _ = inputs.make_activations((2048,), "f16", 32)
+    Xb, _ = inputs.make_activations((16, 2048), "bf16", 33)
+    x = act_tensor(xb, "f16")
+    X = act_tensor(Xb, "bf16")
+    ws = sl.gemm_workspace(L["fmt"], 16)
+    y = torch.empty(512, device="cuda")
+    Y = torch.empty((16, 512), device="cuda")
+    sl.gemv(L["fmt"], rec, None, x, y)
+    sl.gemm_smallM(L["fmt"], rec, None, X, Y, workspace=ws)
+    torch.cuda.synchronize()
+    y0, Y0 = y.clone(), Y.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            sl.gemv(L["fmt"], rec, None, x, y, stream=s)
+            sl.gemm_smallM(L["fmt"], rec, None, X, Y, workspace=ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        y.fill_(float("nan"))
+        Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y0) and torch.equal(Y, Y0)
+    assert sl.device_error() == 0
+    del g
