@@ -296,7 +296,9 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issue
-    if (lane == 0) {
+    // The whole warp runs this loop with warp-uniform values (so they can
+    // stay in uniform registers); one elected lane issues each MMA/commit.
+    {
       const uint32_t idesc = tc::idesc_f16(NB, PC == 3 ? 1 : 0);
       const uint64_t bdesc0 = tc::smem_desc(tc::smem_u32(smem), 128, L::SBO);  // slab 0, K slice 0
       int seg = 0;
@@ -312,10 +314,11 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           ok = tc::mbar_wait_or_abort(xfull(xs), (i / XS) & 1, kWaitLimit, abort_flag) && ok;
           ok = tc::mbar_wait_or_abort(afull(as), (i / AS) & 1, kWaitLimit, abort_flag) && ok;
         }
+        __syncwarp();  // reconverge before the elected issue
         tc::fence_after_sync();
-        // This thread's issue rate bounds the kernel (an MMA of this shape
-        // takes the tensor core about 45 cycles), so everything but the MMAs
-        // is computed up front.
+        // The issue rate bounds the kernel (an MMA of this shape takes the
+        // tensor core about 45 cycles), so everything but the MMAs is
+        // computed up front.
         const uint32_t a0 = tmem + as * L::STAGE_COLS;
         const uint32_t d = tmem + L::D_COL + 64 * db;
         const uint64_t bd = bdesc0 + (uint64_t)((xs * L::XB) >> 4);
@@ -324,10 +327,10 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         for (int kk = 0; kk < KC / 16; ++kk)
 #pragma unroll
           for (int pc = 0; pc < PC; ++pc)
-            tc::mma_f16_ts(d, a0 + pc * L::PIECE_COLS + 8 * kk, bd + 16 * kk, idesc,
-                           (kk == 0 && pc == 0) ? acc0 : 1u);
-        tc::mma_commit(afree(as));  // A stage free; at a segment's end the accumulator is final
-        tc::mma_commit(xfree(xs));  // X slab free
+            tc::mma_f16_ts_warp(d, a0 + pc * L::PIECE_COLS + 8 * kk, bd + 16 * kk, idesc,
+                                (kk == 0 && pc == 0) ? acc0 : 1u);
+        tc::mma_commit_warp(afree(as));  // A stage free; at a segment's end the accumulator is final
+        tc::mma_commit_warp(xfree(xs));  // X slab free
       }
       // The CTA releases TMEM only after its last MMAs have completed
       // (bounded, not cut short by the give-up flag).

@@ -85,6 +85,30 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         "r"(0u), "r"(0u));
 }
 
+// Whole-warp forms: every lane of a converged warp calls them with the same
+// (warp-uniform) operands and one elected lane issues the instruction, so the
+// operands can stay in uniform registers.
+__device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
+        "r"(0u), "r"(0u));
+}
+__device__ __forceinline__ void mma_commit_warp(uint32_t mbar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n"
+      :
+      : "r"(mbar)
+      : "memory");
+}
+
 // Arrive once on `mbar` when all tcgen05.mma issued so far by this thread
 // have completed.
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
