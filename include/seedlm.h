@@ -109,9 +109,11 @@ SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const 
 
 /* Y = X W^T for a small batch: X is M x cols (row-major, type x_dtype), Y is
  * M x rows fp32 (row-major), 1 <= M <= 64.  M = 1 runs the GEMV kernel; for
- * M >= 2 the rebuilt weight tiles feed the tcgen05 tensor cores (tf32 hi/lo
- * pieces, exact products, fp32 accumulation in TMEM) -- two launches: X is
- * first converted into the operand layout, then one CTA per SM runs the GEMM.
+ * M >= 2 the rebuilt weight tiles feed the tcgen05 tensor cores (kind::f16
+ * MMAs in the activations' type: W split exactly into three bf16 pieces for
+ * bf16 X, two fp16 pieces of 2^6 W for fp16 X; exact products, fp32
+ * accumulation in TMEM) -- two launches: X is first copied into the operand
+ * layout, then one CTA per SM runs the GEMM.
  * `workspace` is device memory of at least
  * seedlm_gemm_smallM_workspace_bytes(fmt, M) bytes, 256-byte aligned.  It
  * holds per-tile counters, X in the operand layout and the partial tiles of
