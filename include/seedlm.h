@@ -102,14 +102,17 @@ SEEDLM_API int seedlm_decompress(const seedlm_format* fmt, const uint32_t* rec, 
 /* y = W x (batch 1).  x: cols elements of type x_dtype (SEEDLM_F16 or
  * SEEDLM_BF16); y: rows fp32.  The blocks are rebuilt on the fly and never
  * written out (paperhub.cn thread, authors' replies on inference and on the
- * custom decoding that avoids full-precision weights in memory).  cols up to
- * 56,320 (4-bit) or 40,960 (3-bit): x is held in shared memory as fp32. */
+ * custom decoding that avoids full-precision weights in memory).  x is held
+ * in shared memory as fp32, so cols is limited by it: up to 56,320 (4-bit)
+ * or 42,240 (3-bit) on a B200 (227 KB per block); wider x returns
+ * SEEDLM_EUNSUPPORTED (seedlm_gemm_smallM with M = 1 has no such limit). */
 SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
                 const void* x, int x_dtype, float* y, seedlm_stream stream);
 
 /* Y = X W^T for a small batch: X is M x cols (row-major, type x_dtype), Y is
- * M x rows fp32 (row-major), 1 <= M <= 64.  M = 1 runs the GEMV kernel; for
- * M >= 2 the rebuilt weight tiles feed the tcgen05 tensor cores (kind::f16
+ * M x rows fp32 (row-major), 1 <= M <= 64.  M = 1 runs the GEMV kernel
+ * (unless x is too wide for it); otherwise the rebuilt weight tiles feed the
+ * tcgen05 tensor cores (kind::f16
  * MMAs in the activations' type: W split exactly into three bf16 pieces for
  * bf16 X, two fp16 pieces of 2^6 W for fp16 X; exact products, fp32
  * accumulation in TMEM) -- two launches: X is first copied into the operand
@@ -125,8 +128,8 @@ SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec,
                        int64_t workspace_bytes, seedlm_stream stream);
 
 /* Workspace bytes seedlm_gemm_smallM needs for this format and M on the
- * current device (HOST function; 0 for M = 1 or an empty matrix, negative on
- * error). */
+ * current device (HOST function; 0 for an empty matrix or when M = 1 runs the
+ * GEMV, negative on error). */
 SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M);
 
 /* Same result as seedlm_gemm_smallM, for callers that cannot allocate device

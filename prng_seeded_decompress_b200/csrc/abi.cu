@@ -152,7 +152,8 @@ int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint
     return record_cuda_error(
         cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), (cudaStream_t)stream));
   const uint16_t* Xh = static_cast<const uint16_t*>(X);
-  if (M == 1)
+  // M = 1 runs the GEMV unless x is too wide for its shared memory.
+  if (M == 1 && gemv_smem_bytes(*fmt, dev.max_smem_optin) > 0)
     return launch_gemv(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, Y, (cudaStream_t)stream,
                        dev);
   return launch_gemm_tc(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, M, Y, workspace,
@@ -161,10 +162,11 @@ int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint
 
 int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M) {
   if (check_format(fmt) || M < 1 || M > 64) return SEEDLM_EINVAL;
-  if (M == 1 || fmt->rows == 0 || fmt->cols == 0) return 0;
+  if (fmt->rows == 0 || fmt->cols == 0) return 0;
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
+  if (M == 1 && gemv_smem_bytes(*fmt, dev.max_smem_optin) > 0) return 0;  // the GEMV
   return gemm_tc_workspace_bytes(*fmt, M, dev);
 }
 

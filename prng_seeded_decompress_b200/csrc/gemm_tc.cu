@@ -750,7 +750,8 @@ extern "C" SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt,
     return record_cuda_error(cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), st));
   const uint16_t* Xh = static_cast<const uint16_t*>(X);
   const int is_bf16 = x_dtype == SEEDLM_BF16;
-  if (M == 1) return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
+  if (M == 1 && gemv_smem_bytes(*fmt, dev.max_smem_optin) > 0)
+    return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
 
   int ctas = 1;
   const TcGeom g = make_tc_geom(*fmt, M, dev, &ctas);

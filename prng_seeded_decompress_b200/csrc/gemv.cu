@@ -49,12 +49,14 @@ struct Tune {
   static constexpr int kPrefetch = (C == 8) ? 1 : 2;
 };
 constexpr int kRowsPerTask = 4;
-constexpr int kMaxGroups = 128;  // row groups per partial-sum pass
+constexpr int kMaxGroups = 128;  // row groups per partial-sum pass (fewer if x needs the room)
 
 struct GemvGeom {
   int rows, cols, nb, rec_pitch, e_pitch;
   int n_spans;      // ceil(ceil(nb / 2) / 32): 32 record pairs (one per lane) per span
   int groups;       // ceil(rows / 4)
+  int pass_groups;  // row groups per partial-sum pass (<= kMaxGroups)
+  int x_off;        // byte offset of the x slots in shared memory
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -63,14 +65,15 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Shared-memory map: [jump tables][partial sums][x slots].
+// Shared-memory map: [jump tables][partial sums][x slots].  The partial-sum
+// buffer holds pass_groups row groups; x starts at x_off (both chosen by the
+// launcher so that x fits).
 template <int C>
 struct Smem {
   // C = 8: jump tables (2 KB) + coefficient tables (4 KB); C = 12: jump tables.
   static constexpr int kJumpBytes = (C == 8) ? 2 * 256 * 4 : 2 * 256 * 8;
   static constexpr int kTableBytes = (C == 8) ? kJumpBytes + 2 * 256 * 8 : kJumpBytes;
-  static constexpr int kPartBytes = kMaxGroups * kRowsPerTask * Tune<C>::kWarps * 4;
-  static constexpr int kHead = kTableBytes + kPartBytes;
+  static constexpr int kPartBytesPerGroup = kRowsPerTask * Tune<C>::kWarps * 4;
   static constexpr int kSlotFloats = (C == 8) ? 16 : 32;  // per record pair
 };
 
@@ -101,7 +104,7 @@ __device__ void stage_x_and_tables(unsigned char* smem, const uint16_t* __restri
     }
   }
   // x, zero-padded to n_spans * 32 record pairs.
-  float* xs = reinterpret_cast<float*>(smem + Smem<C>::kHead);
+  float* xs = reinterpret_cast<float*>(smem + g.x_off);
   const int ncols_pad = g.n_spans * 32 * 2 * C;
   for (int j = threadIdx.x; j < ncols_pad; j += blockDim.x) {
     int rp = j / (2 * C);
@@ -206,7 +209,7 @@ __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const floa
 // reduces its 4 row sums with shuffles into shared memory.  After a barrier
 // the partial sums of each row are added in warp order -- the same order on
 // every call -- and written.  Groups are processed in passes of at most
-// kMaxGroups so the partial-sum buffer stays small.
+// pass_groups so the partial-sum buffer stays small.
 template <int C>
 __global__ void __launch_bounds__(Tune<C>::kWarps * 32, 1)
 gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
@@ -215,7 +218,7 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
   const void* t_lo = smem;
   const void* t_hi = smem + Smem<C>::kJumpBytes / 2;
   float* part = reinterpret_cast<float*>(smem + Smem<C>::kTableBytes);
-  const float* xs = reinterpret_cast<const float*>(smem + Smem<C>::kHead);
+  const float* xs = reinterpret_cast<const float*>(smem + g.x_off);
 
   const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,8 +227,8 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
   const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
 
   bool first_pass = true;
-  for (int p0 = g0; p0 < g1; p0 += kMaxGroups) {
-    const int p1 = min(p0 + kMaxGroups, g1);
+  for (int p0 = g0; p0 < g1; p0 += g.pass_groups) {
+    const int p1 = min(p0 + g.pass_groups, g1);
     const int items = (p1 - p0) * g.n_spans;
     const int i0 = (int)((int64_t)warp * items / nw), i1 = (int)((int64_t)(warp + 1) * items / nw);
     // The first record sets are requested before anything else: they do not
@@ -295,7 +298,17 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
   }
 }
 
-GemvGeom make_geom(const seedlm_format& f) {
+// Shared memory of one CTA for a given pass size.
+template <int C>
+size_t smem_for(int n_spans, int pass_groups) {
+  return (size_t)Smem<C>::kTableBytes + (size_t)pass_groups * Smem<C>::kPartBytesPerGroup +
+         (size_t)n_spans * 32 * Smem<C>::kSlotFloats * 4;
+}
+
+// The geometry, with the largest partial-sum pass (<= kMaxGroups, halving)
+// that leaves room for x; pass_groups = 0 if x alone does not fit.
+template <int C>
+GemvGeom make_geom(const seedlm_format& f, int max_smem) {
   GemvGeom g;
   g.rows = f.rows;
   g.cols = f.cols;
@@ -305,24 +318,31 @@ GemvGeom make_geom(const seedlm_format& f) {
   g.n_spans = ((f.nb + 1) / 2 + 31) / 32;
   if (g.n_spans < 1) g.n_spans = 1;
   g.groups = (f.rows + kRowsPerTask - 1) / kRowsPerTask;
+  g.pass_groups = kMaxGroups;
+  while (g.pass_groups > 0 && smem_for<C>(g.n_spans, g.pass_groups) > (size_t)max_smem)
+    g.pass_groups >>= 1;
+  g.x_off = Smem<C>::kTableBytes + g.pass_groups * Smem<C>::kPartBytesPerGroup;
   return g;
 }
 
 }  // namespace
 
-size_t gemv_smem_bytes(const seedlm_format& f) {
-  int n_spans = ((f.nb + 1) / 2 + 31) / 32;
-  if (n_spans < 1) n_spans = 1;
-  if (f.C == 8) return (size_t)Smem<8>::kHead + (size_t)n_spans * 32 * Smem<8>::kSlotFloats * 4;
-  return (size_t)Smem<12>::kHead + (size_t)n_spans * 32 * Smem<12>::kSlotFloats * 4;
+size_t gemv_smem_bytes(const seedlm_format& f, int max_smem) {
+  if (f.C == 8) {
+    const GemvGeom g = make_geom<8>(f, max_smem);
+    return g.pass_groups ? smem_for<8>(g.n_spans, g.pass_groups) : 0;
+  }
+  const GemvGeom g = make_geom<12>(f, max_smem);
+  return g.pass_groups ? smem_for<12>(g.n_spans, g.pass_groups) : 0;
 }
 
 int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                 const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
                 const DeviceInfo& dev) {
-  const GemvGeom g = make_geom(f);
-  const size_t smem = gemv_smem_bytes(f);
-  if (smem > (size_t)dev.max_smem_optin) return SEEDLM_EUNSUPPORTED;
+  const GemvGeom g = (f.C == 8) ? make_geom<8>(f, dev.max_smem_optin)
+                                : make_geom<12>(f, dev.max_smem_optin);
+  if (g.pass_groups == 0) return SEEDLM_EUNSUPPORTED;  // x does not fit in shared memory
+  const size_t smem = gemv_smem_bytes(f, dev.max_smem_optin);
   if (g.groups < 1) return SEEDLM_OK;
   // One CTA per SM (at most one per row group); fewer warps per CTA when
   // each CTA has only a few (group, span) items, so small matrices still

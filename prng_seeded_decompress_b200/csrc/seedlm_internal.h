@@ -27,7 +27,8 @@ void count_launch();
 // per kernel and device, outside any stream capture the caller may start later.
 int allow_max_smem(const void* kernel, const DeviceInfo& dev);
 
-size_t gemv_smem_bytes(const seedlm_format& f);
+// Shared memory the GEMV needs for f within max_smem bytes (0: x does not fit).
+size_t gemv_smem_bytes(const seedlm_format& f, int max_smem);
 int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                 const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
                 const DeviceInfo& dev);

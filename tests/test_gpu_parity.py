@@ -330,3 +330,33 @@ def test_graph_replay_matches_eager_calls(sl):
         assert torch.equal(y, y0) and torch.equal(Y, Y0)
     assert sl.device_error() == 0
     del g
+
+
+# ------------------------------------------------------------ widest x
+
+@pytest.mark.parametrize("cp,cols", [(C8, 56320), (C12, 42240)])
+def test_gemv_at_its_widest_x_and_one_block_past_it(sl, oracle_mod, cp, cols):
+    # x is staged in shared memory as fp32: the widest x the GEMV takes
+    # (the partial-sum buffer shrinks to make room) matches the oracle; one
+    # more block is refused, and gemm_smallM with M = 1 then runs it on the
+    # tensor cores instead.
+    rows = 40
+    L = inputs.make_layer(rows, cols, *cp, seed=cols)
+    xb, xv = inputs.make_activations((cols,), "f16", 3)
+    y = gpu_gemv(sl, L, xb)
+    ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv)
+    assert_within(y, ref, refabs)
+
+    wide = cols + cp[0]
+    L = inputs.make_layer(rows, wide, *cp, seed=wide)
+    rec, ep = planes(L)
+    xb, xv = inputs.make_activations((wide,), "bf16", 4)
+    x = act_tensor(xb, "bf16")
+    y = torch.empty(rows, device="cuda")
+    with pytest.raises(sl.SeedLMError) as exc:
+        sl.gemv(L["fmt"], rec, ep, x, y)
+    assert exc.value.code == -2
+    assert sl.gemm_workspace_bytes(L["fmt"], 1) > 0
+    got = gpu_gemm(sl, L, xb.reshape(1, wide))
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], xv.reshape(1, wide))
+    assert_within(got[0], ref[0], refabs[0])
