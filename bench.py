@@ -317,6 +317,42 @@ def extras(torch, sl, args):
                              "compressed_gbs_cold": round(comp / cold / 1e3, 1)}
     out["square_sweep_4bit"] = sweep
 
+    # The 70B layer's four GEMVs as one CUDA graph vs launched one by one
+    # (4 resident copies rotating, 428 MB of records each, so L2 stays cold):
+    # how much a fused layer launch could save.
+    layer = make_layer_on_device(torch, LAYER_70B, (8, 3), 1300)
+    copies = replicate(torch, layer, 4)
+    fm = [sl.Format.from_dict(m["fmt"]) for m in layer]
+    xl = {}
+    for _, _, N in LAYER_70B:
+        if N not in xl:
+            xb, _ = inputs.make_activations((N,), "f16", 1400 + N)
+            xl[N] = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+    yl = [torch.empty(R, device="cuda") for _, R, _ in LAYER_70B]
+
+    def run70(lay, stream=None):
+        for m, f, y in zip(lay, fm, yl):
+            sl.gemv(f, m["rec"], None, xl[m["N"]], y, stream=stream)
+    for i in range(8):
+        run70(copies[i % 4])
+    eager = time_region(torch, lambda i: run70(copies[i % 4]), 400) / 400 * 1e3
+    graphs = []
+    gs = torch.cuda.Stream()
+    gs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(gs):
+        for c in copies:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gs):
+                run70(c, stream=gs)
+            graphs.append(g)
+    torch.cuda.current_stream().wait_stream(gs)
+    for i in range(8):
+        graphs[i % 4].replay()
+    graph = time_region(torch, lambda i: graphs[i % 4].replay(), 400) / 400 * 1e3
+    out["llama3_70b_layer_graph_vs_eager"] = {"us_per_layer_eager": round(eager, 2),
+                                             "us_per_layer_graph": round(graph, 2)}
+    del graphs, copies, layer
+
     # 3-bit Llama-3-8B layer: as specified (one layer) and 32 copies (cold).
     layer = make_layer_on_device(torch, LAYER_8B, (12, 4), 700)
     xs = {}

@@ -163,6 +163,27 @@ def test_gemv_empty_shapes(sl):
             sl.gemv(L["fmt"], rec, ep, act_tensor(xb, "f16"), y)
 
 
+def test_gemm_decompress_encode_empty_shapes(sl):
+    # rows = 0: nothing is launched or written; cols = 0: Y is all zeros (an
+    # empty sum), decompression and encoding have nothing to do.
+    for rows, cols in ((0, 64), (5, 0)):
+        L = inputs.make_layer(rows, cols, *C8, seed=2)
+        rec, ep = planes(L)
+        X = torch.zeros((3, max(cols, 1)), dtype=torch.bfloat16, device="cuda")
+        Y = torch.full((3, max(rows, 1)), float("nan"), device="cuda")
+        sl.gemm_smallM(L["fmt"], rec, ep, X, Y)
+        W = torch.full((max(rows, 1), max(cols, 1)), float("nan"), device="cuda")
+        sl.decompress(L["fmt"], rec, ep, W, ldw=max(cols, 1))
+        sl.encode(L["fmt"], W, rec, ep, ldw=max(cols, 1))
+        torch.cuda.synchronize()
+        if rows:
+            assert torch.equal(Y, torch.zeros_like(Y))
+        else:
+            assert torch.isnan(Y).all()
+        assert torch.isnan(W).all()
+    assert sl.device_error() == 0
+
+
 @pytest.mark.parametrize("cp,rows,cols", [(C8, 8192, 28672), (C8, 10240, 8192),
                                           (C12, 28672, 4096), (C12, 4096, 14336)])
 def test_gemv_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols):
