@@ -25,7 +25,10 @@
 // chunk.  All search arithmetic is fp64 and uses the expansion
 //   err = ||w||^2 - 2^(1-e) q.(U^T w) + 2^(-2e) q^T G q,
 // so a candidate costs a handful of fp64 operations once U^T w and t* of the
-// seed are known.  The winner's error is recomputed directly at the end.
+// seed are known.  A seed whose least-squares residual ||w||^2 - (U^T w).t*
+// (a lower bound on every quantised candidate's error) already exceeds the
+// best error found is skipped without scoring its exponents.  The winner's
+// error is recomputed directly at the end.
 #include <cuda_runtime.h>
 
 #include "seedlm_device.cuh"
@@ -174,13 +177,19 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
           b[p] = acc;
         }
         double t[P];
+        double bt = 0.0;
 #pragma unroll
         for (int p = 0; p < P; ++p) {
           double acc = 0.0;
 #pragma unroll
           for (int r = 0; r < P; ++r) acc = fma(ch.Gi[j][p * P + r], b[r], acc);
           t[p] = acc;
+          bt = fma(b[p], acc, bt);
         }
+        // No quantised candidate of this seed beats its least-squares
+        // residual ||w||^2 - b.t*; once that is above the best error so far
+        // (beyond fp64 rounding), the seed's exponents need no scoring.
+        if (ww[k] - bt > best[k].err + 1e-13 * ww[k]) continue;
         // Exponents in descending order: on an exact tie the larger e, met
         // first, stays.  |t* 2^e| shrinks with e, so once every q rounds to
         // 0 all smaller exponents give that same candidate (error ||w||^2,
