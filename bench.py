@@ -721,6 +721,15 @@ def profile_case(name: str):
         for _ in range(2):
             for f, rec, x, y in lay:
                 sl.gemv(f, rec, None, x, y)
+    elif name == "encode":
+        # Full seed / coefficient / exponent search of a Gaussian 512 x 1024
+        # matrix at 4 bits (65,536 blocks), twice.
+        rng = np.random.default_rng(11)
+        We = torch.from_numpy((rng.standard_normal((512, 1024)) * 0.02).astype(np.float32)).cuda()
+        fe = inputs.make_format(512, 1024, 8, 3)
+        rec_e = torch.empty((512, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
+        for _ in range(2):
+            sl.encode(fe, We, rec_e)
     elif name == "dense":
         W = torch.randn((57344, 8192), device="cuda").half()
         x = torch.randn(8192, device="cuda").half()
@@ -744,7 +753,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
-    ap.add_argument("--case", choices=("gemv", "decompress", "gemm64", "gemm16", "dense"),
+    ap.add_argument("--case", choices=("gemv", "decompress", "gemm64", "gemm16", "dense", "encode"),
                     help="run one small single-kernel workload (for ncu) and exit")
     args = ap.parse_args()
     if args.case:

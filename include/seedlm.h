@@ -177,10 +177,26 @@ SEEDLM_API int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t l
  * stuck hand-over surfaces to the caller, without a trap or a hang. */
 SEEDLM_API int seedlm_selftest_wait_timeout(int64_t limit_ns, seedlm_stream stream);
 
-/* Reads and clears the device-side error flag of the current device: 1 if a
- * kernel gave up waiting on one of its own barriers (the outputs of that call
- * are then undefined), else 0.  HOST function; synchronous. */
+/* Reads and clears the device-side error flags of the current device into
+ * *flag: bit 0 (value 1) if a kernel gave up waiting on one of its own
+ * barriers, bit 1 (value 2) if a kernel of a checked build (below) computed a
+ * memory index outside the buffers its arguments describe, or a
+ * shared-memory index outside its launch's allocation, and skipped that
+ * access.  The outputs of such a call are undefined.  0 if neither happened.
+ * HOST function; synchronous. */
 SEEDLM_API int seedlm_device_error(int* flag);
+
+/* Failure-path self test of the checked build: one kernel thread compares
+ * index with extent exactly as the kernels' bounds checks do, with no memory
+ * access behind it.  In a checked build, index >= extent then makes
+ * seedlm_device_error report bit 1; other builds compile the check away and
+ * report nothing.  Negative arguments return SEEDLM_EINVAL. */
+SEEDLM_API int seedlm_selftest_bounds_check(int64_t index, int64_t extent, seedlm_stream stream);
+
+/* 1 if this library was compiled with -DSEEDLM_CHECK=1: every kernel then
+ * compares each global and shared memory index it computes with the extent
+ * of the buffer before the access (slower; for testing), else 0. */
+SEEDLM_API int seedlm_checked_build(void);
 
 /* Reference point, not part of the method: y = W x with W dense fp16
  * (rows x cols, row-major, leading dimension ldw halves, 16-byte aligned with

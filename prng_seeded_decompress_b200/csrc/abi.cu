@@ -191,6 +191,14 @@ int seedlm_selftest_wait_timeout(int64_t limit_ns, seedlm_stream stream) {
   return launch_wait_timeout((uint64_t)limit_ns, (cudaStream_t)stream);
 }
 
+int seedlm_selftest_bounds_check(int64_t index, int64_t extent, seedlm_stream stream) {
+  if (index < 0 || extent < 0) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  return launch_bounds_check(index, extent, (cudaStream_t)stream);
+}
+
 int seedlm_device_error(int* flag) {
   if (!flag) return SEEDLM_EINVAL;
   DeviceInfo dev;
@@ -198,9 +206,21 @@ int seedlm_device_error(int* flag) {
   if (rc) return rc;
   unsigned int v = 0;
   if ((rc = read_and_clear_tc_error(&v))) return rc;
-  *flag = v ? 1 : 0;
+  int out = v ? 1 : 0;
+  // Bounds violations recorded by a checked build (always 0 otherwise).
+  int (*const readers[])(unsigned int*) = {read_and_clear_check_gemv, read_and_clear_check_decompress,
+                                           read_and_clear_check_gemm_tc, read_and_clear_check_encode,
+                                           read_and_clear_check_dense};
+  for (auto read : readers) {
+    unsigned int c = 0;
+    if ((rc = read(&c))) return rc;
+    if (c) out |= 2;
+  }
+  *flag = out;
   return SEEDLM_OK;
 }
+
+int seedlm_checked_build(void) { return SEEDLM_CHECK ? 1 : 0; }
 
 int seedlm_dense_gemv_f16(int32_t rows, int32_t cols, const uint16_t* W, int64_t ldw,
                           const uint16_t* x, float* y, seedlm_stream stream) {

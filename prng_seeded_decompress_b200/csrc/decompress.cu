@@ -14,6 +14,8 @@
 
 namespace seedlm {
 
+SEEDLM_CHECK_FLAG(decompress)
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -27,10 +29,13 @@ struct Chunk {
 
 template <int C>
 __device__ __forceinline__ Chunk load_chunk(const uint32_t* __restrict__ rec,
-                                            const uint8_t* __restrict__ eplane, int rec_pitch,
-                                            int e_pitch, int r, int k) {
-  Chunk ch;
-  ch.rec = ld_stream_u4(rec + (size_t)r * rec_pitch + kRecs * k);
+                                            const uint8_t* __restrict__ eplane, int rows,
+                                            int rec_pitch, int e_pitch, int r, int k) {
+  Chunk ch{};
+  // The chunk's last record word, and its exponent bytes, lie inside row r.
+  if (SEEDLM_IN_BOUNDS(g_check_flag, r, rows) &&
+      SEEDLM_IN_BOUNDS(g_check_flag, kRecs * k + kRecs - 1, rec_pitch))
+    ch.rec = ld_stream_u4(rec + (size_t)r * rec_pitch + kRecs * k);
   ch.e = 0;
   if constexpr (C == 12) {
     const uint8_t* ep = eplane + (size_t)r * e_pitch + 2 * k;
@@ -98,6 +103,9 @@ decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ 
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float4* stage = reinterpret_cast<float4*>(dsm + 512 * 8) + warp * 32 * (F + 1);
+  // float4 slots of this warp's staging buffer that the launch provides.
+  SEEDLM_CHECK_ONLY(const int stage_slots =
+                        (int)(seedlm_dynamic_smem_bytes() - 512 * 8) / 16 - warp * 32 * (F + 1);)
   const int cpr = (nb + kRecs - 1) / kRecs;  // chunks per row
   const int ipr = (cpr + 31) / 32;           // warp items per row
   const int64_t items = (int64_t)rows * ipr;
@@ -110,14 +118,14 @@ decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ 
   };
   int r, k;
   locate(it, r, k);
-  Chunk cur = k < cpr ? load_chunk<C>(rec, eplane, rec_pitch, e_pitch, r, k) : Chunk{};
+  Chunk cur = k < cpr ? load_chunk<C>(rec, eplane, rows, rec_pitch, e_pitch, r, k) : Chunk{};
   while (true) {
     const int64_t inext = it + wstep;
     int rn = 0, kn = 0;
     Chunk nxt{};
     if (inext < items) {
       locate(inext, rn, kn);
-      if (kn < cpr) nxt = load_chunk<C>(rec, eplane, rec_pitch, e_pitch, rn, kn);
+      if (kn < cpr) nxt = load_chunk<C>(rec, eplane, rows, rec_pitch, e_pitch, rn, kn);
     }
     const uint32_t words[kRecs] = {cur.rec.x, cur.rec.y, cur.rec.z, cur.rec.w};
 #pragma unroll
@@ -125,14 +133,19 @@ decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ 
       float w[C];
       rebuild_block<C>(words[q], (cur.e >> (4 * q)) & 15u, t32, t64, w);
 #pragma unroll
-      for (int v = 0; v < C / 4; ++v)
-        stage[lane * (F + 1) + q * (C / 4) + v] =
-            make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      for (int v = 0; v < C / 4; ++v) {
+        const int si = lane * (F + 1) + q * (C / 4) + v;
+        if (SEEDLM_IN_BOUNDS(g_check_flag, si, stage_slots))
+          stage[si] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
     }
     __syncwarp();
     const int j = (k - lane) / 32;  // item index within the row
     float* dst_row = W + (size_t)r * (size_t)ldw + (size_t)128 * j * C;
     const int col0 = 128 * j * C;
+    // Elements of W the call covers: rows - 1 full pitches plus one row.
+    SEEDLM_CHECK_ONLY(const size_t w_extent = (size_t)(rows - 1) * (size_t)ldw + (size_t)cols;
+                      const size_t row_base = (size_t)r * (size_t)ldw + (size_t)col0;)
 #pragma unroll
     for (int q = 0; q < F; ++q) {
       const int ff = q * 32 + lane;
@@ -140,12 +153,14 @@ decompress_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ 
       const float4 val = stage[c * (F + 1) + v];
       const int j0 = col0 + 4 * ff;
       if (vec && j0 + 4 <= cols) {
-        __stcs(reinterpret_cast<float4*>(dst_row + 4 * ff), val);
+        if (SEEDLM_IN_BOUNDS(g_check_flag, row_base + 4 * ff + 3, w_extent))
+          __stcs(reinterpret_cast<float4*>(dst_row + 4 * ff), val);
       } else if (j0 < cols) {
         const float e4[4] = {val.x, val.y, val.z, val.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          if (j0 + u < cols) dst_row[4 * ff + u] = e4[u];
+          if (j0 + u < cols && SEEDLM_IN_BOUNDS(g_check_flag, row_base + 4 * ff + u, w_extent))
+            dst_row[4 * ff + u] = e4[u];
       }
     }
     __syncwarp();

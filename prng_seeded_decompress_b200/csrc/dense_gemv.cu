@@ -15,6 +15,8 @@
 
 namespace seedlm {
 
+SEEDLM_CHECK_FLAG(dense)
+
 namespace {
 
 constexpr int kWarps = 16;
@@ -38,8 +40,10 @@ dense_gemv_f16_kernel(int rows, int cols, const uint16_t* __restrict__ W, int64_
                       const uint16_t* __restrict__ x, float* __restrict__ y) {
   extern __shared__ __align__(16) float xs[];
   const int cols8 = (cols + 7) / 8 * 8;
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = seedlm_dynamic_smem_bytes() / 4;)
   for (int j = threadIdx.x; j < cols8; j += kThreads)
-    xs[j] = j < cols ? __half2float(__ushort_as_half(x[j])) : 0.f;
+    if (SEEDLM_IN_BOUNDS(g_check_flag, j, xs_floats))
+      xs[j] = j < cols ? __half2float(__ushort_as_half(x[j])) : 0.f;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int gwarp = blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -55,8 +59,10 @@ dense_gemv_f16_kernel(int rows, int cols, const uint16_t* __restrict__ W, int64_
       uint4 a[kUnroll], b[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        a[u] = ld_stream_u4(w0 + 8 * (k + 32 * u));
-        b[u] = ld_stream_u4(w1 + 8 * (k + 32 * u));
+        // The chunk's last element lies inside the row.
+        const bool ok = SEEDLM_IN_BOUNDS(g_check_flag, 8 * (k + 32 * u) + 7, cols);
+        a[u] = ok ? ld_stream_u4(w0 + 8 * (k + 32 * u)) : make_uint4(0u, 0u, 0u, 0u);
+        b[u] = ok ? ld_stream_u4(w1 + 8 * (k + 32 * u)) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
@@ -66,6 +72,7 @@ dense_gemv_f16_kernel(int rows, int cols, const uint16_t* __restrict__ W, int64_
       }
     }
     for (; k < full8; k += 32) {
+      if (!SEEDLM_IN_BOUNDS(g_check_flag, 8 * k + 7, cols)) continue;
       uint4 a = ld_stream_u4(w0 + 8 * k), b = ld_stream_u4(w1 + 8 * k);
       s0 += dot8(a, xs + 8 * k);
       s1 += dot8(b, xs + 8 * k);
@@ -80,8 +87,8 @@ dense_gemv_f16_kernel(int rows, int cols, const uint16_t* __restrict__ W, int64_
       s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     }
     if (lane == 0) {
-      y[r0] = s0;
-      if (two) y[r0 + 1] = s1;
+      if (SEEDLM_IN_BOUNDS(g_check_flag, r0, rows)) y[r0] = s0;
+      if (two && SEEDLM_IN_BOUNDS(g_check_flag, r0 + 1, rows)) y[r0 + 1] = s1;
     }
   }
 }

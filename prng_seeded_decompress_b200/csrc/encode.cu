@@ -36,6 +36,8 @@
 
 namespace seedlm {
 
+SEEDLM_CHECK_FLAG(encode)
+
 namespace {
 
 constexpr int kEncThreads = 128;
@@ -148,7 +150,9 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       const int col = (b0 + k) * C + c;
-      const bool in = active && b0 + k < nb && col < cols;
+      const bool in = active && b0 + k < nb && col < cols &&
+                      SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * ldw + col,
+                                       (size_t)(rows - 1) * ldw + cols);
       w[k][c] = in ? (double)W[(size_t)row * ldw + col] : 0.0;
       ww[k] = fma(w[k][c], w[k][c], ww[k]);
     }
@@ -249,14 +253,17 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
 #pragma unroll
     for (int p = 0; p < P; ++p) r |= ((uint32_t)best[k].q[p] & 15u) << (4 * p);
     if constexpr (C == 8) r |= (uint32_t)best[k].e << 12;
-    rec[(size_t)row * rec_pitch + blk] = r;
-    if (err_out) err_out[(size_t)row * nb + blk] = err;
+    if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, blk, rec_pitch))
+      rec[(size_t)row * rec_pitch + blk] = r;
+    if (err_out && SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * nb + blk, (size_t)rows * nb))
+      err_out[(size_t)row * nb + blk] = err;
   }
   if constexpr (C == 12) {
     // The pair's exponent byte: block b0 in the low nibble, b0 + 1 (or 0).
     uint32_t byte = (uint32_t)best[0].e & 15u;
     if (b0 + 1 < nb) byte |= ((uint32_t)best[1].e & 15u) << 4;
-    eplane[(size_t)row * e_pitch + (b0 >> 1)] = (uint8_t)byte;
+    if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, e_pitch))
+      eplane[(size_t)row * e_pitch + (b0 >> 1)] = (uint8_t)byte;
   }
 }
 

@@ -61,6 +61,8 @@ namespace seedlm {
 
 __device__ unsigned int g_tc_error = 0;
 
+SEEDLM_CHECK_FLAG(gemm_tc)
+
 namespace {
 
 constexpr int kTileM = 128;
@@ -154,8 +156,9 @@ stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks,
       const uint32_t b = (n < M && col + 2 * u + 1 < cols) ? X[(size_t)n * cols + col + 2 * u + 1] : 0u;
       v[u] = a | (b << 16);
     }
-    *reinterpret_cast<uint4*>(Xs + (size_t)chunk * (NB * KC * 2) + slab_byte<KC>(n, 8 * k8)) =
-        make_uint4(v[0], v[1], v[2], v[3]);
+    const size_t xb = (size_t)chunk * (NB * KC * 2) + slab_byte<KC>(n, 8 * k8);
+    if (SEEDLM_IN_BOUNDS(g_check_flag, xb + 15, (size_t)nchunks * (NB * KC * 2)))
+      *reinterpret_cast<uint4*>(Xs + xb) = make_uint4(v[0], v[1], v[2], v[3]);
   }
 }
 
@@ -227,6 +230,9 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ctas = gridDim.x;
+  // The whole shared-memory layout lies inside the launch's allocation
+  // (checked before any barrier or TMEM exists, so leaving is safe).
+  if (!SEEDLM_IN_BOUNDS(g_check_flag, L::TOTAL - 1, seedlm_dynamic_smem_bytes())) return;
   const long long u_begin = unit_begin(blockIdx.x, g.units, ctas);
   const int n_units = (int)(unit_begin(blockIdx.x + 1, g.units, ctas) - u_begin);
   const int t_first = (int)(u_begin / g.nchunks);
@@ -288,8 +294,12 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         const int s = j % XS;
         if (j >= XS)  // the slab's previous unit (j - XS) has finished its MMAs
           ok = tc::mbar_wait_or_abort(xfree(s), ((j / XS) - 1) & 1, kWaitLimit, abort_flag) && ok;
-        tc::mbar_arrive_expect_tx(xfull(s), L::XB);
-        tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)xc.chunk * L::XB, L::XB, xfull(s));
+        if (SEEDLM_IN_BOUNDS(g_check_flag, xc.chunk, g.nchunks)) {
+          tc::mbar_arrive_expect_tx(xfull(s), L::XB);
+          tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)xc.chunk * L::XB, L::XB, xfull(s));
+        } else {
+          tc::mbar_arrive(xfull(s));  // checked build: no copy, the hand-over still completes
+        }
       }
       // Every copy this thread issued has landed before the CTA may exit
       // (bounded, and not cut short by the give-up flag).
@@ -352,7 +362,10 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     auto load_rec = [&](const UnitCursor& u, RecUnit<C>& p) {
       const int gr = u.tile * kTileM + prow;
       const int b0 = u.chunk * (KC / C) + kq * BPT;  // a multiple of BPT
-      const bool ok_ = gr < g.rows && b0 < g.nb;
+      // The thread's last record and its exponent byte lie inside row gr.
+      const bool ok_ = gr < g.rows && b0 < g.nb &&
+                       SEEDLM_IN_BOUNDS(g_check_flag, b0 + BPT - 1, g.rec_pitch) &&
+                       (C == 8 || SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, g.e_pitch));
       const uint32_t* src = rec + (size_t)gr * g.rec_pitch + b0;
       if constexpr (C == 8) {
         const uint4 v = ok_ ? ld_stream_u4(src) : make_uint4(0u, 0u, 0u, 0u);
@@ -444,6 +457,11 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       const int first = unit_owner((long long)tile * g.nchunks, g.units, ctas);
       const int last = unit_owner((long long)(tile + 1) * g.nchunks - 1, g.units, ctas);
       float* mine = partial + ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);
+      // Extents: Y holds M x rows floats; the partial tiles ctas x segs_max
+      // tiles of NB x 128 floats (one per segment of each CTA).
+      SEEDLM_CHECK_ONLY(const size_t y_n = (size_t)g.M * g.rows;
+                        const size_t part_n = (size_t)ctas * g.segs_max * (NB * kTileM);
+                        const size_t mine_off = ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);)
 #pragma unroll
       for (int n16 = 0; n16 < NB / 16; ++n16) {
         float v[16];
@@ -452,11 +470,16 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           if (gr < g.rows) {
 #pragma unroll
             for (int q = 0; q < 16; ++q)
-              if (16 * n16 + q < g.M) Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q] * kYScale;
+              if (16 * n16 + q < g.M &&
+                  SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(16 * n16 + q) * g.rows + gr, y_n))
+                Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q] * kYScale;
           }
         } else {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) mine[(16 * n16 + q) * kTileM + row] = v[q] * kYScale;
+          for (int q = 0; q < 16; ++q)
+            if (SEEDLM_IN_BOUNDS(g_check_flag, seg, g.segs_max) &&
+                SEEDLM_IN_BOUNDS(g_check_flag, mine_off + (16 * n16 + q) * kTileM + row, part_n))
+              mine[(16 * n16 + q) * kTileM + row] = v[q] * kYScale;
         }
       }
       tc::fence_before_sync();
@@ -466,7 +489,10 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       __threadfence();
       tc::named_sync(128);
       if (tid == 0)
-        slot[1] = (atomicAdd(&counters[tile], 1u) == (unsigned)(last - first)) ? 1u : 0u;
+        slot[1] = SEEDLM_IN_BOUNDS(g_check_flag, tile, g.tiles) &&
+                          atomicAdd(&counters[tile], 1u) == (unsigned)(last - first)
+                      ? 1u
+                      : 0u;
       tc::named_sync(128);
       if (slot[1]) {
         __threadfence();
@@ -475,6 +501,12 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           for (int c = first; c <= last; ++c) {
             const int cseg = tile - (int)(unit_begin(c, g.units, ctas) / g.nchunks);
             const float* p = partial + ((size_t)c * g.segs_max + cseg) * (NB * kTileM) + row;
+            if (!SEEDLM_IN_BOUNDS(g_check_flag, cseg, g.segs_max) ||
+                !SEEDLM_IN_BOUNDS(g_check_flag,
+                                  ((size_t)c * g.segs_max + cseg) * (NB * kTileM) +
+                                      (size_t)(g.M - 1) * kTileM + row,
+                                  part_n))
+              continue;
             for (int n = 0; n < g.M; ++n) {
               float* y = Y + (size_t)n * g.rows + gr;
               *y = (c == first) ? p[n * kTileM] : *y + p[n * kTileM];
@@ -677,7 +709,20 @@ __global__ void __launch_bounds__(64, 1) wait_timeout_kernel(uint64_t limit_ns) 
   }
 }
 
+// One bounds check evaluated on the device, with no memory access behind it:
+// shows that a checked build's comparison and flag reach seedlm_device_error.
+__global__ void bounds_check_kernel(long long index, long long extent) {
+  if (SEEDLM_IN_BOUNDS(g_check_flag, index, extent)) {
+  }
+}
+
 }  // namespace
+
+int launch_bounds_check(int64_t index, int64_t extent, cudaStream_t stream) {
+  bounds_check_kernel<<<1, 1, 0, stream>>>(index, extent);
+  count_launch();
+  return record_cuda_error(cudaGetLastError());
+}
 
 int launch_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
   wait_timeout_kernel<<<1, 64, 0, stream>>>(limit_ns);

@@ -37,6 +37,8 @@
 
 namespace seedlm {
 
+SEEDLM_CHECK_FLAG(gemv)
+
 namespace {
 
 // Warps per CTA (one CTA per SM) and record sets in flight ahead of the one
@@ -106,13 +108,15 @@ __device__ void stage_x_and_tables(unsigned char* smem, const uint16_t* __restri
   // x, zero-padded to n_spans * 32 record pairs.
   float* xs = reinterpret_cast<float*>(smem + g.x_off);
   const int ncols_pad = g.n_spans * 32 * 2 * C;
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (seedlm_dynamic_smem_bytes() - g.x_off) / 4;)
   for (int j = threadIdx.x; j < ncols_pad; j += blockDim.x) {
     int rp = j / (2 * C);
     int w = j - rp * 2 * C;
     int h = w / C;
     int c = w - h * C;
     float v = j < g.cols ? act_to_float(x[j], is_bf16) : 0.f;
-    xs[x_slot_index<C>(rp, c, h)] = v;
+    const int si = x_slot_index<C>(rp, c, h);
+    if (SEEDLM_IN_BOUNDS(g_check_flag, si, xs_floats)) xs[si] = v;
   }
 }
 
@@ -136,11 +140,17 @@ __device__ __forceinline__ void load_set(RecSet<C>& o, const uint32_t* __restric
   const uint32_t* p = rec + (size_t)row0 * g.rec_pitch + 2 * rp;
 #pragma unroll
   for (int j = 0; j < kRowsPerTask; ++j) {
-    const bool ok = pair_ok && row0 + j < g.rows;
+    // The pair's second record is the last word read.
+    const bool ok = pair_ok && row0 + j < g.rows &&
+                    SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(row0 + j) * g.rec_pitch + 2 * rp + 1,
+                                     (size_t)g.rows * g.rec_pitch);
     o.r[j] = ok ? ld_stream_u2(p + (size_t)j * g.rec_pitch) : make_uint2(0u, 0u);
     if constexpr (C == 12)
-      o.e[j] = (ok && rp < g.e_pitch) ? ld_stream_u8(eplane + (size_t)(row0 + j) * g.e_pitch + rp)
-                                      : 0u;
+      o.e[j] = (ok && rp < g.e_pitch &&
+                SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(row0 + j) * g.e_pitch + rp,
+                                 (size_t)g.rows * g.e_pitch))
+                   ? ld_stream_u8(eplane + (size_t)(row0 + j) * g.e_pitch + rp)
+                   : 0u;
   }
 }
 
@@ -219,6 +229,8 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
   const void* t_hi = smem + Smem<C>::kJumpBytes / 2;
   float* part = reinterpret_cast<float*>(smem + Smem<C>::kTableBytes);
   const float* xs = reinterpret_cast<const float*>(smem + g.x_off);
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (seedlm_dynamic_smem_bytes() - g.x_off) / 4;
+                    const int part_floats = (g.x_off - Smem<C>::kTableBytes) / 4;)
 
   const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -249,7 +261,8 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
       stage_x_and_tables<C>(smem, x, is_bf16, g);
       first_pass = false;
     }
-    for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x) part[i] = 0.f;
+    for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x)
+      if (SEEDLM_IN_BOUNDS(g_check_flag, i, part_floats)) part[i] = 0.f;
     __syncthreads();  // x, tables and zeroed partials ready
     if (i0 < i1) {
       float2 acc[kRowsPerTask];
@@ -261,7 +274,10 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
 #pragma unroll
         for (int k = 0; k <= Tune<C>::kPrefetch; ++k) {
           if (!done) {
-            rebuild_and_dot<C>(buf[k], xs, span * 32 + lane, swz, t_lo, t_hi, acc);
+            // Every x slot of the lane's record pair lies in its kSlotFloats row.
+            if (SEEDLM_IN_BOUNDS(g_check_flag,
+                                 (span * 32 + lane + 1) * Smem<C>::kSlotFloats - 1, xs_floats))
+              rebuild_and_dot<C>(buf[k], xs, span * 32 + lane, swz, t_lo, t_hi, acc);
             if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
             ++li;
             if (++lspan == g.n_spans) { lspan = 0; ++lgrp; }
@@ -271,7 +287,8 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
 #pragma unroll
               for (int j = 0; j < kRowsPerTask; ++j) {
                 const float s = warp_sum(acc[j].x + acc[j].y);
-                if (lane == 0) part[((grp - p0) * kRowsPerTask + j) * nw + warp] = s;
+                const int pi = ((grp - p0) * kRowsPerTask + j) * nw + warp;
+                if (lane == 0 && SEEDLM_IN_BOUNDS(g_check_flag, pi, part_floats)) part[pi] = s;
                 acc[j] = make_float2(0.f, 0.f);
               }
               if (end_group) { span = 0; ++grp; }
@@ -291,7 +308,7 @@ gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane
       if (r < g.rows) {
         float s = 0.f;
         for (int w = 0; w < nw; ++w) s += part[t * nw + w];
-        y[r] = s;
+        if (SEEDLM_IN_BOUNDS(g_check_flag, r, g.rows)) y[r] = s;
       }
     }
     __syncthreads();  // partials read before the next pass clears them

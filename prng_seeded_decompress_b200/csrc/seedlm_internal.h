@@ -7,7 +7,56 @@
 
 #include "../../include/seedlm.h"
 
+// Bounds-checked build (-DSEEDLM_CHECK=1, `python -m
+// prng_seeded_decompress_b200.build --check`): every memory index a kernel
+// computes is compared with the extent its arguments (or its shared-memory
+// layout) define before the access; a violation sets the kernel file's check
+// flag, which seedlm_device_error reports, and the access is skipped.  In
+// normal builds the checks compile to nothing.
+#ifndef SEEDLM_CHECK
+#define SEEDLM_CHECK 0
+#endif
+#if SEEDLM_CHECK
+#define SEEDLM_IN_BOUNDS(flag, idx, extent)                                              \
+  (((unsigned long long)(idx) < (unsigned long long)(extent)) ? true                     \
+                                                              : (atomicOr(&(flag), 1u), false))
+// One check flag per kernel file, with a host reader that clears it.
+#define SEEDLM_CHECK_FLAG(name)                                                          \
+  namespace {                                                                            \
+  __device__ unsigned int g_check_flag;                                                  \
+  }                                                                                      \
+  int read_and_clear_check_##name(unsigned int* out) {                                   \
+    unsigned int v = 0, zero = 0;                                                        \
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_check_flag, sizeof(v));                 \
+    if (err == cudaSuccess && v) err = cudaMemcpyToSymbol(g_check_flag, &zero, sizeof(zero)); \
+    *out = v;                                                                            \
+    return record_cuda_error(err);                                                       \
+  }
+// Code that only the checked build compiles (extents computed for the checks).
+#define SEEDLM_CHECK_ONLY(...) __VA_ARGS__
+// Bytes of dynamic shared memory the running kernel was launched with.
+__device__ __forceinline__ unsigned int seedlm_dynamic_smem_bytes() {
+  unsigned int r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+#else
+#define SEEDLM_IN_BOUNDS(flag, idx, extent) true
+#define SEEDLM_CHECK_ONLY(...)
+#define SEEDLM_CHECK_FLAG(name)                                                          \
+  int read_and_clear_check_##name(unsigned int* out) {                                   \
+    *out = 0;                                                                            \
+    return 0;                                                                            \
+  }
+#endif
+
 namespace seedlm {
+
+int read_and_clear_check_gemv(unsigned int* out);
+int read_and_clear_check_decompress(unsigned int* out);
+int read_and_clear_check_gemm_tc(unsigned int* out);
+int read_and_clear_check_encode(unsigned int* out);
+int read_and_clear_check_dense(unsigned int* out);
 
 struct DeviceInfo {
   int device;
@@ -42,6 +91,7 @@ int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* e
                    int64_t workspace_bytes, cudaStream_t stream, const DeviceInfo& dev);
 int read_and_clear_tc_error(unsigned int* out);
 int launch_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+int launch_bounds_check(int64_t index, int64_t extent, cudaStream_t stream);
 int launch_encode(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
                   uint8_t* eplane, double* err, cudaStream_t stream);
 

@@ -11,7 +11,9 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libseedlm.so")
+#: SEEDLM_CHECKED=1 loads the bounds-checked build (`build --check`) instead.
+CHECKED = os.environ.get("SEEDLM_CHECKED", "0") == "1"
+LIB_PATH = os.path.join(PKG, "libseedlm_check.so" if CHECKED else "libseedlm.so")
 
 F16 = 0
 BF16 = 1
@@ -22,7 +24,8 @@ EXPORTS = (
     "seedlm_gemm_smallM_workspace_bytes", "seedlm_gemm_smallM_noalloc", "seedlm_device_error",
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
-    "seedlm_encode", "seedlm_selftest_wait_timeout",
+    "seedlm_encode", "seedlm_selftest_wait_timeout", "seedlm_checked_build",
+    "seedlm_selftest_bounds_check",
 )
 
 
@@ -45,8 +48,8 @@ class Format(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m prng_seeded_decompress_b200.build`"
-            " (the SeedLM kernels have no CPU fallback)")
+            f"{LIB_PATH} is missing: build it with `python -m prng_seeded_decompress_b200.build"
+            f"{' --check' if CHECKED else ''}` (the SeedLM kernels have no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     fmtp = ctypes.POINTER(Format)
@@ -69,6 +72,8 @@ def _load():
         "seedlm_last_cuda_error": (ctypes.c_int, []),
         "seedlm_launch_count": (i64, []),
         "seedlm_shutdown": (None, []),
+        "seedlm_checked_build": (ctypes.c_int, []),
+        "seedlm_selftest_bounds_check": (ctypes.c_int, [i64, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -206,11 +211,24 @@ def gemm_smallM_noalloc(fmt, rec, eplane, X, Y, stream=None):
 
 
 def device_error() -> int:
-    """1 if a kernel gave up on one of its own bounded waits since the last
-    check (and clears the flag), else 0.  Synchronous."""
+    """Reads and clears the device error flags: bit 0 if a kernel gave up on
+    one of its own bounded waits, bit 1 if a kernel of the checked build
+    skipped an out-of-bounds access.  Synchronous."""
     flag = ctypes.c_int(0)
     _check("seedlm_device_error", lib.seedlm_device_error(ctypes.byref(flag)))
     return int(flag.value)
+
+
+def checked_build() -> bool:
+    """True if the loaded library is the bounds-checked build."""
+    return bool(lib.seedlm_checked_build())
+
+
+def selftest_bounds_check(index: int, extent: int, stream=None):
+    """Evaluate one bounds check on the device (no memory access): in the
+    checked build index >= extent raises bit 1 of device_error()."""
+    _check("seedlm_selftest_bounds_check",
+           lib.seedlm_selftest_bounds_check(int(index), int(extent), _stream(stream)))
 
 
 def selftest_wait_timeout(limit_ns: int = 2_000_000, stream=None):

@@ -17,3 +17,21 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def device_flags_stay_clear(request):
+    """After every GPU test: no kernel gave up on a bounded wait and, in the
+    bounds-checked build, none skipped an out-of-bounds access (tests that
+    raise a flag on purpose read and clear it themselves)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    mod = sys.modules.get("prng_seeded_decompress_b200.seedlm")
+    if mod is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    torch.cuda.synchronize()
+    assert mod.device_error() == 0, "a kernel raised the device error flag during this test"

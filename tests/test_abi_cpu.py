@@ -45,6 +45,23 @@ def test_library_exports_every_declared_symbol(sl):
     assert exported == set(names)
 
 
+def test_checked_build_exports_the_same_symbols(sl):
+    # The bounds-checked build (-DSEEDLM_CHECK=1) is the same boundary; only
+    # seedlm_checked_build tells the two apart.
+    from prng_seeded_decompress_b200 import build
+    path = build.build(check=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
+                         text=True, check=True).stdout
+    assert set(re.findall(r"\bT (seedlm_\w+)", out)) == set(declared_functions())
+    assert ctypes.CDLL(path).seedlm_checked_build() == 1
+    assert sl.lib.seedlm_checked_build() == (1 if sl.CHECKED else 0)
+
+
+def test_selftest_arguments_are_checked_before_cuda(sl):
+    assert sl.lib.seedlm_selftest_bounds_check(-1, 4, None) == -1
+    assert sl.lib.seedlm_selftest_bounds_check(0, -4, None) == -1
+
+
 def test_strerror_and_counters(sl):
     assert sl.strerror(0) == "success"
     for c in (-1, -2, -3, 7):
