@@ -722,12 +722,12 @@ def profile_case(name: str):
             for f, rec, x, y in lay:
                 sl.gemv(f, rec, None, x, y)
     elif name == "encode":
-        # Full seed / coefficient / exponent search of a Gaussian 512 x 1024
-        # matrix at 4 bits (65,536 blocks), twice.
+        # Full seed / coefficient / exponent search of a Gaussian 2048 x 2048
+        # matrix at 4 bits (524,288 blocks), twice.
         rng = np.random.default_rng(11)
-        We = torch.from_numpy((rng.standard_normal((512, 1024)) * 0.02).astype(np.float32)).cuda()
-        fe = inputs.make_format(512, 1024, 8, 3)
-        rec_e = torch.empty((512, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
+        We = torch.from_numpy((rng.standard_normal((2048, 2048)) * 0.02).astype(np.float32)).cuda()
+        fe = inputs.make_format(2048, 2048, 8, 3)
+        rec_e = torch.empty((2048, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
         for _ in range(2):
             sl.encode(fe, We, rec_e)
     elif name == "dense":

@@ -180,7 +180,7 @@ int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_
   if (err && !aligned(err, 8)) return SEEDLM_EINVAL;
   DeviceInfo dev;
   if ((rc = device_info(&dev))) return rc;
-  return launch_encode(*fmt, W, ldw, rec, eplane, err, (cudaStream_t)stream);
+  return launch_encode(*fmt, W, ldw, rec, eplane, err, (cudaStream_t)stream, dev);
 }
 
 int seedlm_selftest_wait_timeout(int64_t limit_ns, seedlm_stream stream) {

@@ -5,8 +5,9 @@
 // parameter optimisation): each block is matched against every seed's
 // pseudo-random matrix U(s) (C x P), the coefficients are fitted and
 // quantised, and the seed with the smallest reconstruction error wins; the
-// search is parallel over blocks and seeds.  The pages fix no exponent or
-// rounding rule; the reading used throughout this library:
+// search is parallel over blocks and seeds, with per-seed data computed once
+// and cached.  The pages fix no exponent or rounding rule; the reading used
+// throughout this library:
 //
 //   t*(s) = pinv(U(s)) w              (U(s) has full column rank for every s,
 //                                      so pinv(U) w = G^-1 U^T w, G = U^T U)
@@ -17,19 +18,40 @@
 // largest exponent.  A tail block (cols not a multiple of C) is fitted with
 // its missing weights taken as zero.
 //
-// One thread owns one block (C = 8) or the two blocks that share an exponent
-// byte (C = 12).  A CTA walks all 65,535 seeds in chunks: for each chunk it
-// first builds U, G and G^-1 of every seed in shared memory (from the same
-// bit stream the decoder uses, seedlm_device.cuh; G is exact in fp64 because
-// U's entries are k / 32768), then every thread scores its blocks against the
-// chunk.  All search arithmetic is fp64 and uses the expansion
-//   err = ||w||^2 - 2^(1-e) q.(U^T w) + 2^(-2e) q^T G q,
-// so a candidate costs a handful of fp64 operations once U^T w and t* of the
-// seed are known.  A seed whose least-squares residual ||w||^2 - (U^T w).t*
-// (a lower bound on every quantised candidate's error) already exceeds the
-// best error found is skipped without scoring its exponents.  The winner's
-// error is recomputed directly at the end.
+// Two kernels.  basis_table_kernel computes, once per call, an orthonormal
+// basis Q(s) of every seed's column space (Gram-Schmidt in fp64, each column
+// orthogonalised twice) and stores it rounded to fp32: one float4 per row c
+// of U, (Q[c][0], Q[c][1], Q[c][2], Q[c][3]) for P = 4 and
+// (Q[c][0], Q[c][1], Q[c][2], Q[c][2]) for P = 3.
+//
+// encode_kernel: one thread owns two neighbouring blocks of a row (for C = 12
+// the two that share an exponent byte).  A CTA streams the table through
+// shared memory in chunks of 128 seeds (cp.async, double-buffered), and for
+// every seed each thread first evaluates, in fp32, the least-squares residual
+//   r(s) = ||w||^2 - ||Q(s)^T w||^2,
+// a lower bound on the error of every quantised candidate of that seed.  Only
+// when r(s) is not above the block's best error so far plus a margin does the
+// thread score the seed exactly (score_seed: fp64, U, G exact, G^-1 by
+// Gauss-Jordan, the exponents in descending order with the expansion
+//   err = ||w||^2 - 2^(1-e) q.(U^T w) + 2^(-2e) q^T G q ).
+// On Gaussian blocks about 3 in 10^4 seeds get that far, so the search costs
+// one fp32 projection per seed and block: 3 (C = 8) or 4 (C = 12) packed
+// fp32x2 FMAs per basis row for both blocks, on a row read once.
+//
+// The filter never changes the result.  The block is scaled by 2^-E (exact)
+// so that max|w| lies in [1, 2).  With u = 2^-24, each fp32 coordinate of
+// Q^T w is within (C + 1) u ||w|| of the exact one (C fused products, plus
+// the rounding of Q to fp32; the columns of Q have unit norm), so the squared
+// norm is within about 2 sqrt(P) (C + 1) u ||w||^2 + P u ||w||^2, and ||w||^2
+// in fp32 within C u ||w||^2: |r_fp32 - r| < 5e-6 ||w||^2 for both formats.
+// The basis itself is orthonormal to fp64 rounding, and spans U(s)'s column
+// space to within kappa(U) 2^-53 < 1e-10 (kappa(U) < 4e5 over all seeds), so
+// a seed is skipped only if r_fp32 > best + 3e-5 ||w||^2, where no candidate
+// of it can reach the best error (candidates are compared with strict <).
+// The winner's error is recomputed directly at the end.
 #include <cuda_runtime.h>
+
+#include <cmath>
 
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
@@ -41,15 +63,15 @@ SEEDLM_CHECK_FLAG(encode)
 namespace {
 
 constexpr int kEncThreads = 128;
-constexpr int kSeedChunk = 32;
 constexpr int kNumSeeds = 65535;
-
-template <int C, int P>
-struct EncChunk {
-  double U[kSeedChunk][C * P];  // U[c][p] at c * P + p
-  double G[kSeedChunk][P * P];
-  double Gi[kSeedChunk][P * P];
-};
+constexpr int kTableRows = 65536;  // row i holds seed i + 1; the last row is zero padding
+constexpr int kChunk = 128;        // seeds per shared-memory chunk
+constexpr int kChunks = kTableRows / kChunk;
+constexpr double kPruneMargin = 3e-5;  // relative to ||w||^2, six times the fp32 error bound
+#ifndef SEEDLM_ENC_GROUP
+#define SEEDLM_ENC_GROUP 4
+#endif
+constexpr int kGroup = SEEDLM_ENC_GROUP;  // seeds tested per survivor branch
 
 // The seed's bit stream, bits [0, 64): state_k = bits [k, k + 16).
 __device__ __forceinline__ uint64_t seed_stream(uint32_t seed) {
@@ -65,8 +87,8 @@ __device__ __forceinline__ double basis_entry(uint64_t stream, int c, int p) {
   return (double)(state - 32768) * (1.0 / 32768.0);
 }
 
-// In-place inverse of a symmetric positive definite P x P matrix by
-// Gauss-Jordan elimination (no pivoting needed for SPD).
+// Inverse of a symmetric positive definite P x P matrix by Gauss-Jordan
+// elimination (no pivoting needed for SPD).
 template <int P>
 __device__ void spd_inverse(const double* g, double* gi) {
   double a[P][2 * P];
@@ -96,163 +118,348 @@ __device__ void spd_inverse(const double* g, double* gi) {
     for (int j = 0; j < P; ++j) gi[i * P + j] = a[i][P + j];
 }
 
+// fp64 data of one seed for exact scoring: G = U^T U (exact; row-major,
+// upper triangle used) and G^-1 (Gauss-Jordan), padded to 20 or 32 doubles.
+template <int P>
+struct SeedExact {
+  static constexpr int kDoubles = (2 * P * P + 3) / 4 * 4;
+  static_assert(kDoubles >= 2 * P * P, "G and G^-1 fit one row");
+};
+
+// Row i of the tables: the orthonormal basis of seed i + 1, one float4 per
+// row c of U (see the file comment), and its G and G^-1.
 template <int C, int P>
-__device__ void build_seed(EncChunk<C, P>& ch, int j, uint32_t seed) {
-  const uint64_t st = seed_stream(seed);
-  double u[C][P];
+__global__ void __launch_bounds__(256) basis_table_kernel(float4* __restrict__ table,
+                                                          double* __restrict__ exact) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= kTableRows) return;
+  float4* out = table + (size_t)i * C;
+  if (i >= kNumSeeds) {
+#pragma unroll
+    for (int c = 0; c < C; ++c) out[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const uint64_t st = seed_stream((uint32_t)(i + 1));
+  double q[C][P];
 #pragma unroll
   for (int c = 0; c < C; ++c)
 #pragma unroll
-    for (int p = 0; p < P; ++p) {
-      u[c][p] = basis_entry<C, P>(st, c, p);
-      ch.U[j][c * P + p] = u[c][p];
+    for (int p = 0; p < P; ++p) q[c][p] = basis_entry<C, P>(st, c, p);
+  {
+    double g[P * P], gi[P * P];
+#pragma unroll
+    for (int p = 0; p < P; ++p)
+#pragma unroll
+      for (int r = 0; r < P; ++r) {
+        double acc = 0.0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc = fma(q[c][p], q[c][r], acc);  // exact
+        g[p * P + r] = acc;
+      }
+    spd_inverse<P>(g, gi);
+    double* ex = exact + (size_t)i * SeedExact<P>::kDoubles;
+#pragma unroll
+    for (int k = 0; k < P * P; ++k) {
+      ex[k] = g[k];
+      ex[P * P + k] = gi[k];
     }
-  double g[P * P];
+  }
 #pragma unroll
-  for (int p = 0; p < P; ++p)
+  for (int p = 0; p < P; ++p) {
 #pragma unroll
-    for (int r = 0; r < P; ++r) {
-      double acc = 0.0;
+    for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
-      for (int c = 0; c < C; ++c) acc = fma(u[c][p], u[c][r], acc);  // exact
-      g[p * P + r] = acc;
-      ch.G[j][p * P + r] = acc;
-    }
-  spd_inverse<P>(g, ch.Gi[j]);
+      for (int j = 0; j < p; ++j) {
+        double d = 0.0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) d = fma(q[c][j], q[c][p], d);
+#pragma unroll
+        for (int c = 0; c < C; ++c) q[c][p] = fma(-d, q[c][j], q[c][p]);
+      }
+    double n = 0.0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) n = fma(q[c][p], q[c][p], n);
+    const double inv = 1.0 / sqrt(n);
+#pragma unroll
+    for (int c = 0; c < C; ++c) q[c][p] *= inv;
+  }
+#pragma unroll
+  for (int c = 0; c < C; ++c)
+    out[c] = make_float4((float)q[c][0], (float)q[c][1], (float)q[c][2], (float)q[c][P - 1]);
 }
 
 template <int P>
-struct Best {
+struct BestSlot {
   double err;
   uint32_t seed;
   int e;
   int q[P];
 };
 
-template <int C, int P, int NBLK>
+// The filter threshold of a block in its scaled domain (rounded up): a seed
+// whose fp32 residual exceeds it cannot beat the best error.  Once the best
+// error is 0 nothing can (strict <).
+__device__ __forceinline__ float prune_threshold(double best, double ww, double s2) {
+  if (best == 0.0) return -INFINITY;
+  return __double2float_ru((best + kPruneMargin * ww) * s2);
+}
+
+// Exact fp64 scoring of one seed for one block (the seeds the filter could
+// not rule out).  Updates *best on a strictly smaller error; returns the
+// block's new filter threshold.
+template <int C, int P>
+__device__ __noinline__ float score_seed(uint32_t seed, const float* __restrict__ wsrc,
+                                         int nvalid, double ww, double s2, BestSlot<P>* best,
+                                         const double* __restrict__ exact) {
+  double w[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) w[c] = c < nvalid ? (double)wsrc[c] : 0.0;
+  const uint64_t st = seed_stream(seed);
+  const double* ex = exact + (size_t)(seed - 1) * SeedExact<P>::kDoubles;
+  double g[P * P], gi[P * P], b[P], t[P];
+#pragma unroll
+  for (int k = 0; k < P * P; ++k) {
+    g[k] = __ldg(ex + k);
+    gi[k] = __ldg(ex + P * P + k);
+  }
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    double acc = 0.0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) acc = fma(basis_entry<C, P>(st, c, p), w[c], acc);
+    b[p] = acc;
+  }
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    double acc = 0.0;
+#pragma unroll
+    for (int r = 0; r < P; ++r) acc = fma(gi[p * P + r], b[r], acc);
+    t[p] = acc;
+  }
+  // Exponents in descending order: on an exact tie the larger e, met first,
+  // stays.  |t* 2^e| shrinks with e, so once every q rounds to 0 all smaller
+  // exponents give that same candidate (error ||w||^2): the loop ends there.
+  for (int e = 15; e >= 0; --e) {
+    const double sc = (double)(1 << e), inv = 1.0 / (double)(1 << e);
+    double q[P];
+    bool zero = true;
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      q[p] = fmin(fmax(rint(t[p] * sc), -8.0), 7.0);
+      zero = zero && q[p] == 0.0;
+    }
+    // q.b and q^T G q (G symmetric: diagonal once, off-diagonal twice).
+    double qb = 0.0, qgq = 0.0;
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      qb = fma(q[p], b[p], qb);
+      double row = 0.5 * g[p * P + p] * q[p];
+#pragma unroll
+      for (int r = p + 1; r < P; ++r) row = fma(g[p * P + r], q[r], row);
+      qgq = fma(q[p], row, qgq);
+    }
+    const double err = fma(2.0 * inv * inv, qgq, fma(-2.0 * inv, qb, ww));
+    if (err < best->err) {
+      best->err = err;
+      best->seed = seed;
+      best->e = e;
+#pragma unroll
+      for (int p = 0; p < P; ++p) best->q[p] = (int)q[p];
+    }
+    if (zero) break;
+  }
+  return prune_threshold(best->err, ww, s2);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Chunk k of the table (kChunk seeds x C float4, contiguous) into buf.
+template <int C>
+__device__ __forceinline__ void load_chunk(float4* buf, const float4* __restrict__ table, int k,
+                                           int tid) {
+  const float4* src = table + (size_t)k * kChunk * C;
+#pragma unroll
+  for (int i = 0; i < C; ++i) {
+    const int j = tid + i * kEncThreads;  // kChunk * C = C * kEncThreads float4
+    if (SEEDLM_IN_BOUNDS(g_check_flag, (size_t)k * kChunk * C + j, (size_t)kTableRows * C))
+      cp_async16(buf + j, src + j);
+  }
+}
+
+template <int C, int P>
 __global__ void __launch_bounds__(kEncThreads)
 encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int nb,
               int rec_pitch, int e_pitch, uint32_t* __restrict__ rec,
-              uint8_t* __restrict__ eplane, double* __restrict__ err_out, long long n_items) {
-  __shared__ EncChunk<C, P> ch;
-  const int ipr = (nb + NBLK - 1) / NBLK;  // items per row
-  const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+              uint8_t* __restrict__ eplane, double* __restrict__ err_out, long long n_items,
+              const float4* __restrict__ table, const double* __restrict__ exact) {
+  static_assert(kChunk == kEncThreads, "one float4 per thread and basis row");
+  static_assert(kChunk % kGroup == 0, "whole seed groups per chunk");
+  extern __shared__ __align__(16) unsigned char smem[];
+  float4* qbuf = reinterpret_cast<float4*>(smem);  // [2][kChunk * C]
+  BestSlot<P>* slots = reinterpret_cast<BestSlot<P>*>(smem + 2 * kChunk * C * sizeof(float4));
+  const int tid = threadIdx.x;
+  load_chunk<C>(qbuf, table, 0, tid);
+  cp_async_commit();
+
+  const int ipr = (nb + 1) / 2;  // items (block pairs) per row
+  const long long item = (long long)blockIdx.x * kEncThreads + tid;
   const bool active = item < n_items;
   const int row = active ? (int)(item / ipr) : 0;
-  const int b0 = active ? (int)(item - (long long)row * ipr) * NBLK : 0;
+  const int b0 = active ? (int)(item - (long long)row * ipr) * 2 : 0;
 
-  double w[NBLK][C];
-  double ww[NBLK];
-  Best<P> best[NBLK];
+  // Per block: the weights scaled by 2^-E (max |w| in [1, 2)) as (w, w)
+  // pairs, ||w||^2 in fp64 and in the scaled fp32 domain, 2^-2E, the filter
+  // threshold, and where the weights are in W.
+  float2 wd[2][C];
+  float ww32[2], thr[2];
+  double ww64[2], s2[2];
+  const float* wsrc[2];
+  int nvalid[2];
 #pragma unroll
-  for (int k = 0; k < NBLK; ++k) {
-    ww[k] = 0.0;
+  for (int k = 0; k < 2; ++k) {
+    const int blk = b0 + k;
+    const bool valid = active && blk < nb;
+    nvalid[k] = valid ? min(C, cols - blk * C) : 0;
+    wsrc[k] = W + (size_t)row * ldw + (size_t)blk * C;
+    if (nvalid[k] > 0 &&
+        !SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * ldw + (size_t)blk * C + nvalid[k] - 1,
+                          (size_t)(rows - 1) * ldw + cols))
+      nvalid[k] = 0;
+    float w[C];
+    float maxabs = 0.f;
+    double acc = 0.0;
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-      const int col = (b0 + k) * C + c;
-      const bool in = active && b0 + k < nb && col < cols &&
-                      SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * ldw + col,
-                                       (size_t)(rows - 1) * ldw + cols);
-      w[k][c] = in ? (double)W[(size_t)row * ldw + col] : 0.0;
-      ww[k] = fma(w[k][c], w[k][c], ww[k]);
+      w[c] = c < nvalid[k] ? wsrc[k][c] : 0.f;
+      maxabs = fmaxf(maxabs, fabsf(w[c]));
+      acc = fma((double)w[c], (double)w[c], acc);
     }
-    best[k].err = __longlong_as_double(0x7ff0000000000000ll);  // +inf
-    best[k].seed = 1;
-    best[k].e = 15;
+    ww64[k] = acc;
+    const int E = maxabs > 0.f ? ilogbf(maxabs) : 0;
+    s2[k] = ldexp(1.0, -2 * E);
+    float a = 0.f;
 #pragma unroll
-    for (int p = 0; p < P; ++p) best[k].q[p] = 0;
+    for (int c = 0; c < C; ++c) {
+      const float v = scalbnf(w[c], -E);
+      wd[k][c] = make_float2(v, v);
+      a = fmaf(v, v, a);
+    }
+    ww32[k] = a;
+    BestSlot<P>& sl = slots[2 * tid + k];
+    sl.seed = 1;
+    sl.e = 15;
+#pragma unroll
+    for (int p = 0; p < P; ++p) sl.q[p] = 0;
+    if (nvalid[k] == 0 || acc == 0.0 || !isfinite(acc)) {
+      // Nothing to search: an all-zero block's canonical fit is seed 1,
+      // e = 15, q = 0 with error 0 (every candidate ties at 0).
+      sl.err = acc;
+      thr[k] = -INFINITY;
+    } else {
+      sl.err = INFINITY;
+      thr[k] = INFINITY;
+    }
   }
+  // (w0, w1) pairs: the third basis column of C = 8 meets both blocks in one FMA.
+  float2 wp[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) wp[c] = make_float2(wd[0][c].x, wd[1][c].x);
 
-  for (int s0 = 1; s0 <= kNumSeeds; s0 += kSeedChunk) {
-    const int ns = min(kSeedChunk, kNumSeeds + 1 - s0);
-    __syncthreads();  // the previous chunk is no longer read
-    if (threadIdx.x < ns) build_seed<C, P>(ch, threadIdx.x, (uint32_t)(s0 + threadIdx.x));
-    __syncthreads();
-    for (int j = 0; j < ns; ++j) {
-      const uint32_t seed = (uint32_t)(s0 + j);
+  for (int k = 0; k < kChunks; ++k) {
+    cp_async_wait_all();
+    __syncthreads();  // chunk k landed everywhere; chunk k - 1's buffer is free
+    if (k + 1 < kChunks) load_chunk<C>(qbuf + ((k + 1) & 1) * kChunk * C, table, k + 1, tid);
+    cp_async_commit();
+    if (thr[0] == -INFINITY && thr[1] == -INFINITY) continue;
+    const float4* qc = qbuf + (k & 1) * kChunk * C;
+    const int s_first = k * kChunk + 1;
+    const int ns = min(kChunk, kNumSeeds + 1 - s_first);  // the last table row is padding
+    for (int j0 = 0; j0 < kChunk; j0 += kGroup) {
+      // Residuals of kGroup seeds, then one branch for the rare survivors.
+      float r0[kGroup], r1[kGroup];
+      bool any = false;
 #pragma unroll
-      for (int k = 0; k < NBLK; ++k) {
-        double b[P];
+      for (int u = 0; u < kGroup; ++u) {
+        const float4* qs = qc + (j0 + u) * C;
+        if constexpr (P == 3) {
+          float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0;
 #pragma unroll
-        for (int p = 0; p < P; ++p) {
-          double acc = 0.0;
+          for (int c = 0; c < C; ++c) {
+            const float4 q = qs[c];
+            const float2 q01 = make_float2(q.x, q.y), q22 = make_float2(q.z, q.w);
+            a0 = __ffma2_rn(q01, wd[0][c], a0);
+            a1 = __ffma2_rn(q01, wd[1][c], a1);
+            a2 = __ffma2_rn(q22, wp[c], a2);
+          }
+          r0[u] = fmaf(-a0.x, a0.x, fmaf(-a0.y, a0.y, fmaf(-a2.x, a2.x, ww32[0])));
+          r1[u] = fmaf(-a1.x, a1.x, fmaf(-a1.y, a1.y, fmaf(-a2.y, a2.y, ww32[1])));
+        } else {
+          float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
 #pragma unroll
-          for (int c = 0; c < C; ++c) acc = fma(ch.U[j][c * P + p], w[k][c], acc);
-          b[p] = acc;
+          for (int c = 0; c < C; ++c) {
+            const float4 q = qs[c];
+            const float2 q01 = make_float2(q.x, q.y), q23 = make_float2(q.z, q.w);
+            a0 = __ffma2_rn(q01, wd[0][c], a0);
+            a1 = __ffma2_rn(q23, wd[0][c], a1);
+            a2 = __ffma2_rn(q01, wd[1][c], a2);
+            a3 = __ffma2_rn(q23, wd[1][c], a3);
+          }
+          r0[u] = fmaf(-a0.x, a0.x, fmaf(-a0.y, a0.y, fmaf(-a1.x, a1.x, fmaf(-a1.y, a1.y, ww32[0]))));
+          r1[u] = fmaf(-a2.x, a2.x, fmaf(-a2.y, a2.y, fmaf(-a3.x, a3.x, fmaf(-a3.y, a3.y, ww32[1]))));
         }
-        double t[P];
-        double bt = 0.0;
+        // !(r > thr) keeps a NaN residual in play.
+        any = any || !(r0[u] > thr[0]) || !(r1[u] > thr[1]);
+      }
+      if (any) {
+        // Seeds in ascending order, each tested again against the threshold
+        // the previous ones left.
 #pragma unroll
-        for (int p = 0; p < P; ++p) {
-          double acc = 0.0;
-#pragma unroll
-          for (int r = 0; r < P; ++r) acc = fma(ch.Gi[j][p * P + r], b[r], acc);
-          t[p] = acc;
-          bt = fma(b[p], acc, bt);
-        }
-        // No quantised candidate of this seed beats its least-squares
-        // residual ||w||^2 - b.t*; once that is above the best error so far
-        // (beyond fp64 rounding), the seed's exponents need no scoring.
-        if (ww[k] - bt > best[k].err + 1e-13 * ww[k]) continue;
-        // Exponents in descending order: on an exact tie the larger e, met
-        // first, stays.  |t* 2^e| shrinks with e, so once every q rounds to
-        // 0 all smaller exponents give that same candidate (error ||w||^2,
-        // met later): the loop ends there.
-#pragma unroll 4
-        for (int e = 15; e >= 0; --e) {
-          const double sc = (double)(1 << e), inv = 1.0 / (double)(1 << e);
-          double q[P];
-          bool zero = true;
-#pragma unroll
-          for (int p = 0; p < P; ++p) {
-            q[p] = fmin(fmax(rint(t[p] * sc), -8.0), 7.0);
-            zero = zero && q[p] == 0.0;
-          }
-          // q.b and q^T G q (G symmetric: diagonal once, off-diagonal twice).
-          double qb = 0.0, qgq = 0.0;
-#pragma unroll
-          for (int p = 0; p < P; ++p) {
-            qb = fma(q[p], b[p], qb);
-            double row = 0.5 * ch.G[j][p * P + p] * q[p];
-#pragma unroll
-            for (int r = p + 1; r < P; ++r) row = fma(ch.G[j][p * P + r], q[r], row);
-            qgq = fma(q[p], row, qgq);
-          }
-          const double err = fma(2.0 * inv * inv, qgq, fma(-2.0 * inv, qb, ww[k]));
-          if (err < best[k].err) {
-            best[k].err = err;
-            best[k].seed = seed;
-            best[k].e = e;
-#pragma unroll
-            for (int p = 0; p < P; ++p) best[k].q[p] = (int)q[p];
-          }
-          if (zero) break;
+        for (int u = 0; u < kGroup; ++u) {
+          const int j = j0 + u;
+          const uint32_t seed = (uint32_t)(s_first + j);
+          if (j < ns && !(r0[u] > thr[0]))
+            thr[0] = score_seed<C, P>(seed, wsrc[0], nvalid[0], ww64[0], s2[0], &slots[2 * tid], exact);
+          if (j < ns && !(r1[u] > thr[1]))
+            thr[1] = score_seed<C, P>(seed, wsrc[1], nvalid[1], ww64[1], s2[1], &slots[2 * tid + 1],
+                                      exact);
         }
       }
     }
   }
+  cp_async_wait_all();
   if (!active) return;
 
 #pragma unroll
-  for (int k = 0; k < NBLK; ++k) {
+  for (int k = 0; k < 2; ++k) {
     const int blk = b0 + k;
     if (blk >= nb) break;
+    const BestSlot<P>& best = slots[2 * tid + k];
     // The winner's error, computed directly.
-    const uint64_t st = seed_stream(best[k].seed);
-    const double inv = 1.0 / (double)(1 << best[k].e);
+    const uint64_t st = seed_stream(best.seed);
+    const double inv = 1.0 / (double)(1 << best.e);
     double err = 0.0;
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       double what = 0.0;
 #pragma unroll
-      for (int p = 0; p < P; ++p) what = fma(basis_entry<C, P>(st, c, p), (double)best[k].q[p], what);
-      const double d = w[k][c] - what * inv;
+      for (int p = 0; p < P; ++p) what = fma(basis_entry<C, P>(st, c, p), (double)best.q[p], what);
+      const double wc = c < nvalid[k] ? (double)wsrc[k][c] : 0.0;
+      const double d = wc - what * inv;
       err = fma(d, d, err);
     }
-    uint32_t r = best[k].seed << 16;
+    uint32_t r = best.seed << 16;
 #pragma unroll
-    for (int p = 0; p < P; ++p) r |= ((uint32_t)best[k].q[p] & 15u) << (4 * p);
-    if constexpr (C == 8) r |= (uint32_t)best[k].e << 12;
+    for (int p = 0; p < P; ++p) r |= ((uint32_t)best.q[p] & 15u) << (4 * p);
+    if constexpr (C == 8) r |= (uint32_t)best.e << 12;
     if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, blk, rec_pitch))
       rec[(size_t)row * rec_pitch + blk] = r;
     if (err_out && SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * nb + blk, (size_t)rows * nb))
@@ -260,32 +467,50 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
   }
   if constexpr (C == 12) {
     // The pair's exponent byte: block b0 in the low nibble, b0 + 1 (or 0).
-    uint32_t byte = (uint32_t)best[0].e & 15u;
-    if (b0 + 1 < nb) byte |= ((uint32_t)best[1].e & 15u) << 4;
+    uint32_t byte = (uint32_t)slots[2 * tid].e & 15u;
+    if (b0 + 1 < nb) byte |= ((uint32_t)slots[2 * tid + 1].e & 15u) << 4;
     if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, e_pitch))
       eplane[(size_t)row * e_pitch + (b0 >> 1)] = (uint8_t)byte;
   }
 }
 
-template <int C, int P, int NBLK>
+template <int C, int P>
 int launch_encode_t(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
-                    uint8_t* eplane, double* err, cudaStream_t stream) {
-  const long long ipr = (f.nb + NBLK - 1) / NBLK;
+                    uint8_t* eplane, double* err, cudaStream_t stream, const DeviceInfo& dev) {
+  const long long ipr = (f.nb + 1) / 2;
   const long long items = ipr * f.rows;
+  if (items == 0) return SEEDLM_OK;
   const long long grid = (items + kEncThreads - 1) / kEncThreads;
   if (grid > 0x7fffffffll) return SEEDLM_EUNSUPPORTED;
-  encode_kernel<C, P, NBLK><<<(unsigned)grid, kEncThreads, 0, stream>>>(
-      W, ldw, f.rows, f.cols, f.nb, f.rec_pitch, f.e_pitch, rec, eplane, err, items);
+  const size_t smem = 2 * kChunk * C * sizeof(float4) + 2 * kEncThreads * sizeof(BestSlot<P>);
+  int rc = allow_max_smem((const void*)encode_kernel<C, P>, dev);
+  if (rc) return rc;
+  // The seed tables live for this call only (one stream-ordered allocation:
+  // fp32 bases, then fp64 G and G^-1).
+  const size_t basis_bytes = (size_t)kTableRows * C * sizeof(float4);
+  const size_t exact_bytes = (size_t)kTableRows * SeedExact<P>::kDoubles * sizeof(double);
+  unsigned char* tables = nullptr;
+  if ((rc = record_cuda_error(cudaMallocAsync(reinterpret_cast<void**>(&tables),
+                                              basis_bytes + exact_bytes, stream))))
+    return rc;
+  float4* table = reinterpret_cast<float4*>(tables);
+  double* exact = reinterpret_cast<double*>(tables + basis_bytes);
+  basis_table_kernel<C, P><<<kTableRows / 256, 256, 0, stream>>>(table, exact);
   count_launch();
-  return record_cuda_error(cudaGetLastError());
+  encode_kernel<C, P><<<(unsigned)grid, kEncThreads, smem, stream>>>(
+      W, ldw, f.rows, f.cols, f.nb, f.rec_pitch, f.e_pitch, rec, eplane, err, items, table, exact);
+  count_launch();
+  rc = record_cuda_error(cudaGetLastError());
+  const int rc_free = record_cuda_error(cudaFreeAsync(tables, stream));
+  return rc ? rc : rc_free;
 }
 
 }  // namespace
 
 int launch_encode(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
-                  uint8_t* eplane, double* err, cudaStream_t stream) {
-  if (f.C == 8) return launch_encode_t<8, 3, 1>(f, W, ldw, rec, eplane, err, stream);
-  return launch_encode_t<12, 4, 2>(f, W, ldw, rec, eplane, err, stream);
+                  uint8_t* eplane, double* err, cudaStream_t stream, const DeviceInfo& dev) {
+  if (f.C == 8) return launch_encode_t<8, 3>(f, W, ldw, rec, eplane, err, stream, dev);
+  return launch_encode_t<12, 4>(f, W, ldw, rec, eplane, err, stream, dev);
 }
 
 }  // namespace seedlm

@@ -93,6 +93,6 @@ int read_and_clear_tc_error(unsigned int* out);
 int launch_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 int launch_bounds_check(int64_t index, int64_t extent, cudaStream_t stream);
 int launch_encode(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
-                  uint8_t* eplane, double* err, cudaStream_t stream);
+                  uint8_t* eplane, double* err, cudaStream_t stream, const DeviceInfo& dev);
 
 }  // namespace seedlm
