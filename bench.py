@@ -428,19 +428,23 @@ def extras(torch, sl, args):
     del W, m
 
     # Encoder (offline): full seed / coefficient / exponent search of a
-    # Gaussian 1024 x 1024 matrix at 4 bits (131,072 blocks x 65,535 seeds x
-    # 16 exponents), one call after a warm-up call.
+    # Gaussian 4096 x 4096 matrix at 4 and 3 bits (2.1 M / 1.4 M blocks x
+    # 65,535 seeds x 16 exponents), one call after a warm-up call.
     rng = np.random.default_rng(11)
-    We = torch.from_numpy((rng.standard_normal((1024, 1024)) * 0.02).astype(np.float32)).cuda()
-    fe = inputs.make_format(1024, 1024, 8, 3)
-    rec_e = torch.empty((1024, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
-    sl.encode(fe, We, rec_e)
-    ms = time_region(torch, lambda i: sl.encode(fe, We, rec_e), 1)
-    blocks = 1024 * fe["nb"]
-    out["encode_4bit_1024x1024"] = {
-        "ms_per_call": round(ms, 1), "blocks_per_s": round(blocks / (ms / 1e3)),
-        "candidates_per_s_e9": round(blocks * 65535 * 16 / (ms / 1e3) / 1e9, 2)}
-    del We, rec_e
+    We = torch.from_numpy((rng.standard_normal((4096, 4096)) * 0.02).astype(np.float32)).cuda()
+    for bits, (C, P) in ((4, (8, 3)), (3, (12, 4))):
+        fe = inputs.make_format(4096, 4096, C, P)
+        rec_e = torch.empty((4096, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
+        ep_e = (torch.empty((4096, fe["e_pitch"]), dtype=torch.uint8, device="cuda")
+                if P == 4 else None)
+        sl.encode(fe, We, rec_e, ep_e)
+        ms = time_region(torch, lambda i: sl.encode(fe, We, rec_e, ep_e), 1)
+        blocks = 4096 * fe["nb"]
+        out[f"encode_{bits}bit_4096x4096"] = {
+            "ms_per_call": round(ms, 1), "blocks_per_s": round(blocks / (ms / 1e3)),
+            "seeds_per_s_e9": round(blocks * 65535 / (ms / 1e3) / 1e9, 1)}
+        del rec_e, ep_e
+    del We
 
     # Dense fp16 GEMV (in-house) on the 70B layer shapes, 4 rotating copies.
     rng = np.random.default_rng(3)
