@@ -638,6 +638,21 @@ def seedlm_arm(args):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5)},
         "gpu_launches": int(launches),
     }
+    # The same kernel against its instruction-issue bound: blocks per second if
+    # every warp scheduler issued one instruction per cycle at the measured SM
+    # clock, with the kernel's own instruction count per block (ncu, same
+    # source hash as the traffic figure).
+    sm_mhz = result["clocks"].get("sm_mhz")
+    if traffic is not None and traffic.get("thread_instructions_per_block") and sm_mhz:
+        ipb = traffic["thread_instructions_per_block"]
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        peak_bps = sms * 4 * 32 * sm_mhz * 1e6 / ipb
+        got_bps = achieved * 1e9 / 4  # 4 record bytes per 8-weight block
+        result["roofline_issue"] = {
+            "bound": "alu", "achieved": round(got_bps / 1e9, 2), "peak": round(peak_bps / 1e9, 2),
+            "unit": "Gblock/s", "frac": round(got_bps / peak_bps, 4),
+            "thread_instructions_per_block": ipb, "sm_mhz": sm_mhz, "sms": sms,
+            "kernel": "gemv_kernel<8>"}
     del layers, base
     torch.cuda.empty_cache()
     if world == 1 and not args.no_extras:
