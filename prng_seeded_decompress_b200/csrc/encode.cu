@@ -188,12 +188,18 @@ __global__ void __launch_bounds__(256) basis_table_kernel(float4* __restrict__ t
     out[c] = make_float4((float)q[c][0], (float)q[c][1], (float)q[c][2], (float)q[c][P - 1]);
 }
 
+// One block's search state, in shared memory where the whole warp can read
+// it: the best candidate so far, and what exact scoring needs (||w||^2 in
+// fp64, where the weights are, how many of them the row has).
 template <int P>
-struct BestSlot {
+struct BlockSlot {
   double err;
+  double ww;
+  const float* wsrc;
   uint32_t seed;
   int e;
   int q[P];
+  int nvalid;
 };
 
 // The filter threshold of a block in its scaled domain (rounded up): a seed
@@ -204,13 +210,17 @@ __device__ __forceinline__ float prune_threshold(double best, double ww, double 
   return __double2float_ru((best + kPruneMargin * ww) * s2);
 }
 
-// Exact fp64 scoring of one seed for one block (the seeds the filter could
-// not rule out).  Updates *best on a strictly smaller error; returns the
-// block's new filter threshold.
+// A seed's best candidate for one block, scored exactly in fp64: err and
+// (e, q) packed as e | q_p << (4 + 4p) (q as 4-bit two's complement).
+struct Cand {
+  double err;
+  uint32_t eq;
+};
+
 template <int C, int P>
-__device__ __noinline__ float score_seed(uint32_t seed, const float* __restrict__ wsrc,
-                                         int nvalid, double ww, double s2, BestSlot<P>* best,
-                                         const double* __restrict__ exact) {
+__device__ __noinline__ Cand seed_candidate(uint32_t seed, const float* __restrict__ wsrc,
+                                            int nvalid, double ww,
+                                            const double* __restrict__ exact) {
   double w[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) w[c] = c < nvalid ? (double)wsrc[c] : 0.0;
@@ -236,6 +246,7 @@ __device__ __noinline__ float score_seed(uint32_t seed, const float* __restrict_
     for (int r = 0; r < P; ++r) acc = fma(gi[p * P + r], b[r], acc);
     t[p] = acc;
   }
+  Cand best{INFINITY, 15u};
   // Exponents in descending order: on an exact tie the larger e, met first,
   // stays.  |t* 2^e| shrinks with e, so once every q rounds to 0 all smaller
   // exponents give that same candidate (error ||w||^2): the loop ends there.
@@ -259,16 +270,73 @@ __device__ __noinline__ float score_seed(uint32_t seed, const float* __restrict_
       qgq = fma(q[p], row, qgq);
     }
     const double err = fma(2.0 * inv * inv, qgq, fma(-2.0 * inv, qb, ww));
-    if (err < best->err) {
-      best->err = err;
-      best->seed = seed;
-      best->e = e;
+    if (err < best.err) {
+      best.err = err;
+      uint32_t eq = (uint32_t)e;
 #pragma unroll
-      for (int p = 0; p < P; ++p) best->q[p] = (int)q[p];
+      for (int p = 0; p < P; ++p) eq |= ((uint32_t)(int)q[p] & 15u) << (4 + 4 * p);
+      best.eq = eq;
     }
     if (zero) break;
   }
-  return prune_threshold(best->err, ww, s2);
+  return best;
+}
+
+// Per-warp queue of (seed, block) pairs the filter let through, scored 32 at
+// a time with every lane busy.  Entry: seed | lane << 16 | k << 21 (block k
+// of that lane).
+constexpr int kQueue = 96;  // < 32 left over + at most 64 added per seed
+struct WarpQueue {
+  uint32_t ent[kQueue];
+  double err[32];
+  uint32_t eq[32];
+};
+
+// Scores the queued pairs in batches of 32 (all of them if min_batch is 1,
+// else while at least min_batch remain) and merges each result into its
+// block's slot in queue order -- ascending seeds for every block, so a
+// strictly smaller error replaces the best exactly as a sequential scan
+// would.  Called by the whole warp; returns the entries left.
+template <int C, int P>
+__device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
+                                        BlockSlot<P>* wslots, const double* __restrict__ exact,
+                                        int lane) {
+  int base = 0;
+  while (count - base > 0 && count - base >= min_batch) {
+    const int n = min(32, count - base);
+    if (lane < n) {
+      const uint32_t en = wq->ent[base + lane];
+      const BlockSlot<P>& bs = wslots[2 * ((en >> 16) & 31u) + (en >> 21)];
+      const Cand cd = seed_candidate<C, P>(en & 0xffffu, bs.wsrc, bs.nvalid, bs.ww, exact);
+      wq->err[lane] = cd.err;
+      wq->eq[lane] = cd.eq;
+    }
+    __syncwarp();
+    for (int i = 0; i < n; ++i) {
+      const uint32_t en = wq->ent[base + i];
+      if (((en >> 16) & 31u) == (uint32_t)lane) {
+        BlockSlot<P>& bs = wslots[2 * lane + (en >> 21)];
+        if (wq->err[i] < bs.err) {
+          const uint32_t eq = wq->eq[i];
+          bs.err = wq->err[i];
+          bs.seed = en & 0xffffu;
+          bs.e = (int)(eq & 15u);
+#pragma unroll
+          for (int p = 0; p < P; ++p) bs.q[p] = ((int)(eq << (24 - 4 * p))) >> 28;
+        }
+      }
+    }
+    __syncwarp();
+    base += n;
+  }
+  const int left = count - base;
+  if (base > 0) {
+    const uint32_t v = lane < left ? wq->ent[base + lane] : 0u;
+    __syncwarp();
+    if (lane < left) wq->ent[lane] = v;
+  }
+  __syncwarp();
+  return left;
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -305,8 +373,12 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
   static_assert(kChunk % kGroup == 0, "whole seed groups per chunk");
   extern __shared__ __align__(16) unsigned char smem[];
   float4* qbuf = reinterpret_cast<float4*>(smem);  // [2][kChunk * C]
-  BestSlot<P>* slots = reinterpret_cast<BestSlot<P>*>(smem + 2 * kChunk * C * sizeof(float4));
-  const int tid = threadIdx.x;
+  BlockSlot<P>* slots =
+      reinterpret_cast<BlockSlot<P>*>(smem + 2 * kChunk * C * sizeof(float4));  // [threads][2]
+  WarpQueue* queues = reinterpret_cast<WarpQueue*>(slots + 2 * kEncThreads);  // [warps]
+  const int tid = threadIdx.x, lane = tid & 31;
+  WarpQueue* wq = queues + (tid >> 5);
+  BlockSlot<P>* wslots = slots + 2 * (tid & ~31);  // this warp's 64 slots
   load_chunk<C>(qbuf, table, 0, tid);
   cp_async_commit();
 
@@ -354,11 +426,14 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
       a = fmaf(v, v, a);
     }
     ww32[k] = a;
-    BestSlot<P>& sl = slots[2 * tid + k];
+    BlockSlot<P>& sl = slots[2 * tid + k];
     sl.seed = 1;
     sl.e = 15;
 #pragma unroll
     for (int p = 0; p < P; ++p) sl.q[p] = 0;
+    sl.ww = acc;
+    sl.wsrc = wsrc[k];
+    sl.nvalid = nvalid[k];
     if (nvalid[k] == 0 || acc == 0.0 || !isfinite(acc)) {
       // Nothing to search: an all-zero block's canonical fit is seed 1,
       // e = 15, q = 0 with error 0 (every candidate ties at 0).
@@ -373,13 +448,17 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
   float2 wp[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) wp[c] = make_float2(wd[0][c].x, wd[1][c].x);
+  const bool live0 = thr[0] != -INFINITY, live1 = thr[1] != -INFINITY;
+  const unsigned lanes_below = (1u << lane) - 1u;
+  int queued = 0;  // entries in this warp's queue (warp-uniform)
+  __syncwarp();    // the warp's slots are written
 
   for (int k = 0; k < kChunks; ++k) {
     cp_async_wait_all();
     __syncthreads();  // chunk k landed everywhere; chunk k - 1's buffer is free
     if (k + 1 < kChunks) load_chunk<C>(qbuf + ((k + 1) & 1) * kChunk * C, table, k + 1, tid);
     cp_async_commit();
-    if (thr[0] == -INFINITY && thr[1] == -INFINITY) continue;
+    if (__all_sync(0xffffffffu, thr[0] == -INFINITY && thr[1] == -INFINITY)) continue;
     const float4* qc = qbuf + (k & 1) * kChunk * C;
     const int s_first = k * kChunk + 1;
     const int ns = min(kChunk, kNumSeeds + 1 - s_first);  // the last table row is padding
@@ -419,22 +498,34 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
         // !(r > thr) keeps a NaN residual in play.
         any = any || !(r0[u] > thr[0]) || !(r1[u] > thr[1]);
       }
-      if (any) {
-        // Seeds in ascending order, each tested again against the threshold
-        // the previous ones left.
+      if (__any_sync(0xffffffffu, any)) {
+        // Queue the survivors seed by seed (ascending), scoring a batch
+        // whenever 32 are waiting; the thresholds then come from the slots.
 #pragma unroll
         for (int u = 0; u < kGroup; ++u) {
-          const int j = j0 + u;
-          const uint32_t seed = (uint32_t)(s_first + j);
-          if (j < ns && !(r0[u] > thr[0]))
-            thr[0] = score_seed<C, P>(seed, wsrc[0], nvalid[0], ww64[0], s2[0], &slots[2 * tid], exact);
-          if (j < ns && !(r1[u] > thr[1]))
-            thr[1] = score_seed<C, P>(seed, wsrc[1], nvalid[1], ww64[1], s2[1], &slots[2 * tid + 1],
-                                      exact);
+          const uint32_t seed = (uint32_t)(s_first + j0 + u);
+          const bool in = j0 + u < ns;
+          const bool want0 = in && live0 && !(r0[u] > thr[0]);
+          const bool want1 = in && live1 && !(r1[u] > thr[1]);
+          const unsigned m0 = __ballot_sync(0xffffffffu, want0);
+          const unsigned m1 = __ballot_sync(0xffffffffu, want1);
+          if (want0) wq->ent[queued + __popc(m0 & lanes_below)] = seed | ((uint32_t)lane << 16);
+          queued += __popc(m0);
+          if (want1)
+            wq->ent[queued + __popc(m1 & lanes_below)] = seed | ((uint32_t)lane << 16) | (1u << 21);
+          queued += __popc(m1);
+          if (queued >= 32) {
+            __syncwarp();
+            queued = drain_queue<C, P>(wq, queued, 32, wslots, exact, lane);
+            if (live0) thr[0] = prune_threshold(slots[2 * tid].err, ww64[0], s2[0]);
+            if (live1) thr[1] = prune_threshold(slots[2 * tid + 1].err, ww64[1], s2[1]);
+          }
         }
       }
     }
   }
+  __syncwarp();
+  drain_queue<C, P>(wq, queued, 1, wslots, exact, lane);
   cp_async_wait_all();
   if (!active) return;
 
@@ -442,7 +533,7 @@ encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int 
   for (int k = 0; k < 2; ++k) {
     const int blk = b0 + k;
     if (blk >= nb) break;
-    const BestSlot<P>& best = slots[2 * tid + k];
+    const BlockSlot<P>& best = slots[2 * tid + k];
     // The winner's error, computed directly.
     const uint64_t st = seed_stream(best.seed);
     const double inv = 1.0 / (double)(1 << best.e);
@@ -482,7 +573,8 @@ int launch_encode_t(const seedlm_format& f, const float* W, int64_t ldw, uint32_
   if (items == 0) return SEEDLM_OK;
   const long long grid = (items + kEncThreads - 1) / kEncThreads;
   if (grid > 0x7fffffffll) return SEEDLM_EUNSUPPORTED;
-  const size_t smem = 2 * kChunk * C * sizeof(float4) + 2 * kEncThreads * sizeof(BestSlot<P>);
+  const size_t smem = 2 * kChunk * C * sizeof(float4) + 2 * kEncThreads * sizeof(BlockSlot<P>) +
+                      (kEncThreads / 32) * sizeof(WarpQueue);
   int rc = allow_max_smem((const void*)encode_kernel<C, P>, dev);
   if (rc) return rc;
   // The seed tables live for this call only (one stream-ordered allocation:
