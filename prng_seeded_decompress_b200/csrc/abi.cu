@@ -207,6 +207,8 @@ int seedlm_device_error(int* flag) {
   unsigned int v = 0;
   if ((rc = read_and_clear_tc_error(&v))) return rc;
   int out = v ? 1 : 0;
+  if ((rc = read_and_clear_encode_error(&v))) return rc;
+  if (v) out |= 1;
   // Bounds violations recorded by a checked build (always 0 otherwise).
   int (*const readers[])(unsigned int*) = {read_and_clear_check_gemv, read_and_clear_check_decompress,
                                            read_and_clear_check_gemm_tc, read_and_clear_check_encode,

@@ -18,60 +18,49 @@
 // largest exponent.  A tail block (cols not a multiple of C) is fitted with
 // its missing weights taken as zero.
 //
-// Two kernels.  basis_table_kernel computes, once per call, an orthonormal
-// basis Q(s) of every seed's column space (Gram-Schmidt in fp64, each column
-// orthogonalised twice) and stores it rounded to fp32: one float4 per row c
-// of U, (Q[c][0], Q[c][1], Q[c][2], Q[c][3]) for P = 4 and
-// (Q[c][0], Q[c][1], Q[c][2], Q[c][2]) for P = 3.
+// Two kernels.  seed_table_kernel computes, once per call and for every seed,
+// G (exact in fp64: U's entries are k / 32768) and G^-1, and an orthonormal
+// basis Q(s) of U(s)'s column space (Gram-Schmidt in fp64, each column
+// orthogonalised twice), stored as the B operand of the tensor-core filter.
 //
-// encode_kernel: one thread owns two neighbouring blocks of a row (for C = 12
-// the two that share an exponent byte).  A CTA streams the table through
-// shared memory in chunks of 128 seeds (cp.async, double-buffered), and for
-// every seed each thread first evaluates, in fp32, the least-squares residual
-//   r(s) = ||w||^2 - ||Q(s)^T w||^2,
-// a lower bound on the error of every quantised candidate of that seed.  Only
-// when r(s) is not above the block's best error so far plus a margin does the
-// thread score the seed exactly (score_seed: fp64, U, G exact, G^-1 by
-// Gauss-Jordan, the exponents in descending order with the expansion
-//   err = ||w||^2 - 2^(1-e) q.(U^T w) + 2^(-2e) q^T G q ).
-// On Gaussian blocks about 3 in 10^4 seeds get that far, so the search costs
-// one fp32 projection per seed and block: 3 (C = 8) or 4 (C = 12) packed
-// fp32x2 FMAs per basis row for both blocks, on a row read once.
+// encode_tc_kernel: a least-squares filter on the tensor cores, then exact
+// scoring of the few seeds it cannot rule out.  For every block and seed the
+// residual r(s) = ||w||^2 - ||Q(s)^T w||^2 is a lower bound on the error of
+// every quantised candidate of that seed; only a seed whose residual is not
+// above the block's best error so far plus a margin is scored exactly
+// (seed_candidate: fp64, t* = G^-1 U^T w, the exponents in descending order
+// with err = ||w||^2 - 2^(1-e) q.(U^T w) + 2^(-2e) q^T G q).  On Gaussian
+// blocks about 3 in 10^4 seeds get that far.  The projections Q(s)^T w come
+// from tcgen05 MMAs (description at the kernel); the exact scoring runs in
+// warp-wide batches.
 //
-// The filter never changes the result.  The block is scaled by 2^-E (exact)
-// so that max|w| lies in [1, 2).  With u = 2^-24, each fp32 coordinate of
-// Q^T w is within (C + 1) u ||w|| of the exact one (C fused products, plus
-// the rounding of Q to fp32; the columns of Q have unit norm), so the squared
-// norm is within about 2 sqrt(P) (C + 1) u ||w||^2 + P u ||w||^2, and ||w||^2
-// in fp32 within C u ||w||^2: |r_fp32 - r| < 5e-6 ||w||^2 for both formats.
-// The basis itself is orthonormal to fp64 rounding, and spans U(s)'s column
-// space to within kappa(U) 2^-53 < 1e-10 (kappa(U) < 4e5 over all seeds), so
-// a seed is skipped only if r_fp32 > best + 3e-5 ||w||^2, where no candidate
-// of it can reach the best error (candidates are compared with strict <).
-// The winner's error is recomputed directly at the end.
+// The filter never changes the result: a seed is skipped only when its
+// residual, computed within a proven error bound, exceeds the best error by
+// more than that bound, so none of its candidates can reach the best error
+// (candidates replace the best only on a strictly smaller error).  The
+// winner's error is recomputed directly at the end.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
+#include "tcgen05.cuh"
 
 namespace seedlm {
 
 SEEDLM_CHECK_FLAG(encode)
 
+// Set when a bounded wait of the search gave up.
+__device__ unsigned int g_enc_error = 0;
+
 namespace {
 
-constexpr int kEncThreads = 128;
 constexpr int kNumSeeds = 65535;
 constexpr int kTableRows = 65536;  // row i holds seed i + 1; the last row is zero padding
-constexpr int kChunk = 128;        // seeds per shared-memory chunk
-constexpr int kChunks = kTableRows / kChunk;
-constexpr double kPruneMargin = 3e-5;  // relative to ||w||^2, six times the fp32 error bound
-#ifndef SEEDLM_ENC_GROUP
-#define SEEDLM_ENC_GROUP 4
-#endif
-constexpr int kGroup = SEEDLM_ENC_GROUP;  // seeds tested per survivor branch
+constexpr double kPruneMargin = 2e-4;  // relative to ||w||^2, ten times the filter's error bound
+constexpr uint64_t kEncWaitLimit = 2000000000ull;  // ns a hand-over wait may take
 
 // The seed's bit stream, bits [0, 64): state_k = bits [k, k + 16).
 __device__ __forceinline__ uint64_t seed_stream(uint32_t seed) {
@@ -126,68 +115,6 @@ struct SeedExact {
   static_assert(kDoubles >= 2 * P * P, "G and G^-1 fit one row");
 };
 
-// Row i of the tables: the orthonormal basis of seed i + 1, one float4 per
-// row c of U (see the file comment), and its G and G^-1.
-template <int C, int P>
-__global__ void __launch_bounds__(256) basis_table_kernel(float4* __restrict__ table,
-                                                          double* __restrict__ exact) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= kTableRows) return;
-  float4* out = table + (size_t)i * C;
-  if (i >= kNumSeeds) {
-#pragma unroll
-    for (int c = 0; c < C; ++c) out[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  const uint64_t st = seed_stream((uint32_t)(i + 1));
-  double q[C][P];
-#pragma unroll
-  for (int c = 0; c < C; ++c)
-#pragma unroll
-    for (int p = 0; p < P; ++p) q[c][p] = basis_entry<C, P>(st, c, p);
-  {
-    double g[P * P], gi[P * P];
-#pragma unroll
-    for (int p = 0; p < P; ++p)
-#pragma unroll
-      for (int r = 0; r < P; ++r) {
-        double acc = 0.0;
-#pragma unroll
-        for (int c = 0; c < C; ++c) acc = fma(q[c][p], q[c][r], acc);  // exact
-        g[p * P + r] = acc;
-      }
-    spd_inverse<P>(g, gi);
-    double* ex = exact + (size_t)i * SeedExact<P>::kDoubles;
-#pragma unroll
-    for (int k = 0; k < P * P; ++k) {
-      ex[k] = g[k];
-      ex[P * P + k] = gi[k];
-    }
-  }
-#pragma unroll
-  for (int p = 0; p < P; ++p) {
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-      for (int j = 0; j < p; ++j) {
-        double d = 0.0;
-#pragma unroll
-        for (int c = 0; c < C; ++c) d = fma(q[c][j], q[c][p], d);
-#pragma unroll
-        for (int c = 0; c < C; ++c) q[c][p] = fma(-d, q[c][j], q[c][p]);
-      }
-    double n = 0.0;
-#pragma unroll
-    for (int c = 0; c < C; ++c) n = fma(q[c][p], q[c][p], n);
-    const double inv = 1.0 / sqrt(n);
-#pragma unroll
-    for (int c = 0; c < C; ++c) q[c][p] *= inv;
-  }
-#pragma unroll
-  for (int c = 0; c < C; ++c)
-    out[c] = make_float4((float)q[c][0], (float)q[c][1], (float)q[c][2], (float)q[c][P - 1]);
-}
-
 // One block's search state, in shared memory where the whole warp can read
 // it: the best candidate so far, and what exact scoring needs (||w||^2 in
 // fp64, where the weights are, how many of them the row has).
@@ -203,8 +130,8 @@ struct BlockSlot {
 };
 
 // The filter threshold of a block in its scaled domain (rounded up): a seed
-// whose fp32 residual exceeds it cannot beat the best error.  Once the best
-// error is 0 nothing can (strict <).
+// whose residual exceeds it cannot beat the best error.  Once the best error
+// is 0 nothing can (strict <).
 __device__ __forceinline__ float prune_threshold(double best, double ww, double s2) {
   if (best == 0.0) return -INFINITY;
   return __double2float_ru((best + kPruneMargin * ww) * s2);
@@ -283,9 +210,9 @@ __device__ __noinline__ Cand seed_candidate(uint32_t seed, const float* __restri
 }
 
 // Per-warp queue of (seed, block) pairs the filter let through, scored 32 at
-// a time with every lane busy.  Entry: seed | lane << 16 | k << 21 (block k
-// of that lane).
-constexpr int kQueue = 96;  // < 32 left over + at most 64 added per seed
+// a time with every lane busy.  Entry: seed | lane << 16 (the block of that
+// lane).
+constexpr int kQueue = 64;  // < 32 left over + at most 32 added per seed
 struct WarpQueue {
   uint32_t ent[kQueue];
   double err[32];
@@ -306,7 +233,7 @@ __device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
     const int n = min(32, count - base);
     if (lane < n) {
       const uint32_t en = wq->ent[base + lane];
-      const BlockSlot<P>& bs = wslots[2 * ((en >> 16) & 31u) + (en >> 21)];
+      const BlockSlot<P>& bs = wslots[(en >> 16) & 31u];
       const Cand cd = seed_candidate<C, P>(en & 0xffffu, bs.wsrc, bs.nvalid, bs.ww, exact);
       wq->err[lane] = cd.err;
       wq->eq[lane] = cd.eq;
@@ -315,7 +242,7 @@ __device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
     for (int i = 0; i < n; ++i) {
       const uint32_t en = wq->ent[base + i];
       if (((en >> 16) & 31u) == (uint32_t)lane) {
-        BlockSlot<P>& bs = wslots[2 * lane + (en >> 21)];
+        BlockSlot<P>& bs = wslots[lane];
         if (wq->err[i] < bs.err) {
           const uint32_t eq = wq->eq[i];
           bs.err = wq->err[i];
@@ -339,258 +266,487 @@ __device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
   return left;
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
+// ---------------------------------------------------------------- tensor-core filter
+//
+// The projections on the tensor cores: D[block][(p, s)] = sum_c w[c] Q(s)[c][p]
+// for 128 blocks (the TMEM lanes) against 32 seeds at a time, kind::f16 with
+// fp32 accumulation, every operand split exactly into an fp16 high part and
+// an fp16 rest: D = A_hi B_hi + A_hi B_lo + A_lo B_hi.  For C = 8 the two B
+// parts share one K = 16 row ([Q_hi | Q_lo] against [w_hi | w_hi] and
+// [w_lo | 0]), so a stage is two MMAs; for C = 12 (K padded to 16) three.
+// The block is scaled by 2^-E (exact) so that max|w| lies in [1, 2), and
+// |Q| <= 1.  The dropped A_lo B_lo term and the fp16 rounding of the rests
+// are below 2^-22 of each product (plus 2^-25 absolute, fp16's smallest
+// step); the accumulation adds at most about 20 fp32 roundings of
+// sum_c |w_c Q_cp| <= ||w||, so each coordinate is within 4e-6 ||w||, and
+// with ||w||^2 in fp32 and the final subtraction the residual is within
+// 2e-5 ||w||^2.  Q itself is orthonormal to fp64 rounding and spans U(s)'s
+// column space to within kappa(U) 2^-53 < 1e-10 (kappa(U) < 4e5 over all
+// seeds).  A seed is skipped when r > best + 2e-4 ||w||^2.
+//
+// Warps 0-3 (one TMEM lane quarter each, one block per thread) write A,
+// read each stage's 32 x P accumulator columns and test the residuals
+// against the threshold, queueing survivors for exact scoring; warp 4 issues
+// the MMAs (one elected lane); warp 5 copies the B stages, precomputed in the
+// MMA's shared-memory layout, with bulk copies.  All hand-overs are
+// mbarriers with bounded waits.
+
+template <int C>
+struct TcEnc {
+  static constexpr int P = (C == 8) ? 3 : 4;
+  static constexpr int kSeeds = 32;                    // seeds per stage
+  static constexpr int kStages = kTableRows / kSeeds;  // per sweep
+  static constexpr int N = kSeeds * P;                 // MMA columns: (p, s), p-major
+  static constexpr int kPiecesB = (C == 8) ? 1 : 2;
+  static constexpr int kSlabBytes = N * 16 * 2;        // one N x 16 fp16 operand
+  static constexpr int kStageBytes = kSlabBytes * kPiecesB;
+  static constexpr int kBS = (C == 8) ? 8 : 4;         // B stages in shared memory
+  static constexpr int kDS = 2;                        // accumulator stages in TMEM
+  static constexpr int kACols = 16;                    // A: two pieces of 8 columns
+  static constexpr int kTmemCols = (kACols + kDS * N <= 256) ? 256 : 512;
+  static constexpr int kCtasPerSm = 512 / kTmemCols;
+  static_assert(kACols + kDS * N <= kTmemCols, "TMEM budget");
+  static constexpr int kThreads = 6 * 32;
+  static constexpr int kMmaWarp = 4, kLoaderWarp = 5;
+  static_assert(N % 16 == 0 && N <= 256, "M = 128 MMA shape");
+};
+
+// Byte offset of element (n, k) in an N x 16 fp16 operand, K-major core
+// matrices (8 rows x 16 bytes; K neighbours 128 B apart, 8-row groups 256 B).
+__host__ __device__ constexpr int slab16_byte(int n, int k) {
+  return (n >> 3) * 256 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
 }
 
-// Chunk k of the table (kChunk seeds x C float4, contiguous) into buf.
-template <int C>
-__device__ __forceinline__ void load_chunk(float4* buf, const float4* __restrict__ table, int k,
-                                           int tid) {
-  const float4* src = table + (size_t)k * kChunk * C;
+// Row i of the tables (seed i + 1): G = U^T U and G^-1 for exact scoring,
+// and the orthonormal basis split into fp16 high parts and rests at
+// (n = p * 32 + s, k) of its stage's B operand(s).
+template <int C, int P>
+__global__ void __launch_bounds__(256) seed_table_kernel(unsigned char* __restrict__ btab,
+                                                         double* __restrict__ exact) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= kTableRows) return;
+  using T = TcEnc<C>;
+  unsigned char* stage = btab + (size_t)(i / T::kSeeds) * T::kStageBytes;
+  const int s = i % T::kSeeds;
+  double q[C][P];
+  if (i < kNumSeeds) {
+    const uint64_t st = seed_stream((uint32_t)(i + 1));
 #pragma unroll
-  for (int i = 0; i < C; ++i) {
-    const int j = tid + i * kEncThreads;  // kChunk * C = C * kEncThreads float4
-    if (SEEDLM_IN_BOUNDS(g_check_flag, (size_t)k * kChunk * C + j, (size_t)kTableRows * C))
-      cp_async16(buf + j, src + j);
+    for (int c = 0; c < C; ++c)
+#pragma unroll
+      for (int p = 0; p < P; ++p) q[c][p] = basis_entry<C, P>(st, c, p);
+    {
+      double g[P * P], gi[P * P];
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int r = 0; r < P; ++r) {
+          double acc = 0.0;
+#pragma unroll
+          for (int c = 0; c < C; ++c) acc = fma(q[c][p], q[c][r], acc);  // exact
+          g[p * P + r] = acc;
+        }
+      spd_inverse<P>(g, gi);
+      double* ex = exact + (size_t)i * SeedExact<P>::kDoubles;
+#pragma unroll
+      for (int k = 0; k < P * P; ++k) {
+        ex[k] = g[k];
+        ex[P * P + k] = gi[k];
+      }
+    }
+    // Gram-Schmidt, each column orthogonalised twice against the previous ones.
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+        for (int j = 0; j < p; ++j) {
+          double d = 0.0;
+#pragma unroll
+          for (int c = 0; c < C; ++c) d = fma(q[c][j], q[c][p], d);
+#pragma unroll
+          for (int c = 0; c < C; ++c) q[c][p] = fma(-d, q[c][j], q[c][p]);
+        }
+      double n = 0.0;
+#pragma unroll
+      for (int c = 0; c < C; ++c) n = fma(q[c][p], q[c][p], n);
+      const double inv = 1.0 / sqrt(n);
+#pragma unroll
+      for (int c = 0; c < C; ++c) q[c][p] *= inv;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < C; ++c)
+#pragma unroll
+      for (int p = 0; p < P; ++p) q[c][p] = 0.0;
   }
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    const int n = p * T::kSeeds + s;
+    __half hi[16], lo[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) hi[k] = lo[k] = __float2half_rn(0.f);
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      hi[c] = __double2half(q[c][p]);
+      lo[c] = __double2half(q[c][p] - (double)__half2float(hi[c]));
+    }
+    if constexpr (C == 8) {
+      // One operand: k < 8 the high parts, k >= 8 the rests.
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        *reinterpret_cast<__half*>(stage + slab16_byte(n, k)) = (k < 8) ? hi[k] : lo[k - 8];
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        *reinterpret_cast<__half*>(stage + slab16_byte(n, k)) = hi[k];
+        *reinterpret_cast<__half*>(stage + T::kSlabBytes + slab16_byte(n, k)) = lo[k];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
 template <int C, int P>
-__global__ void __launch_bounds__(kEncThreads)
-encode_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int nb,
-              int rec_pitch, int e_pitch, uint32_t* __restrict__ rec,
-              uint8_t* __restrict__ eplane, double* __restrict__ err_out, long long n_items,
-              const float4* __restrict__ table, const double* __restrict__ exact) {
-  static_assert(kChunk == kEncThreads, "one float4 per thread and basis row");
-  static_assert(kChunk % kGroup == 0, "whole seed groups per chunk");
+__global__ void __launch_bounds__(TcEnc<C>::kThreads)
+encode_tc_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int nb,
+                 int rec_pitch, int e_pitch, uint32_t* __restrict__ rec,
+                 uint8_t* __restrict__ eplane, double* __restrict__ err_out, long long n_items,
+                 int tiles, const unsigned char* __restrict__ btab,
+                 const double* __restrict__ exact) {
+  using T = TcEnc<C>;
+  constexpr int BS = T::kBS, DS = T::kDS, N = T::N;
   extern __shared__ __align__(16) unsigned char smem[];
-  float4* qbuf = reinterpret_cast<float4*>(smem);  // [2][kChunk * C]
-  BlockSlot<P>* slots =
-      reinterpret_cast<BlockSlot<P>*>(smem + 2 * kChunk * C * sizeof(float4));  // [threads][2]
-  WarpQueue* queues = reinterpret_cast<WarpQueue*>(slots + 2 * kEncThreads);  // [warps]
-  const int tid = threadIdx.x, lane = tid & 31;
-  WarpQueue* wq = queues + (tid >> 5);
-  BlockSlot<P>* wslots = slots + 2 * (tid & ~31);  // this warp's 64 slots
-  load_chunk<C>(qbuf, table, 0, tid);
-  cp_async_commit();
-
-  const int ipr = (nb + 1) / 2;  // items (block pairs) per row
-  const long long item = (long long)blockIdx.x * kEncThreads + tid;
-  const bool active = item < n_items;
-  const int row = active ? (int)(item / ipr) : 0;
-  const int b0 = active ? (int)(item - (long long)row * ipr) * 2 : 0;
-
-  // Per block: the weights scaled by 2^-E (max |w| in [1, 2)) as (w, w)
-  // pairs, ||w||^2 in fp64 and in the scaled fp32 domain, 2^-2E, the filter
-  // threshold, and where the weights are in W.
-  float2 wd[2][C];
-  float ww32[2], thr[2];
-  double ww64[2], s2[2];
-  const float* wsrc[2];
-  int nvalid[2];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int blk = b0 + k;
-    const bool valid = active && blk < nb;
-    nvalid[k] = valid ? min(C, cols - blk * C) : 0;
-    wsrc[k] = W + (size_t)row * ldw + (size_t)blk * C;
-    if (nvalid[k] > 0 &&
-        !SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * ldw + (size_t)blk * C + nvalid[k] - 1,
-                          (size_t)(rows - 1) * ldw + cols))
-      nvalid[k] = 0;
-    float w[C];
-    float maxabs = 0.f;
-    double acc = 0.0;
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-      w[c] = c < nvalid[k] ? wsrc[k][c] : 0.f;
-      maxabs = fmaxf(maxabs, fabsf(w[c]));
-      acc = fma((double)w[c], (double)w[c], acc);
+  unsigned char* bring = smem;  // [BS][kStageBytes]
+  BlockSlot<P>* slots = reinterpret_cast<BlockSlot<P>*>(smem + BS * T::kStageBytes);  // [128]
+  WarpQueue* queues = reinterpret_cast<WarpQueue*>(slots + 128);                      // [4]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(queues + 4);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * BS + 2 * DS + 1);  // TMEM base, abort
+  const uint32_t bar0 = tc::smem_u32(bars);
+  auto bfull = [&](int b) { return bar0 + 8 * b; };
+  auto bempty = [&](int b) { return bar0 + 8 * (BS + b); };
+  auto dfull = [&](int d) { return bar0 + 8 * (2 * BS + d); };
+  auto dempty = [&](int d) { return bar0 + 8 * (2 * BS + DS + d); };
+  const uint32_t afull = bar0 + 8 * (2 * BS + 2 * DS);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (!SEEDLM_IN_BOUNDS(g_check_flag,
+                        (size_t)(reinterpret_cast<unsigned char*>(tslot + 2) - smem) - 1,
+                        seedlm_dynamic_smem_bytes()))
+    return;
+  if (tid == 0) {
+    for (int b = 0; b < BS; ++b) {
+      tc::mbar_init(bfull(b), 1);
+      tc::mbar_init(bempty(b), 1);
     }
-    ww64[k] = acc;
-    const int E = maxabs > 0.f ? ilogbf(maxabs) : 0;
-    s2[k] = ldexp(1.0, -2 * E);
-    float a = 0.f;
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-      const float v = scalbnf(w[c], -E);
-      wd[k][c] = make_float2(v, v);
-      a = fmaf(v, v, a);
+    for (int d = 0; d < DS; ++d) {
+      tc::mbar_init(dfull(d), 1);
+      tc::mbar_init(dempty(d), 4);
     }
-    ww32[k] = a;
-    BlockSlot<P>& sl = slots[2 * tid + k];
-    sl.seed = 1;
-    sl.e = 15;
-#pragma unroll
-    for (int p = 0; p < P; ++p) sl.q[p] = 0;
-    sl.ww = acc;
-    sl.wsrc = wsrc[k];
-    sl.nvalid = nvalid[k];
-    if (nvalid[k] == 0 || acc == 0.0 || !isfinite(acc)) {
-      // Nothing to search: an all-zero block's canonical fit is seed 1,
-      // e = 15, q = 0 with error 0 (every candidate ties at 0).
-      sl.err = acc;
-      thr[k] = -INFINITY;
-    } else {
-      sl.err = INFINITY;
-      thr[k] = INFINITY;
-    }
+    tc::mbar_init(afull, 4);
+    tc::fence_mbar_init();
+    tslot[1] = 0u;
   }
-  // (w0, w1) pairs: the third basis column of C = 8 meets both blocks in one FMA.
-  float2 wp[C];
-#pragma unroll
-  for (int c = 0; c < C; ++c) wp[c] = make_float2(wd[0][c].x, wd[1][c].x);
-  const bool live0 = thr[0] != -INFINITY, live1 = thr[1] != -INFINITY;
-  const unsigned lanes_below = (1u << lane) - 1u;
-  int queued = 0;  // entries in this warp's queue (warp-uniform)
-  __syncwarp();    // the warp's slots are written
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tslot), T::kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tslot[0];
+  volatile uint32_t* abort_flag = tslot + 1;
+  bool ok = true;
+  const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int total = my_tiles * T::kStages;  // stages this CTA runs
 
-  for (int k = 0; k < kChunks; ++k) {
-    cp_async_wait_all();
-    __syncthreads();  // chunk k landed everywhere; chunk k - 1's buffer is free
-    if (k + 1 < kChunks) load_chunk<C>(qbuf + ((k + 1) & 1) * kChunk * C, table, k + 1, tid);
-    cp_async_commit();
-    if (__all_sync(0xffffffffu, thr[0] == -INFINITY && thr[1] == -INFINITY)) continue;
-    const float4* qc = qbuf + (k & 1) * kChunk * C;
-    const int s_first = k * kChunk + 1;
-    const int ns = min(kChunk, kNumSeeds + 1 - s_first);  // the last table row is padding
-    for (int j0 = 0; j0 < kChunk; j0 += kGroup) {
-      // Residuals of kGroup seeds, then one branch for the rare survivors.
-      float r0[kGroup], r1[kGroup];
-      bool any = false;
-#pragma unroll
-      for (int u = 0; u < kGroup; ++u) {
-        const float4* qs = qc + (j0 + u) * C;
-        if constexpr (P == 3) {
-          float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0;
-#pragma unroll
-          for (int c = 0; c < C; ++c) {
-            const float4 q = qs[c];
-            const float2 q01 = make_float2(q.x, q.y), q22 = make_float2(q.z, q.w);
-            a0 = __ffma2_rn(q01, wd[0][c], a0);
-            a1 = __ffma2_rn(q01, wd[1][c], a1);
-            a2 = __ffma2_rn(q22, wp[c], a2);
-          }
-          r0[u] = fmaf(-a0.x, a0.x, fmaf(-a0.y, a0.y, fmaf(-a2.x, a2.x, ww32[0])));
-          r1[u] = fmaf(-a1.x, a1.x, fmaf(-a1.y, a1.y, fmaf(-a2.y, a2.y, ww32[1])));
+  if (warp == T::kLoaderWarp) {
+    if (lane == 0) {
+      for (int gs = 0; gs < total; ++gs) {
+        const int b = gs % BS, g = gs % T::kStages;
+        if (gs >= BS) ok = tc::mbar_spin_or_abort(bempty(b), ((gs / BS) - 1) & 1, kEncWaitLimit, abort_flag) && ok;
+        if (SEEDLM_IN_BOUNDS(g_check_flag, g, T::kStages)) {
+          tc::mbar_arrive_expect_tx(bfull(b), T::kStageBytes);
+          tc::bulk_g2s(tc::smem_u32(bring + b * T::kStageBytes), btab + (size_t)g * T::kStageBytes,
+                       T::kStageBytes, bfull(b));
         } else {
-          float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-#pragma unroll
-          for (int c = 0; c < C; ++c) {
-            const float4 q = qs[c];
-            const float2 q01 = make_float2(q.x, q.y), q23 = make_float2(q.z, q.w);
-            a0 = __ffma2_rn(q01, wd[0][c], a0);
-            a1 = __ffma2_rn(q23, wd[0][c], a1);
-            a2 = __ffma2_rn(q01, wd[1][c], a2);
-            a3 = __ffma2_rn(q23, wd[1][c], a3);
-          }
-          r0[u] = fmaf(-a0.x, a0.x, fmaf(-a0.y, a0.y, fmaf(-a1.x, a1.x, fmaf(-a1.y, a1.y, ww32[0]))));
-          r1[u] = fmaf(-a2.x, a2.x, fmaf(-a2.y, a2.y, fmaf(-a3.x, a3.x, fmaf(-a3.y, a3.y, ww32[1]))));
+          tc::mbar_arrive(bfull(b));
         }
-        // !(r > thr) keeps a NaN residual in play.
-        any = any || !(r0[u] > thr[0]) || !(r1[u] > thr[1]);
       }
-      if (__any_sync(0xffffffffu, any)) {
-        // Queue the survivors seed by seed (ascending), scoring a batch
-        // whenever 32 are waiting; the thresholds then come from the slots.
-#pragma unroll
-        for (int u = 0; u < kGroup; ++u) {
-          const uint32_t seed = (uint32_t)(s_first + j0 + u);
-          const bool in = j0 + u < ns;
-          const bool want0 = in && live0 && !(r0[u] > thr[0]);
-          const bool want1 = in && live1 && !(r1[u] > thr[1]);
-          const unsigned m0 = __ballot_sync(0xffffffffu, want0);
-          const unsigned m1 = __ballot_sync(0xffffffffu, want1);
-          if (want0) wq->ent[queued + __popc(m0 & lanes_below)] = seed | ((uint32_t)lane << 16);
-          queued += __popc(m0);
-          if (want1)
-            wq->ent[queued + __popc(m1 & lanes_below)] = seed | ((uint32_t)lane << 16) | (1u << 21);
-          queued += __popc(m1);
-          if (queued >= 32) {
-            __syncwarp();
-            queued = drain_queue<C, P>(wq, queued, 32, wslots, exact, lane);
-            if (live0) thr[0] = prune_threshold(slots[2 * tid].err, ww64[0], s2[0]);
-            if (live1) thr[1] = prune_threshold(slots[2 * tid + 1].err, ww64[1], s2[1]);
-          }
-        }
+      // Every copy has landed before the CTA may exit.
+      for (int k = 0; k < BS && k < total; ++k) {
+        const int gs = total - 1 - k;
+        ok = tc::mbar_wait(bfull(gs % BS), (gs / BS) & 1, kEncWaitLimit) && ok;
       }
     }
-  }
-  __syncwarp();
-  drain_queue<C, P>(wq, queued, 1, wslots, exact, lane);
-  cp_async_wait_all();
-  if (!active) return;
+    __syncwarp();
+  } else if (warp == T::kMmaWarp) {
+    const uint32_t idesc = tc::idesc_f16(N, 0);
+    for (int gs = 0; gs < total; ++gs) {
+      const int b = gs % BS, d = gs % DS;
+      if (gs % T::kStages == 0)  // a new tile: its A pieces are in TMEM
+        ok = tc::mbar_spin_or_abort(afull, (gs / T::kStages) & 1, kEncWaitLimit, abort_flag) && ok;
+      ok = tc::mbar_spin_or_abort(bfull(b), (gs / BS) & 1, kEncWaitLimit, abort_flag) && ok;
+      if (gs >= DS) ok = tc::mbar_spin_or_abort(dempty(d), ((gs / DS) - 1) & 1, kEncWaitLimit, abort_flag) && ok;
+      __syncwarp();
+      tc::fence_after_sync();
+      const uint32_t dt = tmem + T::kACols + d * N;
+      const uint32_t sb = tc::smem_u32(bring + b * T::kStageBytes);
+      const uint64_t bhi = tc::smem_desc(sb, 128, 256);
+      if constexpr (C == 8) {
+        tc::mma_f16_ts_warp(dt, tmem, bhi, idesc, 0u);      // [w_hi | w_hi] . [Q_hi | Q_lo]
+        tc::mma_f16_ts_warp(dt, tmem + 8, bhi, idesc, 1u);  // [w_lo | 0] . [Q_hi | Q_lo]
+      } else {
+        const uint64_t blo = tc::smem_desc(sb + T::kSlabBytes, 128, 256);
+        tc::mma_f16_ts_warp(dt, tmem, bhi, idesc, 0u);
+        tc::mma_f16_ts_warp(dt, tmem, blo, idesc, 1u);
+        tc::mma_f16_ts_warp(dt, tmem + 8, bhi, idesc, 1u);
+      }
+      tc::mma_commit_warp(bempty(b));
+      tc::mma_commit_warp(dfull(d));
+    }
+    // The last commits have arrived before the CTA may exit.
+    for (int k = 0; k < BS && k < total; ++k) {
+      const int gs = total - 1 - k;
+      ok = tc::mbar_wait(bempty(gs % BS), (gs / BS) & 1, kEncWaitLimit) && ok;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue: one block per thread
+    const unsigned lanes_below = (1u << lane) - 1u;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    WarpQueue* wq = queues + warp;
+    BlockSlot<P>* wslots = slots + 32 * warp;
+    BlockSlot<P>& sl = slots[tid];
+    const int ipr = (nb + 1) / 2;
+    int gs = 0;
+    for (int it = 0; it < my_tiles; ++it) {
+      const int tile = (int)blockIdx.x + it * (int)gridDim.x;
+      const long long item = (long long)tile * 64 + (tid >> 1);
+      const int k = tid & 1;
+      const bool active = item < n_items;
+      const int row = active ? (int)(item / ipr) : 0;
+      const int blk = active ? (int)(item - (long long)row * ipr) * 2 + k : 0;
+      const bool valid = active && blk < nb;
+      int nvalid = valid ? min(C, cols - blk * C) : 0;
+      const float* wsrc = W + (size_t)row * ldw + (size_t)blk * C;
+      if (nvalid > 0 &&
+          !SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * ldw + (size_t)blk * C + nvalid - 1,
+                            (size_t)(rows - 1) * ldw + cols))
+        nvalid = 0;
+      float w[C];
+      float maxabs = 0.f;
+      double ww64 = 0.0;
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        w[c] = c < nvalid ? wsrc[c] : 0.f;
+        maxabs = fmaxf(maxabs, fabsf(w[c]));
+        ww64 = fma((double)w[c], (double)w[c], ww64);
+      }
+      const int E = maxabs > 0.f ? ilogbf(maxabs) : 0;
+      const double s2 = ldexp(1.0, -2 * E);
+      float ww32 = 0.f;
+      __half hi[16], lo[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) hi[c] = lo[c] = __float2half_rn(0.f);
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const float v = scalbnf(w[c], -E);
+        ww32 = fmaf(v, v, ww32);
+        hi[c] = __float2half_rn(v);
+        lo[c] = __float2half_rn(v - __half2float(hi[c]));
+      }
+      // A: columns 0-7 the high parts (C = 8: repeated at k = 8..15),
+      // columns 8-15 the rests.
+      uint32_t a[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        a[j] = (C == 8) ? pack_half2(hi[(2 * j) & 7], hi[(2 * j + 1) & 7])
+                        : pack_half2(hi[2 * j], hi[2 * j + 1]);
+        a[8 + j] = pack_half2(lo[2 * j], lo[2 * j + 1]);
+      }
+      tc::tmem_st16(tmem + lane_base, a);
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(afull);
 
+      sl.seed = 1;
+      sl.e = 15;
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int blk = b0 + k;
-    if (blk >= nb) break;
-    const BlockSlot<P>& best = slots[2 * tid + k];
-    // The winner's error, computed directly.
-    const uint64_t st = seed_stream(best.seed);
-    const double inv = 1.0 / (double)(1 << best.e);
-    double err = 0.0;
+      for (int p = 0; p < P; ++p) sl.q[p] = 0;
+      sl.ww = ww64;
+      sl.wsrc = wsrc;
+      sl.nvalid = nvalid;
+      const bool live = !(nvalid == 0 || ww64 == 0.0 || !isfinite(ww64));
+      sl.err = live ? INFINITY : ww64;  // a dead block keeps seed 1, e = 15, q = 0
+      float thr = live ? INFINITY : -INFINITY;
+      float base = ww32 - thr;  // r' = base - sum of squares < 0  <=>  r < thr
+      int queued = 0;
+      __syncwarp();
+
+      // Pipelined over half stages (16 seeds): the TMEM loads of the next
+      // half are in flight while the current half is tested.
+      auto dcol = [&](int dd, int p, int h) {
+        return tmem + lane_base + T::kACols + dd * N + p * T::kSeeds + 16 * h;
+      };
+      uint32_t vb[2][P][16];
+      ok = tc::mbar_spin_or_abort(dfull(gs % DS), (gs / DS) & 1, kEncWaitLimit, abort_flag) && ok;
+      __syncwarp();
+      tc::fence_after_sync();
 #pragma unroll
-    for (int c = 0; c < C; ++c) {
-      double what = 0.0;
+      for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(gs % DS, p, 0), vb[0][p]);
+      for (int g = 0; g < T::kStages; ++g, ++gs) {
+        const int d = gs % DS;
+        float rp[2][16];
+        uint32_t neg = 0;
 #pragma unroll
-      for (int p = 0; p < P; ++p) what = fma(basis_entry<C, P>(st, c, p), (double)best.q[p], what);
-      const double wc = c < nvalid[k] ? (double)wsrc[k][c] : 0.0;
-      const double d = wc - what * inv;
-      err = fma(d, d, err);
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int p = 0; p < P; ++p) tc::tmem_wait_ld_tie(vb[h][p]);
+          if (h == 0) {
+#pragma unroll
+            for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(d, p, 1), vb[1][p]);
+          } else {
+            // Both halves of this stage are in registers: release it and
+            // start the next stage's loads.
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(dempty(d));
+            if (g + 1 < T::kStages) {
+              const int d2 = (gs + 1) % DS;
+              ok = tc::mbar_spin_or_abort(dfull(d2), ((gs + 1) / DS) & 1, kEncWaitLimit, abort_flag) && ok;
+              __syncwarp();
+              tc::fence_after_sync();
+#pragma unroll
+              for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(d2, p, 0), vb[0][p]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float2 r2 = make_float2(base, base);
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+              const float2 x =
+                  make_float2(__uint_as_float(vb[h][p][2 * j]), __uint_as_float(vb[h][p][2 * j + 1]));
+              r2 = __ffma2_rn(make_float2(-x.x, -x.y), x, r2);
+            }
+            rp[h][2 * j] = r2.x;
+            rp[h][2 * j + 1] = r2.y;
+            neg |= __float_as_uint(r2.x) | __float_as_uint(r2.y);
+          }
+        }
+        if (__any_sync(0xffffffffu, live && (neg >> 31))) {
+          // Queue this stage's survivors in seed order (tested against the
+          // threshold the residuals were computed with: never tighter than
+          // the current one), visiting only seeds some lane kept.
+          uint32_t mine = 0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) mine |= (__float_as_uint(rp[h][j]) >> 31) << (16 * h + j);
+          if (!live) mine = 0;
+          if (g == T::kStages - 1) mine &= 0x7fffffffu;  // the padding row is no seed
+          uint32_t todo = __reduce_or_sync(0xffffffffu, mine);
+          while (todo) {
+            const int j = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const bool want = (mine >> j) & 1u;
+            const unsigned m = __ballot_sync(0xffffffffu, want);
+            if (want)
+              wq->ent[queued + __popc(m & lanes_below)] =
+                  (uint32_t)(g * T::kSeeds + j + 1) | ((uint32_t)lane << 16);
+            queued += __popc(m);
+            if (queued >= 32) {
+              __syncwarp();
+              queued = drain_queue<C, P>(wq, queued, 32, wslots, exact, lane);
+              if (live) {
+                thr = prune_threshold(sl.err, ww64, s2);
+                base = ww32 - thr;
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      drain_queue<C, P>(wq, queued, 1, wslots, exact, lane);
+
+      // The block's record (and error), the winner's error computed directly.
+      uint32_t e_me = (uint32_t)sl.e & 15u;
+      if (valid) {
+        const uint64_t st = seed_stream(sl.seed);
+        const double inv = 1.0 / (double)(1 << sl.e);
+        double err = 0.0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+          double what = 0.0;
+#pragma unroll
+          for (int p = 0; p < P; ++p) what = fma(basis_entry<C, P>(st, c, p), (double)sl.q[p], what);
+          const double wc = c < nvalid ? (double)wsrc[c] : 0.0;
+          const double dd = wc - what * inv;
+          err = fma(dd, dd, err);
+        }
+        uint32_t r = sl.seed << 16;
+#pragma unroll
+        for (int p = 0; p < P; ++p) r |= ((uint32_t)sl.q[p] & 15u) << (4 * p);
+        if constexpr (C == 8) r |= (uint32_t)sl.e << 12;
+        if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, blk, rec_pitch))
+          rec[(size_t)row * rec_pitch + blk] = r;
+        if (err_out && SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * nb + blk, (size_t)rows * nb))
+          err_out[(size_t)row * nb + blk] = err;
+      } else {
+        e_me = 0u;
+      }
+      if constexpr (C == 12) {
+        // The pair's exponent byte: even lane (block 2j) low nibble, its
+        // neighbour (block 2j + 1, or nothing) high nibble.
+        const uint32_t e_hi = __shfl_down_sync(0xffffffffu, e_me, 1);
+        if (k == 0 && valid &&
+            SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, blk >> 1, e_pitch))
+          eplane[(size_t)row * e_pitch + (blk >> 1)] = (uint8_t)(e_me | (e_hi << 4));
+      }
+      __syncwarp();
     }
-    uint32_t r = best.seed << 16;
-#pragma unroll
-    for (int p = 0; p < P; ++p) r |= ((uint32_t)best.q[p] & 15u) << (4 * p);
-    if constexpr (C == 8) r |= (uint32_t)best.e << 12;
-    if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, blk, rec_pitch))
-      rec[(size_t)row * rec_pitch + blk] = r;
-    if (err_out && SEEDLM_IN_BOUNDS(g_check_flag, (size_t)row * nb + blk, (size_t)rows * nb))
-      err_out[(size_t)row * nb + blk] = err;
   }
-  if constexpr (C == 12) {
-    // The pair's exponent byte: block b0 in the low nibble, b0 + 1 (or 0).
-    uint32_t byte = (uint32_t)slots[2 * tid].e & 15u;
-    if (b0 + 1 < nb) byte |= ((uint32_t)slots[2 * tid + 1].e & 15u) << 4;
-    if (SEEDLM_IN_BOUNDS(g_check_flag, row, rows) && SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, e_pitch))
-      eplane[(size_t)row * e_pitch + (b0 >> 1)] = (uint8_t)byte;
+
+  if (!ok) atomicOr(&g_enc_error, 1u);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, T::kTmemCols);
   }
 }
 
 template <int C, int P>
 int launch_encode_t(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
                     uint8_t* eplane, double* err, cudaStream_t stream, const DeviceInfo& dev) {
+  using T = TcEnc<C>;
   const long long ipr = (f.nb + 1) / 2;
   const long long items = ipr * f.rows;
   if (items == 0) return SEEDLM_OK;
-  const long long grid = (items + kEncThreads - 1) / kEncThreads;
-  if (grid > 0x7fffffffll) return SEEDLM_EUNSUPPORTED;
-  const size_t smem = 2 * kChunk * C * sizeof(float4) + 2 * kEncThreads * sizeof(BlockSlot<P>) +
-                      (kEncThreads / 32) * sizeof(WarpQueue);
-  int rc = allow_max_smem((const void*)encode_kernel<C, P>, dev);
+  const long long tiles = (items + 63) / 64;  // 128 blocks per tile
+  if (tiles > 0x7fffffffll) return SEEDLM_EUNSUPPORTED;
+  int rc = allow_max_smem((const void*)encode_tc_kernel<C, P>, dev);
   if (rc) return rc;
   // The seed tables live for this call only (one stream-ordered allocation:
-  // fp32 bases, then fp64 G and G^-1).
-  const size_t basis_bytes = (size_t)kTableRows * C * sizeof(float4);
+  // fp64 G and G^-1, then the tensor-core B operands).
   const size_t exact_bytes = (size_t)kTableRows * SeedExact<P>::kDoubles * sizeof(double);
+  const size_t btab_bytes = (size_t)T::kStages * T::kStageBytes;
   unsigned char* tables = nullptr;
   if ((rc = record_cuda_error(cudaMallocAsync(reinterpret_cast<void**>(&tables),
-                                              basis_bytes + exact_bytes, stream))))
+                                              exact_bytes + btab_bytes, stream))))
     return rc;
-  float4* table = reinterpret_cast<float4*>(tables);
-  double* exact = reinterpret_cast<double*>(tables + basis_bytes);
-  basis_table_kernel<C, P><<<kTableRows / 256, 256, 0, stream>>>(table, exact);
+  double* exact = reinterpret_cast<double*>(tables);
+  unsigned char* btab = tables + exact_bytes;
+  seed_table_kernel<C, P><<<kTableRows / 256, 256, 0, stream>>>(btab, exact);
   count_launch();
-  encode_kernel<C, P><<<(unsigned)grid, kEncThreads, smem, stream>>>(
-      W, ldw, f.rows, f.cols, f.nb, f.rec_pitch, f.e_pitch, rec, eplane, err, items, table, exact);
+  const long long cap = (long long)dev.num_sms * T::kCtasPerSm;
+  const int grid = (int)(tiles < cap ? tiles : cap);
+  const size_t smem = (size_t)T::kBS * T::kStageBytes + 128 * sizeof(BlockSlot<P>) +
+                      4 * sizeof(WarpQueue) + (2 * T::kBS + 2 * T::kDS + 1) * 8 + 8;
+  encode_tc_kernel<C, P><<<grid, T::kThreads, smem, stream>>>(
+      W, ldw, f.rows, f.cols, f.nb, f.rec_pitch, f.e_pitch, rec, eplane, err, items, (int)tiles,
+      btab, exact);
   count_launch();
   rc = record_cuda_error(cudaGetLastError());
   const int rc_free = record_cuda_error(cudaFreeAsync(tables, stream));
@@ -598,6 +754,14 @@ int launch_encode_t(const seedlm_format& f, const float* W, int64_t ldw, uint32_
 }
 
 }  // namespace
+
+int read_and_clear_encode_error(unsigned int* out) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t err = cudaMemcpyFromSymbol(&v, g_enc_error, sizeof(v));
+  if (err == cudaSuccess && v) err = cudaMemcpyToSymbol(g_enc_error, &zero, sizeof(zero));
+  *out = v;
+  return record_cuda_error(err);
+}
 
 int launch_encode(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
                   uint8_t* eplane, double* err, cudaStream_t stream, const DeviceInfo& dev) {

@@ -90,6 +90,7 @@ int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* e
                    const uint16_t* X, int is_bf16, int M, float* Y, void* workspace,
                    int64_t workspace_bytes, cudaStream_t stream, const DeviceInfo& dev);
 int read_and_clear_tc_error(unsigned int* out);
+int read_and_clear_encode_error(unsigned int* out);
 int launch_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 int launch_bounds_check(int64_t index, int64_t extent, cudaStream_t stream);
 int launch_encode(const seedlm_format& f, const float* W, int64_t ldw, uint32_t* rec,
