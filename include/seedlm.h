@@ -164,11 +164,11 @@ SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt, const uint32
  * use the layout of seedlm_format; record slots past nb and exponent-plane
  * bytes past ceil(nb / 2) are left untouched.  err (optional, NULL or device
  * memory of rows x nb doubles, 8-byte aligned) receives each block's squared
- * error.  Each call allocates its seed tables (18 MiB for (8,3), 28 MiB for
+ * error.  Each call allocates its seed tables (16 MiB for (8,3), 32 MiB for
  * (12,4)) on the stream with cudaMallocAsync and frees them the same way.
- * The search scores 65,535 seeds per block (an fp32 least-squares bound
- * first, exact fp64 scoring for the seeds it cannot rule out), so this is an
- * offline (model-load) step, not part of the hot path. */
+ * The search scores 65,535 seeds per block (a least-squares bound on the
+ * tensor cores first, exact fp64 scoring for the seeds it cannot rule out),
+ * so this is an offline (model-load) step, not part of the hot path. */
 SEEDLM_API int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_t* rec,
                              uint8_t* eplane, double* err, seedlm_stream stream);
 
