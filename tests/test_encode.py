@@ -176,3 +176,22 @@ def test_encode_decode_roundtrip_through_the_gemv(sl, oracle_mod):
     what = oracle_mod.decompress(fmt, rec, ep)
     rel = np.linalg.norm(what - W) / np.linalg.norm(W)
     assert rel < 0.5, rel
+
+
+@pytest.mark.parametrize("cp,rows,cols", [(C8, 640, 512), (C12, 400, 576)])
+def test_many_tiles_per_cta_sampled_blocks(sl, oracle_mod, cp, rows, cols):
+    # More 128-block tiles than the grid has CTAs (4-bit: 320 tiles on two
+    # CTAs per SM; 3-bit: 150 tiles on one per SM), so CTAs run several tiles
+    # and reuse their tensor memory, queues and barrier phases.  Blocks
+    # sampled across the matrix (first, last, tile edges, random) must reach
+    # the oracle's minimum error.
+    rng = np.random.default_rng(21 + cp[0])
+    W = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    fmt = inputs.make_format(rows, cols, *cp)
+    rec, ep, err = gpu_encode(sl, fmt, W)
+    nb = fmt["nb"]
+    flat = [0, 127, 128, rows * nb - 1, 64 * 296 * 2 - 1, 64 * 296 * 2]
+    flat += [int(v) for v in rng.integers(0, rows * nb, 12)]
+    blocks = sorted({(f // nb, f % nb) for f in flat if f < rows * nb})
+    check_against_oracle(oracle_mod, fmt, W.astype(np.float64), rec, ep, err, blocks)
+    assert np.all(np.isfinite(err)) and np.all(err >= 0)
