@@ -21,7 +21,7 @@
  * authors' reply on how inference uses Eq (1)).
  *
  * Concrete parameters the pages leave open, fixed as the workload
- * specification fixes them (every reading is listed in the design doc):
+ * specification fixes them:
  *   K = 16, Fibonacci LFSR with taps 16,14,13,11:
  *       bit = (s ^ s>>2 ^ s>>3 ^ s>>5) & 1 ;  s = (s >> 1) | (bit << 15)
  *   state_0 = seed;  U[c][p] = (state_{p*C + c} - 32768) / 32768.

@@ -4,7 +4,7 @@
 
 Every ``csrc/*.cu`` is compiled separately (in parallel) into ``_build/`` and
 linked into ``prng_seeded_decompress_b200/libseedlm.so`` with the CUDA runtime
-linked statically, so the library needs nothing but the driver at run time.
+linked statically, so the library needs nothing but the NVIDIA driver at run time.
 
 ``--check`` builds ``libseedlm_check.so`` (objects in ``_build_check/``) with
 -DSEEDLM_CHECK=1: every kernel compares each memory index it computes with
