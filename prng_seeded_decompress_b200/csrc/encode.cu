@@ -58,7 +58,7 @@ __device__ unsigned int g_enc_error = 0;
 namespace {
 
 constexpr int kNumSeeds = 65535;
-constexpr int kTableRows = 65536;  // row i holds seed i + 1; the last row is zero padding
+constexpr int kTableRows = 65536;  // exact-table rows: row i holds seed i + 1
 constexpr double kPruneMargin = 2e-4;  // relative to ||w||^2, ten times the filter's error bound
 constexpr uint64_t kEncWaitLimit = 2000000000ull;  // ns a hand-over wait may take
 
@@ -296,9 +296,15 @@ __device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
 template <int C>
 struct TcEnc {
   static constexpr int P = (C == 8) ? 3 : 4;
-  static constexpr int kSeeds = 32;                    // seeds per stage
-  static constexpr int kStages = kTableRows / kSeeds;  // per sweep
+  // Seeds per stage: N = 96 MMA columns either way, so the accumulators of
+  // two stages (and A) fit in 256 TMEM columns and two CTAs share an SM.
+  static constexpr int kSeeds = (C == 8) ? 32 : 24;
+  static constexpr int kStages = (kNumSeeds + kSeeds - 1) / kSeeds;  // per sweep
+  static constexpr int kRows = kStages * kSeeds;       // table rows incl. zero padding
   static constexpr int N = kSeeds * P;                 // MMA columns: (p, s), p-major
+  // Seeds of the last stage that exist (the rest are padding rows).
+  static constexpr int kLastSeeds = kNumSeeds - (kStages - 1) * kSeeds;
+  static constexpr uint32_t kLastMask = (kLastSeeds == 32) ? 0xffffffffu : ((1u << kLastSeeds) - 1u);
   static constexpr int kPiecesB = (C == 8) ? 1 : 2;
   static constexpr int kSlabBytes = N * 16 * 2;        // one N x 16 fp16 operand
   static constexpr int kStageBytes = kSlabBytes * kPiecesB;
@@ -321,13 +327,13 @@ __host__ __device__ constexpr int slab16_byte(int n, int k) {
 
 // Row i of the tables (seed i + 1): G = U^T U and G^-1 for exact scoring,
 // and the orthonormal basis split into fp16 high parts and rests at
-// (n = p * 32 + s, k) of its stage's B operand(s).
+// (n = p * kSeeds + s, k) of its stage's B operand(s).
 template <int C, int P>
 __global__ void __launch_bounds__(256) seed_table_kernel(unsigned char* __restrict__ btab,
                                                          double* __restrict__ exact) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= kTableRows) return;
   using T = TcEnc<C>;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T::kRows) return;
   unsigned char* stage = btab + (size_t)(i / T::kSeeds) * T::kStageBytes;
   const int s = i % T::kSeeds;
   double q[C][P];
@@ -413,7 +419,7 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
 }
 
 template <int C, int P>
-__global__ void __launch_bounds__(TcEnc<C>::kThreads)
+__global__ void __launch_bounds__(TcEnc<C>::kThreads, TcEnc<C>::kCtasPerSm)
 encode_tc_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, int nb,
                  int rec_pitch, int e_pitch, uint32_t* __restrict__ rec,
                  uint8_t* __restrict__ eplane, double* __restrict__ err_out, long long n_items,
@@ -589,6 +595,8 @@ encode_tc_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, i
       // Pipelined over half stages (16 seeds): the TMEM loads of the next
       // half are in flight while the current half is tested.
       auto dcol = [&](int dd, int p, int h) {
+        // (with 24 seeds the second half's last 8 columns belong to the next
+        // p or stage: read, never used)
         return tmem + lane_base + T::kACols + dd * N + p * T::kSeeds + 16 * h;
       };
       uint32_t vb[2][P][16];
@@ -634,7 +642,7 @@ encode_tc_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, i
             }
             rp[h][2 * j] = r2.x;
             rp[h][2 * j + 1] = r2.y;
-            neg |= __float_as_uint(r2.x) | __float_as_uint(r2.y);
+            if (16 * h + 2 * j < T::kSeeds) neg |= __float_as_uint(r2.x) | __float_as_uint(r2.y);
           }
         }
         if (__any_sync(0xffffffffu, live && (neg >> 31))) {
@@ -645,9 +653,10 @@ encode_tc_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, i
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int j = 0; j < 16; ++j) mine |= (__float_as_uint(rp[h][j]) >> 31) << (16 * h + j);
+            for (int j = 0; j < 16; ++j)
+              if (16 * h + j < T::kSeeds) mine |= (__float_as_uint(rp[h][j]) >> 31) << (16 * h + j);
           if (!live) mine = 0;
-          if (g == T::kStages - 1) mine &= 0x7fffffffu;  // the padding row is no seed
+          if (g == T::kStages - 1) mine &= T::kLastMask;  // padding rows are no seeds
           uint32_t todo = __reduce_or_sync(0xffffffffu, mine);
           while (todo) {
             const int j = __ffs(todo) - 1;
@@ -733,14 +742,14 @@ int launch_encode_t(const seedlm_format& f, const float* W, int64_t ldw, uint32_
   // The seed tables live for this call only (one stream-ordered allocation:
   // fp64 G and G^-1, then the tensor-core B operands).
   const size_t exact_bytes = (size_t)kTableRows * SeedExact<P>::kDoubles * sizeof(double);
-  const size_t btab_bytes = (size_t)T::kStages * T::kStageBytes;
+  const size_t btab_bytes = (size_t)T::kStages * T::kStageBytes;  // kRows seeds
   unsigned char* tables = nullptr;
   if ((rc = record_cuda_error(cudaMallocAsync(reinterpret_cast<void**>(&tables),
                                               exact_bytes + btab_bytes, stream))))
     return rc;
   double* exact = reinterpret_cast<double*>(tables);
   unsigned char* btab = tables + exact_bytes;
-  seed_table_kernel<C, P><<<kTableRows / 256, 256, 0, stream>>>(btab, exact);
+  seed_table_kernel<C, P><<<(T::kRows + 255) / 256, 256, 0, stream>>>(btab, exact);
   count_launch();
   const long long cap = (long long)dev.num_sms * T::kCtasPerSm;
   const int grid = (int)(tiles < cap ? tiles : cap);
