@@ -269,9 +269,9 @@ __device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
 // ---------------------------------------------------------------- tensor-core filter
 //
 // The projections on the tensor cores: D[block][(p, s)] = sum_c w[c] Q(s)[c][p]
-// for 128 blocks (the TMEM lanes) against 32 seeds at a time, kind::f16 with
-// fp32 accumulation, every operand split exactly into an fp16 high part and
-// an fp16 rest: D = A_hi B_hi + A_hi B_lo + A_lo B_hi.  For C = 8 the two B
+// for 128 blocks (the TMEM lanes) against 32 (C = 8) or 24 (C = 12) seeds at
+// a time, kind::f16 with fp32 accumulation, every operand split exactly into
+// an fp16 high part and an fp16 rest: D = A_hi B_hi + A_hi B_lo + A_lo B_hi.  For C = 8 the two B
 // parts share one K = 16 row ([Q_hi | Q_lo] against [w_hi | w_hi] and
 // [w_lo | 0]), so a stage is two MMAs; for C = 12 (K padded to 16) three.
 // The block is scaled by 2^-E (exact) so that max|w| lies in [1, 2), and
@@ -285,7 +285,7 @@ __device__ __noinline__ int drain_queue(WarpQueue* wq, int count, int min_batch,
 // seeds).  A seed is skipped when r > best + 2e-4 ||w||^2.
 //
 // Warps 0-3 (one TMEM lane quarter each, one block per thread) write A,
-// read each stage's 32 x P accumulator columns and test the residuals
+// read each stage's 96 accumulator columns and test the residuals
 // against the threshold, queueing survivors for exact scoring; warp 4 issues
 // the MMAs (one elected lane); warp 5 copies the B stages, precomputed in the
 // MMA's shared-memory layout, with bulk copies.  All hand-overs are
