@@ -195,3 +195,27 @@ def test_many_tiles_per_cta_sampled_blocks(sl, oracle_mod, cp, rows, cols):
     blocks = sorted({(f // nb, f % nb) for f in flat if f < rows * nb})
     check_against_oracle(oracle_mod, fmt, W.astype(np.float64), rec, ep, err, blocks)
     assert np.all(np.isfinite(err)) and np.all(err >= 0)
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_leading_dimension_gives_the_same_records(sl, cp):
+    # W as a column slice of a wider matrix (ldw > cols, ragged tail block)
+    # encodes exactly as its contiguous copy: same records, exponents, errors.
+    C = cp[0]
+    rows, cols, wide = 37, 5 * C + 3, 8 * C + 4
+    g = torch.Generator(device="cuda").manual_seed(17)
+    Wwide = torch.randn((rows, wide), device="cuda", generator=g) * 0.02
+    fmt = inputs.make_format(rows, cols, *cp)
+    outs = []
+    for W in (Wwide[:, :cols], Wwide[:, :cols].contiguous()):
+        rec = torch.zeros((rows, fmt["rec_pitch"]), dtype=torch.int32, device="cuda")
+        ep = (torch.zeros((rows, fmt["e_pitch"]), dtype=torch.uint8, device="cuda")
+              if cp[1] == 4 else None)
+        err = torch.empty((rows, fmt["nb"]), dtype=torch.float64, device="cuda")
+        sl.encode(fmt, W, rec, ep, err)
+        torch.cuda.synchronize()
+        outs.append((rec.cpu(), None if ep is None else ep.cpu(), err.cpu()))
+    assert Wwide[:, :cols].stride(0) == wide
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][2], outs[1][2])
+    if cp[1] == 4:
+        assert torch.equal(outs[0][1], outs[1][1])
