@@ -1,7 +1,7 @@
 // tcgen05.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core path:
-// shared-memory matrix descriptors, tcgen05.mma (kind::tf32, A from shared
-// or tensor memory), TMEM allocation, loads and stores, bulk copies and
-// mbarriers with bounded waits.
+// shared-memory matrix descriptors, tcgen05.mma (kind::f16, A from tensor
+// memory, issued by one elected lane of a converged warp), TMEM allocation,
+// loads and stores, bulk copies and mbarriers with bounded waits.
 #pragma once
 
 #include <stdint.h>
@@ -28,40 +28,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   return d;
 }
 
-// Instruction descriptor for kind::tf32: D fp32, A and B tf32, both K-major,
-// M = 128, N = n (multiple of 8, <= 256).
-__host__ __device__ constexpr uint32_t idesc_tf32(int n) {
-  return (1u << 4)                        // D format: f32
-         | (2u << 7)                      // A format: tf32
-         | (2u << 10)                     // B format: tf32
-         | ((uint32_t)(n >> 3) << 17)     // N >> 3
-         | ((uint32_t)(128 >> 4) << 24);  // M >> 4
-}
-
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
-      :
-      : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
-        "r"(0u), "r"(0u));
-}
-
-// Same with A taken from tensor memory: A is 128 lanes (rows) x 8 columns
-// (one tf32 per column) starting at TMEM address `a_tmem`.
-__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
-      :
-      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
-        "r"(0u), "r"(0u));
-}
-
 // Instruction descriptor for kind::f16: D fp32, A and B both fp16 (bf16 = 0)
 // or both bf16 (bf16 = 1), K-major, M = 128, N = n (multiple of 16, <= 256).
 __host__ __device__ constexpr uint32_t idesc_f16(int n, int bf16) {
@@ -72,22 +38,12 @@ __host__ __device__ constexpr uint32_t idesc_f16(int n, int bf16) {
          | ((uint32_t)(128 >> 4) << 24);  // M >> 4
 }
 
-// kind::f16 MMA, K = 16, A from tensor memory: 128 lanes (rows) x 8 columns,
-// each column two 16-bit elements (lower K index in the low half).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
-      :
-      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
-        "r"(0u), "r"(0u));
-}
-
-// Whole-warp forms: every lane of a converged warp calls them with the same
-// (warp-uniform) operands and one elected lane issues the instruction, so the
-// operands can stay in uniform registers.
+// kind::f16 MMA, K = 16, A from tensor memory (128 lanes = rows x 8 columns,
+// each column two 16-bit elements, the lower K index in the low half), B from
+// shared memory through its descriptor, D (fp32) in tensor memory.  Both
+// this and the commit below are whole-warp forms: every lane of a converged
+// warp calls them with the same (warp-uniform) operands and one elected lane
+// issues the instruction, so the operands can stay in uniform registers.
 __device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -109,26 +65,12 @@ __device__ __forceinline__ void mma_commit_warp(uint32_t mbar) {
       : "memory");
 }
 
-// Arrive once on `mbar` when all tcgen05.mma issued so far by this thread
-// have completed.
-__device__ __forceinline__ void mma_commit(uint32_t mbar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               :
-               : "r"(mbar)
-               : "memory");
-}
-
 __device__ __forceinline__ void fence_before_sync() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// Generic-proxy shared-memory writes -> visible to the async (tensor) proxy.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // TMEM allocation (one full warp).  The allocated base address is written to
 // shared memory at `slot`.
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
@@ -192,14 +134,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
         "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
         "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-      :
-      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
-        "r"(r[6]), "r"(r[7])
       : "memory");
 }
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
@@ -329,19 +263,6 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint32_t mbar, uint32_t parit
       return false;
     }
   }
-}
-
-// Non-blocking test of the phase (never suspends the thread).
-__device__ __forceinline__ bool mbar_test_wait(uint32_t mbar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done)
-      : "r"(mbar), "r"(parity)
-      : "memory");
-  return done != 0;
 }
 
 // As mbar_wait_or_abort but spinning on plain try_wait, with no suspend
