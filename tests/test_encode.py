@@ -219,3 +219,27 @@ def test_leading_dimension_gives_the_same_records(sl, cp):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][2], outs[1][2])
     if cp[1] == 4:
         assert torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("cp,seed", [(C8, 48395), (C8, 38137), (C12, 62544), (C12, 1596)])
+def test_planted_fit_on_the_worst_conditioned_seeds(sl, oracle_mod, cp, seed):
+    # The seeds whose U is closest to rank-deficient (condition number of
+    # U^T U about 1e11 at 4 bits, 3e9 at 3 bits, checked here on the CPU):
+    # a block planted on one of them still comes back as an exact fit with
+    # the oracle's canonical triple -- the exact scoring's G^-1 is accurate
+    # enough to round t* 2^e to the planted q.
+    C, P = cp
+    U = oracle_mod.block_basis(seed, C, P)
+    assert np.linalg.cond(U.T @ U) > 1e9
+    q = np.array([5, -3, 7, -6][:P], dtype=np.int64)
+    e = 10
+    fmt = inputs.make_format(1, C, *cp)
+    w = (U @ q) * 2.0 ** -e
+    assert np.array_equal(w.astype(np.float32).astype(np.float64), w)
+    rec, ep, err = gpu_encode(sl, fmt, w.reshape(1, C).astype(np.float32))
+    from oracle.search import seed_search
+    s, qo, eo, e_err, _ = seed_search(w, C, P)
+    gs, gq, ge = oracle_mod.block_fields(fmt, rec, ep, 0, 0)
+    assert e_err == 0.0 and err[0, 0] == 0.0
+    assert (gs, ge) == (s, eo) and np.array_equal(np.asarray(gq), np.asarray(qo))
+    assert np.array_equal(oracle_mod.reconstruct_block(fmt, rec, ep, 0, 0), w)
