@@ -298,7 +298,9 @@ struct TcEnc {
   static constexpr int P = (C == 8) ? 3 : 4;
   // Seeds per stage: N = 96 MMA columns either way, so the accumulators of
   // two stages (and A) fit in 256 TMEM columns and two CTAs share an SM.
+  // (16 seeds per stage with 4 or 3 stages measured 15-25 % slower.)
   static constexpr int kSeeds = (C == 8) ? 32 : 24;
+  static constexpr int kHalves = (kSeeds + 15) / 16;  // 16-seed halves of a stage
   static constexpr int kStages = (kNumSeeds + kSeeds - 1) / kSeeds;  // per sweep
   static constexpr int kRows = kStages * kSeeds;       // table rows incl. zero padding
   static constexpr int N = kSeeds * P;                 // MMA columns: (p, s), p-major
@@ -317,6 +319,10 @@ struct TcEnc {
   static constexpr int kThreads = 6 * 32;
   static constexpr int kMmaWarp = 4, kLoaderWarp = 5;
   static_assert(N % 16 == 0 && N <= 256, "M = 128 MMA shape");
+  // The epilogue reads whole 16-column halves: the last one may run past its
+  // stage, never past the allocation.
+  static_assert(kACols + (kDS - 1) * N + (P - 1) * kSeeds + 16 * kHalves <= kTmemCols,
+                "TMEM reads stay inside the allocation");
 };
 
 // Byte offset of element (n, k) in an N x 16 fp16 operand, K-major core
@@ -595,87 +601,100 @@ encode_tc_kernel(const float* __restrict__ W, int64_t ldw, int rows, int cols, i
       // Pipelined over half stages (16 seeds): the TMEM loads of the next
       // half are in flight while the current half is tested.
       auto dcol = [&](int dd, int p, int h) {
-        // (with 24 seeds the second half's last 8 columns belong to the next
-        // p or stage: read, never used)
+        // (a last half of fewer than 16 seeds reads columns of the next p or
+        // stage as well: read, never used)
         return tmem + lane_base + T::kACols + dd * N + p * T::kSeeds + 16 * h;
       };
+      // Halves of 16 seeds: the loads of the next half are in flight while
+      // the current one is tested.  With one half per stage the stage loop
+      // is unrolled by two so that the register buffer of every half is
+      // known at compile time.
+      constexpr int H = T::kHalves;
+      constexpr int U = (H == 1) ? 2 : 1;
+      static_assert(T::kStages % U == 0, "whole unrolled stage pairs");
       uint32_t vb[2][P][16];
       ok = tc::mbar_spin_or_abort(dfull(gs % DS), (gs / DS) & 1, kEncWaitLimit, abort_flag) && ok;
       __syncwarp();
       tc::fence_after_sync();
 #pragma unroll
       for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(gs % DS, p, 0), vb[0][p]);
-      for (int g = 0; g < T::kStages; ++g, ++gs) {
-        const int d = gs % DS;
-        float rp[2][16];
-        uint32_t neg = 0;
+      for (int g0 = 0; g0 < T::kStages; g0 += U) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int u = 0; u < U; ++u) {
+          const int g = g0 + u;
+          const int d = gs % DS;
+          float rp[H][16];
+          uint32_t neg = 0;
 #pragma unroll
-          for (int p = 0; p < P; ++p) tc::tmem_wait_ld_tie(vb[h][p]);
-          if (h == 0) {
+          for (int h = 0; h < H; ++h) {
+            const int b = (H == 1) ? u : h;  // buffer of this half
 #pragma unroll
-            for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(d, p, 1), vb[1][p]);
-          } else {
-            // Both halves of this stage are in registers: release it and
-            // start the next stage's loads.
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(dempty(d));
-            if (g + 1 < T::kStages) {
-              const int d2 = (gs + 1) % DS;
-              ok = tc::mbar_spin_or_abort(dfull(d2), ((gs + 1) / DS) & 1, kEncWaitLimit, abort_flag) && ok;
+            for (int p = 0; p < P; ++p) tc::tmem_wait_ld_tie(vb[b][p]);
+            if (h + 1 < H) {
+#pragma unroll
+              for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(d, p, h + 1), vb[1 - b][p]);
+            } else {
+              // The whole stage is in registers: release it and start the
+              // next stage's loads.
+              tc::fence_before_sync();
               __syncwarp();
-              tc::fence_after_sync();
+              if (lane == 0) tc::mbar_arrive(dempty(d));
+              if (g + 1 < T::kStages) {
+                const int d2 = (gs + 1) % DS;
+                ok = tc::mbar_spin_or_abort(dfull(d2), ((gs + 1) / DS) & 1, kEncWaitLimit, abort_flag) && ok;
+                __syncwarp();
+                tc::fence_after_sync();
 #pragma unroll
-              for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(d2, p, 0), vb[0][p]);
+                for (int p = 0; p < P; ++p) tc::tmem_ld16_async(dcol(d2, p, 0), vb[1 - b][p]);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float2 r2 = make_float2(base, base);
+#pragma unroll
+              for (int p = 0; p < P; ++p) {
+                const float2 x =
+                    make_float2(__uint_as_float(vb[b][p][2 * j]), __uint_as_float(vb[b][p][2 * j + 1]));
+                r2 = __ffma2_rn(make_float2(-x.x, -x.y), x, r2);
+              }
+              rp[h][2 * j] = r2.x;
+              rp[h][2 * j + 1] = r2.y;
+              if (16 * h + 2 * j < T::kSeeds) neg |= __float_as_uint(r2.x) | __float_as_uint(r2.y);
             }
           }
+          if (__any_sync(0xffffffffu, live && (neg >> 31))) {
+            // Queue this stage's survivors in seed order (tested against the
+            // threshold the residuals were computed with: never tighter than
+            // the current one), visiting only seeds some lane kept.
+            uint32_t mine = 0;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float2 r2 = make_float2(base, base);
+            for (int h = 0; h < H; ++h)
 #pragma unroll
-            for (int p = 0; p < P; ++p) {
-              const float2 x =
-                  make_float2(__uint_as_float(vb[h][p][2 * j]), __uint_as_float(vb[h][p][2 * j + 1]));
-              r2 = __ffma2_rn(make_float2(-x.x, -x.y), x, r2);
-            }
-            rp[h][2 * j] = r2.x;
-            rp[h][2 * j + 1] = r2.y;
-            if (16 * h + 2 * j < T::kSeeds) neg |= __float_as_uint(r2.x) | __float_as_uint(r2.y);
-          }
-        }
-        if (__any_sync(0xffffffffu, live && (neg >> 31))) {
-          // Queue this stage's survivors in seed order (tested against the
-          // threshold the residuals were computed with: never tighter than
-          // the current one), visiting only seeds some lane kept.
-          uint32_t mine = 0;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (16 * h + j < T::kSeeds) mine |= (__float_as_uint(rp[h][j]) >> 31) << (16 * h + j);
-          if (!live) mine = 0;
-          if (g == T::kStages - 1) mine &= T::kLastMask;  // padding rows are no seeds
-          uint32_t todo = __reduce_or_sync(0xffffffffu, mine);
-          while (todo) {
-            const int j = __ffs(todo) - 1;
-            todo &= todo - 1;
-            const bool want = (mine >> j) & 1u;
-            const unsigned m = __ballot_sync(0xffffffffu, want);
-            if (want)
-              wq->ent[queued + __popc(m & lanes_below)] =
-                  (uint32_t)(g * T::kSeeds + j + 1) | ((uint32_t)lane << 16);
-            queued += __popc(m);
-            if (queued >= 32) {
-              __syncwarp();
-              queued = drain_queue<C, P>(wq, queued, 32, wslots, exact, lane);
-              if (live) {
-                thr = prune_threshold(sl.err, ww64, s2);
-                base = ww32 - thr;
+              for (int j = 0; j < 16; ++j)
+                if (16 * h + j < T::kSeeds) mine |= (__float_as_uint(rp[h][j]) >> 31) << (16 * h + j);
+            if (!live) mine = 0;
+            if (g == T::kStages - 1) mine &= T::kLastMask;  // padding rows are no seeds
+            uint32_t todo = __reduce_or_sync(0xffffffffu, mine);
+            while (todo) {
+              const int j = __ffs(todo) - 1;
+              todo &= todo - 1;
+              const bool want = (mine >> j) & 1u;
+              const unsigned m = __ballot_sync(0xffffffffu, want);
+              if (want)
+                wq->ent[queued + __popc(m & lanes_below)] =
+                    (uint32_t)(g * T::kSeeds + j + 1) | ((uint32_t)lane << 16);
+              queued += __popc(m);
+              if (queued >= 32) {
+                __syncwarp();
+                queued = drain_queue<C, P>(wq, queued, 32, wslots, exact, lane);
+                if (live) {
+                  thr = prune_threshold(sl.err, ww64, s2);
+                  base = ww32 - thr;
+                }
               }
             }
           }
+          ++gs;
         }
       }
       __syncwarp();
