@@ -33,7 +33,8 @@ _FORMATS = {(8, 3, 16), (12, 4, 16)}
 
 
 def check_format(fmt: dict) -> dict:
-    """The format's fields as ints, or ValueError if they are inconsistent."""
+    """The format's fields as ints, or ValueError if they are inconsistent
+    (the same rules the library applies to ``seedlm_format``)."""
     try:
         f = {k: int(fmt[k]) for k in _FIELDS}
     except (KeyError, TypeError, ValueError) as exc:
@@ -46,11 +47,8 @@ def check_format(fmt: dict) -> dict:
         raise ValueError("nb is not ceil(cols / C)")
     if f["rec_pitch"] < f["nb"] or f["rec_pitch"] % 4:
         raise ValueError("rec_pitch must be >= nb and a multiple of 4")
-    if f["P"] == 4:
-        if f["e_pitch"] < (f["nb"] + 1) // 2 or f["e_pitch"] % 16:
-            raise ValueError("e_pitch must be >= ceil(nb / 2) and a multiple of 16")
-    elif f["e_pitch"] != 0:
-        raise ValueError("e_pitch must be 0 when e is packed in the record")
+    if f["P"] == 4 and f["e_pitch"] < (f["nb"] + 1) // 2:
+        raise ValueError("e_pitch must be >= ceil(nb / 2)")
     return f
 
 
