@@ -437,13 +437,18 @@ def extras(torch, sl, args):
         rec_e = torch.empty((4096, fe["rec_pitch"]), dtype=torch.int32, device="cuda")
         ep_e = (torch.empty((4096, fe["e_pitch"]), dtype=torch.uint8, device="cuda")
                 if P == 4 else None)
-        sl.encode(fe, We, rec_e, ep_e)
+        err_e = torch.empty((4096, fe["nb"]), dtype=torch.float64, device="cuda")
+        sl.encode(fe, We, rec_e, ep_e, err_e)
         ms = time_region(torch, lambda i: sl.encode(fe, We, rec_e, ep_e), 1)
         blocks = 4096 * fe["nb"]
+        # Relative reconstruction error of the fit (Gaussian weights, as in
+        # the pages' design-space exploration): ||W - W_hat|| / ||W||.
+        rel = math.sqrt(float(err_e.sum()) / float((We.double() ** 2).sum()))
         out[f"encode_{bits}bit_4096x4096"] = {
             "ms_per_call": round(ms, 1), "blocks_per_s": round(blocks / (ms / 1e3)),
-            "seeds_per_s_e9": round(blocks * 65535 / (ms / 1e3) / 1e9, 1)}
-        del rec_e, ep_e
+            "seeds_per_s_e9": round(blocks * 65535 / (ms / 1e3) / 1e9, 1),
+            "relative_reconstruction_error": round(rel, 4)}
+        del rec_e, ep_e, err_e
     del We
 
     # Dense fp16 GEMV (in-house) on the 70B layer shapes, 4 rotating copies.
