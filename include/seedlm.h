@@ -35,7 +35,10 @@
  *
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers, unless a function says HOST.
- *     The caller owns every buffer; the library allocates no device memory.
+ *     The caller owns every buffer.  No call allocates device memory except
+ *     seedlm_encode, which takes its seed tables from the stream-ordered
+ *     allocator for the duration of the call (seedlm_gemm_smallM_noalloc's
+ *     scratch is an array inside the library image).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and runs asynchronously; the call returns once it is enqueued.
  *   - Return value 0 = success, negative = error (SEEDLM_E*), with no work
