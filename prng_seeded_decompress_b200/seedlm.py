@@ -137,6 +137,20 @@ def _fmt(fmt) -> Format:
     return fmt if isinstance(fmt, Format) else Format.from_dict(fmt)
 
 
+def _row_major_ld(t, cols: int) -> int:
+    """Leading dimension of a row-major matrix argument (unit column stride)."""
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError("expected a 2-D row-major tensor with unit column stride")
+    return int(t.stride(0)) if t.shape[0] > 1 else max(int(t.stride(0)), cols)
+
+
+def _dense(t, name: str):
+    """Arguments the library reads or writes as one dense array."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
 def init():
     _check("seedlm_init", lib.seedlm_init())
 
@@ -144,7 +158,7 @@ def init():
 def decompress(fmt, rec, eplane, W, ldw: int | None = None, stream=None):
     """W[:rows, :cols] = the rebuilt weights (fp32)."""
     f = _fmt(fmt)
-    ld = ldw if ldw is not None else (W.stride(0) if W.dim() == 2 else f.cols)
+    ld = ldw if ldw is not None else _row_major_ld(W, f.cols)
     _check("seedlm_decompress", lib.seedlm_decompress(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(W), ld, _stream(stream, W)))
 
@@ -156,7 +170,7 @@ def encode(fmt, W, rec, eplane=None, err=None, ldw: int | None = None, stream=No
     given, is a float64 (rows x nb) tensor that receives each block's squared
     reconstruction error."""
     f = _fmt(fmt)
-    ld = ldw if ldw is not None else (W.stride(0) if W.dim() == 2 else f.cols)
+    ld = ldw if ldw is not None else _row_major_ld(W, f.cols)
     _check("seedlm_encode", lib.seedlm_encode(
         ctypes.byref(f), _ptr(W), ld, _ptr(rec), _ptr(eplane), _ptr(err), _stream(stream, W)))
 
@@ -164,6 +178,7 @@ def encode(fmt, W, rec, eplane=None, err=None, ldw: int | None = None, stream=No
 def gemv(fmt, rec, eplane, x, y, stream=None):
     """y = W x; x float16/bfloat16 (cols), y float32 (rows)."""
     f = _fmt(fmt)
+    _dense(x, "x"), _dense(y, "y")
     _check("seedlm_gemv", lib.seedlm_gemv(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(x), _act_dtype(x), _ptr(y),
         _stream(stream, y)))
@@ -191,6 +206,7 @@ def gemm_smallM(fmt, rec, eplane, X, Y, workspace=None, stream=None):
 
     `workspace` comes from gemm_workspace(); if omitted a fresh one is made."""
     f = _fmt(fmt)
+    _dense(X, "X"), _dense(Y, "Y")
     M = int(X.shape[0])
     if workspace is None:
         workspace = gemm_workspace(f, M, device=Y.device)
@@ -205,6 +221,7 @@ def gemm_smallM_noalloc(fmt, rec, eplane, X, Y, stream=None):
     tiles; 16 MiB + 64 KiB) is an array inside the library; calls sharing it
     must not overlap."""
     f = _fmt(fmt)
+    _dense(X, "X"), _dense(Y, "Y")
     _check("seedlm_gemm_smallM_noalloc", lib.seedlm_gemm_smallM_noalloc(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), int(X.shape[0]),
         _ptr(Y), _stream(stream, Y)))
@@ -240,8 +257,9 @@ def selftest_wait_timeout(limit_ns: int = 2_000_000, stream=None):
 
 def dense_gemv_f16(W, x, y, stream=None):
     """y = W x with dense fp16 W (rows, cols) -- the reference point."""
+    _dense(x, "x"), _dense(y, "y")
     _check("seedlm_dense_gemv_f16", lib.seedlm_dense_gemv_f16(
-        int(W.shape[0]), int(W.shape[1]), _ptr(W), int(W.stride(0)), _ptr(x), _ptr(y),
+        int(W.shape[0]), int(W.shape[1]), _ptr(W), _row_major_ld(W, int(W.shape[1])), _ptr(x), _ptr(y),
         _stream(stream, y)))
 
 

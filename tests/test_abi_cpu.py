@@ -143,3 +143,21 @@ def test_binding_refuses_to_run_without_the_library(tmp_path):
         (pkg / f).write_text(open(os.path.join(ROOT, "prng_seeded_decompress_b200", f)).read())
     res = subprocess.run(["python", "-c", code], capture_output=True, text=True)
     assert res.returncode != 0 and "libseedlm.so is missing" in res.stderr
+
+
+def test_binding_refuses_layouts_the_library_cannot_read(sl):
+    # Row-major with unit column stride is what the library addresses; a
+    # transposed or strided tensor is refused before any call (CPU tensors
+    # stand in for device ones: only the layout is looked at).
+    torch = pytest.importorskip("torch")
+    W = torch.empty((6, 10))
+    assert sl._row_major_ld(W, 10) == 10
+    assert sl._row_major_ld(torch.empty((6, 16))[:, :10], 10) == 16
+    assert sl._row_major_ld(torch.empty((1, 10)), 10) == 10
+    with pytest.raises(ValueError, match="unit column stride"):
+        sl._row_major_ld(W.t(), 6)
+    with pytest.raises(ValueError, match="unit column stride"):
+        sl._row_major_ld(torch.empty(10), 10)
+    with pytest.raises(ValueError, match="contiguous"):
+        sl._dense(torch.empty((4, 8))[:, ::2], "X")
+    assert sl._dense(torch.empty(5), "x").numel() == 5
