@@ -243,3 +243,27 @@ def test_planted_fit_on_the_worst_conditioned_seeds(sl, oracle_mod, cp, seed):
     assert e_err == 0.0 and err[0, 0] == 0.0
     assert (gs, ge) == (s, eo) and np.array_equal(np.asarray(gq), np.asarray(qo))
     assert np.array_equal(oracle_mod.reconstruct_block(fmt, rec, ep, 0, 0), w)
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_encode_save_load_then_gemv(sl, oracle_mod, tmp_path, cp):
+    # The offline workflow: encode on the GPU, save the planes, load them
+    # back (format, sizes and SHA-256 checked), then the GEMV on the loaded
+    # planes matches the oracle GEMV on the same planes.
+    from prng_seeded_decompress_b200 import store
+    rng = np.random.default_rng(31 + cp[0])
+    rows, cols = 48, 200
+    W = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    fmt = inputs.make_format(rows, cols, *cp)
+    rec, ep, _ = gpu_encode(sl, fmt, W)
+    store.save_layer(str(tmp_path / "layer"), fmt, rec, ep)
+    fmt2, rec2, ep2 = store.load_layer(str(tmp_path / "layer"))
+    assert fmt2 == fmt and np.array_equal(rec2, rec)
+    xb, xv = inputs.make_activations((cols,), "f16", 5)
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+    y = torch.empty(rows, device="cuda")
+    sl.gemv(fmt2, torch.from_numpy(rec2.view(np.int32)).cuda(),
+            None if ep2 is None else torch.from_numpy(ep2).cuda(), x, y)
+    torch.cuda.synchronize()
+    ref, refabs = oracle_mod.gemv(fmt2, rec2, ep2, xv)
+    assert np.all(np.abs(y.cpu().numpy().astype(np.float64) - ref) <= 1e-5 * refabs + 1e-30)
