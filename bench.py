@@ -618,7 +618,8 @@ def seedlm_arm(args):
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+        # Arithmetic: weights rebuilt exactly in int32, products and sums in fp32.
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded PCG64 records and N(0,1) fp16 activations; runtime does not "
                 "depend on weight values)",
         "config": {"workload": WORKLOAD, "format": "C=8, P=3, K=16 (32 bits per 8 weights)",
