@@ -51,6 +51,7 @@ struct Tune {
   static constexpr int kPrefetch = (C == 8) ? 1 : 2;
 };
 constexpr int kRowsPerTask = 4;
+constexpr int kMinWarps = 8;      // warps per CTA however few items it has
 constexpr int kMaxGroups = 128;  // row groups per partial-sum pass (fewer if x needs the room)
 
 struct GemvGeom {
@@ -368,6 +369,10 @@ int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* epla
   int items_per_cta = (g.groups + grid - 1) / grid * g.n_spans;
   const int max_warps = (f.C == 8) ? Tune<8>::kWarps : Tune<12>::kWarps;
   int wpc = items_per_cta < max_warps ? items_per_cta : max_warps;
+  // At least 8 warps: on small matrices the CTA's setup (x and the tables
+  // into shared memory) outweighs its one or two items, and warps without
+  // items still share it.
+  if (wpc < kMinWarps) wpc = kMinWarps;
   const void* kern = (f.C == 8) ? (const void*)gemv_kernel<8> : (const void*)gemv_kernel<12>;
   int rc = allow_max_smem(kern, dev);
   if (rc) return rc;
