@@ -12,6 +12,7 @@ the planted-seed pin.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import subprocess
 import threading
@@ -69,6 +70,15 @@ def _load():
             lib.oracle_gemm.argtypes = [P(_Fmt), ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_int]
+            u32 = ctypes.c_uint32
+            lib.oracle_lfsr_next_k.restype = u32
+            lib.oracle_lfsr_next_k.argtypes = [u32, ctypes.c_int, u32]
+            lib.oracle_lfsr_period_k.restype = ctypes.c_uint64
+            lib.oracle_lfsr_period_k.argtypes = [ctypes.c_int, u32]
+            lib.oracle_block_basis_k.argtypes = [u32, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 u32, ctypes.c_void_p]
+            lib.oracle_basis_all_k.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u32,
+                                               ctypes.c_void_p]
             _lib = lib
     return _lib
 
@@ -131,6 +141,50 @@ def basis_all(C: int, P: int) -> np.ndarray:
     """U(s) for s = 1..65535 as a (65535, C, P) float64 array."""
     U = np.zeros((65535, C, P), np.float64)
     _load().oracle_basis_all(C, P, _ptr(U))
+    return U
+
+
+# ------------------------------------------------------ design-space variants
+
+#: Taps of the 16-bit register the workload specifies (bits 0, 2, 3, 5:
+#: s ^ s>>2 ^ s>>3 ^ s>>5).
+TAPS_K16 = 0x2D
+
+
+def lfsr_next_k(s: int, K: int, taps: int) -> int:
+    return int(_load().oracle_lfsr_next_k(s, K, taps))
+
+
+def lfsr_period_k(K: int, taps: int) -> int:
+    """Steps from state 1 back to 1 (0 if it never returns within 2^K)."""
+    return int(_load().oracle_lfsr_period_k(K, taps))
+
+
+@functools.lru_cache(maxsize=None)
+def primitive_taps(K: int) -> int:
+    """Taps of the K-bit register used for the design-space variants: the
+    spec's taps for K = 16, otherwise the smallest odd tap mask whose register
+    visits all 2^K - 1 nonzero states (found by brute force; the pages give
+    no polynomial for any K)."""
+    if K == 16:
+        return TAPS_K16
+    full = (1 << K) - 1
+    for taps in range(1, 1 << K, 2):
+        if lfsr_period_k(K, taps) == full:
+            return taps
+    raise ValueError(f"no maximal-length register for K = {K}")
+
+
+def block_basis_k(seed: int, C: int, P: int, K: int, taps: int) -> np.ndarray:
+    U = np.zeros((C, P), np.float64)
+    _load().oracle_block_basis_k(seed, C, P, K, taps, _ptr(U))
+    return U
+
+
+def basis_all_k(C: int, P: int, K: int, taps: int) -> np.ndarray:
+    """U(s) for s = 1 .. 2^K - 1 as a (2^K - 1, C, P) float64 array."""
+    U = np.zeros(((1 << K) - 1, C, P), np.float64)
+    _load().oracle_basis_all_k(C, P, K, taps, _ptr(U))
     return U
 
 

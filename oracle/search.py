@@ -19,7 +19,7 @@ import functools
 
 import numpy as np
 
-from . import basis_all
+from . import basis_all, basis_all_k
 
 
 @functools.lru_cache(maxsize=4)
@@ -29,11 +29,28 @@ def _tables(C: int, P: int):
     return U, Upinv
 
 
+@functools.lru_cache(maxsize=4)
+def _tables_k(C: int, P: int, K: int, taps: int):
+    U = basis_all_k(C, P, K, taps)      # (2^K - 1, C, P)
+    Upinv = np.linalg.pinv(U)           # (2^K - 1, P, C)
+    return U, Upinv
+
+
 def seed_search(w, C: int, P: int):
     """Best (seed, q, e, err, w_hat) for the length-C block ``w``."""
+    return _search(w, C, *_tables(C, P))
+
+
+def seed_search_k(w, C: int, P: int, K: int, taps: int):
+    """The same search over the 2^K - 1 seeds of a K-bit register with the
+    given taps (design-space variants: other block sizes C, latent
+    dimensions P and seed widths K)."""
+    return _search(w, C, *_tables_k(C, P, K, taps))
+
+
+def _search(w, C: int, U, Upinv):
     w = np.asarray(w, dtype=np.float64)
     assert w.shape == (C,)
-    U, Upinv = _tables(C, P)
     tstar = Upinv @ w                   # (65535, P)
     best = None
     for e in range(15, -1, -1):         # descending so that ties keep the largest e

@@ -78,6 +78,45 @@ void oracle_basis_all(int C, int P, double* U_all) {
     oracle_block_basis((uint16_t)s, C, P, U_all + (size_t)(s - 1) * (size_t)(C * P));
 }
 
+/* The general register of seedlm_oracle.h, one step. */
+uint32_t oracle_lfsr_next_k(uint32_t s, int K, uint32_t taps) {
+  uint32_t v = s & taps, parity = 0;
+  while (v) {
+    parity ^= v & 1u;
+    v >>= 1;
+  }
+  return (s >> 1) | (parity << (K - 1));
+}
+
+uint64_t oracle_lfsr_period_k(int K, uint32_t taps) {
+  const uint64_t limit = (uint64_t)1 << K;
+  uint32_t s = 1;
+  for (uint64_t n = 1; n <= limit; ++n) {
+    s = oracle_lfsr_next_k(s, K, taps);
+    if (s == 1) return n;
+  }
+  return 0;
+}
+
+void oracle_block_basis_k(uint32_t seed, int C, int P, int K, uint32_t taps, double* U) {
+  uint32_t* st = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)(C * P));
+  uint32_t s = seed;
+  for (int k = 0; k < C * P; ++k) {
+    st[k] = s;
+    s = oracle_lfsr_next_k(s, K, taps);
+  }
+  const double half = ldexp(1.0, K - 1);
+  for (int c = 0; c < C; ++c)
+    for (int p = 0; p < P; ++p) U[c * P + p] = ((double)st[p * C + c] - half) / half;
+  free(st);
+}
+
+void oracle_basis_all_k(int C, int P, int K, uint32_t taps, double* U_all) {
+  const uint32_t n = (1u << K) - 1u;
+  for (uint32_t s = 1; s <= n; ++s)
+    oracle_block_basis_k(s, C, P, K, taps, U_all + (size_t)(s - 1) * (size_t)(C * P));
+}
+
 /* Eq (1) of the paperhub.cn thread: W_blk = U t, with t_p = q_p * 2^-e. */
 int oracle_reconstruct_block(const oracle_format* f, const uint32_t* rec, const uint8_t* eplane,
                              int r, int b, double* wblk) {

@@ -74,6 +74,26 @@ void oracle_block_basis(uint16_t seed, int C, int P, double* U);
 /* U(seed) for every seed 1..65535, seed s at U_all + (s-1)*C*P. */
 void oracle_basis_all(int C, int P, double* U_all);
 
+/* Design-space variants (the pages' discussion of seed bit-width, block size
+ * and latent dimension; review thread on paperhub.cn and the atlas.scime.ai
+ * summary, "Limitations"): a K-bit Fibonacci register, 2 <= K <= 24, that
+ * shifts right and feeds the parity of the tapped bits in at the top:
+ *     bit = parity(s & taps);  s <- (s >> 1) | (bit << (K - 1)).
+ * For K = 16 and taps = 0x2D this is the register above. */
+uint32_t oracle_lfsr_next_k(uint32_t s, int K, uint32_t taps);
+
+/* Steps from state 1 until the register first returns to 1; 0 if it has not
+ * returned after 2^K steps (the taps are then not invertible). */
+uint64_t oracle_lfsr_period_k(int K, uint32_t taps);
+
+/* U(seed), C x P row-major, for a K-bit register: column p holds states
+ * p*C .. p*C + C - 1 (state_0 = seed), each mapped to
+ * (state - 2^(K-1)) / 2^(K-1). */
+void oracle_block_basis_k(uint32_t seed, int C, int P, int K, uint32_t taps, double* U);
+
+/* U(s) for every seed 1 .. 2^K - 1, seed s at U_all + (s-1)*C*P. */
+void oracle_basis_all_k(int C, int P, int K, uint32_t taps, double* U_all);
+
 /* W_blk = U t for block b of row r (all C weights, including any past cols). */
 int oracle_reconstruct_block(const oracle_format* f, const uint32_t* rec, const uint8_t* eplane,
                              int r, int b, double* wblk);
