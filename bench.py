@@ -180,6 +180,29 @@ def oracle_sample(shapes, fmt_cp, rows_per_shape, threads, seed=5):
     return weights, secs
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_single_thread(shapes, fmt_cp, target_s=3.0):
+    """The oracle on one host thread: GB/s FP16-equivalent on the first rows
+    of each layer shape, about `target_s` of work."""
+    w0, s0 = oracle_sample(shapes, fmt_cp, 8, 1)
+    rows = max(8, int(8 * target_s / max(s0, 1e-3)))
+    w, s = oracle_sample(shapes, fmt_cp, rows, 1)
+    return {"value": round(2 * w / s / 1e9, 6), "unit": UNIT, "cores": 1,
+            "sample": f"first {rows} rows of each of the 4 layer shapes: "
+                      f"{w / 1e6:.1f} M weights in {s:.1f} s, fp64, 1 host thread"}
+
+
 def cpu_baseline(shapes, fmt_cp, target_s=12.0):
     """The oracle on the host cores: the first rows of each layer shape (all
     rows if that is quick), repeated until about `target_s` of CPU work."""
@@ -197,6 +220,8 @@ def cpu_baseline(shapes, fmt_cp, target_s=12.0):
             "kind": "oracle",
             "sample": f"first {rows} rows of each of the 4 layer shapes, {passes} pass(es): "
                       f"{w / 1e6:.1f} M weights in {s:.1f} s, fp64, {threads} host threads",
+            "cpu_model": cpu_model(),
+            "single_thread": cpu_single_thread(shapes, fmt_cp),
             "encode": cpu_encode_baseline()}
 
 
@@ -241,6 +266,11 @@ def replicate(torch, layer, copies):
         res.append([dict(m, rec=m["rec"].clone(), ep=None if m["ep"] is None else m["ep"].clone())
                     for m in layer])
     return res
+
+
+def time_median(torch, fn, reps, regions=5):
+    """Median over `regions` timed regions of `reps` calls each: ms per call."""
+    return statistics.median(time_region(torch, fn, reps) / reps for _ in range(regions))
 
 
 def time_region(torch, fn, reps):
@@ -292,7 +322,7 @@ def extras(torch, sl, args):
         call = lambda i: sl.gemv(f, layer["rec"], None, x, y)  # noqa: E731
         for i in range(20):
             call(i)
-        warm = time_region(torch, call, 1000) / 1000 * 1e3
+        warm = time_median(torch, call, 1000) * 1e3
         g = torch.cuda.CUDAGraph()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
@@ -303,12 +333,12 @@ def extras(torch, sl, args):
                     sl.gemv(f, layer["rec"], None, x, y, stream=s)
         torch.cuda.current_stream().wait_stream(s)
         g.replay()
-        graph = time_region(torch, lambda i: g.replay(), 3) / 3000 * 1e3
+        graph = time_median(torch, lambda i: g.replay(), 1) / 1000 * 1e3
         del g
         copies = max(2, math.ceil(4 * l2 / layer["rec"].numel() / 4))
         recs = [layer["rec"].clone() for _ in range(copies)]
-        cold = time_region(torch, lambda i: sl.gemv(f, recs[i % copies], None, x, y),
-                           max(1000, copies)) / max(1000, copies) * 1e3
+        cold = time_median(torch, lambda i: sl.gemv(f, recs[i % copies], None, x, y),
+                           max(1000, copies)) * 1e3
         del recs
         comp = n * layer["fmt"]["rec_pitch"] * 4
         sweep[f"{n}x{n}"] = {"us_per_call": round(warm, 3), "us_per_call_graph": round(graph, 3),
@@ -335,7 +365,7 @@ def extras(torch, sl, args):
             sl.gemv(f, m["rec"], None, xl[m["N"]], y, stream=stream)
     for i in range(8):
         run70(copies[i % 4])
-    eager = time_region(torch, lambda i: run70(copies[i % 4]), 400) / 400 * 1e3
+    eager = time_median(torch, lambda i: run70(copies[i % 4]), 80) * 1e3
     graphs = []
     gs = torch.cuda.Stream()
     gs.wait_stream(torch.cuda.current_stream())
@@ -348,7 +378,7 @@ def extras(torch, sl, args):
     torch.cuda.current_stream().wait_stream(gs)
     for i in range(8):
         graphs[i % 4].replay()
-    graph = time_region(torch, lambda i: graphs[i % 4].replay(), 400) / 400 * 1e3
+    graph = time_median(torch, lambda i: graphs[i % 4].replay(), 80) * 1e3
     out["llama3_70b_layer_graph_vs_eager"] = {"us_per_layer_eager": round(eager, 2),
                                              "us_per_layer_graph": round(graph, 2)}
     del graphs, copies, layer
@@ -368,9 +398,9 @@ def extras(torch, sl, args):
             sl.gemv(f, m["rec"], m["ep"], xs[m["N"]], y)
     for i in range(5):
         run_layer(layer)
-    one = time_region(torch, lambda i: run_layer(layer), 200) / 200 * 1e3
+    one = time_median(torch, lambda i: run_layer(layer), 100) * 1e3
     copies = replicate(torch, layer, 32)
-    cold = time_region(torch, lambda i: run_layer(copies[i % 32]), 320) / 320 * 1e3
+    cold = time_median(torch, lambda i: run_layer(copies[i % 32]), 64) * 1e3
     del copies
     w, comp, _ = layer_bytes(LAYER_8B, (12, 4))
     out["llama3_8b_layer_3bit"] = {
@@ -380,14 +410,18 @@ def extras(torch, sl, args):
         "compressed_gbs": round(comp / cold / 1e3, 1)}
     del layer
 
-    # Small-M GEMM on the 70B MLP shapes, 4-bit and 3-bit, M in {1,8,16,64}.
+    # Small-M GEMM on the 70B MLP shapes, 4-bit and 3-bit, M in {1,8,16,64},
+    # rotating over distinct record copies totalling >= 4x L2.
     gemm = {}
     for cp, tag in (((8, 3), "4bit"), ((12, 4), "3bit")):
         for name, R, N in (("up_28672x8192", 28672, 8192), ("down_8192x28672", 8192, 28672)):
-            mats = make_layer_on_device(torch, [(name, R, N)], cp, 900 + R)
-            mats = [mats[0], dict(mats[0], rec=mats[0]["rec"].clone(),
-                                  ep=None if mats[0]["ep"] is None else mats[0]["ep"].clone())]
-            f = sl.Format.from_dict(mats[0]["fmt"])
+            base = make_layer_on_device(torch, [(name, R, N)], cp, 900 + R)[0]
+            nbytes = base["rec"].numel() * 4 + (0 if base["ep"] is None else base["ep"].numel())
+            ncp = max(2, math.ceil(4 * l2 / nbytes))
+            mats = [base] + [dict(base, rec=base["rec"].clone(),
+                                  ep=None if base["ep"] is None else base["ep"].clone())
+                             for _ in range(ncp - 1)]
+            f = sl.Format.from_dict(base["fmt"])
             # bf16 activations (three bf16 pieces of W) at every M, fp16 (two
             # fp16 pieces) at M = 16 and 64.
             for M, dt in ((1, "bf16"), (8, "bf16"), (16, "bf16"), (64, "bf16"), (16, "f16"),
@@ -397,31 +431,54 @@ def extras(torch, sl, args):
                     torch.bfloat16 if dt == "bf16" else torch.float16)
                 Y = torch.empty((M, R), device="cuda")
                 ws = sl.gemm_workspace(f, M)
-                fn = lambda i: sl.gemm_smallM(f, mats[i % 2]["rec"], mats[i % 2]["ep"], X, Y,  # noqa
+                fn = lambda i: sl.gemm_smallM(f, mats[i % ncp]["rec"], mats[i % ncp]["ep"], X, Y,  # noqa
                                               workspace=ws)
                 fn(0)
-                reps = 50
-                us = time_region(torch, fn, reps) / reps * 1e3
+                us = time_median(torch, fn, 4 * ncp) * 1e3
                 key = f"{tag}/{name}/M={M}" + ("" if dt == "bf16" else "/f16")
                 gemm[key] = {
                     "us_per_call": round(us, 2), "weights_per_s_e9": round(R * N / us / 1e3, 2),
-                    "tflops_useful": round(2 * M * R * N / us / 1e6, 2)}
+                    "tflops_useful": round(2 * M * R * N / us / 1e6, 2), "copies": ncp}
             xb, _ = inputs.make_activations((N,), "bf16", 990)
             x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
             y = torch.empty(R, device="cuda")
-            fn = lambda i: sl.gemv(f, mats[i % 2]["rec"], mats[i % 2]["ep"], x, y)  # noqa
+            fn = lambda i: sl.gemv(f, mats[i % ncp]["rec"], mats[i % ncp]["ep"], x, y)  # noqa
             fn(0)
-            gemm[f"{tag}/{name}/gemv_bf16"] = {"us_per_call": round(time_region(torch, fn, 50)
-                                                                    / 50 * 1e3, 2)}
-            del mats
+            gemm[f"{tag}/{name}/gemv_bf16"] = {"us_per_call": round(time_median(torch, fn, 4 * ncp)
+                                                                    * 1e3, 2)}
+            del mats, base
     out["gemm_smallM"] = gemm
+
+    # Dense fp16 reference for the crossover on the same shapes: the weights
+    # as fp16 (2 bytes each), Y = X W^T through cuBLAS (torch.matmul, fp32
+    # accumulation) at M in {8, 16, 64} and the in-house dense GEMV at M = 1,
+    # rotating over copies totalling >= 4x L2.
+    dense_mm = {}
+    for name, R, N in (("up_28672x8192", 28672, 8192), ("down_8192x28672", 8192, 28672)):
+        Wd = torch.randn((R, N), device="cuda", dtype=torch.float16) * 0.02
+        ncp = max(2, math.ceil(4 * l2 / (Wd.numel() * 2)))
+        Ws = [Wd] + [Wd.clone() for _ in range(ncp - 1)]
+        for M in (1, 8, 16, 64):
+            X = torch.randn((M, N), device="cuda", dtype=torch.float16)
+            if M == 1:
+                y = torch.empty(R, device="cuda")
+                fn = lambda i: sl.dense_gemv_f16(Ws[i % ncp], X[0], y)  # noqa
+            else:
+                fn = lambda i: torch.matmul(X, Ws[i % ncp].t())  # noqa
+            fn(0)
+            us = time_median(torch, fn, 4 * ncp) * 1e3
+            dense_mm[f"{name}/M={M}"] = {"us_per_call": round(us, 2),
+                                         "hbm_gbs": round(2 * R * N / us / 1e3, 1),
+                                         "impl": "in-house GEMV" if M == 1 else "cuBLAS"}
+        del Ws, Wd
+    out["dense_fp16_smallM"] = dense_mm
 
     # Decompression of the 70B down projection (fp32 output).
     m = make_layer_on_device(torch, [("down", 8192, 28672)], (8, 3), 1100)[0]
     f = sl.Format.from_dict(m["fmt"])
     W = torch.empty((8192, 28672), device="cuda")
     sl.decompress(f, m["rec"], None, W)
-    us = time_region(torch, lambda i: sl.decompress(f, m["rec"], None, W), 20) / 20 * 1e3
+    us = time_median(torch, lambda i: sl.decompress(f, m["rec"], None, W), 10) * 1e3
     moved = W.numel() * 4 + m["rec"].numel() * 4
     out["decompress_4bit_8192x28672"] = {"us_per_call": round(us, 1),
                                         "hbm_gbs_read_plus_write": round(moved / us / 1e3, 1)}
@@ -451,6 +508,30 @@ def extras(torch, sl, args):
         del rec_e, ep_e, err_e
     del We
 
+    # Design-space sweep: exhaustive search (all 2^K - 1 seeds, 16 exponents)
+    # on Gaussian blocks for other block sizes C, latent dimensions P and
+    # seed widths K; relative reconstruction error against bits per weight
+    # ((K + 4P + 4) / C).
+    sweep_ds = {}
+    for C, P, K, nblk in ((8, 3, 16, 16384), (8, 4, 16, 16384), (8, 2, 16, 16384),
+                          (12, 3, 16, 16384), (12, 4, 16, 16384), (16, 4, 16, 16384),
+                          (16, 3, 16, 16384), (8, 3, 12, 16384), (8, 3, 14, 16384),
+                          (8, 3, 18, 4096), (8, 3, 20, 1024)):
+        rng = np.random.default_rng(1000 + C * 100 + P * 10 + K)
+        Wb = torch.from_numpy((rng.standard_normal((nblk, C)) * 0.02).astype(np.float32)).cuda()
+        sd = torch.empty(nblk, dtype=torch.int32, device="cuda")
+        qd = torch.empty((nblk, P), dtype=torch.int8, device="cuda")
+        ed = torch.empty(nblk, dtype=torch.uint8, device="cuda")
+        er = torch.empty(nblk, dtype=torch.float64, device="cuda")
+        sl.search_blocks(C, P, K, Wb, sd, qd, ed, er)
+        ms = time_region(torch, lambda i: sl.search_blocks(C, P, K, Wb, sd, qd, ed, er), 1)
+        rel = math.sqrt(float(er.sum()) / float((Wb.double() ** 2).sum()))
+        sweep_ds[f"C={C},P={P},K={K}"] = {
+            "bits_per_weight": round((K + 4 * P + 4) / C, 3), "relative_error": round(rel, 4),
+            "blocks": nblk, "ms": round(ms, 1)}
+        del Wb, sd, qd, ed, er
+    out["design_space_sweep"] = sweep_ds
+
     # Dense fp16 GEMV (in-house) on the 70B layer shapes, 4 rotating copies.
     rng = np.random.default_rng(3)
     dense = []
@@ -466,11 +547,62 @@ def extras(torch, sl, args):
             sl.dense_gemv_f16(cps[i % 4], xsd[N], y)
     for i in range(4):
         dense_layer(i)
-    us = time_region(torch, dense_layer, 40) / 40 * 1e3
+    us = time_median(torch, dense_layer, 20) * 1e3
     w, _, _ = layer_bytes(LAYER_70B, (8, 3))
     out["dense_fp16_gemv_70b_layer"] = {"us_per_layer": round(us, 2),
                                        "hbm_gbs": round(2 * w / us / 1e3, 1)}
     del dense
+
+    # The same reference on the Llama-3-8B layer shapes (the 3-bit workload).
+    dense8 = []
+    for name, R, N in LAYER_8B:
+        Wh = (torch.randn((R, N), device="cuda") * 0.02).half()
+        dense8.append([Wh] + [Wh.clone() for _ in range(7)])
+    xs8 = {N: torch.randn(N, device="cuda").half() for N in (4096, 14336)}
+    ys8 = [torch.empty(R, device="cuda") for _, R, _ in LAYER_8B]
+
+    def dense_layer8(i):
+        for cps, (_, R, N), y in zip(dense8, LAYER_8B, ys8):
+            sl.dense_gemv_f16(cps[i % 8], xs8[N], y)
+    for i in range(8):
+        dense_layer8(i)
+    us = time_median(torch, dense_layer8, 40) * 1e3
+    w8, _, _ = layer_bytes(LAYER_8B, (12, 4))
+    out["dense_fp16_gemv_8b_layer"] = {"us_per_layer": round(us, 2),
+                                      "hbm_gbs": round(2 * w8 / us / 1e3, 1)}
+    del dense8
+    return out
+
+
+def summarize(result, hbm_peak):
+    """The figures a reader looks for first, compact, at the end of the line."""
+    ex = result["extras"]
+    out = {"llama3_70b_4bit_us_per_layer": round(result["ms_per_step"] * 1e3, 2),
+           "llama3_70b_4bit_roofline_frac": result["roofline"]["frac"]}
+    d70 = ex.get("dense_fp16_gemv_70b_layer", {}).get("us_per_layer")
+    if d70:
+        out["llama3_70b_speedup_vs_dense_fp16"] = round(d70 / (result["ms_per_step"] * 1e3), 3)
+    l8 = ex.get("llama3_8b_layer_3bit")
+    if l8:
+        _, comp8, alg8 = layer_bytes(LAYER_8B, (12, 4))
+        us8 = l8["us_per_layer_32_copies"]
+        out["llama3_8b_3bit_us_per_layer"] = us8
+        out["llama3_8b_3bit_roofline_frac"] = round(alg8 / us8 / 1e3 / hbm_peak, 4)
+        d8 = ex.get("dense_fp16_gemv_8b_layer", {}).get("us_per_layer")
+        if d8:
+            out["llama3_8b_speedup_vs_dense_fp16"] = round(d8 / us8, 3)
+    g = ex.get("gemm_smallM", {})
+    dm = ex.get("dense_fp16_smallM", {})
+    for M in (8, 16, 64):
+        k = f"4bit/up_28672x8192/M={M}"
+        if k in g:
+            out[f"gemm_4bit_28672x8192_M{M}_us"] = g[k]["us_per_call"]
+        kd = f"up_28672x8192/M={M}"
+        if kd in dm:
+            out[f"dense_fp16_28672x8192_M{M}_us"] = dm[kd]["us_per_call"]
+    sq = ex.get("square_sweep_4bit", {})
+    for n, v in sq.items():
+        out[f"square_{n}_us_graph"] = v["us_per_call_graph"]
     return out
 
 
@@ -665,6 +797,8 @@ def seedlm_arm(args):
         result["extras"] = extras(torch, sl, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(shapes, cp, target_s=args.cpu_seconds)
+    if "extras" in result:
+        result["summary"] = summarize(result, hbm_peak)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -746,6 +880,20 @@ def profile_case(name: str):
         for _ in range(2):
             for f, rec, x, y in lay:
                 sl.gemv(f, rec, None, x, y)
+    elif name == "gemv3":
+        # The four GEMVs of one 3-bit Llama-3-8B layer, twice (capture with
+        # -s 4 -c 4; the third launch is gate+up, 28672 x 4096).
+        lay = []
+        for i, (_, R, N) in enumerate(LAYER_8B):
+            L = inputs.make_layer(R, N, 12, 4, seed=30 + i)
+            xb, _ = inputs.make_activations((N,), "f16", 40 + i)
+            lay.append((L["fmt"], torch.from_numpy(L["rec"].view(np.int32)).cuda(),
+                        torch.from_numpy(L["eplane"]).cuda(),
+                        torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16),
+                        torch.empty(R, device="cuda")))
+        for _ in range(2):
+            for f, rec, ep, x, y in lay:
+                sl.gemv(f, rec, ep, x, y)
     elif name == "encode":
         # Full seed / coefficient / exponent search of a Gaussian 2048 x 2048
         # matrix at 4 bits (524,288 blocks), twice.
@@ -778,7 +926,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
-    ap.add_argument("--case", choices=("gemv", "decompress", "gemm64", "gemm16", "dense", "encode"),
+    ap.add_argument("--case", choices=("gemv", "gemv3", "decompress", "gemm64", "gemm16", "dense",
+                                       "encode"),
                     help="run one small single-kernel workload (for ncu) and exit")
     args = ap.parse_args()
     if args.case:

@@ -112,8 +112,30 @@ SEEDLM_API int seedlm_decompress(const seedlm_format* fmt, const uint32_t* rec, 
 SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
                 const void* x, int x_dtype, float* y, seedlm_stream stream);
 
+/* Several independent GEMVs in one launch (at most 8; all of one storage
+ * format, the same C, P, K): y_k = W_k x_k for k < n.  fmts is a HOST array
+ * of n formats; recs, eplanes (may be NULL for (8,3)), xs and ys are HOST
+ * arrays of n DEVICE pointers, with the rules of seedlm_gemv for each entry
+ * and one activation type for all.  The result equals n seedlm_gemv calls
+ * bit for bit; the kernel's setup (its decode tables in shared memory) is
+ * paid once, and each CTA moves straight from its share of one product to
+ * the next, with no launch or tail between them.  The pages name the extra
+ * kernel launches of memory-bound work as a GPU cost of the method
+ * (paperhub.cn review thread, authors' reply on GPU implementation
+ * challenges); this is the library's answer for products that do not
+ * depend on each other, e.g. the projections that share one input.  Empty
+ * entries (rows == 0) are skipped; cols == 0 zeroes y_k. */
+SEEDLM_API int seedlm_gemv_batch(int32_t n, const seedlm_format* fmts,
+                                 const uint32_t* const* recs, const uint8_t* const* eplanes,
+                                 const void* const* xs, int x_dtype, float* const* ys,
+                                 seedlm_stream stream);
+
 /* Y = X W^T for a small batch: X is M x cols (row-major, type x_dtype), Y is
- * M x rows fp32 (row-major), 1 <= M <= 64.  M = 1 runs the GEMV kernel
+ * M x rows fp32 (row-major), 1 <= M <= 64 -- the batched form of the
+ * inference step of the paperhub.cn review thread (authors' reply on how
+ * inference uses s and t: the blocks are rebuilt from seed and coefficients
+ * and multiplied with the activations; a batch of M activation rows shares
+ * every rebuilt block).  M = 1 runs the GEMV kernel
  * (unless x is too wide for it); otherwise the rebuilt weight tiles feed the
  * tcgen05 tensor cores (kind::f16
  * MMAs in the activations' type: W split exactly into three bf16 pieces for
@@ -145,9 +167,11 @@ SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, 
  * call allocates or frees anything.  Calls whose workspace would not fit
  * (seedlm_gemm_smallM_workspace_bytes(fmt, M) > 16 MiB + 64 KiB) return
  * SEEDLM_EUNSUPPORTED; use seedlm_gemm_smallM with a workspace for those.
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) -- make that first call before any stream capture on
- * that device.  Every call clears the counters and then reuses the same
+ * Outside a stream capture every call looks up the array's device address
+ * (cudaGetSymbolAddress); inside a capture the address from an earlier call
+ * on the same device is used, so make one call on each device before
+ * capturing it into a graph (a first call inside a capture returns
+ * SEEDLM_EUNSUPPORTED).  Every call clears the counters and then reuses the same
  * array, so calls that overlap on the GPU (two streams, or unordered host
  * threads) race and give wrong results: order them, for example on one
  * stream. */
@@ -174,6 +198,32 @@ SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt, const uint32
  * so this is an offline (model-load) step, not part of the hot path. */
 SEEDLM_API int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_t* rec,
                              uint8_t* eplane, double* err, seedlm_stream stream);
+
+/* Design-space search (the pages' discussion of seed bit-width K, block
+ * size C and latent dimension P: paperhub.cn review thread, authors'
+ * replies on compression time against those parameters; atlas.scime.ai
+ * summary, "Limitations": the design was explored on Gaussian weights).
+ * For each of nblocks blocks of C weights (W: nblocks x C fp32, row-major,
+ * device memory) the search over all 2^K - 1 seeds of a K-bit register and
+ * e = 0..15 returns the seed, the P coefficients q (int8, nblocks x P), the
+ * exponent e and, if err != NULL (nblocks doubles, 8-byte aligned), the
+ * squared error ||w - U(s) q 2^-e||^2, under the rounding and tie rules of
+ * seedlm_encode.  The register shifts right and feeds the parity of its
+ * tapped bits in at the top (taps: seedlm_lfsr_taps(K)); U(s)[c][p] =
+ * (state_{pC+c} - 2^(K-1)) / 2^(K-1).  Supported: C in {8, 12, 16}, P in
+ * {2, 3, 4}, 8 <= K <= 20 (else SEEDLM_EUNSUPPORTED).  The call allocates
+ * its per-seed tables ((P*C + P*P) * (2^K - 1) doubles; 640 MiB at C = 16,
+ * P = 4, K = 20) with cudaMallocAsync on the stream and frees them the same
+ * way.  An offline tool (model-load or design time), not the hot path. */
+SEEDLM_API int seedlm_search_blocks(int32_t C, int32_t P, int32_t K, const float* W,
+                                    int64_t nblocks, uint32_t* seed, int8_t* q, uint8_t* e,
+                                    double* err, seedlm_stream stream);
+
+/* Tap mask of the K-bit register seedlm_search_blocks uses: 0x2D (bits 0, 2,
+ * 3, 5, the workload's register) for K = 16; for other K, whose polynomial
+ * the pages do not give, the smallest odd mask whose register visits all
+ * 2^K - 1 nonzero states.  0 for K outside 8..20.  HOST function. */
+SEEDLM_API uint32_t seedlm_lfsr_taps(int32_t K);
 
 /* Failure-path self test (no counterpart in the pages): launches one small
  * kernel whose bounded mbarrier wait -- the wait the tensor-core GEMM uses,

@@ -49,6 +49,8 @@ int device_info(DeviceInfo* out) {
   return SEEDLM_OK;
 }
 
+}  // namespace
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int check_format(const seedlm_format* f) {
@@ -69,8 +71,6 @@ int check_planes(const seedlm_format* f, const uint32_t* rec, const uint8_t* epl
   if (f->P == 4 && !eplane) return SEEDLM_EINVAL;
   return SEEDLM_OK;
 }
-
-}  // namespace
 
 int record_cuda_error(cudaError_t err) {
   if (err == cudaSuccess) return SEEDLM_OK;
@@ -135,6 +135,47 @@ int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* ep
                      x_dtype == SEEDLM_BF16, y, (cudaStream_t)stream, dev);
 }
 
+int seedlm_gemv_batch(int32_t n, const seedlm_format* fmts, const uint32_t* const* recs,
+                      const uint8_t* const* eplanes, const void* const* xs, int x_dtype,
+                      float* const* ys, seedlm_stream stream) {
+  if (n < 0 || n > 8 || (n > 0 && (!fmts || !recs || !xs || !ys))) return SEEDLM_EINVAL;
+  if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
+  int rc;
+  for (int k = 0; k < n; ++k) {
+    const seedlm_format* f = &fmts[k];
+    if ((rc = check_format(f))) return rc;
+    if (f->C != fmts[0].C) return SEEDLM_EUNSUPPORTED;
+    if ((rc = check_planes(f, recs[k], eplanes ? eplanes[k] : nullptr))) return rc;
+    if (f->rows == 0) continue;
+    if (!ys[k] || !aligned(ys[k], 4)) return SEEDLM_EINVAL;
+    if (f->cols > 0 && (!xs[k] || !aligned(xs[k], 2))) return SEEDLM_EINVAL;
+  }
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const seedlm_format* f[8];
+  const uint32_t* r[8];
+  const uint8_t* e[8];
+  const uint16_t* x[8];
+  float* y[8];
+  int m = 0;
+  for (int k = 0; k < n; ++k) {
+    if (fmts[k].rows == 0) continue;
+    if (fmts[k].cols == 0) {
+      if ((rc = record_cuda_error(cudaMemsetAsync(ys[k], 0, (size_t)fmts[k].rows * sizeof(float),
+                                                  (cudaStream_t)stream))))
+        return rc;
+      continue;
+    }
+    f[m] = &fmts[k];
+    r[m] = recs[k];
+    e[m] = eplanes ? eplanes[k] : nullptr;
+    x[m] = static_cast<const uint16_t*>(xs[k]);
+    y[m] = ys[k];
+    ++m;
+  }
+  return launch_gemv_batch(m, f, r, e, x, x_dtype == SEEDLM_BF16, y, (cudaStream_t)stream, dev);
+}
+
 int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
                        const void* X, int x_dtype, int M, float* Y, void* workspace,
                        int64_t workspace_bytes, seedlm_stream stream) {
@@ -153,7 +194,7 @@ int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint
         cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), (cudaStream_t)stream));
   const uint16_t* Xh = static_cast<const uint16_t*>(X);
   // M = 1 runs the GEMV unless x is too wide for its shared memory.
-  if (M == 1 && gemv_smem_bytes(*fmt, dev.max_smem_optin) > 0)
+  if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0)
     return launch_gemv(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, Y, (cudaStream_t)stream,
                        dev);
   return launch_gemm_tc(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, M, Y, workspace,
@@ -166,7 +207,7 @@ int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M) {
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
-  if (M == 1 && gemv_smem_bytes(*fmt, dev.max_smem_optin) > 0) return 0;  // the GEMV
+  if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0) return 0;  // the GEMV
   return gemm_tc_workspace_bytes(*fmt, M, dev);
 }
 
@@ -208,6 +249,8 @@ int seedlm_device_error(int* flag) {
   if ((rc = read_and_clear_tc_error(&v))) return rc;
   int out = v ? 1 : 0;
   if ((rc = read_and_clear_encode_error(&v))) return rc;
+  if (v) out |= 1;
+  if ((rc = read_and_clear_gemv_error(&v))) return rc;
   if (v) out |= 1;
   // Bounds violations recorded by a checked build (always 0 otherwise).
   int (*const readers[])(unsigned int*) = {read_and_clear_check_gemv, read_and_clear_check_decompress,

@@ -756,17 +756,26 @@ namespace {
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[64] = {};
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the name is only a host-side stand-in for it).
-int noalloc_scratch(const DeviceInfo& dev, unsigned char** out) {
+// Device address of g_noalloc_scratch on the current device (the name is only
+// a host-side stand-in for it).  Outside a stream capture it is looked up on
+// every call, so a context that was reset and reloaded the module is seen;
+// during a capture the address found by an earlier call on this device is
+// used (a lookup there could load the module inside the capture), and there
+// must have been one.
+int noalloc_scratch(const DeviceInfo& dev, cudaStream_t st, unsigned char** out) {
   if (dev.device < 0 || dev.device >= 64) return SEEDLM_EUNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t err = cudaStreamIsCapturing(st, &cap);
+  if (err != cudaSuccess) return record_cuda_error(err);
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev.device]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
-    cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (err != cudaSuccess) return record_cuda_error(err);
     if (!p) return SEEDLM_ECUDA;
     g_noalloc_addr[dev.device] = p;
+  } else if (!g_noalloc_addr[dev.device]) {
+    return SEEDLM_EUNSUPPORTED;  // first call on this device inside a capture
   }
   *out = static_cast<unsigned char*>(g_noalloc_addr[dev.device]);
   return SEEDLM_OK;
@@ -782,30 +791,22 @@ extern "C" SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt,
                                                      const uint32_t* rec, const uint8_t* eplane,
                                                      const void* X, int x_dtype, int M, float* Y,
                                                      seedlm_stream stream) {
-  if (!fmt) return SEEDLM_EINVAL;
-  const bool c8 = fmt->C == 8 && fmt->P == 3 && fmt->K == 16;
-  const bool c12 = fmt->C == 12 && fmt->P == 4 && fmt->K == 16;
-  if (!c8 && !c12) return SEEDLM_EUNSUPPORTED;
-  if (fmt->rows < 0 || fmt->cols < 0 || fmt->nb != (fmt->cols + fmt->C - 1) / fmt->C ||
-      fmt->rec_pitch < fmt->nb || fmt->rec_pitch % 4 != 0 ||
-      (c12 && fmt->e_pitch < (fmt->nb + 1) / 2))
-    return SEEDLM_EINVAL;
+  int rc = check_format(fmt);
+  if (rc) return rc;
+  if ((rc = check_planes(fmt, rec, eplane))) return rc;
   if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
   if (M < 1 || M > 64) return SEEDLM_EINVAL;
   if (fmt->rows == 0) return SEEDLM_OK;
-  if (fmt->nb > 0 && (!rec || (reinterpret_cast<uintptr_t>(rec) & 15u))) return SEEDLM_EINVAL;
-  if (fmt->nb > 0 && c12 && !eplane) return SEEDLM_EINVAL;
-  if (!Y || (reinterpret_cast<uintptr_t>(Y) & 3u)) return SEEDLM_EINVAL;
-  if (fmt->cols > 0 && (!X || (reinterpret_cast<uintptr_t>(X) & 1u))) return SEEDLM_EINVAL;
+  if (!Y || !aligned(Y, 4)) return SEEDLM_EINVAL;
+  if (fmt->cols > 0 && (!X || !aligned(X, 2))) return SEEDLM_EINVAL;
   DeviceInfo dev;
-  int rc = current_device_info(&dev);
-  if (rc) return rc;
+  if ((rc = current_device_info(&dev))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if (fmt->cols == 0)
     return record_cuda_error(cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), st));
   const uint16_t* Xh = static_cast<const uint16_t*>(X);
   const int is_bf16 = x_dtype == SEEDLM_BF16;
-  if (M == 1 && gemv_smem_bytes(*fmt, dev.max_smem_optin) > 0)
+  if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0)
     return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
 
   int ctas = 1;
@@ -813,7 +814,7 @@ extern "C" SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt,
   const TcWorkspace w = tc_workspace(g, fmt->C, ctas);
   if (w.total() > kNoAllocBytes) return SEEDLM_EUNSUPPORTED;  // needs more than the library holds
   unsigned char* base = nullptr;
-  if ((rc = noalloc_scratch(dev, &base))) return rc;
+  if ((rc = noalloc_scratch(dev, st, &base))) return rc;
   // The counters must start at zero; the last call may have left them in any
   // state if it failed part-way.
   if ((rc = record_cuda_error(cudaMemsetAsync(base, 0, (size_t)w.cnt_bytes, st)))) return rc;

@@ -4,35 +4,87 @@
 // uses Eq (1)): the seed and coefficients of each block are read from memory,
 // the block is rebuilt and consumed at once; W never exists in full precision.
 //
-// Work decomposition (one CTA per SM, up to 16 warps, persistent):
-//   * x is converted to fp32 once per CTA into shared memory, zero-padded, in
-//     a swizzled "record pair" layout: for records 2rp and 2rp+1 of a row the
-//     x values of column c of both blocks sit side by side, so one packed
-//     fp32x2 FMA consumes weight c of both blocks.  The XOR swizzle makes the
-//     lanes of a quarter-warp hit distinct banks.
+// On B200 this product is bound by the SM, not by HBM: a 4-bit block of 8
+// weights costs 16 dp2a, 8 funnel shifts and 8 packed fp32 operations of
+// arithmetic (seedlm_device.cuh) plus its decode, and the decode's table
+// lookups are random.  The kernel is organised around two facts:
+//
+//   * Lane-replicated tables, conflict-free.  Every decode table (the stream
+//     jump tables, and for C = 8 the coefficient tables) is stored once per
+//     lane, in rows of 256 bytes: row v holds entry v for each lane side by
+//     side (4-byte entries: lanes 0..31; 8-byte entries: lanes 0..15, one
+//     half-warp at a time).  Lane l therefore always reads its own bank (bank
+//     pair) whatever index it looks up: one shared-memory wavefront per
+//     lookup instead of ~3.2 for random indices into a single copy, which
+//     saturated the shared-memory pipe before.
+//   * One-instruction table addresses.  The table rows start at fixed shared
+//     addresses (kTabJump, kTabCoef), so the address of (row v, lane l) is
+//     (v << 8) | lane_offset: one prmt moves the index byte of the record
+//     next to the lane's offset byte, and the table base rides in the load's
+//     immediate offset.  The dynamic shared allocation must start at shared
+//     address kSmemBase for this (checked at entry; a mismatch raises the
+//     device error flag and the kernel does nothing).
+//
+// Work decomposition (one CTA per SM, persistent):
+//   * x is converted to fp32 into shared memory in a swizzled "record pair"
+//     layout: for records 2rp and 2rp+1 of a row the x values of column c of
+//     both blocks sit side by side, so one packed fp32x2 FMA consumes weight
+//     c of both blocks.  x is staged in column segments of at most
+//     kMaxSegSpans<C> spans (32 record pairs each), so any width works.
 //   * An item is a group of 4 rows x one span of 32 record pairs (one pair
 //     per lane): the lane loads the two records of each row (8 bytes,
 //     coalesced across the warp), keeps the pair's x values in registers for
 //     all 4 rows, and accumulates one fp32x2 sum per row.  Record sets are
-//     loaded two items ahead of the one being rebuilt.
-//   * Each CTA owns a contiguous range of row groups and splits its items
-//     evenly over its warps, so every SM and every warp gets the same work
-//     to within one item.  Row sums are reduced with warp shuffles and then
-//     across warps in shared memory, in a fixed order, so every call gives
-//     the same bits.
-//   * Launched with programmatic stream serialization: the first record
-//     loads are issued before griddepcontrol.wait, so back-to-back GEMVs
-//     overlap one kernel's tail with the next one's prologue; x is read only
-//     after the wait.
+//     loaded ahead of the one being rebuilt.
+//   * Each CTA owns a contiguous range of row groups and splits the items of
+//     each (pass, segment) evenly over its warps.  Row sums are reduced with
+//     warp shuffles and added into a per-warp slot in shared memory; after a
+//     barrier the slots of each row are added in warp order -- the same
+//     order on every call -- and written.
+//   * Launched with programmatic stream serialization: the table fill runs
+//     before griddepcontrol.wait and overlaps the previous kernel's tail;
+//     records and x are read only after the wait, so they may be written by
+//     the previous kernel in the stream.
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
 
-// 1: take the C = 8 coefficient decode from two 256-entry shared tables;
-// 0: compute it with byte arithmetic and dp2a.
-#ifndef SEEDLM_GEMV_COEF_TABLES
-#define SEEDLM_GEMV_COEF_TABLES 1
+// Float operations per pair of weights (one in each of the lane's two
+// blocks): 0 = one packed fp32x2 add (int -> float) + one packed fp32x2 FMA;
+// 1 = two scalar adds + one packed FMA (moves the adds off the pipe the dp2a
+// instructions use).
+#ifndef SEEDLM_GEMV_FP_MODE
+#define SEEDLM_GEMV_FP_MODE 0
+#endif
+
+// How a C = 8 block gets its stream bits 16..47 (the LFSR states past the
+// seed).  The pages name the LFSR as the generator and note that GPUs lack
+// hardware for it (paperhub.cn review thread, authors' reply on GPU
+// implementation challenges); three ways to run it on the SM:
+//   0 = GF(2) jump tables: two lane-replicated 256-entry tables indexed by
+//       the seed's bytes, xor-ed (the library's choice);
+//   1 = register stepping: the recurrence b[m+16] = b[m]^b[m+2]^b[m+3]^b[m+5]
+//       applied to 32-bit words, three passes of shifts and xors;
+//   2 = one table of the whole 65,535-state cycle: records then hold the
+//       seed's position in the cycle instead of the seed (a one-time
+//       relabelling, a bijection), and a block's window is one 8-byte load
+//       at that position.  For comparisons only: the library's record format
+//       stores seeds, so this build does not compute the library's product.
+#ifndef SEEDLM_GEMV_LFSR
+#define SEEDLM_GEMV_LFSR 0
+#endif
+
+// Record sets in flight ahead of the one being rebuilt, C = 8.
+#ifndef SEEDLM_GEMV_PREFETCH8
+#define SEEDLM_GEMV_PREFETCH8 1
+#endif
+
+// Blocks per lane and row for C = 8 (2 or 4); see Tune below.
+#ifndef SEEDLM_GEMV_BPL8
+#define SEEDLM_GEMV_BPL8 4
 #endif
 
 namespace seedlm {
@@ -41,26 +93,75 @@ SEEDLM_CHECK_FLAG(gemv)
 
 namespace {
 
-// Warps per CTA (one CTA per SM) and record sets in flight ahead of the one
-// being rebuilt.  C = 8 runs 24 warps with one set ahead; C = 12 needs more
-// registers per lane (four dp2a windows per weight) and spills at 24 warps, so
-// it keeps 16 warps with two sets ahead.
+__device__ unsigned int g_gemv_error = 0;
+
+// Blocks of one row a lane takes per item (one 8- or 16-byte record load),
+// warps per CTA (one CTA per SM) and record sets in flight ahead of the one
+// being rebuilt.  C = 8 takes 4 blocks (a quad) per lane and row, so the
+// per-item work (addresses, loads, loop) is spread over 16 blocks; with 32
+// x values per lane that needs the register file of 16 warps.  C = 12 takes
+// 2 blocks (a pair): its four dp2a windows per weight already fill 128
+// registers.
 template <int C>
 struct Tune {
-  static constexpr int kWarps = (C == 8) ? 24 : 16;
-  static constexpr int kPrefetch = (C == 8) ? 1 : 2;
+  static constexpr int kBPL = (C == 8) ? SEEDLM_GEMV_BPL8 : 2;
+  static constexpr int kWarps = (C == 8 && kBPL == 2) ? 24 : 16;
+  static constexpr int kPrefetch = (C == 8) ? SEEDLM_GEMV_PREFETCH8 : 2;
 };
 constexpr int kRowsPerTask = 4;
 constexpr int kMinWarps = 8;      // warps per CTA however few items it has
-constexpr int kMaxGroups = 128;  // row groups per partial-sum pass (fewer if x needs the room)
+constexpr int kSpanUnits = 32;    // lane units (pairs or quads of blocks) per span
+
+// Shared-memory map (absolute shared addresses):
+//   C = 8:  [kSmemBase, 0x10000)  x slots of one column segment
+//           [0x10000, 0x20000)    stream jump-table rows
+//           [0x20000, 0x30000)    coefficient-table rows
+//   C = 12: [kSmemBase, 0x20000)  x slots of one column segment
+//           [0x20000, 0x30000)    stream jump-table rows
+//   both:   [0x30000, ...)        partial row sums of one pass
+constexpr uint32_t kSmemBase = 1024;
+constexpr uint32_t kTabCoef = 0x20000;
+template <int C>
+struct Smem {
+  static constexpr uint32_t kJump = (C == 8) ? 0x10000u : 0x20000u;
+  static constexpr uint32_t kPart = 0x30000u;
+  static constexpr uint32_t kXEnd = kJump;  // x slots end here
+  // x floats per lane unit: C * kBPL, rounded up to 32 for C = 12 (swizzle).
+  static constexpr int kSlotFloats = (C == 8) ? 8 * Tune<C>::kBPL : 32;
+  static constexpr int kSpanBytes = kSpanUnits * kSlotFloats * 4;
+  static constexpr int kMaxSegSpans = (int)(kXEnd - kSmemBase) / kSpanBytes;
+  static constexpr int kPartBytesPerGroup = kRowsPerTask * 4;  // per warp
+};
+constexpr uint32_t kTabJump = Smem<8>::kJump;
 
 struct GemvGeom {
   int rows, cols, nb, rec_pitch, e_pitch;
-  int n_spans;      // ceil(ceil(nb / 2) / 32): 32 record pairs (one per lane) per span
+  int n_spans;      // ceil(ceil(nb / kBPL) / 32)
   int groups;       // ceil(rows / 4)
-  int pass_groups;  // row groups per partial-sum pass (<= kMaxGroups)
-  int x_off;        // byte offset of the x slots in shared memory
+  int full_groups;  // groups with all 4 rows inside the matrix
+  int full_spans;   // spans whose every unit lies inside the row pitch
+  int seg_spans;    // spans per x segment (the last one may be shorter)
+  int n_segs;
+  int pass_groups;  // row groups per partial-sum pass
 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+  return v;
+}
+
+template <uint32_t OFF>
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
+  return v;
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -68,330 +169,654 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Shared-memory map: [jump tables][partial sums][x slots].  The partial-sum
-// buffer holds pass_groups row groups; x starts at x_off (both chosen by the
-// launcher so that x fits).
-template <int C>
-struct Smem {
-  // C = 8: jump tables (2 KB) + coefficient tables (4 KB); C = 12: jump tables.
-  static constexpr int kJumpBytes = (C == 8) ? 2 * 256 * 4 : 2 * 256 * 8;
-  static constexpr int kTableBytes = (C == 8) ? kJumpBytes + 2 * 256 * 8 : kJumpBytes;
-  static constexpr int kPartBytesPerGroup = kRowsPerTask * Tune<C>::kWarps * 4;
-  static constexpr int kSlotFloats = (C == 8) ? 16 : 32;  // per record pair
-};
-
-template <int C>
-__device__ __forceinline__ int x_slot_index(int rp, int c, int h) {
-  // Float index of column (record 2rp+h, weight c) in the swizzled layout.
-  if constexpr (C == 8) {
-    return rp * 16 + (((c >> 1) ^ ((rp >> 1) & 3)) << 2) + ((c & 1) << 1) + h;
-  } else {
-    return rp * 32 + (((c >> 1) ^ (rp & 7)) << 2) + ((c & 1) << 1) + h;
-  }
+#if SEEDLM_GEMV_LFSR == 1
+// One pass of the recurrence on a 32-bit word X whose bits [0, n) are stream
+// bits [0, n): bit m of the result is stream bit 16 + m for m + 5 < n.
+// x>>3 ^ x>>5 = (x ^ x>>2) >> 3, so a pass is two shift-xor pairs.
+__device__ __forceinline__ uint32_t lfsr_pass(uint32_t x) {
+  const uint32_t u = x ^ (x >> 2);
+  return u ^ (u >> 3);
 }
+#endif
 
+#if SEEDLM_GEMV_LFSR == 2
+// Seed at positions 0, 8, 16, ... of the cycle that starts at seed 1.
+struct CycleSeeds {
+  uint16_t s[8192];
+};
+constexpr CycleSeeds make_cycle_seeds() {
+  CycleSeeds t{};
+  uint32_t st = 1;
+  for (int p = 0; p < 8192 * 8; ++p) {
+    if ((p & 7) == 0) t.s[p >> 3] = (uint16_t)st;
+    const uint32_t bit = (st ^ (st >> 2) ^ (st >> 3) ^ (st >> 5)) & 1u;
+    st = (st >> 1) | (bit << 15);
+  }
+  return t;
+}
+__device__ const CycleSeeds kCycleSeeds = make_cycle_seeds();
+#endif
+
+// Fills the table rows.  Row v (256 bytes) holds, for C = 8,
+//   jump rows:  ext_lo(v) for lanes 0..31, then ext_hi(v) for lanes 0..31
+//               (4 bytes each: stream bits 16..47 of the seed bytes v and v<<8)
+//   coef rows:  tq1(v) for lanes 0..15, then tq2(v) for lanes 0..15 (8 bytes)
+// and for C = 12 the jump rows only, with 8-byte entries (stream bits 16..79)
+// for lanes 0..15.  Coefficient entries, with q the signed nibble values:
+//   tq1(v), v = q0 | q1 << 4: (kappa0, kappa1) = (q0, 256 q0 + q1) and
+//           bits(1.5 * 2^8) - 32768 (q0 + q1)
+//   tq2(v), v = q1 | q2 << 4: (kappa2, kappa3) = (256 q1 + q2, 256 q2) and
+//           -32768 q2
+// so that the block's integer start value is tq1.y + tq2.y - (e << 23).
 template <int C>
-__device__ void stage_x_and_tables(unsigned char* smem, const uint16_t* __restrict__ x, int is_bf16,
-                                   const GemvGeom& g) {
+__device__ void fill_tables(unsigned char* smem) {
+  uint4* jr = reinterpret_cast<uint4*>(smem + (Smem<C>::kJump - kSmemBase));
+#if SEEDLM_GEMV_LFSR == 2
   if constexpr (C == 8) {
-    uint32_t* t = reinterpret_cast<uint32_t*>(smem);
-    for (int i = threadIdx.x; i < 512; i += blockDim.x)
-      t[i] = (uint32_t)(i < 256 ? kStreamTables.lo[i] : kStreamTables.hi[i - 256]);
-    uint2* tq = reinterpret_cast<uint2*>(smem + Smem<8>::kJumpBytes);
-    fill_coef_tables_c8(tq, tq + 256, threadIdx.x, blockDim.x);
-  } else {
-    uint2* t = reinterpret_cast<uint2*>(smem);
-    for (int i = threadIdx.x; i < 512; i += blockDim.x) {
-      uint64_t v = i < 256 ? kStreamTables.lo[i] : kStreamTables.hi[i - 256];
-      t[i] = make_uint2((uint32_t)v, (uint32_t)(v >> 32));
+    // Cycle-window table: entry k = the seed at position 8k followed by its
+    // stream bits 16..63 (64 KB in place of the jump rows).
+    uint2* cw = reinterpret_cast<uint2*>(jr);
+    for (int i = threadIdx.x; i < 8192; i += blockDim.x) {
+      const uint32_t sd = kCycleSeeds.s[i];
+      const uint64_t ext = kStreamTables.lo[sd & 0xffu] ^ kStreamTables.hi[sd >> 8];
+      const uint64_t e = (uint64_t)sd | (ext << 16);
+      cw[i] = make_uint2((uint32_t)e, (uint32_t)(e >> 32));
+    }
+  } else
+#endif
+  // One thread per (row v, table): one 8-byte read of the jump table, eight
+  // 16-byte stores of its lane copies.
+  for (int t = threadIdx.x; t < 512; t += blockDim.x) {
+    const int v = t & 255, which = t >> 8;
+    const uint64_t e = which ? kStreamTables.hi[v] : kStreamTables.lo[v];
+    const uint32_t lo = (uint32_t)e, hi = (uint32_t)(e >> 32);
+    const uint4 q = (C == 8) ? make_uint4(lo, lo, lo, lo) : make_uint4(lo, hi, lo, hi);
+    uint4* row = jr + v * 16 + which * 8;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) row[k] = q;
+  }
+  if constexpr (C == 8) {
+    uint4* cr = reinterpret_cast<uint4*>(smem + (kTabCoef - kSmemBase));
+    for (int t = threadIdx.x; t < 512; t += blockDim.x) {
+      const int v = t & 255, which = t >> 8;
+      const int32_t a = nibble_value(v), b = nibble_value(v >> 4);
+      const uint2 e = which == 0 ? make_uint2(pack_s16(a, 256 * a + b),
+                                              kMagicBits - (uint32_t)(32768 * (a + b)))
+                                 : make_uint2(pack_s16(256 * a + b, 256 * b),
+                                              (uint32_t)(-32768 * b));
+      const uint4 q = make_uint4(e.x, e.y, e.x, e.y);
+      uint4* row = cr + v * 16 + which * 8;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) row[k] = q;
     }
   }
-  // x, zero-padded to n_spans * 32 record pairs.
-  float* xs = reinterpret_cast<float*>(smem + g.x_off);
-  const int ncols_pad = g.n_spans * 32 * 2 * C;
-  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (seedlm_dynamic_smem_bytes() - g.x_off) / 4;)
-  for (int j = threadIdx.x; j < ncols_pad; j += blockDim.x) {
-    int rp = j / (2 * C);
-    int w = j - rp * 2 * C;
-    int h = w / C;
-    int c = w - h * C;
-    float v = j < g.cols ? act_to_float(x[j], is_bf16) : 0.f;
-    const int si = x_slot_index<C>(rp, c, h);
-    if (SEEDLM_IN_BOUNDS(g_check_flag, si, xs_floats)) xs[si] = v;
+}
+
+// C = 8 decode from the replicated tables.  The record's byte 2 and byte 3
+// are the seed's low and high bytes, byte 0 is q0 | q1 << 4 and bits 4..11
+// are q1 | q2 << 4.
+__device__ __forceinline__ BlockC8 decode_c8_rep(uint32_t rec, uint32_t lane4, uint32_t lane8) {
+  BlockC8 b;
+#if SEEDLM_GEMV_LFSR == 1
+  b.lo = rec;
+  // Passes over 16, 27 and 32 valid stream bits: stream bits 16..42.
+  const uint32_t t1 = lfsr_pass(rec);                     // bits 16..26 valid at 16..26
+  const uint32_t t2 = lfsr_pass(prmt<0x7632u>(rec, t1));  // stream 0..26 -> 16..37 at 0..21
+  b.hi = lfsr_pass(prmt<0x5432u>(rec, t2));               // stream 0..31 -> 16..42 at 0..26
+#elif SEEDLM_GEMV_LFSR == 2
+  // rec bits [16,32) = position P in the cycle; the table entry k holds
+  // cycle bits [8k, 8k + 64).
+  const uint32_t pos = rec >> 16;
+  const uint2 w = lds64<kTabJump>(pos & 0xfff8u);
+  const uint32_t sh = pos & 7u;
+  const uint32_t s_lo = __funnelshift_r(w.x, w.y, sh), s_hi = w.y >> sh;  // bits [P, P+56)
+  b.lo = s_lo << 16;
+  b.hi = __funnelshift_r(s_lo, s_hi, 16);
+#else
+  b.lo = rec;
+  b.hi = lds32<kTabJump>(prmt<0x5524u>(rec, lane4)) ^
+         lds32<kTabJump + 128>(prmt<0x5534u>(rec, lane4));
+#endif
+  const uint2 c1 = lds64<kTabCoef>(prmt<0x5504u>(rec, lane8));
+  const uint2 c2 = lds64<kTabCoef + 128>(prmt<0x5514u>(rec << 4, lane8));
+  b.a01 = c1.x;
+  b.a23 = c2.x;
+  const uint32_t e23 = (rec << 11) & 0x07800000u;  // e << 23
+  b.init = (int32_t)(c1.y + c2.y - e23);
+  b.negm = kNegMagicBits - e23;
+  return b;
+}
+
+// C = 12 decode: stream windows from the replicated 8-byte jump tables, the
+// coefficients computed from the record's nibbles (seedlm_device.cuh).
+__device__ __forceinline__ BlockC12 decode_c12_rep(uint32_t rec, uint32_t e4, uint32_t lane8) {
+  BlockC12 b;
+  b.lo = rec;
+  const uint2 x0 = lds64<Smem<12>::kJump>(prmt<0x5524u>(rec, lane8));
+  const uint2 x1 = lds64<Smem<12>::kJump + 128>(prmt<0x5534u>(rec, lane8));
+  b.mid = x0.x ^ x1.x;
+  b.hi = x0.y ^ x1.y;
+  coef_c12(b, rec, e4);
+  return b;
+}
+
+// x slot layout, per lane unit u (kBPL consecutive blocks of a row):
+//   C = 8, pairs:  16 floats; float4 i holds column 2i and 2i+1 of both
+//                  blocks (h = 0, 1 interleaved), at float4 i ^ ((u >> 1) & 3)
+//   C = 8, quads:  32 floats; float4 c holds column c of blocks 0..3, at
+//                  float4 c ^ (u & 7)
+//   C = 12, pairs: 32 floats (24 used); float4 i holds columns 2i, 2i+1 of
+//                  both blocks, at float4 i ^ (u & 7)
+// so each lane reads its unit with 16-byte loads and one packed fp32x2 FMA
+// takes weight c of two blocks; the XOR swizzles keep the 8 lanes of a
+// quarter-warp on distinct bank groups.
+template <int C>
+__device__ __forceinline__ int x_slot_index(int u, int c, int h) {
+  if constexpr (C == 8 && Tune<8>::kBPL == 4) {
+    return u * 32 + ((c ^ (u & 7)) << 2) + h;
+  } else if constexpr (C == 8) {
+    return u * 16 + (((c >> 1) ^ ((u >> 1) & 3)) << 2) + ((c & 1) << 1) + h;
+  } else {
+    return u * 32 + (((c >> 1) ^ (u & 7)) << 2) + ((c & 1) << 1) + h;
   }
 }
 
-// The records one lane needs for one (row group, span) item: the pair of
-// blocks (2rp, 2rp+1) in each of the group's 4 rows, plus for C = 12 the
-// exponent byte of the pair.  Rows past `rows` and pairs past the row pitch
-// read as zero records (their x is zero, so they add nothing).
+// x columns of spans [s0, s0 + sl), zero past cols, into the segment's
+// slots.  One thread per lane unit; 16-byte loads when x is 16-byte aligned
+// and the unit lies inside x.
+template <int C>
+__device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, const GemvGeom& g,
+                        int s0, int sl) {
+  constexpr int kBPL = Tune<C>::kBPL;
+  constexpr int kVals = C * kBPL;  // x values of one unit (16, 24 or 32)
+  const int units = sl * kSpanUnits;
+  const int col_base = s0 * kSpanUnits * kVals;
+  const bool vec = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (Smem<C>::kXEnd - kSmemBase) / 4;)
+  for (int u = threadIdx.x; u < units; u += blockDim.x) {
+    const int col0 = col_base + u * kVals;
+    uint16_t v16[kVals];
+    if (vec && col0 + kVals <= g.cols) {
+#pragma unroll
+      for (int k = 0; k < kVals / 8; ++k) {
+        const uint4 q = *reinterpret_cast<const uint4*>(x + col0 + 8 * k);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          v16[8 * k + 2 * m] = (uint16_t)w[m];
+          v16[8 * k + 2 * m + 1] = (uint16_t)(w[m] >> 16);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kVals; ++k) v16[k] = col0 + k < g.cols ? x[col0 + k] : (uint16_t)0;
+    }
+#pragma unroll
+    for (int k = 0; k < kVals; ++k) {
+      const int h = k / C, c = k - h * C;
+      const int si = x_slot_index<C>(u, c, h);
+      const float f = act_to_float(v16[k], is_bf16);
+      if (SEEDLM_IN_BOUNDS(g_check_flag, si, xs_floats)) xs[si] = f;
+    }
+  }
+}
+
+// The records one lane needs for one (row group, span) item: its unit of
+// kBPL blocks in each of the group's 4 rows, plus for C = 12 the exponent
+// byte of the pair.  Rows past `rows` and units past the row pitch read as
+// zero records (their x is zero, so they add nothing).
 template <int C>
 struct RecSet {
-  uint2 r[kRowsPerTask];
+  using Unit = typename std::conditional<Tune<C>::kBPL == 4, uint4, uint2>::type;
+  Unit r[kRowsPerTask];
   uint32_t e[C == 12 ? kRowsPerTask : 1];
 };
+
+template <int C>
+__device__ __forceinline__ void load_unit(typename RecSet<C>::Unit& o, const uint32_t* p) {
+  if constexpr (Tune<C>::kBPL == 4) o = ld_stream_u4(p);
+  else o = ld_stream_u2(p);
+}
 
 template <int C>
 __device__ __forceinline__ void load_set(RecSet<C>& o, const uint32_t* __restrict__ rec,
                                          const uint8_t* __restrict__ eplane, const GemvGeom& g,
                                          int grp, int span, int lane) {
+  constexpr int kBPL = Tune<C>::kBPL;
   const int row0 = grp * kRowsPerTask;
-  const int rp = span * 32 + lane;
-  const bool pair_ok = 2 * rp < g.rec_pitch;
-  const uint32_t* p = rec + (size_t)row0 * g.rec_pitch + 2 * rp;
+  const int u = span * kSpanUnits + lane;
+  const uint32_t* p = rec + (size_t)row0 * g.rec_pitch + kBPL * u;
+  if (grp < g.full_groups && span < g.full_spans && !SEEDLM_CHECK) {
+    // Every row of the group and every unit of the span is inside the plane.
 #pragma unroll
-  for (int j = 0; j < kRowsPerTask; ++j) {
-    // The pair's second record is the last word read.
-    const bool ok = pair_ok && row0 + j < g.rows &&
-                    SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(row0 + j) * g.rec_pitch + 2 * rp + 1,
-                                     (size_t)g.rows * g.rec_pitch);
-    o.r[j] = ok ? ld_stream_u2(p + (size_t)j * g.rec_pitch) : make_uint2(0u, 0u);
-    if constexpr (C == 12)
-      o.e[j] = (ok && rp < g.e_pitch &&
-                SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(row0 + j) * g.e_pitch + rp,
+    for (int j = 0; j < kRowsPerTask; ++j) load_unit<C>(o.r[j], p + (size_t)j * g.rec_pitch);
+  } else {
+    const bool unit_ok = kBPL * u < g.rec_pitch;
+#pragma unroll
+    for (int j = 0; j < kRowsPerTask; ++j) {
+      // The unit's last record is the last word read.
+      const bool ok = unit_ok && row0 + j < g.rows &&
+                      SEEDLM_IN_BOUNDS(g_check_flag,
+                                       (size_t)(row0 + j) * g.rec_pitch + kBPL * u + kBPL - 1,
+                                       (size_t)g.rows * g.rec_pitch);
+      if (ok) load_unit<C>(o.r[j], p + (size_t)j * g.rec_pitch);
+      else o.r[j] = typename RecSet<C>::Unit{};
+    }
+  }
+  if constexpr (C == 12) {
+#pragma unroll
+    for (int j = 0; j < kRowsPerTask; ++j)
+      o.e[j] = (row0 + j < g.rows && u < g.e_pitch &&
+                SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(row0 + j) * g.e_pitch + u,
                                  (size_t)g.rows * g.e_pitch))
-                   ? ld_stream_u8(eplane + (size_t)(row0 + j) * g.e_pitch + rp)
+                   ? ld_stream_u8(eplane + (size_t)(row0 + j) * g.e_pitch + u)
                    : 0u;
   }
 }
 
-// Rebuild the lane's 2 x C weights of each of the 4 rows and accumulate
-// w * x into one fp32x2 sum per row.
+#ifndef SEEDLM_GEMV_C12_ORDER
+#define SEEDLM_GEMV_C12_ORDER 1
+#endif
+
+
+#if SEEDLM_GEMV_C12_ORDER == 1
+// Window k (stream bits [k, k+32)) of a C = 12 block holds state k in its
+// low half and state k+16 in its high half; state 12p + c belongs to weight
+// c with coefficient q_p.  Windows 0..31 cover all 48 states.
+template <int k>
+__device__ __forceinline__ void c12_windows(const BlockC12& A, const BlockC12& B, int32_t (&va)[12],
+                                            int32_t (&vb)[12]) {
+  if constexpr (k < 32) {
+    const uint32_t wa = window_c12<k>(A), wb = window_c12<k>(B);
+    constexpr int lo_p = k / 12, lo_c = k % 12;              // state k
+    constexpr int hi_p = (k + 16) / 12, hi_c = (k + 16) % 12;  // state k + 16
+    if constexpr (lo_p < 4 && k < 24) {
+      va[lo_c] = dp2a_lo_su(A.a[lo_p], wa, va[lo_c]);
+      vb[lo_c] = dp2a_lo_su(B.a[lo_p], wb, vb[lo_c]);
+    }
+    if constexpr (hi_p < 4 && k >= 8) {
+      va[hi_c] = dp2a_hi_su(A.a[hi_p], wa, va[hi_c]);
+      vb[hi_c] = dp2a_hi_su(B.a[hi_p], wb, vb[hi_c]);
+    }
+    c12_windows<k + 1>(A, B, va, vb);
+  }
+}
+#endif
+
+// Weight pair (c of block A, c of block B) -> fp32x2, accumulated against
+// the pair's x values.
+__device__ __forceinline__ float2 fma_pair(int32_t bits_a, int32_t bits_b, float2 negm, float2 xv,
+                                           float2 acc) {
+#if SEEDLM_GEMV_FP_MODE == 1
+  const float2 w = make_float2(__int_as_float(bits_a) + negm.x, __int_as_float(bits_b) + negm.y);
+  return __ffma2_rn(w, xv, acc);
+#else
+  const float2 w = make_float2(__int_as_float(bits_a), __int_as_float(bits_b));
+  return __ffma2_rn(__fadd2_rn(w, negm), xv, acc);
+#endif
+}
+
+// Blocks A and B of one row (x pairs xv[c] = (x of A's column c, x of B's)).
+__device__ __forceinline__ float2 dot_c8(uint32_t ra, uint32_t rb, const float2 (&xv)[8],
+                                         uint32_t lane4, uint32_t lane8, float2 a) {
+  const BlockC8 A = decode_c8_rep(ra, lane4, lane8);
+  const BlockC8 B = decode_c8_rep(rb, lane4, lane8);
+  const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
+#define SEEDLM_C8_STEP(c) a = fma_pair(weight_bits_c8<c>(A), weight_bits_c8<c>(B), negm, xv[c], a);
+  SEEDLM_C8_STEP(0) SEEDLM_C8_STEP(1) SEEDLM_C8_STEP(2) SEEDLM_C8_STEP(3)
+  SEEDLM_C8_STEP(4) SEEDLM_C8_STEP(5) SEEDLM_C8_STEP(6) SEEDLM_C8_STEP(7)
+#undef SEEDLM_C8_STEP
+  return a;
+}
+
+// Rebuild the lane's kBPL x C weights of each of the 4 rows and accumulate
+// w * x into one fp32x2 sum per row.  ul is the lane's unit within the
+// staged segment.
 template <int C>
 __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const float* __restrict__ xs,
-                                                int rp, int swz, const void* t_lo, const void* t_hi,
+                                                int ul, int lane, uint32_t lane4, uint32_t lane8,
                                                 float2 (&acc)[kRowsPerTask]) {
-  float2 xp[C];
+  const float* slot = xs + ul * Smem<C>::kSlotFloats;
+  if constexpr (C == 8 && Tune<8>::kBPL == 4) {
+    const int swz = lane & 7;
+    float2 x01[8], x23[8];
 #pragma unroll
-  for (int i = 0; i < C / 2; ++i) {
-    float4 v = *reinterpret_cast<const float4*>(xs + rp * Smem<C>::kSlotFloats + ((i ^ swz) << 2));
-    xp[2 * i] = make_float2(v.x, v.y);
-    xp[2 * i + 1] = make_float2(v.z, v.w);
-  }
+    for (int c = 0; c < 8; ++c) {
+      const float4 v = *reinterpret_cast<const float4*>(slot + ((c ^ swz) << 2));
+      x01[c] = make_float2(v.x, v.y);
+      x23[c] = make_float2(v.z, v.w);
+    }
 #pragma unroll
-  for (int j = 0; j < kRowsPerTask; ++j) {
-    float2 a = acc[j];
-    if constexpr (C == 8) {
-      const uint32_t* tl = static_cast<const uint32_t*>(t_lo);
-      const uint32_t* th = static_cast<const uint32_t*>(t_hi);
-#if SEEDLM_GEMV_COEF_TABLES
-      const uint2* tq1 = reinterpret_cast<const uint2*>(th + 256);
-      const BlockC8 A = decode_c8_tab(cur.r[j].x, tl, th, tq1, tq1 + 256);
-      const BlockC8 B = decode_c8_tab(cur.r[j].y, tl, th, tq1, tq1 + 256);
+    for (int j = 0; j < kRowsPerTask; ++j) {
+      float2 a = dot_c8(cur.r[j].x, cur.r[j].y, x01, lane4, lane8, acc[j]);
+      acc[j] = dot_c8(cur.r[j].z, cur.r[j].w, x23, lane4, lane8, a);
+    }
+  } else if constexpr (C == 8) {
+    const int swz = (lane >> 1) & 3;
+    float2 xp[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = *reinterpret_cast<const float4*>(slot + ((i ^ swz) << 2));
+      xp[2 * i] = make_float2(v.x, v.y);
+      xp[2 * i + 1] = make_float2(v.z, v.w);
+    }
+#pragma unroll
+    for (int j = 0; j < kRowsPerTask; ++j)
+      acc[j] = dot_c8(cur.r[j].x, cur.r[j].y, xp, lane4, lane8, acc[j]);
+  } else {
+    const int swz = lane & 7;
+    float2 xp[C];
+#pragma unroll
+    for (int i = 0; i < C / 2; ++i) {
+      const float4 v = *reinterpret_cast<const float4*>(slot + ((i ^ swz) << 2));
+      xp[2 * i] = make_float2(v.x, v.y);
+      xp[2 * i + 1] = make_float2(v.z, v.w);
+    }
+#pragma unroll
+    for (int j = 0; j < kRowsPerTask; ++j) {
+      float2 a = acc[j];
+      const BlockC12 A = decode_c12_rep(cur.r[j].x, cur.e[j], lane8);
+      const BlockC12 B = decode_c12_rep(cur.r[j].y, cur.e[j] >> 4, lane8);
+      const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
+#if SEEDLM_GEMV_C12_ORDER == 1
+      // Window-major: each of the 32 stream windows is formed once and feeds
+      // the (up to two) states that sit in its halves.
+      int32_t va[12], vb[12];
+#pragma unroll
+      for (int c = 0; c < 12; ++c) { va[c] = A.init; vb[c] = B.init; }
+      c12_windows<0>(A, B, va, vb);
+#pragma unroll
+      for (int c = 0; c < 12; ++c) a = fma_pair(va[c], vb[c], negm, xp[c], a);
 #else
-      const BlockC8 A = decode_c8(cur.r[j].x, tl, th);
-      const BlockC8 B = decode_c8(cur.r[j].y, tl, th);
-#endif
-      const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
-#define SEEDLM_C8_STEP(c)                                                        \
-  {                                                                              \
-    float2 w = make_float2(__int_as_float(weight_bits_c8<c>(A)),                 \
-                           __int_as_float(weight_bits_c8<c>(B)));                \
-    a = __ffma2_rn(__fadd2_rn(w, negm), xp[c], a);                               \
-  }
-      SEEDLM_C8_STEP(0) SEEDLM_C8_STEP(1) SEEDLM_C8_STEP(2) SEEDLM_C8_STEP(3)
-      SEEDLM_C8_STEP(4) SEEDLM_C8_STEP(5) SEEDLM_C8_STEP(6) SEEDLM_C8_STEP(7)
-#undef SEEDLM_C8_STEP
-    } else {
-      const uint2* tl = static_cast<const uint2*>(t_lo);
-      const uint2* th = static_cast<const uint2*>(t_hi);
-      const BlockC12 A = decode_c12(cur.r[j].x, cur.e[j], tl, th);
-      const BlockC12 B = decode_c12(cur.r[j].y, cur.e[j] >> 4, tl, th);
-      const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
-#define SEEDLM_C12_STEP(c)                                                       \
-  {                                                                              \
-    float2 w = make_float2(__int_as_float(weight_bits_c12<c>(A)),                \
-                           __int_as_float(weight_bits_c12<c>(B)));               \
-    a = __ffma2_rn(__fadd2_rn(w, negm), xp[c], a);                               \
-  }
+#define SEEDLM_C12_STEP(c) a = fma_pair(weight_bits_c12<c>(A), weight_bits_c12<c>(B), negm, xp[c], a);
       SEEDLM_C12_STEP(0) SEEDLM_C12_STEP(1) SEEDLM_C12_STEP(2) SEEDLM_C12_STEP(3)
       SEEDLM_C12_STEP(4) SEEDLM_C12_STEP(5) SEEDLM_C12_STEP(6) SEEDLM_C12_STEP(7)
       SEEDLM_C12_STEP(8) SEEDLM_C12_STEP(9) SEEDLM_C12_STEP(10) SEEDLM_C12_STEP(11)
 #undef SEEDLM_C12_STEP
+#endif
+      acc[j] = a;
     }
-    acc[j] = a;
   }
 }
 
-// CTA b owns the contiguous row groups [g0, g1) (sizes differ by at most
-// one group); its (group, span) items are split into equal contiguous ranges,
-// one per warp.  A warp walks its range with record sets loaded Tune<C>::kPrefetch
-// items ahead (across group boundaries), and whenever it leaves a group it
-// reduces its 4 row sums with shuffles into shared memory.  After a barrier
-// the partial sums of each row are added in warp order -- the same order on
-// every call -- and written.  Groups are processed in passes of at most
-// pass_groups so the partial-sum buffer stays small.
-template <int C>
-__global__ void __launch_bounds__(Tune<C>::kWarps * 32, 1)
-gemv_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
-            const uint16_t* __restrict__ x, int is_bf16, float* __restrict__ y, GemvGeom g) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const void* t_lo = smem;
-  const void* t_hi = smem + Smem<C>::kJumpBytes / 2;
-  float* part = reinterpret_cast<float*>(smem + Smem<C>::kTableBytes);
-  const float* xs = reinterpret_cast<const float*>(smem + g.x_off);
-  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (seedlm_dynamic_smem_bytes() - g.x_off) / 4;
-                    const int part_floats = (g.x_off - Smem<C>::kTableBytes) / 4;)
+// One launch may run several independent GEMVs of the same format (a
+// batch): the tables are filled once, and each CTA then takes its share of
+// every GEMV in turn.
+constexpr int kMaxBatch = 8;
+struct GemvBatch {
+  int n;
+  GemvGeom g[kMaxBatch];
+  const uint32_t* rec[kMaxBatch];
+  const uint8_t* ep[kMaxBatch];
+  const uint16_t* x[kMaxBatch];
+  float* y[kMaxBatch];
+};
 
+// For every GEMV of the batch, CTA b owns the contiguous row groups
+// [g0, g1) (sizes differ by at most one group), processed in passes of at
+// most pass_groups groups.  Within a pass, x is staged one column segment at
+// a time (once per GEMV when one segment holds all of x); the (group, span)
+// items of the pass and segment are split into equal contiguous ranges, one
+// per warp.  A warp walks its range with record sets loaded
+// Tune<C>::kPrefetch items ahead (across group boundaries), and whenever it
+// leaves a group it reduces its 4 row sums with shuffles and adds them into
+// its own slot of the pass's partial sums.  At the end of the pass the slots
+// of each row are added in warp order and written.
+template <int C, bool kBatch>
+__global__ void __launch_bounds__(Tune<C>::kWarps * 32, 1)
+gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
+  constexpr int kP = Tune<C>::kPrefetch;
+  extern __shared__ __align__(16) unsigned char smem[];
+  // The table addresses are absolute: the allocation must start at kSmemBase.
+  if (smem_u32(smem) != kSmemBase) {
+    if (threadIdx.x == 0) atomicOr(&g_gemv_error, 1u);
+    return;
+  }
+  float* xs = reinterpret_cast<float*>(smem);
+  float* part = reinterpret_cast<float*>(smem + (Smem<C>::kPart - kSmemBase));
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (Smem<C>::kXEnd - kSmemBase) / 4;
+                    const int part_floats =
+                        (int)(seedlm_dynamic_smem_bytes() - (Smem<C>::kPart - kSmemBase)) / 4;)
   const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int swz = (C == 8) ? ((lane >> 1) & 3) : (lane & 7);
-  const int g0 = (int)((int64_t)blockIdx.x * g.groups / gridDim.x);
-  const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
+  const uint32_t lane4 = (uint32_t)lane << 2, lane8 = (uint32_t)(lane & 15) << 3;
+  RecSet<C> buf[kP + 1];
 
-  bool first_pass = true;
-  for (int p0 = g0; p0 < g1; p0 += g.pass_groups) {
-    const int p1 = min(p0 + g.pass_groups, g1);
-    const int items = (p1 - p0) * g.n_spans;
-    const int i0 = (int)((int64_t)warp * items / nw), i1 = (int)((int64_t)(warp + 1) * items / nw);
-    // The first record sets are requested before anything else: they do not
-    // depend on x, so their latency overlaps the staging of x (and, with
-    // programmatic dependent launch, the tail of the previous kernel).
-    int grp = p0 + (i0 < i1 ? i0 / g.n_spans : 0), span = i0 < i1 ? i0 % g.n_spans : 0;
-    int lgrp = grp, lspan = span, li = i0;
-    RecSet<C> buf[Tune<C>::kPrefetch + 1];
+  fill_tables<C>(smem);
+  // Records and x may be the previous kernel's output: read them only now.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int nbatch = kBatch ? B.n : 1;
+  for (int bi = 0; bi < nbatch; ++bi) {
+    const GemvGeom g = B.g[bi];
+    const uint32_t* __restrict__ rec = B.rec[bi];
+    const uint8_t* __restrict__ eplane = B.ep[bi];
+    const uint16_t* __restrict__ x = B.x[bi];
+    float* __restrict__ y = B.y[bi];
+    const int g0 = (int)((int64_t)blockIdx.x * g.groups / gridDim.x);
+    const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
+    for (int p0 = g0; p0 < g1; p0 += g.pass_groups) {
+      const int p1 = min(p0 + g.pass_groups, g1);
+      for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x)
+        if (SEEDLM_IN_BOUNDS(g_check_flag, i, part_floats)) part[i] = 0.f;
+      for (int sg = 0; sg < g.n_segs; ++sg) {
+        const int s0 = sg * g.seg_spans;
+        const int sl = min(g.seg_spans, g.n_spans - s0);
+        // One segment: x stays staged for every pass of this GEMV.
+        if (g.n_segs > 1 || p0 == g0) stage_x<C>(xs, x, is_bf16, g, s0, sl);
+        __syncthreads();  // x, tables and zeroed partials ready
+        const int items = (p1 - p0) * sl;
+        const int i0 = (int)((int64_t)warp * items / nw);
+        const int i1 = (int)((int64_t)(warp + 1) * items / nw);
+        if (i0 < i1) {
+          // Item cursor (grp, span) and load cursor (lgrp, lspan), kP items ahead.
+          int grp = p0 + i0 / sl, span = i0 % sl;
+          int lgrp = grp, lspan = span;
 #pragma unroll
-    for (int k = 0; k <= Tune<C>::kPrefetch; ++k) {
-      if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
-      ++li;
-      if (++lspan == g.n_spans) { lspan = 0; ++lgrp; }
-    }
-    if (first_pass) {
-      // x may be the previous kernel's output: wait for it only now.
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      stage_x_and_tables<C>(smem, x, is_bf16, g);
-      first_pass = false;
-    }
-    for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x)
-      if (SEEDLM_IN_BOUNDS(g_check_flag, i, part_floats)) part[i] = 0.f;
-    __syncthreads();  // x, tables and zeroed partials ready
-    if (i0 < i1) {
-      float2 acc[kRowsPerTask];
+          for (int k = 0; k <= kP; ++k) {
+            if (i0 + k < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+            if (++lspan == sl) { lspan = 0; ++lgrp; }
+          }
+          float2 acc[kRowsPerTask];
 #pragma unroll
-      for (int j = 0; j < kRowsPerTask; ++j) acc[j] = make_float2(0.f, 0.f);
-      int ci = i0;
-      bool done = false;
-      while (!done) {
+          for (int j = 0; j < kRowsPerTask; ++j) acc[j] = make_float2(0.f, 0.f);
+          int ci = i0;
+          for (;;) {
 #pragma unroll
-        for (int k = 0; k <= Tune<C>::kPrefetch; ++k) {
-          if (!done) {
-            // Every x slot of the lane's record pair lies in its kSlotFloats row.
-            if (SEEDLM_IN_BOUNDS(g_check_flag,
-                                 (span * 32 + lane + 1) * Smem<C>::kSlotFloats - 1, xs_floats))
-              rebuild_and_dot<C>(buf[k], xs, span * 32 + lane, swz, t_lo, t_hi, acc);
-            if (li < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, lspan, lane);
-            ++li;
-            if (++lspan == g.n_spans) { lspan = 0; ++lgrp; }
-            ++ci;
-            const bool end_group = (++span == g.n_spans);
-            if (end_group || ci == i1) {
-#pragma unroll
-              for (int j = 0; j < kRowsPerTask; ++j) {
-                const float s = warp_sum(acc[j].x + acc[j].y);
-                const int pi = ((grp - p0) * kRowsPerTask + j) * nw + warp;
-                if (lane == 0 && SEEDLM_IN_BOUNDS(g_check_flag, pi, part_floats)) part[pi] = s;
-                acc[j] = make_float2(0.f, 0.f);
+            for (int k = 0; k <= kP; ++k) {
+              const int ul = span * kSpanUnits + lane;
+              // Every x slot of the lane's unit lies in its kSlotFloats row.
+              if (SEEDLM_IN_BOUNDS(g_check_flag, (ul + 1) * Smem<C>::kSlotFloats - 1, xs_floats))
+                rebuild_and_dot<C>(buf[k], xs, ul, lane, lane4, lane8, acc);
+              if (ci + kP + 1 < i1) {
+                load_set<C>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+                if (++lspan == sl) { lspan = 0; ++lgrp; }
               }
-              if (end_group) { span = 0; ++grp; }
-              done = (ci == i1);
+              ++ci;
+              const bool end_group = (++span == sl);
+              if (end_group || ci == i1) {
+#pragma unroll
+                for (int j = 0; j < kRowsPerTask; ++j) {
+                  const float sum = warp_sum(acc[j].x + acc[j].y);
+                  const int pi = ((grp - p0) * kRowsPerTask + j) * nw + warp;
+                  if (lane == 0 && SEEDLM_IN_BOUNDS(g_check_flag, pi, part_floats)) part[pi] += sum;
+                  acc[j] = make_float2(0.f, 0.f);
+                }
+                if (end_group) { span = 0; ++grp; }
+                if (ci == i1) goto range_done;
+              }
             }
           }
+        range_done:;
+        }
+        __syncthreads();  // partials complete; x may be restaged
+      }
+      if (bi == nbatch - 1 && p1 == g1) {
+        // The next kernel in the stream may start its prologue now.
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+      }
+      for (int t = threadIdx.x; t < (p1 - p0) * kRowsPerTask; t += blockDim.x) {
+        const int r = p0 * kRowsPerTask + t;
+        if (r < g.rows) {
+          float sum = 0.f;
+          for (int w = 0; w < nw; ++w)
+            if (SEEDLM_IN_BOUNDS(g_check_flag, t * nw + w, part_floats)) sum += part[t * nw + w];
+          if (SEEDLM_IN_BOUNDS(g_check_flag, r, g.rows)) y[r] = sum;
         }
       }
+      __syncthreads();  // partials read before the next pass clears them
     }
-    __syncthreads();
-    if (p1 == g1) {
-      // The next kernel in the stream may start its prologue now.
-      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    }
-    for (int t = threadIdx.x; t < (p1 - p0) * kRowsPerTask; t += blockDim.x) {
-      const int r = p0 * kRowsPerTask + t;
-      if (r < g.rows) {
-        float s = 0.f;
-        for (int w = 0; w < nw; ++w) s += part[t * nw + w];
-        if (SEEDLM_IN_BOUNDS(g_check_flag, r, g.rows)) y[r] = s;
-      }
-    }
-    __syncthreads();  // partials read before the next pass clears them
   }
 }
 
-// Shared memory of one CTA for a given pass size.
 template <int C>
-size_t smem_for(int n_spans, int pass_groups) {
-  return (size_t)Smem<C>::kTableBytes + (size_t)pass_groups * Smem<C>::kPartBytesPerGroup +
-         (size_t)n_spans * 32 * Smem<C>::kSlotFloats * 4;
+int warps_for(int items_per_cta) {
+  int w = items_per_cta < Tune<C>::kWarps ? items_per_cta : Tune<C>::kWarps;
+  // At least kMinWarps: on small matrices the CTA's setup (tables and x into
+  // shared memory) outweighs its one or two items, and warps without items
+  // still share it.
+  return w < kMinWarps ? kMinWarps : w;
 }
 
-// The geometry, with the largest partial-sum pass (<= kMaxGroups, halving)
-// that leaves room for x; pass_groups = 0 if x alone does not fit.
+// The geometry for `nw` warps per CTA and `grid` CTAs, with the largest
+// partial-sum pass that fits; pass_groups = 0 if even one group does not.
 template <int C>
-GemvGeom make_geom(const seedlm_format& f, int max_smem) {
+GemvGeom make_geom(const seedlm_format& f, int max_smem, int nw, int grid) {
+  constexpr int kBPL = Tune<C>::kBPL;
   GemvGeom g;
   g.rows = f.rows;
   g.cols = f.cols;
   g.nb = f.nb;
   g.rec_pitch = f.rec_pitch;
   g.e_pitch = f.e_pitch;
-  g.n_spans = ((f.nb + 1) / 2 + 31) / 32;
+  g.n_spans = ((f.nb + kBPL - 1) / kBPL + kSpanUnits - 1) / kSpanUnits;
   if (g.n_spans < 1) g.n_spans = 1;
   g.groups = (f.rows + kRowsPerTask - 1) / kRowsPerTask;
-  g.pass_groups = kMaxGroups;
-  while (g.pass_groups > 0 && smem_for<C>(g.n_spans, g.pass_groups) > (size_t)max_smem)
-    g.pass_groups >>= 1;
-  g.x_off = Smem<C>::kTableBytes + g.pass_groups * Smem<C>::kPartBytesPerGroup;
+  g.full_groups = f.rows / kRowsPerTask;
+  // Units of the pitch: a span is full when its last unit ends inside it.
+  g.full_spans = f.rec_pitch / (kBPL * kSpanUnits);
+  g.n_segs = (g.n_spans + Smem<C>::kMaxSegSpans - 1) / Smem<C>::kMaxSegSpans;
+  g.seg_spans = (g.n_spans + g.n_segs - 1) / g.n_segs;
+  const int64_t room = (int64_t)max_smem - (int64_t)(Smem<C>::kPart - kSmemBase);
+  const int64_t per_group = (int64_t)Smem<C>::kPartBytesPerGroup * nw;
+  const int max_cta_groups = grid > 0 ? (g.groups + grid - 1) / grid : 1;
+  int64_t pg = room > 0 ? room / per_group : 0;
+  if (pg > max_cta_groups) pg = max_cta_groups;
+  g.pass_groups = (int)pg;
   return g;
+}
+
+template <int C>
+size_t smem_for(const GemvGeom& g, int nw) {
+  return (size_t)(Smem<C>::kPart - kSmemBase) +
+         (size_t)g.pass_groups * Smem<C>::kPartBytesPerGroup * nw;
+}
+
+struct GemvLaunch {
+  GemvBatch b;
+  int grid, warps;
+  size_t smem;
+};
+
+// One launch for n GEMVs of format C: one CTA per SM (fewer if no GEMV has
+// that many row groups), warps for the largest share, and each GEMV's
+// partial-sum pass sized for that warp count.
+template <int C>
+GemvLaunch plan(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
+  constexpr int kBPL = Tune<C>::kBPL;
+  GemvLaunch L{};
+  int max_groups = 1, max_items = 1;
+  for (int k = 0; k < n; ++k) {
+    const int groups = (f[k]->rows + kRowsPerTask - 1) / kRowsPerTask;
+    int n_spans = ((f[k]->nb + kBPL - 1) / kBPL + kSpanUnits - 1) / kSpanUnits;
+    if (n_spans < 1) n_spans = 1;
+    if (groups > max_groups) max_groups = groups;
+    const int grid_k = groups < dev.num_sms ? groups : dev.num_sms;
+    const int items = (groups + grid_k - 1) / (grid_k > 0 ? grid_k : 1) * n_spans;
+    if (items > max_items) max_items = items;
+  }
+  L.grid = max_groups < dev.num_sms ? max_groups : dev.num_sms;
+  L.warps = warps_for<C>(max_items);
+  L.b.n = n;
+  L.smem = 0;
+  for (int k = 0; k < n; ++k) {
+    L.b.g[k] = make_geom<C>(*f[k], dev.max_smem_optin, L.warps, L.grid);
+    if (L.b.g[k].pass_groups == 0) {
+      L.smem = 0;
+      return L;
+    }
+    const size_t s = smem_for<C>(L.b.g[k], L.warps);
+    if (s > L.smem) L.smem = s;
+  }
+  return L;
 }
 
 }  // namespace
 
-size_t gemv_smem_bytes(const seedlm_format& f, int max_smem) {
-  if (f.C == 8) {
-    const GemvGeom g = make_geom<8>(f, max_smem);
-    return g.pass_groups ? smem_for<8>(g.n_spans, g.pass_groups) : 0;
-  }
-  const GemvGeom g = make_geom<12>(f, max_smem);
-  return g.pass_groups ? smem_for<12>(g.n_spans, g.pass_groups) : 0;
+size_t gemv_smem_bytes(const seedlm_format& f, const DeviceInfo& dev) {
+  const seedlm_format* fp = &f;
+  return f.C == 8 ? plan<8>(&fp, 1, dev).smem : plan<12>(&fp, 1, dev).smem;
 }
 
-int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
-                const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
-                const DeviceInfo& dev) {
-  const GemvGeom g = (f.C == 8) ? make_geom<8>(f, dev.max_smem_optin)
-                                : make_geom<12>(f, dev.max_smem_optin);
-  if (g.pass_groups == 0) return SEEDLM_EUNSUPPORTED;  // x does not fit in shared memory
-  const size_t smem = gemv_smem_bytes(f, dev.max_smem_optin);
-  if (g.groups < 1) return SEEDLM_OK;
-  // One CTA per SM (at most one per row group); fewer warps per CTA when
-  // each CTA has only a few (group, span) items, so small matrices still
-  // spread over all SMs.
-  int grid = g.groups < dev.num_sms ? g.groups : dev.num_sms;
-  int items_per_cta = (g.groups + grid - 1) / grid * g.n_spans;
-  const int max_warps = (f.C == 8) ? Tune<8>::kWarps : Tune<12>::kWarps;
-  int wpc = items_per_cta < max_warps ? items_per_cta : max_warps;
-  // At least 8 warps: on small matrices the CTA's setup (x and the tables
-  // into shared memory) outweighs its one or two items, and warps without
-  // items still share it.
-  if (wpc < kMinWarps) wpc = kMinWarps;
-  const void* kern = (f.C == 8) ? (const void*)gemv_kernel<8> : (const void*)gemv_kernel<12>;
+int read_and_clear_gemv_error(unsigned int* out) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t err = cudaMemcpyFromSymbol(&v, g_gemv_error, sizeof(v));
+  if (err != cudaSuccess) return record_cuda_error(err);
+  if (v) {
+    err = cudaMemcpyToSymbol(g_gemv_error, &zero, sizeof(zero));
+    if (err != cudaSuccess) return record_cuda_error(err);
+  }
+  *out = v;
+  return SEEDLM_OK;
+}
+
+int launch_gemv_batch(int n, const seedlm_format* const* f, const uint32_t* const* rec,
+                      const uint8_t* const* eplane, const uint16_t* const* x, int is_bf16,
+                      float* const* y, cudaStream_t stream, const DeviceInfo& dev) {
+  if (n < 1) return SEEDLM_OK;
+  if (n > kMaxBatch) return SEEDLM_EUNSUPPORTED;
+  const int C = f[0]->C;
+  GemvLaunch L = (C == 8) ? plan<8>(f, n, dev) : plan<12>(f, n, dev);
+  if (L.smem == 0) return SEEDLM_EUNSUPPORTED;  // the tables do not fit
+  for (int k = 0; k < n; ++k) {
+    L.b.rec[k] = rec[k];
+    L.b.ep[k] = eplane[k];
+    L.b.x[k] = x[k];
+    L.b.y[k] = y[k];
+  }
+  const bool batch = n > 1;
+  const void* kern = (C == 8) ? (batch ? (const void*)gemv_kernel<8, true>
+                                       : (const void*)gemv_kernel<8, false>)
+                              : (batch ? (const void*)gemv_kernel<12, true>
+                                       : (const void*)gemv_kernel<12, false>);
   int rc = allow_max_smem(kern, dev);
   if (rc) return rc;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(wpc * 32);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(L.grid);
+  cfg.blockDim = dim3(L.warps * 32);
+  cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = (f.C == 8)
-                        ? cudaLaunchKernelEx(&cfg, gemv_kernel<8>, rec, eplane, x, is_bf16, y, g)
-                        : cudaLaunchKernelEx(&cfg, gemv_kernel<12>, rec, eplane, x, is_bf16, y, g);
+  cudaError_t err =
+      (C == 8) ? (batch ? cudaLaunchKernelEx(&cfg, gemv_kernel<8, true>, L.b, is_bf16)
+                        : cudaLaunchKernelEx(&cfg, gemv_kernel<8, false>, L.b, is_bf16))
+               : (batch ? cudaLaunchKernelEx(&cfg, gemv_kernel<12, true>, L.b, is_bf16)
+                        : cudaLaunchKernelEx(&cfg, gemv_kernel<12, false>, L.b, is_bf16));
   if (err != cudaSuccess) return record_cuda_error(err);
   count_launch();
   return record_cuda_error(cudaGetLastError());
+}
+
+int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
+                const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
+                const DeviceInfo& dev) {
+  if (f.rows == 0) return SEEDLM_OK;
+  const seedlm_format* fp = &f;
+  return launch_gemv_batch(1, &fp, &rec, &eplane, &x, is_bf16, &y, stream, dev);
 }
 
 }  // namespace seedlm

@@ -222,16 +222,9 @@ struct BlockC12 {
   uint32_t negm;
 };
 
-// e4 is the block's exponent in bits [0,4).
-__device__ __forceinline__ BlockC12 decode_c12(uint32_t rec, uint32_t e4,
-                                               const uint2* __restrict__ t_lo,
-                                               const uint2* __restrict__ t_hi) {
-  BlockC12 b;
-  b.lo = rec;
-  uint2 x0 = t_lo[(rec >> 16) & 0xffu];
-  uint2 x1 = t_hi[rec >> 24];
-  b.mid = x0.x ^ x1.x;
-  b.hi = x0.y ^ x1.y;
+// The coefficient part of a C = 12 block: (q_p, 256 q_p) pairs, the integer
+// start value and -M_e.  e4 is the block's exponent in bits [0,4).
+__device__ __forceinline__ void coef_c12(BlockC12& b, uint32_t rec, uint32_t e4) {
   uint32_t v = prmt<0x5140u>(rec, rec >> 4) & 0x0f0f0f0fu;  // (q0, q1, q2, q3)
   uint32_t s = sext_nibble_bytes(v);
   // (q_p, sign(q_p), 0x00, q_p): the zero byte is the sign of a byte of v.
@@ -243,6 +236,19 @@ __device__ __forceinline__ BlockC12 decode_c12(uint32_t rec, uint32_t e4,
   uint32_t e23 = (e4 & 15u) << 23;
   b.init = (int32_t)(kMagicBits - e23) - qsum * 32768;
   b.negm = kNegMagicBits - e23;
+}
+
+// e4 is the block's exponent in bits [0,4).
+__device__ __forceinline__ BlockC12 decode_c12(uint32_t rec, uint32_t e4,
+                                               const uint2* __restrict__ t_lo,
+                                               const uint2* __restrict__ t_hi) {
+  BlockC12 b;
+  b.lo = rec;
+  uint2 x0 = t_lo[(rec >> 16) & 0xffu];
+  uint2 x1 = t_hi[rec >> 24];
+  b.mid = x0.x ^ x1.x;
+  b.hi = x0.y ^ x1.y;
+  coef_c12(b, rec, e4);
   return b;
 }
 

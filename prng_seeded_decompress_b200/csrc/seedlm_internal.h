@@ -68,6 +68,14 @@ struct DeviceInfo {
 // Properties of the current device (cached per device); SEEDLM_OK or an error.
 int current_device_info(DeviceInfo* out);
 
+// Argument checks shared by every entry point: p is a multiple of a bytes;
+// the format is one the kernels support and self-consistent (SEEDLM_OK,
+// SEEDLM_EINVAL or SEEDLM_EUNSUPPORTED); the record (and, for (12,4),
+// exponent) planes are present and aligned when the matrix is not empty.
+bool aligned(const void* p, uintptr_t a);
+int check_format(const seedlm_format* f);
+int check_planes(const seedlm_format* f, const uint32_t* rec, const uint8_t* eplane);
+
 // Records err as this thread's last CUDA error; SEEDLM_OK or SEEDLM_ECUDA.
 int record_cuda_error(cudaError_t err);
 // Counts one kernel launch (process-wide).
@@ -76,11 +84,16 @@ void count_launch();
 // per kernel and device, outside any stream capture the caller may start later.
 int allow_max_smem(const void* kernel, const DeviceInfo& dev);
 
-// Shared memory the GEMV needs for f within max_smem bytes (0: x does not fit).
-size_t gemv_smem_bytes(const seedlm_format& f, int max_smem);
+// Shared memory the GEMV kernel needs for f on dev (0: its tables do not fit).
+size_t gemv_smem_bytes(const seedlm_format& f, const DeviceInfo& dev);
+int read_and_clear_gemv_error(unsigned int* out);
 int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                 const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
                 const DeviceInfo& dev);
+// n (<= 8) GEMVs of one format (same C) in one launch; every entry non-empty.
+int launch_gemv_batch(int n, const seedlm_format* const* f, const uint32_t* const* rec,
+                      const uint8_t* const* eplane, const uint16_t* const* x, int is_bf16,
+                      float* const* y, cudaStream_t stream, const DeviceInfo& dev);
 int launch_decompress(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                       float* W, int64_t ldw, cudaStream_t stream, const DeviceInfo& dev);
 int launch_dense_gemv_f16(int rows, int cols, const uint16_t* W, int64_t ldw, const uint16_t* x,

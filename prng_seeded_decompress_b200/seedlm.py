@@ -25,7 +25,8 @@ EXPORTS = (
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
     "seedlm_encode", "seedlm_selftest_wait_timeout", "seedlm_checked_build",
-    "seedlm_selftest_bounds_check",
+    "seedlm_selftest_bounds_check", "seedlm_search_blocks", "seedlm_lfsr_taps",
+    "seedlm_gemv_batch",
 )
 
 
@@ -74,6 +75,9 @@ def _load():
         "seedlm_shutdown": (None, []),
         "seedlm_checked_build": (ctypes.c_int, []),
         "seedlm_selftest_bounds_check": (ctypes.c_int, [i64, i64, vp]),
+        "seedlm_search_blocks": (ctypes.c_int, [i32, i32, i32, vp, i64, vp, vp, vp, vp, vp]),
+        "seedlm_lfsr_taps": (ctypes.c_uint32, [i32]),
+        "seedlm_gemv_batch": (ctypes.c_int, [i32, vp, vp, vp, vp, ctypes.c_int, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -175,6 +179,24 @@ def encode(fmt, W, rec, eplane=None, err=None, ldw: int | None = None, stream=No
         ctypes.byref(f), _ptr(W), ld, _ptr(rec), _ptr(eplane), _ptr(err), _stream(stream, W)))
 
 
+def search_blocks(C: int, P: int, K: int, W, seed, q, e, err=None, stream=None):
+    """Design-space search over the 2^K - 1 seeds of a K-bit register for
+    every row of W (float32, nblocks x C, device): seed (int32/uint32,
+    nblocks), q (int8, nblocks x P), e (uint8, nblocks) and optionally err
+    (float64, nblocks) receive the best fit of each block."""
+    _dense(W, "W")
+    n = int(W.shape[0]) if W.dim() == 2 else int(W.numel()) // int(C)
+    _check("seedlm_search_blocks", lib.seedlm_search_blocks(
+        int(C), int(P), int(K), _ptr(W), n, _ptr(seed), _ptr(q), _ptr(e), _ptr(err),
+        _stream(stream, W)))
+
+
+def lfsr_taps(K: int) -> int:
+    """Tap mask of the K-bit register the design-space search uses (0 if K is
+    unsupported)."""
+    return int(lib.seedlm_lfsr_taps(int(K)))
+
+
 def gemv(fmt, rec, eplane, x, y, stream=None):
     """y = W x; x float16/bfloat16 (cols), y float32 (rows)."""
     f = _fmt(fmt)
@@ -182,6 +204,25 @@ def gemv(fmt, rec, eplane, x, y, stream=None):
     _check("seedlm_gemv", lib.seedlm_gemv(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(x), _act_dtype(x), _ptr(y),
         _stream(stream, y)))
+
+
+def gemv_batch(items, stream=None):
+    """Several independent GEMVs in one launch: items is a list of
+    (fmt, rec, eplane, x, y) tuples, all of one storage format and one
+    activation type."""
+    n = len(items)
+    if n == 0:
+        return
+    fmts = (Format * n)(*[_fmt(it[0]) for it in items])
+    ptrs = lambda vals: (ctypes.c_void_p * n)(*vals)  # noqa: E731
+    for it in items:
+        _dense(it[3], "x"), _dense(it[4], "y")
+    recs = ptrs([_ptr(it[1]) for it in items])
+    eps = ptrs([_ptr(it[2]) for it in items])
+    xs = ptrs([_ptr(it[3]) for it in items])
+    ys = ptrs([_ptr(it[4]) for it in items])
+    _check("seedlm_gemv_batch", lib.seedlm_gemv_batch(
+        n, fmts, recs, eps, xs, _act_dtype(items[0][3]), ys, _stream(stream, items[0][4])))
 
 
 def gemm_workspace_bytes(fmt, M: int) -> int:

@@ -47,20 +47,23 @@ def test_fewer_than_three_warmup_steps_are_refused():
 
 
 def test_traffic_figure_is_dropped_when_its_sources_change(tmp_path, monkeypatch):
+    # A tree with one kernel source and a traffic record carrying that
+    # source's hash: the record is used while the source is unchanged and
+    # dropped (None) once one byte of it changes.
+    import hashlib
+    import json
+
     import bench
-    t = bench.profile_traffic("gemv_kernel<8>")
-    assert t is not None and t["bytes_per_launch"] > 0      # committed and current
-    # A copy of the tree where one source file differs by one byte.
     root = tmp_path / "tree"
     (root / "profiles").mkdir(parents=True)
-    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), root / "profiles")
-    for f in t["sources"]:
-        dst = root / f
-        dst.parent.mkdir(parents=True, exist_ok=True)
-        shutil.copy(os.path.join(ROOT, f), dst)
+    src = root / "k.cu"
+    src.write_bytes(b"__global__ void k() {}\n")
+    rec = {"k": {"bytes_per_launch": 123, "sources": ["k.cu"],
+                 "sources_sha256": hashlib.sha256(src.read_bytes()).hexdigest()}}
+    (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(root))
-    assert bench.profile_traffic("gemv_kernel<8>") is not None
-    src = root / t["sources"][0]
+    t = bench.profile_traffic("k")
+    assert t is not None and t["bytes_per_launch"] == 123
     src.write_bytes(src.read_bytes() + b"\n")
-    assert bench.profile_traffic("gemv_kernel<8>") is None
+    assert bench.profile_traffic("k") is None
     assert bench.profile_traffic("no_such_kernel") is None

@@ -83,6 +83,39 @@ def test_decompress_bit_exact(sl, oracle_mod, cp, rows, cols):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("cp,rows,cols", [(C8, 4096, 4096), (C12, 2048, 6000)])
+def test_decompress_multi_item_loop_bit_exact(sl, oracle_mod, cp, rows, cols):
+    # More warp items (one row's 128 consecutive blocks each) than the grid
+    # has warps (4 CTAs x 8 warps per SM), so every warp walks several items
+    # and takes the next-item prefetch and row/column relocation path.
+    L = inputs.make_layer(rows, cols, *cp, seed=rows * 3 + cols, e_range=(0, 15))
+    rec, ep = planes(L)
+    W = torch.full((rows, cols), float("nan"), device="cuda")
+    sl.decompress(L["fmt"], rec, ep, W)
+    torch.cuda.synchronize()
+    ref = oracle_mod.decompress(L["fmt"], L["rec"], L["eplane"]).astype(np.float32)
+    assert np.array_equal(W.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def test_decompress_full_size_sampled_rows(sl, oracle_mod):
+    # The 70B down projection (8192 x 28672, 4-bit), the shape the benchmark
+    # decompresses: bit patterns of sampled rows (first and last rows plus a
+    # random sample) against the oracle's decompression of those rows' records.
+    rows, cols = 8192, 28672
+    L = inputs.make_layer(rows, cols, *C8, seed=4242, e_range=(0, 15))
+    rec, ep = planes(L)
+    W = torch.full((rows, cols), float("nan"), device="cuda")
+    sl.decompress(L["fmt"], rec, ep, W)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    sample = np.unique(np.concatenate([np.arange(4), np.arange(rows - 4, rows),
+                                       rng.integers(0, rows, 24)]))
+    sub = dict(L["fmt"], rows=int(sample.size))
+    ref = oracle_mod.decompress(sub, np.ascontiguousarray(L["rec"][sample]), None)
+    got = W[torch.from_numpy(sample).cuda()].cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.astype(np.float32).view(np.uint32))
+
+
 def test_decompress_leading_dimension_and_seed_zero(sl, oracle_mod):
     fmt = inputs.make_format(3, 20, 8, 3)
     seeds = np.array([[0, 1, 65535], [0, 0, 0], [12345, 0, 7]])
@@ -195,6 +228,22 @@ def test_gemv_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols):
     rng = np.random.default_rng(0)
     sample = np.unique(np.concatenate([np.arange(8), np.arange(rows - 8, rows),
                                        rng.integers(0, rows, 48)]))
+    ref, refabs = oracle_mod.gemv_rows(L["fmt"], L["rec"], L["eplane"], xv, sample)
+    assert_within(y[sample], ref, refabs)
+
+
+@pytest.mark.parametrize("cp,rows,cols", [(C8, 1800, 56320), (C12, 6000, 42240)])
+def test_gemv_multi_pass_wide_x(sl, oracle_mod, cp, rows, cols):
+    # x this wide leaves room in shared memory for only a few row groups of
+    # partial sums per pass (2 at 4 bits, 8 at 3 bits), so with these row
+    # counts every CTA runs several passes: the later passes re-zero the
+    # partials and reuse the staged x.  Checked on sampled rows.
+    L = inputs.make_layer(rows, cols, *cp, seed=rows + cols)
+    xb, xv = inputs.make_activations((cols,), "f16", 17)
+    y = gpu_gemv(sl, L, xb)
+    rng = np.random.default_rng(1)
+    sample = np.unique(np.concatenate([np.arange(16), np.arange(rows - 16, rows),
+                                       rng.integers(0, rows, 96)]))
     ref, refabs = oracle_mod.gemv_rows(L["fmt"], L["rec"], L["eplane"], xv, sample)
     assert_within(y[sample], ref, refabs)
 
@@ -353,31 +402,71 @@ def test_graph_replay_matches_eager_calls(sl):
     del g
 
 
-# ------------------------------------------------------------ widest x
+# ------------------------------------------------------------ wide x
 
-@pytest.mark.parametrize("cp,cols", [(C8, 56320), (C12, 42240)])
-def test_gemv_at_its_widest_x_and_one_block_past_it(sl, oracle_mod, cp, cols):
-    # x is staged in shared memory as fp32: the widest x the GEMV takes
-    # (the partial-sum buffer shrinks to make room) matches the oracle; one
-    # more block is refused, and gemm_smallM with M = 1 then runs it on the
-    # tensor cores instead.
+@pytest.mark.parametrize("cp,cols", [(C8, 70000), (C12, 50000), (C8, 15872), (C8, 15873),
+                                     (C12, 23808), (C12, 23809)])
+def test_gemv_wide_x_in_column_segments(sl, oracle_mod, cp, cols):
+    # x is staged in shared memory in column segments (31 spans of 512
+    # columns at 4 bits, 31 spans of 768 at 3 bits): 70,000 and 50,000
+    # columns take five and three segments; 15,872 columns (4 bits) and
+    # 23,808 (3 bits) exactly fill one segment, and one more column needs a
+    # second.  gemm_smallM with M = 1 runs the same kernel, same bits.
     rows = 40
     L = inputs.make_layer(rows, cols, *cp, seed=cols)
     xb, xv = inputs.make_activations((cols,), "f16", 3)
     y = gpu_gemv(sl, L, xb)
     ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv)
     assert_within(y, ref, refabs)
+    assert sl.gemm_workspace_bytes(L["fmt"], 1) == 0
+    got = gpu_gemm(sl, L, xb.reshape(1, cols), dtype="f16")
+    assert np.array_equal(got[0].astype(np.float32).view(np.uint32),
+                          y.astype(np.float32).view(np.uint32))
 
-    wide = cols + cp[0]
-    L = inputs.make_layer(rows, wide, *cp, seed=wide)
-    rec, ep = planes(L)
-    xb, xv = inputs.make_activations((wide,), "bf16", 4)
-    x = act_tensor(xb, "bf16")
-    y = torch.empty(rows, device="cuda")
+
+# ------------------------------------------------------------ batched GEMV
+
+@pytest.mark.parametrize("cp,shapes,dtype", [
+    (C8, [(1000, 8192), (40, 70000), (0, 512), (300, 999), (5000, 4096)], "f16"),
+    (C12, [(700, 4096), (33, 30000), (2000, 1000)], "bf16"),
+])
+def test_gemv_batch_equals_separate_calls(sl, oracle_mod, cp, shapes, dtype):
+    # One launch for several GEMVs of one format (shapes with one and several
+    # x segments, fewer row groups than SMs, an empty matrix): every output
+    # has the bits of the separate seedlm_gemv call and is within tolerance
+    # of the oracle.
+    items, refs = [], []
+    for i, (rows, cols) in enumerate(shapes):
+        L = inputs.make_layer(rows, cols, *cp, seed=500 + i)
+        xb, xv = inputs.make_activations((cols,), dtype, 600 + i)
+        rec, ep = planes(L)
+        x = act_tensor(xb, dtype)
+        y = torch.full((rows,), float("nan"), device="cuda")
+        items.append((L["fmt"], rec, ep, x, y))
+        refs.append((L, xv))
+    sl.gemv_batch(items)
+    torch.cuda.synchronize()
+    for (fmt, rec, ep, x, y), (L, xv) in zip(items, refs):
+        ys = torch.full_like(y, float("nan"))
+        sl.gemv(fmt, rec, ep, x, ys)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int32), ys.view(torch.int32))
+        if fmt["rows"]:
+            ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv,
+                                          threads=os.cpu_count() or 1)
+            assert_within(y.cpu().numpy().astype(np.float64), ref, refabs)
+
+
+def test_gemv_batch_rejects_mixed_formats_and_too_many(sl):
+    L8 = inputs.make_layer(8, 64, *C8, seed=1)
+    L12 = inputs.make_layer(8, 72, *C12, seed=2)
+    x = torch.zeros(72, dtype=torch.float16, device="cuda")
+    y = torch.zeros(8, device="cuda")
+    r8, _ = planes(L8)
+    r12, e12 = planes(L12)
     with pytest.raises(sl.SeedLMError) as exc:
-        sl.gemv(L["fmt"], rec, ep, x, y)
+        sl.gemv_batch([(L8["fmt"], r8, None, x, y), (L12["fmt"], r12, e12, x, y)])
     assert exc.value.code == -2
-    assert sl.gemm_workspace_bytes(L["fmt"], 1) > 0
-    got = gpu_gemm(sl, L, xb.reshape(1, wide))
-    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], xv.reshape(1, wide))
-    assert_within(got[0], ref[0], refabs[0])
+    with pytest.raises(sl.SeedLMError) as exc:
+        sl.gemv_batch([(L8["fmt"], r8, None, x, y)] * 9)
+    assert exc.value.code == -1

@@ -4,11 +4,12 @@ GPU's memory pool, or a path that must not pay cudaMalloc's implicit device
 synchronisation), so cannot hand in a workspace.  Its workspace is an array
 inside libseedlm.so.
 
-These tests call the entry point through the C ABI (ctypes) and compare it
-with seedlm_gemm_smallM (caller workspace) on the same inputs, within the
-tolerance the other GPU tests use, on two calls in a row -- the second call
-finds the scratch exactly as the first one left it.  The file is named so
-that pytest collects it last.
+These tests call the entry point through the C ABI (ctypes) on two calls in
+a row -- the second call finds the scratch exactly as the first one left it
+-- and check each result twice: bit for bit against seedlm_gemm_smallM with
+a caller workspace (the same kernel with the same split, so the same bits),
+and against the fp64 CPU oracle within the tolerance every GPU product test
+uses.  The file is named so that pytest collects it last.
 """
 import ctypes
 import os
@@ -81,32 +82,40 @@ def test_noalloc_matches_workspace_entry_on_two_calls(sl, oracle_mod, cp, rows, 
     Y_ws = torch.full((M, rows), float("nan"), device="cuda")
     sl.gemm_smallM(L["fmt"], rec, ep, X, Y_ws, workspace=sl.gemm_workspace(L["fmt"], M))
     torch.cuda.synchronize()
-    ref = Y_ws.cpu().numpy().astype(np.float64)
-    _, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv, threads=os.cpu_count() or 1)
+    ws_bits = Y_ws.cpu().numpy().view(np.uint32)
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv,
+                                  threads=os.cpu_count() or 1)
     for call in range(2):
         Y = torch.full((M, rows), float("nan"), device="cuda")
         assert _noalloc(sl, L, rec, ep, X, Y) == 0
         torch.cuda.synchronize()
         assert sl.device_error() == 0
-        got = Y.cpu().numpy().astype(np.float64)
-        err = np.abs(got - ref)
+        got = Y.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), ws_bits), f"call {call}: differs from the " \
+            "workspace entry point"
+        err = np.abs(got.astype(np.float64) - ref)
         assert np.all(err <= TOL * refabs + 1e-30), f"call {call}: max err {err.max()}"
 
 
 @pytest.mark.gpu
 def test_noalloc_rejects_problems_beyond_its_scratch(sl):
-    # 38400 rows = 300 tiles over 8192 columns at M = 64: one CTA per SM
-    # covers about two tiles, touches up to four, and keeps a 32 KiB partial
-    # tile for each -- more than the 16 MiB + 64 KiB the library holds.
+    # 57344 rows = 448 row tiles over 8192 columns (64 chunks each) at
+    # M = 64: one CTA per SM takes about 194 of the 28,672 (tile, chunk)
+    # units, so it touches up to four row tiles and keeps a 32 KiB partial
+    # tile for each: 148 x 4 x 32 KiB is more than the 16 MiB + 64 KiB the library
+    # holds, and the call must be refused before anything is launched.
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    rows, cols, M = 38400, 8192, 64
+    rows, cols, M = 57344, 8192, 64
     fmt = inputs.make_format(rows, cols, *C8)
     need = sl.gemm_workspace_bytes(fmt, M)
-    if need <= (16 << 20) + (64 << 10):
-        pytest.skip("this device splits the problem so that it fits")
+    assert need > (16 << 20) + (64 << 10), need
     rec = torch.zeros((rows, fmt["rec_pitch"]), dtype=torch.int32, device="cuda")
     X = torch.zeros((M, cols), dtype=torch.bfloat16, device="cuda")
-    Y = torch.zeros((M, rows), device="cuda")
+    Y = torch.full((M, rows), 7.0, device="cuda")
     L = dict(fmt=fmt)
+    n0 = sl.launch_count()
     assert _noalloc(sl, L, rec, None, X, Y) == -2
+    torch.cuda.synchronize()
+    assert sl.launch_count() == n0
+    assert bool((Y == 7.0).all())
