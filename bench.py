@@ -381,6 +381,11 @@ def extras(torch, sl, args):
     graph = time_median(torch, lambda i: graphs[i % 4].replay(), 80) * 1e3
     out["llama3_70b_layer_graph_vs_eager"] = {"us_per_layer_eager": round(eager, 2),
                                              "us_per_layer_graph": round(graph, 2)}
+    # The same four GEMVs as one batched launch (seedlm_gemv_batch).
+    batched = time_median(torch, lambda i: sl.gemv_batch(
+        [(f, m["rec"], None, xl[m["N"]], y) for m, f, y in zip(copies[i % 4], fm, yl)]), 80) * 1e3
+    out["llama3_70b_layer_batched"] = {"us_per_layer": round(batched, 2),
+                                      "us_per_layer_separate_calls": round(eager, 2)}
     del graphs, copies, layer
 
     # 3-bit Llama-3-8B layer: as specified (one layer) and 32 copies (cold).
@@ -513,10 +518,10 @@ def extras(torch, sl, args):
     # seed widths K; relative reconstruction error against bits per weight
     # ((K + 4P + 4) / C).
     sweep_ds = {}
-    for C, P, K, nblk in ((8, 3, 16, 16384), (8, 4, 16, 16384), (8, 2, 16, 16384),
-                          (12, 3, 16, 16384), (12, 4, 16, 16384), (16, 4, 16, 16384),
-                          (16, 3, 16, 16384), (8, 3, 12, 16384), (8, 3, 14, 16384),
-                          (8, 3, 18, 4096), (8, 3, 20, 1024)):
+    for C, P, K, nblk in ((8, 3, 16, 4096), (8, 4, 16, 4096), (8, 2, 16, 4096),
+                          (12, 3, 16, 4096), (12, 4, 16, 4096), (16, 4, 16, 4096),
+                          (16, 3, 16, 4096), (8, 3, 12, 4096), (8, 3, 14, 4096),
+                          (8, 3, 18, 1024), (8, 3, 20, 256)):
         rng = np.random.default_rng(1000 + C * 100 + P * 10 + K)
         Wb = torch.from_numpy((rng.standard_normal((nblk, C)) * 0.02).astype(np.float32)).cuda()
         sd = torch.empty(nblk, dtype=torch.int32, device="cuda")
@@ -600,6 +605,9 @@ def summarize(result, hbm_peak):
         kd = f"up_28672x8192/M={M}"
         if kd in dm:
             out[f"dense_fp16_28672x8192_M{M}_us"] = dm[kd]["us_per_call"]
+    bt = ex.get("llama3_70b_layer_batched")
+    if bt:
+        out["llama3_70b_4bit_us_per_layer_one_batched_launch"] = bt["us_per_layer"]
     sq = ex.get("square_sweep_4bit", {})
     for n, v in sq.items():
         out[f"square_{n}_us_graph"] = v["us_per_call_graph"]
@@ -842,6 +850,17 @@ def reference_arm(args):
     }), flush=True)
 
 
+def flush_l2(torch):
+    """Leave L2 holding clean lines only: the uploads of the inputs are
+    written back now rather than during the captured kernel."""
+    junk = torch.empty(int(4 * torch.cuda.get_device_properties(0).L2_cache_size) // 4,
+                       dtype=torch.float32, device="cuda")
+    junk.zero_()
+    float(junk.sum())  # a read pass over 4x L2 evicts every dirty line
+    del junk
+    torch.cuda.synchronize()
+
+
 def profile_case(name: str):
     """One small single-kernel workload for an ncu capture (inputs > L2)."""
     import numpy as np
@@ -867,16 +886,30 @@ def profile_case(name: str):
         ws = sl.gemm_workspace(L["fmt"], M)
         for _ in range(3):
             sl.gemm_smallM(L["fmt"], rec, None, X, Y, workspace=ws)
-    elif name == "gemv":
+    elif name in ("gemv", "gemv-cycle"):
         # The four GEMVs of one 4-bit Llama-3-70B layer, twice (the first
-        # round warms up; capture with -s 4 -c 4).
+        # round warms up; capture with -s 4 -c 4).  "gemv-cycle" stores each
+        # seed's position in the register's cycle instead of the seed, the
+        # record form of a library built with SEEDLM_GEMV_LFSR=2 (the
+        # full-cycle window table; for the LFSR variant comparison only).
+        pos = None
+        if name == "gemv-cycle":
+            pos = np.zeros(65536, np.uint32)
+            st = 1
+            for p in range(65535):
+                pos[st] = p
+                st = (st >> 1) | (((st ^ (st >> 2) ^ (st >> 3) ^ (st >> 5)) & 1) << 15)
         lay = []
         for i, (_, R, N) in enumerate(LAYER_70B):
             L = inputs.make_layer(R, N, 8, 3, seed=10 + i)
+            rec = L["rec"]
+            if pos is not None:
+                rec = ((pos[rec >> 16] << 16) | (rec & 0xffff)).astype(np.uint32)
             xb, _ = inputs.make_activations((N,), "f16", 20 + i)
-            lay.append((L["fmt"], torch.from_numpy(L["rec"].view(np.int32)).cuda(),
+            lay.append((L["fmt"], torch.from_numpy(rec.view(np.int32)).cuda(),
                         torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16),
                         torch.empty(R, device="cuda")))
+        flush_l2(torch)
         for _ in range(2):
             for f, rec, x, y in lay:
                 sl.gemv(f, rec, None, x, y)
@@ -891,6 +924,7 @@ def profile_case(name: str):
                         torch.from_numpy(L["eplane"]).cuda(),
                         torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16),
                         torch.empty(R, device="cuda")))
+        flush_l2(torch)
         for _ in range(2):
             for f, rec, ep, x, y in lay:
                 sl.gemv(f, rec, ep, x, y)
@@ -926,8 +960,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
-    ap.add_argument("--case", choices=("gemv", "gemv3", "decompress", "gemm64", "gemm16", "dense",
-                                       "encode"),
+    ap.add_argument("--case", choices=("gemv", "gemv3", "gemv-cycle", "decompress", "gemm64",
+                                       "gemm16", "dense", "encode"),
                     help="run one small single-kernel workload (for ncu) and exit")
     args = ap.parse_args()
     if args.case:

@@ -105,10 +105,11 @@ SEEDLM_API int seedlm_decompress(const seedlm_format* fmt, const uint32_t* rec, 
 /* y = W x (batch 1).  x: cols elements of type x_dtype (SEEDLM_F16 or
  * SEEDLM_BF16); y: rows fp32.  The blocks are rebuilt on the fly and never
  * written out (paperhub.cn thread, authors' replies on inference and on the
- * custom decoding that avoids full-precision weights in memory).  x is held
- * in shared memory as fp32, so cols is limited by it: up to 56,320 (4-bit)
- * or 42,240 (3-bit) on a B200 (227 KB per block); wider x returns
- * SEEDLM_EUNSUPPORTED (seedlm_gemm_smallM with M = 1 has no such limit). */
+ * custom decoding that avoids full-precision weights in memory).  Any width:
+ * x is staged in shared memory as fp32 one column segment at a time.  The
+ * kernel is launched with programmatic dependent launch; it reads the
+ * records and x only after waiting for the previous kernel in the stream,
+ * so that kernel may write them (for example seedlm_encode, or a copy). */
 SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
                 const void* x, int x_dtype, float* y, seedlm_stream stream);
 
@@ -116,10 +117,14 @@ SEEDLM_API int seedlm_gemv(const seedlm_format* fmt, const uint32_t* rec, const 
  * format, the same C, P, K): y_k = W_k x_k for k < n.  fmts is a HOST array
  * of n formats; recs, eplanes (may be NULL for (8,3)), xs and ys are HOST
  * arrays of n DEVICE pointers, with the rules of seedlm_gemv for each entry
- * and one activation type for all.  The result equals n seedlm_gemv calls
- * bit for bit; the kernel's setup (its decode tables in shared memory) is
- * paid once, and each CTA moves straight from its share of one product to
- * the next, with no launch or tail between them.  The pages name the extra
+ * and one activation type for all.  One launch configuration serves the
+ * whole batch (chosen from its largest product), so an entry's summation
+ * order may differ from a separate seedlm_gemv call's: results agree with
+ * separate calls within the products' tolerance, and bit for bit when the
+ * entry alone would get the same configuration (as the large matrices of
+ * one decoder layer do).  The kernel's setup (its decode tables in shared
+ * memory) is paid once, and each CTA moves straight from its share of one
+ * product to the next, with no launch or tail between them.  The pages name the extra
  * kernel launches of memory-bound work as a GPU cost of the method
  * (paperhub.cn review thread, authors' reply on GPU implementation
  * challenges); this is the library's answer for products that do not
@@ -135,8 +140,8 @@ SEEDLM_API int seedlm_gemv_batch(int32_t n, const seedlm_format* fmts,
  * inference step of the paperhub.cn review thread (authors' reply on how
  * inference uses s and t: the blocks are rebuilt from seed and coefficients
  * and multiplied with the activations; a batch of M activation rows shares
- * every rebuilt block).  M = 1 runs the GEMV kernel
- * (unless x is too wide for it); otherwise the rebuilt weight tiles feed the
+ * every rebuilt block).  M = 1 runs the GEMV kernel; otherwise the rebuilt
+ * weight tiles feed the
  * tcgen05 tensor cores (kind::f16
  * MMAs in the activations' type: W split exactly into three bf16 pieces for
  * bf16 X, two fp16 pieces of 2^6 W for fp16 X; exact products, fp32

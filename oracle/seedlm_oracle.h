@@ -15,8 +15,8 @@
  * thread on paperhub.cn names U and t the compression matrices of Eq (1)).
  * The coefficients are 4-bit integers q with a 4-bit exponent e shared by the
  * block, t = q * 2^-e (the same thread, authors' reply on data formats with
- * shared exponents; atlas.scime.ai summary, "Approach": "store only the seed
- * and 4-bit quantized coefficients").  At inference the weights are rebuilt
+ * shared exponents; atlas.scime.ai summary, "Approach": only the seed and
+ * the 4-bit coefficients are kept per block).  At inference the weights are rebuilt
  * on the fly and then multiplied with the activations (paperhub.cn thread,
  * authors' reply on how inference uses Eq (1)).
  *

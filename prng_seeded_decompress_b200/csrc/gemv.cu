@@ -102,37 +102,50 @@ __device__ unsigned int g_gemv_error = 0;
 // x values per lane that needs the register file of 16 warps.  C = 12 takes
 // 2 blocks (a pair): its four dp2a windows per weight already fill 128
 // registers.
-template <int C>
+template <int C, int V>
 struct Tune {
-  static constexpr int kBPL = (C == 8) ? SEEDLM_GEMV_BPL8 : 2;
-  static constexpr int kWarps = (C == 8 && kBPL == 2) ? 24 : 16;
+  static constexpr int kBPL = (C == 8 && V == 0) ? SEEDLM_GEMV_BPL8 : 2;
+  static constexpr int kWarps = (V == 1) ? 8 : (C == 8 && kBPL == 2) ? 24 : 16;
   static constexpr int kPrefetch = (C == 8) ? SEEDLM_GEMV_PREFETCH8 : 2;
+  static constexpr int kMinBlocks = (V == 1) ? 2 : 1;  // CTAs per SM the launch bounds ask for
 };
 constexpr int kRowsPerTask = 4;
 constexpr int kMinWarps = 8;      // warps per CTA however few items it has
 constexpr int kSpanUnits = 32;    // lane units (pairs or quads of blocks) per span
 
-// Shared-memory map (absolute shared addresses):
-//   C = 8:  [kSmemBase, 0x10000)  x slots of one column segment
-//           [0x10000, 0x20000)    stream jump-table rows
-//           [0x20000, 0x30000)    coefficient-table rows
-//   C = 12: [kSmemBase, 0x20000)  x slots of one column segment
-//           [0x20000, 0x30000)    stream jump-table rows
-//   both:   [0x30000, ...)        partial row sums of one pass
+// Two variants of the kernel:
+//   V = 0 (large products): the lane-replicated tables at absolute shared
+//     addresses, one CTA per SM.  Shared-memory map:
+//       C = 8:  [kSmemBase, 0x10000)  x slots of one column segment
+//               [0x10000, 0x20000)    stream jump-table rows
+//               [0x20000, 0x30000)    coefficient-table rows
+//       C = 12: [kSmemBase, 0x20000)  x slots of one column segment
+//               [0x20000, 0x30000)    stream jump-table rows
+//       both:   [0x30000, ...)        partial row sums of one pass
+//   V = 1 (small products, a few items per CTA): one copy of each table at
+//     the start of the allocation, 32 KB of x slots after it, then the
+//     partial sums; 8 warps and small allocations, so that several CTAs --
+//     of this launch and of the next one in the stream -- share an SM.  On
+//     a 512 x 512 matrix the replicated tables' setup (128 KB of shared
+//     stores, one CTA per SM) costs more than the product itself.
 constexpr uint32_t kSmemBase = 1024;
 constexpr uint32_t kTabCoef = 0x20000;
-template <int C>
+template <int C, int V>
 struct Smem {
-  static constexpr uint32_t kJump = (C == 8) ? 0x10000u : 0x20000u;
-  static constexpr uint32_t kPart = 0x30000u;
-  static constexpr uint32_t kXEnd = kJump;  // x slots end here
+  static constexpr uint32_t kJump = (C == 8) ? 0x10000u : 0x20000u;  // V = 0
+  // V = 1: jump tables (C = 8: 2 x 256 words; C = 12: 2 x 256 8-byte
+  // entries) then, for C = 8, the two coefficient tables (2 x 256 x 8 B).
+  static constexpr int kTabBytes = (V == 0) ? 0 : (C == 8) ? 2048 + 4096 : 4096;
+  static constexpr int kXOff = kTabBytes;  // bytes from the allocation's start
+  static constexpr int kXBytes = (V == 0) ? (int)(kJump - kSmemBase) : 32768;
+  static constexpr int kPartOff = (V == 0) ? (int)(0x30000u - kSmemBase) : kXOff + kXBytes;
   // x floats per lane unit: C * kBPL, rounded up to 32 for C = 12 (swizzle).
-  static constexpr int kSlotFloats = (C == 8) ? 8 * Tune<C>::kBPL : 32;
+  static constexpr int kSlotFloats = (C == 8) ? 8 * Tune<C, V>::kBPL : 32;
   static constexpr int kSpanBytes = kSpanUnits * kSlotFloats * 4;
-  static constexpr int kMaxSegSpans = (int)(kXEnd - kSmemBase) / kSpanBytes;
+  static constexpr int kMaxSegSpans = kXBytes / kSpanBytes;
   static constexpr int kPartBytesPerGroup = kRowsPerTask * 4;  // per warp
 };
-constexpr uint32_t kTabJump = Smem<8>::kJump;
+constexpr uint32_t kTabJump = Smem<8, 0>::kJump;
 
 struct GemvGeom {
   int rows, cols, nb, rec_pitch, e_pitch;
@@ -208,9 +221,26 @@ __device__ const CycleSeeds kCycleSeeds = make_cycle_seeds();
 //   tq2(v), v = q1 | q2 << 4: (kappa2, kappa3) = (256 q1 + q2, 256 q2) and
 //           -32768 q2
 // so that the block's integer start value is tq1.y + tq2.y - (e << 23).
-template <int C>
+template <int C, int V>
 __device__ void fill_tables(unsigned char* smem) {
-  uint4* jr = reinterpret_cast<uint4*>(smem + (Smem<C>::kJump - kSmemBase));
+  if constexpr (V == 1) {
+    // One copy: C = 8 words t_lo[256], t_hi[256], then tq1[256], tq2[256]
+    // (fill_coef_tables_c8's layout); C = 12 8-byte t_lo[256], t_hi[256].
+    for (int i = threadIdx.x; i < 512; i += blockDim.x) {
+      const uint64_t e = i < 256 ? kStreamTables.lo[i] : kStreamTables.hi[i - 256];
+      if constexpr (C == 8)
+        reinterpret_cast<uint32_t*>(smem)[i] = (uint32_t)e;
+      else
+        reinterpret_cast<uint2*>(smem)[i] = make_uint2((uint32_t)e, (uint32_t)(e >> 32));
+    }
+    if constexpr (C == 8) {
+      // The layout decode_c8_tab reads (it adds bits(M) itself).
+      uint2* tq = reinterpret_cast<uint2*>(smem + 2048);
+      fill_coef_tables_c8(tq, tq + 256, threadIdx.x, blockDim.x);
+    }
+    return;
+  }
+  uint4* jr = reinterpret_cast<uint4*>(smem + (Smem<C, 0>::kJump - kSmemBase));
 #if SEEDLM_GEMV_LFSR == 2
   if constexpr (C == 8) {
     // Cycle-window table: entry k = the seed at position 8k followed by its
@@ -292,8 +322,8 @@ __device__ __forceinline__ BlockC8 decode_c8_rep(uint32_t rec, uint32_t lane4, u
 __device__ __forceinline__ BlockC12 decode_c12_rep(uint32_t rec, uint32_t e4, uint32_t lane8) {
   BlockC12 b;
   b.lo = rec;
-  const uint2 x0 = lds64<Smem<12>::kJump>(prmt<0x5524u>(rec, lane8));
-  const uint2 x1 = lds64<Smem<12>::kJump + 128>(prmt<0x5534u>(rec, lane8));
+  const uint2 x0 = lds64<Smem<12, 0>::kJump>(prmt<0x5524u>(rec, lane8));
+  const uint2 x1 = lds64<Smem<12, 0>::kJump + 128>(prmt<0x5534u>(rec, lane8));
   b.mid = x0.x ^ x1.x;
   b.hi = x0.y ^ x1.y;
   coef_c12(b, rec, e4);
@@ -310,9 +340,9 @@ __device__ __forceinline__ BlockC12 decode_c12_rep(uint32_t rec, uint32_t e4, ui
 // so each lane reads its unit with 16-byte loads and one packed fp32x2 FMA
 // takes weight c of two blocks; the XOR swizzles keep the 8 lanes of a
 // quarter-warp on distinct bank groups.
-template <int C>
+template <int C, int V>
 __device__ __forceinline__ int x_slot_index(int u, int c, int h) {
-  if constexpr (C == 8 && Tune<8>::kBPL == 4) {
+  if constexpr (C == 8 && Tune<8, V>::kBPL == 4) {
     return u * 32 + ((c ^ (u & 7)) << 2) + h;
   } else if constexpr (C == 8) {
     return u * 16 + (((c >> 1) ^ ((u >> 1) & 3)) << 2) + ((c & 1) << 1) + h;
@@ -324,15 +354,15 @@ __device__ __forceinline__ int x_slot_index(int u, int c, int h) {
 // x columns of spans [s0, s0 + sl), zero past cols, into the segment's
 // slots.  One thread per lane unit; 16-byte loads when x is 16-byte aligned
 // and the unit lies inside x.
-template <int C>
+template <int C, int V>
 __device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, const GemvGeom& g,
                         int s0, int sl) {
-  constexpr int kBPL = Tune<C>::kBPL;
+  constexpr int kBPL = Tune<C, V>::kBPL;
   constexpr int kVals = C * kBPL;  // x values of one unit (16, 24 or 32)
   const int units = sl * kSpanUnits;
   const int col_base = s0 * kSpanUnits * kVals;
   const bool vec = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
-  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (Smem<C>::kXEnd - kSmemBase) / 4;)
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = Smem<C, V>::kXBytes / 4;)
   for (int u = threadIdx.x; u < units; u += blockDim.x) {
     const int col0 = col_base + u * kVals;
     uint16_t v16[kVals];
@@ -354,7 +384,7 @@ __device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, 
 #pragma unroll
     for (int k = 0; k < kVals; ++k) {
       const int h = k / C, c = k - h * C;
-      const int si = x_slot_index<C>(u, c, h);
+      const int si = x_slot_index<C, V>(u, c, h);
       const float f = act_to_float(v16[k], is_bf16);
       if (SEEDLM_IN_BOUNDS(g_check_flag, si, xs_floats)) xs[si] = f;
     }
@@ -365,31 +395,31 @@ __device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, 
 // kBPL blocks in each of the group's 4 rows, plus for C = 12 the exponent
 // byte of the pair.  Rows past `rows` and units past the row pitch read as
 // zero records (their x is zero, so they add nothing).
-template <int C>
+template <int C, int V>
 struct RecSet {
-  using Unit = typename std::conditional<Tune<C>::kBPL == 4, uint4, uint2>::type;
+  using Unit = typename std::conditional<Tune<C, V>::kBPL == 4, uint4, uint2>::type;
   Unit r[kRowsPerTask];
   uint32_t e[C == 12 ? kRowsPerTask : 1];
 };
 
-template <int C>
-__device__ __forceinline__ void load_unit(typename RecSet<C>::Unit& o, const uint32_t* p) {
-  if constexpr (Tune<C>::kBPL == 4) o = ld_stream_u4(p);
+template <int C, int V>
+__device__ __forceinline__ void load_unit(typename RecSet<C, V>::Unit& o, const uint32_t* p) {
+  if constexpr (Tune<C, V>::kBPL == 4) o = ld_stream_u4(p);
   else o = ld_stream_u2(p);
 }
 
-template <int C>
-__device__ __forceinline__ void load_set(RecSet<C>& o, const uint32_t* __restrict__ rec,
+template <int C, int V>
+__device__ __forceinline__ void load_set(RecSet<C, V>& o, const uint32_t* __restrict__ rec,
                                          const uint8_t* __restrict__ eplane, const GemvGeom& g,
                                          int grp, int span, int lane) {
-  constexpr int kBPL = Tune<C>::kBPL;
+  constexpr int kBPL = Tune<C, V>::kBPL;
   const int row0 = grp * kRowsPerTask;
   const int u = span * kSpanUnits + lane;
   const uint32_t* p = rec + (size_t)row0 * g.rec_pitch + kBPL * u;
   if (grp < g.full_groups && span < g.full_spans && !SEEDLM_CHECK) {
     // Every row of the group and every unit of the span is inside the plane.
 #pragma unroll
-    for (int j = 0; j < kRowsPerTask; ++j) load_unit<C>(o.r[j], p + (size_t)j * g.rec_pitch);
+    for (int j = 0; j < kRowsPerTask; ++j) load_unit<C, V>(o.r[j], p + (size_t)j * g.rec_pitch);
   } else {
     const bool unit_ok = kBPL * u < g.rec_pitch;
 #pragma unroll
@@ -399,8 +429,8 @@ __device__ __forceinline__ void load_set(RecSet<C>& o, const uint32_t* __restric
                       SEEDLM_IN_BOUNDS(g_check_flag,
                                        (size_t)(row0 + j) * g.rec_pitch + kBPL * u + kBPL - 1,
                                        (size_t)g.rows * g.rec_pitch);
-      if (ok) load_unit<C>(o.r[j], p + (size_t)j * g.rec_pitch);
-      else o.r[j] = typename RecSet<C>::Unit{};
+      if (ok) load_unit<C, V>(o.r[j], p + (size_t)j * g.rec_pitch);
+      else o.r[j] = typename RecSet<C, V>::Unit{};
     }
   }
   if constexpr (C == 12) {
@@ -456,11 +486,38 @@ __device__ __forceinline__ float2 fma_pair(int32_t bits_a, int32_t bits_b, float
 #endif
 }
 
+// The decode of the variant: replicated tables (V = 0) or the single copies
+// at the start of the allocation (V = 1).
+template <int V>
+__device__ __forceinline__ BlockC8 decode_c8_v(uint32_t rec, uint32_t lane4, uint32_t lane8,
+                                               const unsigned char* tabs) {
+  if constexpr (V == 0) {
+    return decode_c8_rep(rec, lane4, lane8);
+  } else {
+    const uint32_t* t = reinterpret_cast<const uint32_t*>(tabs);
+    const uint2* tq = reinterpret_cast<const uint2*>(tabs + 2048);
+    return decode_c8_tab(rec, t, t + 256, tq, tq + 256);
+  }
+}
+
+template <int V>
+__device__ __forceinline__ BlockC12 decode_c12_v(uint32_t rec, uint32_t e4, uint32_t lane8,
+                                                 const unsigned char* tabs) {
+  if constexpr (V == 0) {
+    return decode_c12_rep(rec, e4, lane8);
+  } else {
+    const uint2* t = reinterpret_cast<const uint2*>(tabs);
+    return decode_c12(rec, e4, t, t + 256);
+  }
+}
+
 // Blocks A and B of one row (x pairs xv[c] = (x of A's column c, x of B's)).
+template <int V>
 __device__ __forceinline__ float2 dot_c8(uint32_t ra, uint32_t rb, const float2 (&xv)[8],
-                                         uint32_t lane4, uint32_t lane8, float2 a) {
-  const BlockC8 A = decode_c8_rep(ra, lane4, lane8);
-  const BlockC8 B = decode_c8_rep(rb, lane4, lane8);
+                                         uint32_t lane4, uint32_t lane8,
+                                         const unsigned char* tabs, float2 a) {
+  const BlockC8 A = decode_c8_v<V>(ra, lane4, lane8, tabs);
+  const BlockC8 B = decode_c8_v<V>(rb, lane4, lane8, tabs);
   const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
 #define SEEDLM_C8_STEP(c) a = fma_pair(weight_bits_c8<c>(A), weight_bits_c8<c>(B), negm, xv[c], a);
   SEEDLM_C8_STEP(0) SEEDLM_C8_STEP(1) SEEDLM_C8_STEP(2) SEEDLM_C8_STEP(3)
@@ -472,12 +529,14 @@ __device__ __forceinline__ float2 dot_c8(uint32_t ra, uint32_t rb, const float2 
 // Rebuild the lane's kBPL x C weights of each of the 4 rows and accumulate
 // w * x into one fp32x2 sum per row.  ul is the lane's unit within the
 // staged segment.
-template <int C>
-__device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const float* __restrict__ xs,
-                                                int ul, int lane, uint32_t lane4, uint32_t lane8,
+template <int C, int V>
+__device__ __forceinline__ void rebuild_and_dot(const RecSet<C, V>& cur,
+                                                const float* __restrict__ xs, int ul, int lane,
+                                                uint32_t lane4, uint32_t lane8,
+                                                const unsigned char* tabs,
                                                 float2 (&acc)[kRowsPerTask]) {
-  const float* slot = xs + ul * Smem<C>::kSlotFloats;
-  if constexpr (C == 8 && Tune<8>::kBPL == 4) {
+  const float* slot = xs + ul * Smem<C, V>::kSlotFloats;
+  if constexpr (C == 8 && Tune<8, V>::kBPL == 4) {
     const int swz = lane & 7;
     float2 x01[8], x23[8];
 #pragma unroll
@@ -488,8 +547,8 @@ __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const floa
     }
 #pragma unroll
     for (int j = 0; j < kRowsPerTask; ++j) {
-      float2 a = dot_c8(cur.r[j].x, cur.r[j].y, x01, lane4, lane8, acc[j]);
-      acc[j] = dot_c8(cur.r[j].z, cur.r[j].w, x23, lane4, lane8, a);
+      float2 a = dot_c8<V>(cur.r[j].x, cur.r[j].y, x01, lane4, lane8, tabs, acc[j]);
+      acc[j] = dot_c8<V>(cur.r[j].z, cur.r[j].w, x23, lane4, lane8, tabs, a);
     }
   } else if constexpr (C == 8) {
     const int swz = (lane >> 1) & 3;
@@ -502,7 +561,7 @@ __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const floa
     }
 #pragma unroll
     for (int j = 0; j < kRowsPerTask; ++j)
-      acc[j] = dot_c8(cur.r[j].x, cur.r[j].y, xp, lane4, lane8, acc[j]);
+      acc[j] = dot_c8<V>(cur.r[j].x, cur.r[j].y, xp, lane4, lane8, tabs, acc[j]);
   } else {
     const int swz = lane & 7;
     float2 xp[C];
@@ -515,8 +574,8 @@ __device__ __forceinline__ void rebuild_and_dot(const RecSet<C>& cur, const floa
 #pragma unroll
     for (int j = 0; j < kRowsPerTask; ++j) {
       float2 a = acc[j];
-      const BlockC12 A = decode_c12_rep(cur.r[j].x, cur.e[j], lane8);
-      const BlockC12 B = decode_c12_rep(cur.r[j].y, cur.e[j] >> 4, lane8);
+      const BlockC12 A = decode_c12_v<V>(cur.r[j].x, cur.e[j], lane8, tabs);
+      const BlockC12 B = decode_c12_v<V>(cur.r[j].y, cur.e[j] >> 4, lane8, tabs);
       const float2 negm = make_float2(__uint_as_float(A.negm), __uint_as_float(B.negm));
 #if SEEDLM_GEMV_C12_ORDER == 1
       // Window-major: each of the 32 stream windows is formed once and feeds
@@ -558,31 +617,33 @@ struct GemvBatch {
 // a time (once per GEMV when one segment holds all of x); the (group, span)
 // items of the pass and segment are split into equal contiguous ranges, one
 // per warp.  A warp walks its range with record sets loaded
-// Tune<C>::kPrefetch items ahead (across group boundaries), and whenever it
+// Tune<C, V>::kPrefetch items ahead (across group boundaries), and whenever it
 // leaves a group it reduces its 4 row sums with shuffles and adds them into
 // its own slot of the pass's partial sums.  At the end of the pass the slots
 // of each row are added in warp order and written.
-template <int C, bool kBatch>
-__global__ void __launch_bounds__(Tune<C>::kWarps * 32, 1)
+template <int C, int V, bool kBatch>
+__global__ void __launch_bounds__(Tune<C, V>::kWarps * 32, Tune<C, V>::kMinBlocks)
 gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
-  constexpr int kP = Tune<C>::kPrefetch;
+  constexpr int kP = Tune<C, V>::kPrefetch;
   extern __shared__ __align__(16) unsigned char smem[];
-  // The table addresses are absolute: the allocation must start at kSmemBase.
-  if (smem_u32(smem) != kSmemBase) {
+  // V = 0: the table addresses are absolute, so the allocation must start at
+  // kSmemBase.
+  if (V == 0 && smem_u32(smem) != kSmemBase) {
     if (threadIdx.x == 0) atomicOr(&g_gemv_error, 1u);
     return;
   }
-  float* xs = reinterpret_cast<float*>(smem);
-  float* part = reinterpret_cast<float*>(smem + (Smem<C>::kPart - kSmemBase));
-  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = (Smem<C>::kXEnd - kSmemBase) / 4;
+  const unsigned char* tabs = smem;
+  float* xs = reinterpret_cast<float*>(smem + Smem<C, V>::kXOff);
+  float* part = reinterpret_cast<float*>(smem + Smem<C, V>::kPartOff);
+  SEEDLM_CHECK_ONLY(const unsigned int xs_floats = Smem<C, V>::kXBytes / 4;
                     const int part_floats =
-                        (int)(seedlm_dynamic_smem_bytes() - (Smem<C>::kPart - kSmemBase)) / 4;)
+                        (int)(seedlm_dynamic_smem_bytes() - Smem<C, V>::kPartOff) / 4;)
   const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lane4 = (uint32_t)lane << 2, lane8 = (uint32_t)(lane & 15) << 3;
-  RecSet<C> buf[kP + 1];
+  RecSet<C, V> buf[kP + 1];
 
-  fill_tables<C>(smem);
+  fill_tables<C, V>(smem);
   // Records and x may be the previous kernel's output: read them only now.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
@@ -603,7 +664,7 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
         const int s0 = sg * g.seg_spans;
         const int sl = min(g.seg_spans, g.n_spans - s0);
         // One segment: x stays staged for every pass of this GEMV.
-        if (g.n_segs > 1 || p0 == g0) stage_x<C>(xs, x, is_bf16, g, s0, sl);
+        if (g.n_segs > 1 || p0 == g0) stage_x<C, V>(xs, x, is_bf16, g, s0, sl);
         __syncthreads();  // x, tables and zeroed partials ready
         const int items = (p1 - p0) * sl;
         const int i0 = (int)((int64_t)warp * items / nw);
@@ -614,7 +675,7 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
           int lgrp = grp, lspan = span;
 #pragma unroll
           for (int k = 0; k <= kP; ++k) {
-            if (i0 + k < i1) load_set<C>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+            if (i0 + k < i1) load_set<C, V>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
             if (++lspan == sl) { lspan = 0; ++lgrp; }
           }
           float2 acc[kRowsPerTask];
@@ -626,10 +687,10 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
             for (int k = 0; k <= kP; ++k) {
               const int ul = span * kSpanUnits + lane;
               // Every x slot of the lane's unit lies in its kSlotFloats row.
-              if (SEEDLM_IN_BOUNDS(g_check_flag, (ul + 1) * Smem<C>::kSlotFloats - 1, xs_floats))
-                rebuild_and_dot<C>(buf[k], xs, ul, lane, lane4, lane8, acc);
+              if (SEEDLM_IN_BOUNDS(g_check_flag, (ul + 1) * (Smem<C, V>::kSlotFloats) - 1, xs_floats))
+                rebuild_and_dot<C, V>(buf[k], xs, ul, lane, lane4, lane8, tabs, acc);
               if (ci + kP + 1 < i1) {
-                load_set<C>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+                load_set<C, V>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
                 if (++lspan == sl) { lspan = 0; ++lgrp; }
               }
               ++ci;
@@ -669,20 +730,23 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
   }
 }
 
-template <int C>
+template <int C, int V>
 int warps_for(int items_per_cta) {
-  int w = items_per_cta < Tune<C>::kWarps ? items_per_cta : Tune<C>::kWarps;
+  int w = items_per_cta < Tune<C, V>::kWarps ? items_per_cta : Tune<C, V>::kWarps;
   // At least kMinWarps: on small matrices the CTA's setup (tables and x into
   // shared memory) outweighs its one or two items, and warps without items
   // still share it.
   return w < kMinWarps ? kMinWarps : w;
 }
 
+// Partial-sum bytes the small variant allows itself (keeps several CTAs per SM).
+constexpr int kSmallPartBytes = 16384;
+
 // The geometry for `nw` warps per CTA and `grid` CTAs, with the largest
 // partial-sum pass that fits; pass_groups = 0 if even one group does not.
-template <int C>
+template <int C, int V>
 GemvGeom make_geom(const seedlm_format& f, int max_smem, int nw, int grid) {
-  constexpr int kBPL = Tune<C>::kBPL;
+  constexpr int kBPL = Tune<C, V>::kBPL;
   GemvGeom g;
   g.rows = f.rows;
   g.cols = f.cols;
@@ -695,10 +759,11 @@ GemvGeom make_geom(const seedlm_format& f, int max_smem, int nw, int grid) {
   g.full_groups = f.rows / kRowsPerTask;
   // Units of the pitch: a span is full when its last unit ends inside it.
   g.full_spans = f.rec_pitch / (kBPL * kSpanUnits);
-  g.n_segs = (g.n_spans + Smem<C>::kMaxSegSpans - 1) / Smem<C>::kMaxSegSpans;
+  g.n_segs = (g.n_spans + Smem<C, V>::kMaxSegSpans - 1) / Smem<C, V>::kMaxSegSpans;
   g.seg_spans = (g.n_spans + g.n_segs - 1) / g.n_segs;
-  const int64_t room = (int64_t)max_smem - (int64_t)(Smem<C>::kPart - kSmemBase);
-  const int64_t per_group = (int64_t)Smem<C>::kPartBytesPerGroup * nw;
+  int64_t room = (int64_t)max_smem - Smem<C, V>::kPartOff;
+  if (V == 1 && room > kSmallPartBytes) room = kSmallPartBytes;
+  const int64_t per_group = (int64_t)Smem<C, V>::kPartBytesPerGroup * nw;
   const int max_cta_groups = grid > 0 ? (g.groups + grid - 1) / grid : 1;
   int64_t pg = room > 0 ? room / per_group : 0;
   if (pg > max_cta_groups) pg = max_cta_groups;
@@ -706,49 +771,72 @@ GemvGeom make_geom(const seedlm_format& f, int max_smem, int nw, int grid) {
   return g;
 }
 
-template <int C>
+template <int C, int V>
 size_t smem_for(const GemvGeom& g, int nw) {
-  return (size_t)(Smem<C>::kPart - kSmemBase) +
-         (size_t)g.pass_groups * Smem<C>::kPartBytesPerGroup * nw;
+  return (size_t)Smem<C, V>::kPartOff + (size_t)g.pass_groups * Smem<C, V>::kPartBytesPerGroup * nw;
 }
 
 struct GemvLaunch {
   GemvBatch b;
-  int grid, warps;
+  int grid, warps, variant;
   size_t smem;
 };
 
-// One launch for n GEMVs of format C: one CTA per SM (fewer if no GEMV has
-// that many row groups), warps for the largest share, and each GEMV's
-// partial-sum pass sized for that warp count.
-template <int C>
-GemvLaunch plan(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
-  constexpr int kBPL = Tune<C>::kBPL;
-  GemvLaunch L{};
-  int max_groups = 1, max_items = 1;
+// Work items (row group x span) of the busiest CTA, for a grid of up to
+// max_ctas CTAs.
+template <int C, int V>
+int max_items_per_cta(const seedlm_format* const* f, int n, int max_ctas, int* max_groups) {
+  constexpr int kBPL = Tune<C, V>::kBPL;
+  int mi = 1;
+  *max_groups = 1;
   for (int k = 0; k < n; ++k) {
     const int groups = (f[k]->rows + kRowsPerTask - 1) / kRowsPerTask;
     int n_spans = ((f[k]->nb + kBPL - 1) / kBPL + kSpanUnits - 1) / kSpanUnits;
     if (n_spans < 1) n_spans = 1;
-    if (groups > max_groups) max_groups = groups;
-    const int grid_k = groups < dev.num_sms ? groups : dev.num_sms;
+    if (groups > *max_groups) *max_groups = groups;
+    const int grid_k = groups < max_ctas ? groups : max_ctas;
     const int items = (groups + grid_k - 1) / (grid_k > 0 ? grid_k : 1) * n_spans;
-    if (items > max_items) max_items = items;
+    if (items > mi) mi = items;
   }
-  L.grid = max_groups < dev.num_sms ? max_groups : dev.num_sms;
-  L.warps = warps_for<C>(max_items);
+  return mi;
+}
+
+// One launch for n GEMVs of format C in variant V: one CTA per SM for V = 0
+// (fewer if no GEMV has that many row groups), up to two per SM for V = 1;
+// warps for the largest share, and each GEMV's partial-sum pass sized for
+// that warp count.
+template <int C, int V>
+GemvLaunch plan_v(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
+  GemvLaunch L{};
+  const int max_ctas = (V == 0) ? dev.num_sms : 2 * dev.num_sms;
+  int max_groups = 1;
+  const int max_items = max_items_per_cta<C, V>(f, n, max_ctas, &max_groups);
+  L.variant = V;
+  L.grid = max_groups < max_ctas ? max_groups : max_ctas;
+  L.warps = warps_for<C, V>(max_items);
   L.b.n = n;
   L.smem = 0;
   for (int k = 0; k < n; ++k) {
-    L.b.g[k] = make_geom<C>(*f[k], dev.max_smem_optin, L.warps, L.grid);
+    L.b.g[k] = make_geom<C, V>(*f[k], dev.max_smem_optin, L.warps, L.grid);
     if (L.b.g[k].pass_groups == 0) {
       L.smem = 0;
       return L;
     }
-    const size_t s = smem_for<C>(L.b.g[k], L.warps);
-    if (s > L.smem) L.smem = s;
+    const size_t sm = smem_for<C, V>(L.b.g[k], L.warps);
+    if (sm > L.smem) L.smem = sm;
   }
   return L;
+}
+
+// The small variant when the large one would give each of its 16 warps
+// fewer than 4 items: there the setup of the replicated tables and the
+// one-CTA-per-SM launch, not the rebuild, set the time.
+template <int C>
+GemvLaunch plan(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
+  int max_groups = 1;
+  const int items = max_items_per_cta<C, 0>(f, n, dev.num_sms, &max_groups);
+  if (items < 4 * Tune<C, 0>::kWarps) return plan_v<C, 1>(f, n, dev);
+  return plan_v<C, 0>(f, n, dev);
 }
 
 }  // namespace
@@ -770,6 +858,15 @@ int read_and_clear_gemv_error(unsigned int* out) {
   return SEEDLM_OK;
 }
 
+const void* kernel_for(int C, int V, bool batch) {
+  if (C == 8) {
+    if (V == 0) return batch ? (const void*)gemv_kernel<8, 0, true> : (const void*)gemv_kernel<8, 0, false>;
+    return batch ? (const void*)gemv_kernel<8, 1, true> : (const void*)gemv_kernel<8, 1, false>;
+  }
+  if (V == 0) return batch ? (const void*)gemv_kernel<12, 0, true> : (const void*)gemv_kernel<12, 0, false>;
+  return batch ? (const void*)gemv_kernel<12, 1, true> : (const void*)gemv_kernel<12, 1, false>;
+}
+
 int launch_gemv_batch(int n, const seedlm_format* const* f, const uint32_t* const* rec,
                       const uint8_t* const* eplane, const uint16_t* const* x, int is_bf16,
                       float* const* y, cudaStream_t stream, const DeviceInfo& dev) {
@@ -785,10 +882,7 @@ int launch_gemv_batch(int n, const seedlm_format* const* f, const uint32_t* cons
     L.b.y[k] = y[k];
   }
   const bool batch = n > 1;
-  const void* kern = (C == 8) ? (batch ? (const void*)gemv_kernel<8, true>
-                                       : (const void*)gemv_kernel<8, false>)
-                              : (batch ? (const void*)gemv_kernel<12, true>
-                                       : (const void*)gemv_kernel<12, false>);
+  const void* kern = kernel_for(C, L.variant, batch);
   int rc = allow_max_smem(kern, dev);
   if (rc) return rc;
   cudaLaunchConfig_t cfg = {};
@@ -801,11 +895,8 @@ int launch_gemv_batch(int n, const seedlm_format* const* f, const uint32_t* cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err =
-      (C == 8) ? (batch ? cudaLaunchKernelEx(&cfg, gemv_kernel<8, true>, L.b, is_bf16)
-                        : cudaLaunchKernelEx(&cfg, gemv_kernel<8, false>, L.b, is_bf16))
-               : (batch ? cudaLaunchKernelEx(&cfg, gemv_kernel<12, true>, L.b, is_bf16)
-                        : cudaLaunchKernelEx(&cfg, gemv_kernel<12, false>, L.b, is_bf16));
+  void* args[] = {(void*)&L.b, (void*)&is_bf16};
+  cudaError_t err = cudaLaunchKernelExC(&cfg, kern, args);
   if (err != cudaSuccess) return record_cuda_error(err);
   count_launch();
   return record_cuda_error(cudaGetLastError());

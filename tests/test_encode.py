@@ -178,6 +178,40 @@ def test_encode_decode_roundtrip_through_the_gemv(sl, oracle_mod):
     assert rel < 0.5, rel
 
 
+@pytest.mark.parametrize("cp,rows,cols", [(C8, 2400, 8192), (C12, 96, 1000)])
+def test_encode_then_gemv_on_one_stream(sl, oracle_mod, cp, rows, cols):
+    # The encoder writes the records and the GEMV (programmatic dependent
+    # launch) reads them right after it on the same stream, with no host
+    # synchronisation in between: the GEMV must wait for the encoder's
+    # writes before it reads a record.  Both the large-product kernel (2400
+    # rows) and the small one are covered.  The records start as garbage so
+    # that an early read would show.
+    rng = np.random.default_rng(cols)
+    W = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    fmt = inputs.make_format(rows, cols, *cp)
+    rec = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, fmt["rec_pitch"]), dtype=torch.int32,
+                        device="cuda")
+    ep = None
+    if fmt["P"] == 4:
+        ep = torch.randint(0, 256, (rows, fmt["e_pitch"]), dtype=torch.uint8, device="cuda")
+    xb, xv = inputs.make_activations((cols,), "f16", 5)
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+    y = torch.full((rows,), float("nan"), device="cuda")
+    Wd = torch.from_numpy(W).cuda()
+    torch.cuda.synchronize()
+    sl.encode(fmt, Wd, rec, ep)
+    sl.gemv(fmt, rec, ep, x, y)
+    torch.cuda.synchronize()
+    assert sl.device_error() == 0
+    rec_h = rec.cpu().numpy().view(np.uint32)
+    ep_h = None if ep is None else ep.cpu().numpy()
+    sample = np.unique(np.concatenate([np.arange(8), np.arange(rows - 8, rows),
+                                       rng.integers(0, rows, 48)]))
+    ref, refabs = oracle_mod.gemv_rows(fmt, rec_h, ep_h, xv, sample)
+    got = y.cpu().numpy().astype(np.float64)[sample]
+    assert np.all(np.abs(got - ref) <= 1e-5 * refabs + 1e-30)
+
+
 @pytest.mark.parametrize("cp,rows,cols", [(C8, 640, 512), (C12, 400, 576)])
 def test_many_tiles_per_cta_sampled_blocks(sl, oracle_mod, cp, rows, cols):
     # More 128-block tiles than the grid has CTAs (4-bit: 320 tiles on two

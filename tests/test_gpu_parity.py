@@ -232,12 +232,14 @@ def test_gemv_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols):
     assert_within(y[sample], ref, refabs)
 
 
-@pytest.mark.parametrize("cp,rows,cols", [(C8, 1800, 56320), (C12, 6000, 42240)])
-def test_gemv_multi_pass_wide_x(sl, oracle_mod, cp, rows, cols):
-    # x this wide leaves room in shared memory for only a few row groups of
-    # partial sums per pass (2 at 4 bits, 8 at 3 bits), so with these row
-    # counts every CTA runs several passes: the later passes re-zero the
-    # partials and reuse the staged x.  Checked on sampled rows.
+@pytest.mark.parametrize("cp,rows,cols", [(C8, 100000, 16), (C12, 100000, 24),
+                                          (C8, 1800, 56320), (C12, 6000, 42240)])
+def test_gemv_multi_pass_and_wide_x(sl, oracle_mod, cp, rows, cols):
+    # 100,000 short rows give each CTA about 169 row groups, more than one
+    # partial-sum pass holds (144 for 16 warps), so every CTA runs two
+    # passes: the second re-zeroes the partials and reuses the staged x.
+    # The wide shapes stage x in several column segments.  Checked on
+    # sampled rows.
     L = inputs.make_layer(rows, cols, *cp, seed=rows + cols)
     xb, xv = inputs.make_activations((cols,), "f16", 17)
     y = gpu_gemv(sl, L, xb)
@@ -404,19 +406,26 @@ def test_graph_replay_matches_eager_calls(sl):
 
 # ------------------------------------------------------------ wide x
 
-@pytest.mark.parametrize("cp,cols", [(C8, 70000), (C12, 50000), (C8, 15872), (C8, 15873),
-                                     (C12, 23808), (C12, 23809)])
-def test_gemv_wide_x_in_column_segments(sl, oracle_mod, cp, cols):
-    # x is staged in shared memory in column segments (31 spans of 512
-    # columns at 4 bits, 31 spans of 768 at 3 bits): 70,000 and 50,000
-    # columns take five and three segments; 15,872 columns (4 bits) and
-    # 23,808 (3 bits) exactly fill one segment, and one more column needs a
-    # second.  gemm_smallM with M = 1 runs the same kernel, same bits.
-    rows = 40
-    L = inputs.make_layer(rows, cols, *cp, seed=cols)
+@pytest.mark.parametrize("cp,rows,cols", [
+    # Large-product kernel (one CTA per SM, 16 warps, at least 64 items per
+    # CTA): 15 spans of 1024 columns (4 bits, 4 blocks per lane) or 31 of
+    # 768 (3 bits) per x segment.
+    (C8, 2400, 70000), (C12, 2400, 50000), (C8, 2400, 15360), (C8, 2400, 15361),
+    (C12, 2400, 23808), (C12, 2400, 23809),
+    # Small-product kernel (a few items per CTA): 32 KB of x slots, 16 spans
+    # of 512 columns (4 bits, 2 blocks per lane) or 8 of 768 (3 bits).
+    (C8, 40, 8192), (C8, 40, 8193), (C12, 40, 6144), (C12, 40, 6145),
+])
+def test_gemv_wide_x_in_column_segments(sl, oracle_mod, cp, rows, cols):
+    # x is staged in shared memory in column segments, so any width works;
+    # each kernel variant is checked exactly at, and one column past, its
+    # one-segment width, and the large one at many segments.  gemm_smallM with M = 1 runs the same kernel, same
+    # bits.
+    L = inputs.make_layer(rows, cols, *cp, seed=cols + rows)
     xb, xv = inputs.make_activations((cols,), "f16", 3)
     y = gpu_gemv(sl, L, xb)
-    ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv)
+    ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv,
+                                  threads=os.cpu_count() or 1)
     assert_within(y, ref, refabs)
     assert sl.gemm_workspace_bytes(L["fmt"], 1) == 0
     got = gpu_gemm(sl, L, xb.reshape(1, cols), dtype="f16")
@@ -426,15 +435,22 @@ def test_gemv_wide_x_in_column_segments(sl, oracle_mod, cp, cols):
 
 # ------------------------------------------------------------ batched GEMV
 
-@pytest.mark.parametrize("cp,shapes,dtype", [
-    (C8, [(1000, 8192), (40, 70000), (0, 512), (300, 999), (5000, 4096)], "f16"),
-    (C12, [(700, 4096), (33, 30000), (2000, 1000)], "bf16"),
+@pytest.mark.parametrize("cp,shapes,dtype,same_bits", [
+    # Products large enough that each alone runs the batch's configuration
+    # (the large-product kernel, 148 CTAs x 16 warps), as the projections of
+    # a 70B decoder layer do: the bits must agree.
+    (C8, [(8192, 8192), (10240, 8192), (8192, 28672), (16384, 8192)], "f16", True),
+    # Mixed shapes: one and several x segments, fewer row groups than SMs,
+    # an empty matrix; the batch's configuration may differ from an entry's
+    # own (another summation order), so only the tolerance applies.
+    (C8, [(1000, 8192), (40, 70000), (0, 512), (300, 999), (5000, 4096)], "f16", False),
+    (C12, [(700, 4096), (33, 30000), (2000, 1000)], "bf16", False),
 ])
-def test_gemv_batch_equals_separate_calls(sl, oracle_mod, cp, shapes, dtype):
-    # One launch for several GEMVs of one format (shapes with one and several
-    # x segments, fewer row groups than SMs, an empty matrix): every output
-    # has the bits of the separate seedlm_gemv call and is within tolerance
-    # of the oracle.
+def test_gemv_batch_matches_separate_calls(sl, oracle_mod, cp, shapes, dtype, same_bits):
+    # One launch for several GEMVs of one format.  Every output is within
+    # tolerance of the oracle, repeated batches give the same bits, and when
+    # the launch configuration is the one each entry would get alone, the
+    # bits of the separate seedlm_gemv calls.
     items, refs = [], []
     for i, (rows, cols) in enumerate(shapes):
         L = inputs.make_layer(rows, cols, *cp, seed=500 + i)
@@ -446,11 +462,16 @@ def test_gemv_batch_equals_separate_calls(sl, oracle_mod, cp, shapes, dtype):
         refs.append((L, xv))
     sl.gemv_batch(items)
     torch.cuda.synchronize()
-    for (fmt, rec, ep, x, y), (L, xv) in zip(items, refs):
-        ys = torch.full_like(y, float("nan"))
-        sl.gemv(fmt, rec, ep, x, ys)
-        torch.cuda.synchronize()
-        assert torch.equal(y.view(torch.int32), ys.view(torch.int32))
+    first = [it[4].clone() for it in items]
+    sl.gemv_batch(items)
+    torch.cuda.synchronize()
+    for (fmt, rec, ep, x, y), y0, (L, xv) in zip(items, first, refs):
+        assert torch.equal(y.view(torch.int32), y0.view(torch.int32))
+        if same_bits:
+            ys = torch.full_like(y, float("nan"))
+            sl.gemv(fmt, rec, ep, x, ys)
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int32), ys.view(torch.int32))
         if fmt["rows"]:
             ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv,
                                           threads=os.cpu_count() or 1)
