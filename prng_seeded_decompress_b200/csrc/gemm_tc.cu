@@ -4,55 +4,76 @@
 // Where the batch makes the product a real contraction (several rows of X
 // share every rebuilt weight), the reconstructed tiles feed tcgen05.mma
 // (paperhub.cn review thread: the weights are rebuilt from s and t and then
-// used to compute the activations).  The MMAs are kind::f16 (K = 16) in the
-// activations' own type, with W split exactly into pieces of that type:
+// used to compute the activations).  The MMAs are kind::f16 (K = 16) on
+// fp16 operands:
 //
-//   * bf16 X: W = p1 + p2 + p3, three bf16 pieces (8 significant bits each;
-//     a rebuilt weight has at most 20);
-//   * fp16 X: 2^6 W = p1 + p2, two fp16 pieces (11 significant bits each; the
-//     2^6 keeps the smallest weight quantum, 2^-30, at or above fp16's 2^-24)
-//     and Y is scaled back by 2^-6.
+//   * W: 2^6 W = p1 + p2, two fp16 pieces (11 significant bits each; a
+//     rebuilt weight has at most 20, and the 2^6 keeps the smallest weight
+//     quantum, 2^-30, at or above fp16's 2^-24).  Every product of a piece
+//     and an activation is exact in the fp32 accumulator.
+//   * X: fp16 activations as they are; bf16 activations scaled per row n by
+//     a power of two 2^s_n that brings the row's largest finite magnitude to
+//     [2^15, 2^16) and stored as fp16.  A bf16 value has 8 significant bits,
+//     so every element within a factor 2^33 of its row's largest is exact;
+//     smaller ones round to fp16's subnormal grid, an error below 2^-40 of
+//     the row's largest element.
+//   * Y = acc * 2^-(6 + s_n), applied as two exact power-of-two products.
 //
-// Every product of a piece and an activation is exact in the fp32 accumulator.
+// Two pieces instead of three bf16 pieces cut the MMAs per K step from 3 to
+// 2 and the producers' split from ten instructions per weight pair to six.
+//
 // One call is two launches:
 //
-//   1. stage_x_kernel copies X (M x cols) into the workspace in the
-//      tensor-core operand layout, one contiguous slab per K chunk (NB x KC
-//      16-bit elements, NB = M rounded up to 16, zero-padded), so the GEMM
-//      copies a chunk of X into shared memory with a single bulk copy.
+//   1. stage_x_kernel writes X (M x cols) into the workspace in the
+//      tensor-core operand layout, one contiguous fp16 slab per K chunk (NB x
+//      KC elements, NB = M rounded up to 16, zero-padded), and the two scale
+//      factors of each row.  A CTA covers one row n and a range of its
+//      columns; for bf16 X it first takes the maximum over the whole row.
 //   2. gemm_tc_kernel, one CTA per SM.  The work is the list of
 //      (128-row tile, K chunk) units in tile-major order, cut into equal
 //      contiguous ranges, one per CTA ("stream-K"), so every SM gets the same
 //      number of units whatever the shape.  Inside a CTA:
 //        * 16 producer warps rebuild the unit's 128 x KC weights exactly in
-//          fp32 (seedlm_device.cuh), split them into pieces, pack two K
+//          fp32 (seedlm_device.cuh) with the lane-replicated decode tables
+//          (rep_tables.cuh: one conflict-free shared-memory wavefront per
+//          lookup), split them into the two fp16 pieces, pack two K
 //          neighbours per 32-bit word and store them straight into tensor
-//          memory with tcgen05.st -- A operand stages, 128 lanes = rows.  Warp
-//          w owns TMEM lanes 32(w%4).. and a quarter (w/4) of the chunk's
-//          blocks.
+//          memory with tcgen05.st, one block at a time -- A operand stages,
+//          128 lanes = rows.  Warp w owns TMEM lanes 32(w%4).. and a quarter
+//          (w/4) of the chunk's blocks.
 //        * one thread issues the MMAs (M = 128, N = NB, A from TMEM, B = X
-//          slab from shared memory), all pieces into the same fp32
+//          slab from shared memory), both pieces into the same fp32
 //          accumulator in TMEM.  An MMA of this shape costs the tensor core
-//          about 45 cycles whatever N (<= 64) and K (8 for tf32, 16 here), so
-//          K = 16 halves the MMA count of a tf32 hi/lo split for fp16 X.
+//          about 45 cycles whatever N (<= 64) and K, so the MMA count, not
+//          M*N*K, sets the tensor-core time.
 //        * one thread keeps the X slabs coming, a few chunks ahead, with bulk
 //          copies.
 //        * stages are handed over with mbarriers only (A stage full: all 16
 //          producer warps arrived; A stage / X slab free: tcgen05.commit of the
 //          MMAs that read it), so no warp waits for the whole CTA.
 //        * the accumulator is double-buffered in TMEM.  At the end of each
-//          tile segment warps 0-3 read it out: a tile owned by one CTA goes
-//          straight to Y; otherwise each CTA writes a partial tile to the
-//          workspace and the last of the tile's CTAs to arrive (atomic
-//          counter) adds the partials in CTA order -- a fixed order, so every
-//          call gives the same bits -- writes Y and resets the counter.
+//          tile segment the MMA warp commits to an "accumulator full"
+//          barrier, and four epilogue warps of their own read it out and
+//          scale it while the producers go on with the next segment: a tile
+//          owned by one CTA goes straight to Y; otherwise each CTA writes a
+//          partial tile to the workspace and the last of the tile's CTAs to
+//          arrive (atomic counter) adds the partials in CTA order -- a fixed
+//          order, so every call gives the same bits -- writes Y and resets
+//          the counter.
 //   Every mbarrier wait is bounded; a wait that gives up raises the library's
 //   device error flag, and TMEM is always released.
+//
+//   The GEMM is launched with programmatic stream serialization: its
+//   prologue (tables, barriers, TMEM) and the producers' first units overlap
+//   stage_x_kernel.  The producers read only the records, which the kernel
+//   before stage_x_kernel (a plain launch, so fully finished) may have
+//   written; the X slabs and scale factors are read after griddepcontrol.wait.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
+#include "rep_tables.cuh"
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
 #include "tcgen05.cuh"
@@ -69,31 +90,29 @@ constexpr int kTileM = 128;
 constexpr int kProdWarps = 16;
 constexpr int kMmaWarp = kProdWarps;         // issues the MMAs (one thread)
 constexpr int kLoaderWarp = kProdWarps + 1;  // copies the X slabs (one thread)
-constexpr int kThreads = (kProdWarps + 2) * 32;
+constexpr int kEpiWarp0 = kProdWarps + 2;    // four warps drain the accumulators
+constexpr int kThreads = (kProdWarps + 6) * 32;
 constexpr int kTmemCols = 512;
+constexpr int kAccCols = 64;   // one accumulator (N <= 64); there are two
+constexpr int kShift = 6;      // the pieces are of 2^kShift W
+constexpr int kXS = 5;         // X slabs in shared memory
+constexpr int kHdrBytes = 1024;  // mbarriers, TMEM slot, row scales, at the allocation's start
+constexpr int kRecAhead = 2;   // units of records a producer thread has in flight
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
-// Per format and piece count (PC = 3: bf16 pieces, PC = 2: fp16 pieces):
-// K columns per unit, blocks per producer thread and unit, A stages in TMEM
-// (PC x KC/2 columns each, two 16-bit elements per column), X slabs in
-// shared memory.
-template <int C, int PC>
+// Per format: K columns per unit and blocks per producer thread and unit.
+template <int C>
 struct TcCfg;
-template <int PC>
-struct TcCfg<8, PC> {
+template <>
+struct TcCfg<8> {
   static constexpr int KC = 128;  // 16 blocks
   static constexpr int BPT = 4;
-  static constexpr int AS = (PC == 3) ? 2 : 3;
-  static constexpr int XS = 5;
 };
-template <int PC>
-struct TcCfg<12, PC> {
+template <>
+struct TcCfg<12> {
   static constexpr int KC = 96;  // 8 blocks
   static constexpr int BPT = 2;
-  static constexpr int AS = (PC == 3) ? 2 : 3;
-  static constexpr int XS = 5;
 };
-constexpr int kRecAhead = 2;   // units of records a producer thread has in flight
 
 struct TcGeom {
   int rows, cols, nb, rec_pitch, e_pitch, M;
@@ -102,28 +121,43 @@ struct TcGeom {
   int segs_max;     // most tiles any one CTA touches
 };
 
-template <int C, int NB, int PC>
+// Shared memory, by absolute shared address (the dynamic allocation starts
+// at rep::kSmemBase; checked at entry):
+//   [kSmemBase, +kHdrBytes)           mbarriers, TMEM base, flags, row scales
+//   [kSmemBase + kHdrBytes, tables)   X slabs, as many as fit
+//   [tables, rep::kEnd)               lane-replicated decode tables
+//   [rep::kEnd, ...)                  the remaining X slabs
+// TMEM: AS A stages of two pieces (KC/2 columns each: two fp16 per 32-bit
+// column), then two accumulators of kAccCols fp32 columns.
+template <int C, int NB>
 struct TcSmem {
-  static constexpr int KC = TcCfg<C, PC>::KC;
-  static constexpr int AS = TcCfg<C, PC>::AS;
-  static constexpr int XS = TcCfg<C, PC>::XS;
-  static constexpr int BPT = TcCfg<C, PC>::BPT;
-  static constexpr int SBO = KC * 16;  // bytes between 8-row groups of X (KC/8 core matrices)
-  static constexpr int XB = NB * KC * 2;  // one X slab (16-bit elements)
-  static constexpr int PIECE_COLS = KC / 2;      // TMEM columns of one piece of a stage
-  static constexpr int STAGE_COLS = PC * PIECE_COLS;
-  static constexpr int TABLE_OFF = XS * XB;
-  // C = 8: jump tables (2 KB) + coefficient tables (4 KB); C = 12: jump tables.
-  static constexpr int TABLE_BYTES = (C == 8) ? 512 * 4 + 512 * 8 : 512 * 8;
-  static constexpr int BAR_OFF = TABLE_OFF + TABLE_BYTES;
-  // mbarriers: xfull[XS] xfree[XS] afull[AS] afree[AS] dfree[2]
-  static constexpr int NBAR = 2 * XS + 2 * AS + 2;
-  static constexpr int SLOT_OFF = BAR_OFF + 8 * NBAR;  // TMEM base, last-CTA flag, give-up flag
-  static constexpr int TOTAL = SLOT_OFF + 16;
+  static constexpr int KC = TcCfg<C>::KC;
+  static constexpr int BPT = TcCfg<C>::BPT;
+  static constexpr int SBO = KC * 16;      // bytes between 8-row groups of X (KC/8 core matrices)
+  static constexpr int XB = NB * KC * 2;   // one X slab (fp16)
+  static constexpr int PIECE_COLS = KC / 2;
+  static constexpr int STAGE_COLS = 2 * PIECE_COLS;
+  static constexpr int AS = (kTmemCols - 2 * kAccCols) / STAGE_COLS;  // C = 8: 3, C = 12: 4
   static constexpr int D_COL = AS * STAGE_COLS;  // first accumulator column
-  static_assert(D_COL + 2 * 64 <= kTmemCols, "TMEM budget");
+  // mbarriers: xfull[kXS] xfree[kXS] afull[AS] afree[AS] dfree[2] dfull[2]
+  static constexpr int NBAR = 2 * kXS + 2 * AS + 4;
+  static constexpr uint32_t BAR = rep::kSmemBase;
+  static constexpr uint32_t SLOT = BAR + 8 * NBAR;  // TMEM base, last-CTA flag, give-up flag
+  static constexpr uint32_t YSCALE = rep::kSmemBase + 256;  // NB float2: the rows' output scales
+  static constexpr uint32_t SLAB_A = rep::kSmemBase + kHdrBytes;
+  static constexpr uint32_t TAB = rep::tables_begin<C>();
+  static constexpr int SLABS_A = (int)((TAB - SLAB_A) / XB) < kXS ? (int)((TAB - SLAB_A) / XB) : kXS;
+  static constexpr uint32_t END = rep::kEnd + (uint32_t)(kXS - SLABS_A) * XB;
+  static constexpr int TOTAL = (int)(END - rep::kSmemBase);
+  __host__ __device__ static constexpr uint32_t slab(int s) {
+    return s < SLABS_A ? SLAB_A + (uint32_t)s * XB : rep::kEnd + (uint32_t)(s - SLABS_A) * XB;
+  }
+  static_assert(SLOT + 16 <= YSCALE && YSCALE + 8 * kAccCols <= SLAB_A, "header");
+  static_assert(D_COL + 2 * kAccCols <= kTmemCols, "TMEM budget");
+  static_assert(NB <= kAccCols, "one accumulator holds N <= 64 columns");
   static_assert(KC == 4 * BPT * C, "four producer quarters of BPT blocks per unit");
   static_assert(KC % 16 == 0, "whole K = 16 MMA steps");
+  static_assert(SLAB_A % 16 == 0 && XB % 16 == 0, "bulk copies and descriptors need 16-byte alignment");
 };
 
 // Byte offset of X element (n, k) inside a slab (K-major core matrices:
@@ -134,31 +168,87 @@ __host__ __device__ constexpr int slab_byte(int n, int k) {
   return (n >> 3) * (KC * 16) + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
 }
 
+// 2^k as a float, -126 <= k <= 127.
+__device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(127 + k) << 23); }
+
+// Largest finite magnitude (as bf16 bits without the sign) among two packed
+// bf16 values; inf and NaN count as 0.
+__device__ __forceinline__ uint32_t finite_mag2(uint32_t v) {
+  const uint32_t a = v & 0x7FFFu, b = (v >> 16) & 0x7FFFu;
+  return max(a < 0x7F80u ? a : 0u, b < 0x7F80u ? b : 0u);
+}
+
+// One CTA per (row n of the padded batch, column part).  Writes the row's
+// fp16 slab entries for its part (zeros past M rows and past cols) and, part
+// 0, the row's output scale factors (f1, f2): Y = (acc * f1) * f2.
 template <int KC, int NB>
 __global__ void __launch_bounds__(256)
-stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks,
-               unsigned char* __restrict__ Xs) {
-  // The GEMM may start its prologue at once; it reads Xs only after
+stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks, int is_bf16,
+               int parts, int vec, unsigned char* __restrict__ Xs, float2* __restrict__ yscale) {
+  // The GEMM may start its prologue at once; it reads Xs and yscale only after
   // griddepcontrol.wait, i.e. after this grid has finished.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  constexpr int PER_CHUNK = NB * (KC / 8);  // 16-byte groups per slab
-  const long long total = (long long)nchunks * PER_CHUNK;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int chunk = (int)(i / PER_CHUNK);
-    const int rem = (int)(i - (long long)chunk * PER_CHUNK);
-    const int n = rem / (KC / 8), k8 = rem - n * (KC / 8);  // k fastest: coalesced reads
-    const int col = chunk * KC + 8 * k8;
-    uint32_t v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t a = (n < M && col + 2 * u < cols) ? X[(size_t)n * cols + col + 2 * u] : 0u;
-      const uint32_t b = (n < M && col + 2 * u + 1 < cols) ? X[(size_t)n * cols + col + 2 * u + 1] : 0u;
-      v[u] = a | (b << 16);
+  __shared__ uint32_t red[8];
+  const int n = blockIdx.x / parts, part = blockIdx.x - n * parts;
+  const uint16_t* row = X + (size_t)n * cols;
+  int s = 0;  // x is stored as x * 2^s
+  if (is_bf16 && n < M) {
+    uint32_t m = 0;
+    if (vec) {
+      const uint4* r4 = reinterpret_cast<const uint4*>(row);
+      for (int i = threadIdx.x; i < cols / 8; i += blockDim.x) {
+        const uint4 v = __ldg(r4 + i);
+        m = max(m, max(max(finite_mag2(v.x), finite_mag2(v.y)), max(finite_mag2(v.z), finite_mag2(v.w))));
+      }
+    } else {
+      for (int k = threadIdx.x; k < cols; k += blockDim.x) m = max(m, finite_mag2(row[k]));
     }
-    const size_t xb = (size_t)chunk * (NB * KC * 2) + slab_byte<KC>(n, 8 * k8);
+    m = __reduce_max_sync(0xffffffffu, m);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = max(m, red[w]);
+    if (m) {
+      const int E = max((int)(m >> 7), 1) - 127;  // the largest has its leading bit at or below 2^E
+      s = 15 - E;                                 // -112 <= s <= 141
+    }
+  }
+  const int s1 = s / 2, s2 = s - s1;
+  if (part == 0 && threadIdx.x == 0)
+    yscale[n] = make_float2(exp2i(-(kShift + s1)), exp2i(-s2));
+  const float g1 = exp2i(s1), g2 = exp2i(s2);
+  const int groups = nchunks * (KC / 8);  // 8-column groups of the padded row
+  const int g0 = (int)((long long)part * groups / parts);
+  const int g1e = (int)((long long)(part + 1) * groups / parts);
+  for (int gi = g0 + threadIdx.x; gi < g1e; gi += blockDim.x) {
+    const int col = 8 * gi;
+    uint16_t h[8];
+    if (n < M && vec && col + 8 <= cols) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + col));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u) h[u] = (uint16_t)(w[u >> 1] >> (16 * (u & 1)));
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) h[u] = (n < M && col + u < cols) ? row[col + u] : (uint16_t)0;
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) {
+      uint32_t a = h[u], b = h[u + 1];
+      if (is_bf16) {
+        const __half2 c = __floats2half2_rn(__uint_as_float(a << 16) * g1 * g2,
+                                            __uint_as_float(b << 16) * g1 * g2);
+        o[u >> 1] = *reinterpret_cast<const uint32_t*>(&c);
+      } else {
+        o[u >> 1] = a | (b << 16);
+      }
+    }
+    const int chunk = col / KC;
+    const size_t xb = (size_t)chunk * (NB * KC * 2) + slab_byte<KC>(n, col - chunk * KC);
     if (SEEDLM_IN_BOUNDS(g_check_flag, xb + 15, (size_t)nchunks * (NB * KC * 2)))
-      *reinterpret_cast<uint4*>(Xs + xb) = make_uint4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<uint4*>(Xs + xb) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -170,35 +260,30 @@ __device__ __forceinline__ int unit_owner(long long u, long long units, int ctas
   return (int)(((u + 1) * ctas + units - 1) / units) - 1;
 }
 
-// Pieces of two rebuilt weights (K neighbours) given as magic-biased floats
-// b (weight = b + nm), packed two per 32-bit word, the lower K index in the
-// low half.  All splits are exact.
-template <int PC>
-__device__ __forceinline__ void split_pair(float b0, float b1, float nm, uint32_t (&out)[PC]) {
-  if constexpr (PC == 3) {
-    // bf16: each piece keeps the top 8 significant bits of what is left.
-    const float2 w = __fadd2_rn(make_float2(b0, b1), make_float2(nm, nm));
-    const uint32_t h0 = __float_as_uint(w.x) & 0xFFFF0000u, h1 = __float_as_uint(w.y) & 0xFFFF0000u;
-    const float2 r = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)),
-                                make_float2(-1.f, -1.f), w);
-    const uint32_t m0 = __float_as_uint(r.x) & 0xFFFF0000u, m1 = __float_as_uint(r.y) & 0xFFFF0000u;
-    const float2 l = __ffma2_rn(make_float2(__uint_as_float(m0), __uint_as_float(m1)),
-                                make_float2(-1.f, -1.f), r);
-    out[0] = prmt<0x7632u>(h0, h1);
-    out[1] = prmt<0x7632u>(m0, m1);
-    out[2] = prmt<0x7632u>(__float_as_uint(l.x), __float_as_uint(l.y));
-  } else {
-    // fp16 of 2^6 w: the top 11 significant bits, then the rest.
-    const float2 w = __ffma2_rn(make_float2(b0, b1), make_float2(64.f, 64.f),
-                                make_float2(64.f * nm, 64.f * nm));
-    const uint32_t h0 = __float_as_uint(w.x) & 0xFFFFE000u, h1 = __float_as_uint(w.y) & 0xFFFFE000u;
-    const float2 l = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)),
-                                make_float2(-1.f, -1.f), w);
-    const __half2 ph = __floats2half2_rn(__uint_as_float(h0), __uint_as_float(h1));
-    const __half2 pl = __floats2half2_rn(l.x, l.y);
-    out[0] = *reinterpret_cast<const uint32_t*>(&ph);
-    out[1] = *reinterpret_cast<const uint32_t*>(&pl);
-  }
+// The two pieces of two rebuilt weights (K neighbours) given as
+// magic-biased bit patterns t (weight * 2^6 = t + nm): the top 11
+// significant bits h, then the rest l (at most 9 bits).  Both are exact in
+// fp16 and h + l is exact.  neg1 holds (-1, -1).
+__device__ __forceinline__ void f32_pieces(int32_t t0, int32_t t1, float2 nm, float2 neg1, float& h0,
+                                           float& h1, float& l0, float& l1) {
+  const float2 w = __fadd2_rn(make_float2(__int_as_float(t0), __int_as_float(t1)), nm);
+  h0 = __uint_as_float(__float_as_uint(w.x) & 0xFFFFE000u);
+  h1 = __uint_as_float(__float_as_uint(w.y) & 0xFFFFE000u);
+  const float2 l = __ffma2_rn(make_float2(h0, h1), neg1, w);
+  l0 = l.x;
+  l1 = l.y;
+}
+
+// The same pieces converted to fp16 and packed two per 32-bit word, the
+// lower K index in the low half.
+__device__ __forceinline__ void fp16_pieces(int32_t t0, int32_t t1, float2 nm, float2 neg1,
+                                            uint32_t& hi, uint32_t& lo) {
+  float h0, h1, l0, l1;
+  f32_pieces(t0, t1, nm, neg1, h0, h1, l0, l1);
+  const __half2 ph = __floats2half2_rn(h0, h1);
+  const __half2 pl = __floats2half2_rn(l0, l1);
+  hi = *reinterpret_cast<const uint32_t*>(&ph);
+  lo = *reinterpret_cast<const uint32_t*>(&pl);
 }
 
 // (tile, chunk) of consecutive units, advanced without dividing: a 64-bit
@@ -219,51 +304,45 @@ struct RecUnit {
   uint32_t e;                  // C = 12: their exponent byte
 };
 
-template <int C, int NB, int PC>
+template <int C, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
-               const unsigned char* __restrict__ Xs, float* __restrict__ Y,
-               float* __restrict__ partial, unsigned int* __restrict__ counters, TcGeom g) {
-  using L = TcSmem<C, NB, PC>;
-  constexpr int KC = L::KC, AS = L::AS, XS = L::XS, BPT = L::BPT;
-  constexpr float kYScale = (PC == 2) ? 1.0f / 64.0f : 1.0f;  // undo the fp16 pieces' 2^6
+               const unsigned char* __restrict__ Xs, const float2* __restrict__ yscale,
+               float* __restrict__ Y, float* __restrict__ partial,
+               unsigned int* __restrict__ counters, TcGeom g) {
+  using L = TcSmem<C, NB>;
+  constexpr int KC = L::KC, AS = L::AS, BPT = L::BPT;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ctas = gridDim.x;
-  // The whole shared-memory layout lies inside the launch's allocation
-  // (checked before any barrier or TMEM exists, so leaving is safe).
+  // The shared-memory map is by absolute address: the allocation must start
+  // at rep::kSmemBase and hold the whole map (checked before any barrier or
+  // TMEM exists, so leaving is safe).
+  if (tc::smem_u32(smem) != rep::kSmemBase) {
+    if (tid == 0) atomicOr(&g_tc_error, 1u);
+    return;
+  }
   if (!SEEDLM_IN_BOUNDS(g_check_flag, L::TOTAL - 1, seedlm_dynamic_smem_bytes())) return;
   const long long u_begin = unit_begin(blockIdx.x, g.units, ctas);
   const int n_units = (int)(unit_begin(blockIdx.x + 1, g.units, ctas) - u_begin);
   const int t_first = (int)(u_begin / g.nchunks);
   const UnitCursor c0{t_first, (int)(u_begin - (long long)t_first * g.nchunks)};
 
-  uint32_t* t32 = reinterpret_cast<uint32_t*>(smem + L::TABLE_OFF);
-  uint2* t64 = reinterpret_cast<uint2*>(smem + L::TABLE_OFF);
-  for (int i = tid; i < 512; i += kThreads) {
-    uint64_t v = i < 256 ? kStreamTables.lo[i] : kStreamTables.hi[i - 256];
-    if constexpr (C == 8)
-      t32[i] = (uint32_t)v;
-    else
-      t64[i] = make_uint2((uint32_t)v, (uint32_t)(v >> 32));
-  }
-  if constexpr (C == 8) {
-    uint2* tq = reinterpret_cast<uint2*>(t32 + 512);
-    fill_coef_tables_c8(tq, tq + 256, tid, kThreads);
-  }
-  const uint32_t bar = tc::smem_u32(smem + L::BAR_OFF);
+  rep::fill_rep_tables<C, kShift>(smem, tid, kThreads);
+  const uint32_t bar = L::BAR;
   // xfull: X slab landed.  xfree: the MMAs that read the slab completed.
   // afull: all producer warps stored the A stage.  afree: the unit's MMAs
-  // completed: its A stage may be reused and, at a segment's end, the
-  // accumulator is final.  dfree: warps 0-3 have read an accumulator out.
+  // completed: its A stage may be reused.  dfull: a segment's MMAs completed,
+  // its accumulator is final.  dfree: the epilogue warps have read it out.
   auto xfull = [&](int s) { return bar + 8 * s; };
-  auto xfree = [&](int s) { return bar + 8 * (XS + s); };
-  auto afull = [&](int s) { return bar + 8 * (2 * XS + s); };
-  auto afree = [&](int s) { return bar + 8 * (2 * XS + AS + s); };
-  auto dfree = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + b); };
-  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
+  auto xfree = [&](int s) { return bar + 8 * (kXS + s); };
+  auto afull = [&](int s) { return bar + 8 * (2 * kXS + s); };
+  auto afree = [&](int s) { return bar + 8 * (2 * kXS + AS + s); };
+  auto dfree = [&](int b) { return bar + 8 * (2 * kXS + 2 * AS + b); };
+  auto dfull = [&](int b) { return bar + 8 * (2 * kXS + 2 * AS + 2 + b); };
+  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + (L::SLOT - rep::kSmemBase));
   if (tid == 0) {
-    for (int s = 0; s < XS; ++s) {
+    for (int s = 0; s < kXS; ++s) {
       tc::mbar_init(xfull(s), 1);
       tc::mbar_init(xfree(s), 1);
     }
@@ -271,11 +350,14 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       tc::mbar_init(afull(s), kProdWarps);
       tc::mbar_init(afree(s), 1);
     }
-    for (int b = 0; b < 2; ++b) tc::mbar_init(dfree(b), 4);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(dfree(b), 4);
+      tc::mbar_init(dfull(b), 1);
+    }
     tc::fence_mbar_init();
     slot[2] = 0u;  // give-up flag shared by all bounded waits
   }
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(slot), kTmemCols);
+  if (warp == 0) tc::tmem_alloc(L::SLOT, kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -286,25 +368,24 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   if (warp == kLoaderWarp) {
     // ------------------------------------------------ X slabs
     if (lane == 0) {
-      const uint32_t xs0 = tc::smem_u32(smem);
       UnitCursor xc = c0;
       // Xs is written by the previous kernel on the stream.
       asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j = 0; j < n_units; ++j, xc.next(g.nchunks)) {
-        const int s = j % XS;
-        if (j >= XS)  // the slab's previous unit (j - XS) has finished its MMAs
-          ok = tc::mbar_wait_or_abort(xfree(s), ((j / XS) - 1) & 1, kWaitLimit, abort_flag) && ok;
+        const int s = j % kXS;
+        if (j >= kXS)  // the slab's previous unit (j - kXS) has finished its MMAs
+          ok = tc::mbar_wait_or_abort(xfree(s), ((j / kXS) - 1) & 1, kWaitLimit, abort_flag) && ok;
         if (SEEDLM_IN_BOUNDS(g_check_flag, xc.chunk, g.nchunks)) {
           tc::mbar_arrive_expect_tx(xfull(s), L::XB);
-          tc::bulk_g2s(xs0 + s * L::XB, Xs + (size_t)xc.chunk * L::XB, L::XB, xfull(s));
+          tc::bulk_g2s(L::slab(s), Xs + (size_t)xc.chunk * L::XB, L::XB, xfull(s));
         } else {
           tc::mbar_arrive(xfull(s));  // checked build: no copy, the hand-over still completes
         }
       }
       // Every copy this thread issued has landed before the CTA may exit
       // (bounded, and not cut short by the give-up flag).
-      for (int s = 0; s < XS && s < n_units; ++s) {
-        const int k = (n_units - 1 - s) / XS;  // last load into slab s
+      for (int s = 0; s < kXS && s < n_units; ++s) {
+        const int k = (n_units - 1 - s) / kXS;  // last load into slab s
         ok = tc::mbar_wait(xfull(s), k & 1, kWaitLimit) && ok;
       }
     }
@@ -314,8 +395,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     // The whole warp runs this loop with warp-uniform values (so they can
     // stay in uniform registers); one elected lane issues each MMA/commit.
     {
-      const uint32_t idesc = tc::idesc_f16(NB, PC == 3 ? 1 : 0);
-      const uint64_t bdesc0 = tc::smem_desc(tc::smem_u32(smem), 128, L::SBO);  // slab 0, K slice 0
+      constexpr uint32_t idesc = tc::idesc_f16(NB, 0);
       int seg = 0;
       UnitCursor mc = c0;
       for (int i = 0; i < n_units; ++i, mc.next(g.nchunks)) {
@@ -324,28 +404,36 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         const int db = seg & 1;
         if (first && seg >= 2)  // accumulator db was last used by segment seg - 2
           ok = tc::mbar_wait_or_abort(dfree(db), ((seg >> 1) - 1) & 1, kWaitLimit, abort_flag) && ok;
-        const int xs = i % XS, as = i % AS;
-        if (!tc::mbar_try_wait2(xfull(xs), (i / XS) & 1, afull(as), (i / AS) & 1)) {
-          ok = tc::mbar_wait_or_abort(xfull(xs), (i / XS) & 1, kWaitLimit, abort_flag) && ok;
+        const int xs = i % kXS, as = i % AS;
+        if (!tc::mbar_try_wait2(xfull(xs), (i / kXS) & 1, afull(as), (i / AS) & 1)) {
+          ok = tc::mbar_wait_or_abort(xfull(xs), (i / kXS) & 1, kWaitLimit, abort_flag) && ok;
           ok = tc::mbar_wait_or_abort(afull(as), (i / AS) & 1, kWaitLimit, abort_flag) && ok;
         }
         __syncwarp();  // reconverge before the elected issue
         tc::fence_after_sync();
-        // The issue rate bounds the kernel (an MMA of this shape takes the
-        // tensor core about 45 cycles), so everything but the MMAs is
-        // computed up front.
+        // The issue rate bounds the tensor core here, so everything but the
+        // MMAs is computed up front.
         const uint32_t a0 = tmem + as * L::STAGE_COLS;
-        const uint32_t d = tmem + L::D_COL + 64 * db;
-        const uint64_t bd = bdesc0 + (uint64_t)((xs * L::XB) >> 4);
+        const uint32_t d = tmem + L::D_COL + kAccCols * db;
+        const uint64_t bd = tc::smem_desc(L::slab(xs), 128, L::SBO);
         const uint32_t acc0 = first ? 0u : 1u;
+        if constexpr (C == 8) {
+          // The unit's 16 MMAs in one statement with one elect (measured: the
+          // per-MMA form costs the issuing warp 45 % more cycles).
+          static_assert(KC == 128 && L::PIECE_COLS == 64, "mma_f16_ts_warp_8x2's layout");
+          tc::mma_f16_ts_warp_8x2(d, a0, bd, idesc, acc0);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < KC / 16; ++kk)
+          for (int kk = 0; kk < KC / 16; ++kk)
 #pragma unroll
-          for (int pc = 0; pc < PC; ++pc)
-            tc::mma_f16_ts_warp(d, a0 + pc * L::PIECE_COLS + 8 * kk, bd + 16 * kk, idesc,
-                                (kk == 0 && pc == 0) ? acc0 : 1u);
-        tc::mma_commit_warp(afree(as));  // A stage free; at a segment's end the accumulator is final
+            for (int pc = 0; pc < 2; ++pc)
+              tc::mma_f16_ts_warp_nomask(d, a0 + pc * L::PIECE_COLS + 8 * kk, bd + 16 * kk, idesc,
+                                         (kk == 0 && pc == 0) ? acc0 : 1u);
+        }
+        tc::mma_commit_warp(afree(as));  // A stage free
         tc::mma_commit_warp(xfree(xs));  // X slab free
+        if (i == n_units - 1 || mc.chunk == g.nchunks - 1)
+          tc::mma_commit_warp(dfull(db));  // the segment's accumulator is final
       }
       // The CTA releases TMEM only after its last MMAs have completed
       // (bounded, not cut short by the give-up flag).
@@ -355,10 +443,121 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       }
     }
     __syncwarp();
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------ epilogue
+    // Warp kEpiWarp0 + j reads TMEM lanes 32 (warp % 4).. (a warp reaches
+    // the lane quarter of its warp index modulo 4), so the four warps cover
+    // all 128 rows of the tile.  Each segment's accumulator is read out 16
+    // columns at a time, scaled by the rows' factors and written.
+    const int eq = warp & 3;
+    const int row = 32 * eq + lane;
+    const bool leader = warp == kEpiWarp0 && lane == 0;
+    // The rows' scale factors, written by the previous kernel on the stream,
+    // into shared memory once.
+    float2* ys = reinterpret_cast<float2*>(smem + (L::YSCALE - rep::kSmemBase));
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int et = tid - kEpiWarp0 * 32;  // 0..127
+    if (et < NB) ys[et] = __ldcg(yscale + et);
+    tc::named_sync(128);
+    auto epilogue = [&](int seg, int tile) {
+      const int db = seg & 1;
+      ok = tc::mbar_wait_or_abort(dfull(db), (seg >> 1) & 1, kWaitLimit, abort_flag) && ok;
+      tc::fence_after_sync();
+      const int gr = tile * kTileM + row;
+      const int first = unit_owner((long long)tile * g.nchunks, g.units, ctas);
+      const int last = unit_owner((long long)(tile + 1) * g.nchunks - 1, g.units, ctas);
+      float* mine = partial + ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);
+      // Extents: Y holds M x rows floats; the partial tiles ctas x segs_max
+      // tiles of NB x 128 floats (one per segment of each CTA).
+      SEEDLM_CHECK_ONLY(const size_t y_n = (size_t)g.M * g.rows;
+                        const size_t part_n = (size_t)ctas * g.segs_max * (NB * kTileM);
+                        const size_t mine_off = ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);)
+#pragma unroll
+      for (int n16 = 0; n16 < NB / 16; ++n16) {
+        float v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(32 * eq) << 16) + L::D_COL + kAccCols * db + 16 * n16, v);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float2 f = ys[16 * n16 + q];
+          v[q] = v[q] * f.x * f.y;
+        }
+        if (first == last) {
+          if (gr < g.rows) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              if (16 * n16 + q < g.M &&
+                  SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(16 * n16 + q) * g.rows + gr, y_n))
+                Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q];
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            if (SEEDLM_IN_BOUNDS(g_check_flag, seg, g.segs_max) &&
+                SEEDLM_IN_BOUNDS(g_check_flag, mine_off + (16 * n16 + q) * kTileM + row, part_n))
+              mine[(16 * n16 + q) * kTileM + row] = v[q];
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(dfree(db));
+      if (first == last) return;
+      // The leader publishes the four warps' partial tile (the barrier orders
+      // their stores before its fence) and counts it; the last CTA of the
+      // tile to count reads every partial after its own fence and barrier.
+      tc::named_sync(128);
+      if (leader) {
+        __threadfence();
+        const bool is_last = SEEDLM_IN_BOUNDS(g_check_flag, tile, g.tiles) &&
+                             atomicAdd(&counters[tile], 1u) == (unsigned)(last - first);
+        if (is_last) __threadfence();
+        slot[1] = is_last ? 1u : 0u;
+      }
+      tc::named_sync(128);
+      if (slot[1]) {
+        if (gr < g.rows) {
+          // Y = partial(first) + partial(first + 1) + ... in CTA order, 16
+          // batch rows at a time in registers (independent loads; Y written
+          // once).
+#pragma unroll 1
+          for (int n16 = 0; n16 < NB / 16; ++n16) {
+            float acc[16];
+#pragma unroll 1
+            for (int c = first; c <= last; ++c) {
+              const int cseg = tile - (int)(unit_begin(c, g.units, ctas) / g.nchunks);
+              const size_t off = ((size_t)c * g.segs_max + cseg) * (NB * kTileM) +
+                                 (size_t)(16 * n16) * kTileM + row;
+              const bool in = SEEDLM_IN_BOUNDS(g_check_flag, cseg, g.segs_max) &&
+                              SEEDLM_IN_BOUNDS(g_check_flag, off + 15 * kTileM, part_n);
+              const float* p = partial + (in ? off : 0);
+              if (c == first) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) acc[q] = __ldcg(p + q * kTileM);
+              } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) acc[q] += __ldcg(p + q * kTileM);
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              if (16 * n16 + q < g.M &&
+                  SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(16 * n16 + q) * g.rows + gr, y_n))
+                Y[(size_t)(16 * n16 + q) * g.rows + gr] = acc[q];
+          }
+        }
+        if (leader) counters[tile] = 0u;
+      }
+      tc::named_sync(128);  // slot[1] is rewritten by the next segment
+    };
+    UnitCursor ec = c0;
+    int seg = 0;
+    for (int i = 0; i < n_units; ++i, ec.next(g.nchunks))
+      if (i == n_units - 1 || ec.chunk == g.nchunks - 1) epilogue(seg++, ec.tile);
   } else {
-    // ------------------------------------------------ producers (+ epilogue)
+    // ------------------------------------------------ producers
     const int lq = warp & 3, kq = warp >> 2;
     const int prow = 32 * lq + lane;  // TMEM lane = row in the tile
+    const uint32_t lane4 = (uint32_t)lane << 2, lane8 = (uint32_t)(lane & 15) << 3;
+    const float2 neg1 = make_float2(-1.f, -1.f);
     auto load_rec = [&](const UnitCursor& u, RecUnit<C>& p) {
       const int gr = u.tile * kTileM + prow;
       const int b0 = u.chunk * (KC / C) + kq * BPT;  // a multiple of BPT
@@ -382,140 +581,50 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       const int as = i % AS;
       if (i >= AS) ok = tc::mbar_wait_or_abort(afree(as), ((i / AS) - 1) & 1, kWaitLimit, abort_flag) && ok;
       tc::fence_after_sync();
-      // Piece pc of this thread's BPT * C weights: BPT * C / 2 packed columns.
+      // The thread's BPT * C weights are BPT * C / 2 packed columns of each piece.
       constexpr int NPACK = BPT * C / 2;
       const uint32_t col0 = tmem + ((uint32_t)(32 * lq) << 16) + as * L::STAGE_COLS + kq * NPACK;
-      uint32_t pk[PC][NPACK];
+      if constexpr (C == 8) {
+        // Two blocks at a time: eight packed columns of each piece.
 #pragma unroll
-      for (int j = 0; j < BPT; ++j) {
-        float b[C];
-        float nm;
-        if constexpr (C == 8) {
-          // With bf16 pieces (the busier integer pipe) the coefficient words
-          // come from the shared tables, measured 2 % faster; with fp16
-          // pieces computing them is 2 % faster.
-          const uint2* tq1 = reinterpret_cast<const uint2*>(t32 + 512);
-          const BlockC8 blk = (PC == 3) ? decode_c8_tab(cur.r[j], t32, t32 + 256, tq1, tq1 + 256)
-                                        : decode_c8(cur.r[j], t32, t32 + 256);
-          nm = __uint_as_float(blk.negm);
-          b[0] = __int_as_float(weight_bits_c8<0>(blk));
-          b[1] = __int_as_float(weight_bits_c8<1>(blk));
-          b[2] = __int_as_float(weight_bits_c8<2>(blk));
-          b[3] = __int_as_float(weight_bits_c8<3>(blk));
-          b[4] = __int_as_float(weight_bits_c8<4>(blk));
-          b[5] = __int_as_float(weight_bits_c8<5>(blk));
-          b[6] = __int_as_float(weight_bits_c8<6>(blk));
-          b[7] = __int_as_float(weight_bits_c8<7>(blk));
-        } else {
-          const BlockC12 blk = decode_c12(cur.r[j], (j ? cur.e >> 4 : cur.e) & 15u, t64, t64 + 256);
-          nm = __uint_as_float(blk.negm);
-          b[0] = __int_as_float(weight_bits_c12<0>(blk));
-          b[1] = __int_as_float(weight_bits_c12<1>(blk));
-          b[2] = __int_as_float(weight_bits_c12<2>(blk));
-          b[3] = __int_as_float(weight_bits_c12<3>(blk));
-          b[4] = __int_as_float(weight_bits_c12<4>(blk));
-          b[5] = __int_as_float(weight_bits_c12<5>(blk));
-          b[6] = __int_as_float(weight_bits_c12<6>(blk));
-          b[7] = __int_as_float(weight_bits_c12<7>(blk));
-          b[8] = __int_as_float(weight_bits_c12<8>(blk));
-          b[9] = __int_as_float(weight_bits_c12<9>(blk));
-          b[10] = __int_as_float(weight_bits_c12<10>(blk));
-          b[11] = __int_as_float(weight_bits_c12<11>(blk));
+        for (int j2 = 0; j2 < BPT; j2 += 2) {
+          float h[16], l[16];
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            const BlockC8 blk = rep::decode_c8_rep<kShift>(cur.r[j2 + jj], lane4, lane8);
+            const float2 nm = make_float2(__uint_as_float(blk.negm), __uint_as_float(blk.negm));
+            float* hh = h + 8 * jj;
+            float* ll = l + 8 * jj;
+            f32_pieces(weight_bits_c8<0>(blk), weight_bits_c8<1>(blk), nm, neg1, hh[0], hh[1], ll[0], ll[1]);
+            f32_pieces(weight_bits_c8<2>(blk), weight_bits_c8<3>(blk), nm, neg1, hh[2], hh[3], ll[2], ll[3]);
+            f32_pieces(weight_bits_c8<4>(blk), weight_bits_c8<5>(blk), nm, neg1, hh[4], hh[5], ll[4], ll[5]);
+            f32_pieces(weight_bits_c8<6>(blk), weight_bits_c8<7>(blk), nm, neg1, hh[6], hh[7], ll[6], ll[7]);
+          }
+          tc::tmem_st_f16_pieces_x8(col0 + 4 * j2, col0 + L::PIECE_COLS + 4 * j2, h, l);
+        }
+      } else {
+        uint32_t ph[NPACK], pl[NPACK];
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+          const BlockC12 blk = rep::decode_c12_rep<kShift>(cur.r[j], (j ? cur.e >> 4 : cur.e) & 15u, lane8);
+          const float2 nm = make_float2(__uint_as_float(blk.negm), __uint_as_float(blk.negm));
+          fp16_pieces(weight_bits_c12<0>(blk), weight_bits_c12<1>(blk), nm, neg1, ph[6 * j + 0], pl[6 * j + 0]);
+          fp16_pieces(weight_bits_c12<2>(blk), weight_bits_c12<3>(blk), nm, neg1, ph[6 * j + 1], pl[6 * j + 1]);
+          fp16_pieces(weight_bits_c12<4>(blk), weight_bits_c12<5>(blk), nm, neg1, ph[6 * j + 2], pl[6 * j + 2]);
+          fp16_pieces(weight_bits_c12<6>(blk), weight_bits_c12<7>(blk), nm, neg1, ph[6 * j + 3], pl[6 * j + 3]);
+          fp16_pieces(weight_bits_c12<8>(blk), weight_bits_c12<9>(blk), nm, neg1, ph[6 * j + 4], pl[6 * j + 4]);
+          fp16_pieces(weight_bits_c12<10>(blk), weight_bits_c12<11>(blk), nm, neg1, ph[6 * j + 5], pl[6 * j + 5]);
         }
 #pragma unroll
-        for (int c = 0; c < C; c += 2) {
-          uint32_t o[PC];
-          split_pair<PC>(b[c], b[c + 1], nm, o);
-#pragma unroll
-          for (int pc = 0; pc < PC; ++pc) pk[pc][(j * C + c) / 2] = o[pc];
-        }
-      }
-#pragma unroll
-      for (int pc = 0; pc < PC; ++pc) {
-        if constexpr (C == 8) {
-          tc::tmem_st16(col0 + pc * L::PIECE_COLS, pk[pc]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < NPACK / 4; ++q) tc::tmem_st4(col0 + pc * L::PIECE_COLS + 4 * q, pk[pc] + 4 * q);
+        for (int q = 0; q < NPACK / 4; ++q) {
+          tc::tmem_st4(col0 + 4 * q, ph + 4 * q);
+          tc::tmem_st4(col0 + L::PIECE_COLS + 4 * q, pl + 4 * q);
         }
       }
       tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(afull(as));
-    };
-
-    // Warps 0-3 (all 128 TMEM lanes) drain the accumulator of a segment, 16
-    // columns at a time.
-    auto epilogue = [&](int seg, int tile, int i_last) {
-      const int db = seg & 1;
-      ok = tc::mbar_wait_or_abort(afree(i_last % AS), (i_last / AS) & 1, kWaitLimit, abort_flag) &&
-           ok;
-      tc::fence_after_sync();
-      const int row = 32 * warp + lane;
-      const int gr = tile * kTileM + row;
-      const int first = unit_owner((long long)tile * g.nchunks, g.units, ctas);
-      const int last = unit_owner((long long)(tile + 1) * g.nchunks - 1, g.units, ctas);
-      float* mine = partial + ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);
-      // Extents: Y holds M x rows floats; the partial tiles ctas x segs_max
-      // tiles of NB x 128 floats (one per segment of each CTA).
-      SEEDLM_CHECK_ONLY(const size_t y_n = (size_t)g.M * g.rows;
-                        const size_t part_n = (size_t)ctas * g.segs_max * (NB * kTileM);
-                        const size_t mine_off = ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);)
-#pragma unroll
-      for (int n16 = 0; n16 < NB / 16; ++n16) {
-        float v[16];
-        tc::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + L::D_COL + 64 * db + 16 * n16, v);
-        if (first == last) {
-          if (gr < g.rows) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q)
-              if (16 * n16 + q < g.M &&
-                  SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(16 * n16 + q) * g.rows + gr, y_n))
-                Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q] * kYScale;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            if (SEEDLM_IN_BOUNDS(g_check_flag, seg, g.segs_max) &&
-                SEEDLM_IN_BOUNDS(g_check_flag, mine_off + (16 * n16 + q) * kTileM + row, part_n))
-              mine[(16 * n16 + q) * kTileM + row] = v[q] * kYScale;
-        }
-      }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(dfree(db));
-      if (first == last) return;
-      __threadfence();
-      tc::named_sync(128);
-      if (tid == 0)
-        slot[1] = SEEDLM_IN_BOUNDS(g_check_flag, tile, g.tiles) &&
-                          atomicAdd(&counters[tile], 1u) == (unsigned)(last - first)
-                      ? 1u
-                      : 0u;
-      tc::named_sync(128);
-      if (slot[1]) {
-        __threadfence();
-        if (gr < g.rows) {
-          // Y = partial(first) + partial(first + 1) + ... in CTA order.
-          for (int c = first; c <= last; ++c) {
-            const int cseg = tile - (int)(unit_begin(c, g.units, ctas) / g.nchunks);
-            const float* p = partial + ((size_t)c * g.segs_max + cseg) * (NB * kTileM) + row;
-            if (!SEEDLM_IN_BOUNDS(g_check_flag, cseg, g.segs_max) ||
-                !SEEDLM_IN_BOUNDS(g_check_flag,
-                                  ((size_t)c * g.segs_max + cseg) * (NB * kTileM) +
-                                      (size_t)(g.M - 1) * kTileM + row,
-                                  part_n))
-              continue;
-            for (int n = 0; n < g.M; ++n) {
-              float* y = Y + (size_t)n * g.rows + gr;
-              *y = (c == first) ? p[n * kTileM] : *y + p[n * kTileM];
-            }
-          }
-        }
-        if (tid == 0) counters[tile] = 0u;
-      }
-      tc::named_sync(128);  // slot[1] is rewritten by the next segment
     };
 
     RecUnit<C> ring[kRecAhead];
@@ -526,8 +635,6 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         load_rec(rc, ring[k]);
         rc.next(g.nchunks);
       }
-    UnitCursor pc = c0;  // unit being rebuilt
-    int seg = 0;
     for (int i0 = 0; i0 < n_units; i0 += kRecAhead) {
 #pragma unroll
       for (int k = 0; k < kRecAhead; ++k) {
@@ -538,11 +645,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
             load_rec(rc, ring[k]);
             rc.next(g.nchunks);
           }
-          if (i > 0 && pc.chunk == 0) ++seg;
           produce(i, cur);
-          if (warp < 4 && (i == n_units - 1 || pc.chunk == g.nchunks - 1))
-            epilogue(seg, pc.tile, i);
-          pc.next(g.nchunks);
         }
       }
     }
@@ -557,8 +660,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   }
 }
 
-// K columns per unit (the same for both piece types).
-int kc_of(int C) { return C == 8 ? TcCfg<8, 3>::KC : TcCfg<12, 3>::KC; }
+int kc_of(int C) { return C == 8 ? TcCfg<8>::KC : TcCfg<12>::KC; }
 
 TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev, int* ctas) {
   TcGeom g;
@@ -584,10 +686,11 @@ TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev, int* c
   return g;
 }
 
-// Workspace: [tile counters][X slabs][partial tiles], each part 256-aligned.
+// Workspace: [tile counters][row scale factors][X slabs][partial tiles], each
+// part 256-aligned.
 struct TcWorkspace {
-  int64_t cnt_bytes, xs_bytes, part_bytes;
-  int64_t total() const { return cnt_bytes + xs_bytes + part_bytes; }
+  int64_t cnt_bytes, scale_bytes, xs_bytes, part_bytes;
+  int64_t total() const { return cnt_bytes + scale_bytes + xs_bytes + part_bytes; }
 };
 
 int64_t round256(int64_t v) { return (v + 255) / 256 * 256; }
@@ -596,28 +699,31 @@ TcWorkspace tc_workspace(const TcGeom& g, int C, int ctas) {
   const int NB = (g.M + 15) / 16 * 16;
   TcWorkspace w;
   w.cnt_bytes = round256((int64_t)g.tiles * 4);
+  w.scale_bytes = round256((int64_t)NB * 8);
   w.xs_bytes = round256((int64_t)g.nchunks * NB * kc_of(C) * 2);
   w.part_bytes = round256((int64_t)ctas * g.segs_max * NB * kTileM * 4);
   return w;
 }
 
-template <int C, int NB, int PC>
+template <int C, int NB>
 int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* eplane,
-              const uint16_t* X, float* Y, unsigned char* ws, const TcWorkspace& w,
+              const uint16_t* X, int is_bf16, float* Y, unsigned char* ws, const TcWorkspace& w,
               cudaStream_t stream, const DeviceInfo& dev) {
-  using L = TcSmem<C, NB, PC>;
+  using L = TcSmem<C, NB>;
   if ((size_t)L::TOTAL > (size_t)dev.max_smem_optin) return SEEDLM_EUNSUPPORTED;
-  int rc = allow_max_smem((const void*)gemm_tc_kernel<C, NB, PC>, dev);
+  int rc = allow_max_smem((const void*)gemm_tc_kernel<C, NB>, dev);
   if (rc) return rc;
   unsigned int* counters = reinterpret_cast<unsigned int*>(ws);
-  unsigned char* xs = ws + w.cnt_bytes;
-  float* partial = reinterpret_cast<float*>(ws + w.cnt_bytes + w.xs_bytes);
+  float2* yscale = reinterpret_cast<float2*>(ws + w.cnt_bytes);
+  unsigned char* xs = ws + w.cnt_bytes + w.scale_bytes;
+  float* partial = reinterpret_cast<float*>(ws + w.cnt_bytes + w.scale_bytes + w.xs_bytes);
 
-  const long long groups = (long long)g.nchunks * NB * (L::KC / 8);
-  long long want = (groups + 255) / 256;
-  const long long cap = 8ll * dev.num_sms;
-  const int sgrid = (int)(want < cap ? (want < 1 ? 1 : want) : cap);
-  stage_x_kernel<L::KC, NB><<<sgrid, 256, 0, stream>>>(X, g.M, g.cols, g.nchunks, xs);
+  // stage_x: NB rows x parts CTAs, about 256 column groups of 8 per CTA.
+  const int groups = g.nchunks * (L::KC / 8);
+  const int parts = groups / 256 < 1 ? 1 : (groups / 256 > 64 ? 64 : groups / 256);
+  const int vec = (reinterpret_cast<uintptr_t>(X) % 16 == 0) && (g.cols % 8 == 0);
+  stage_x_kernel<L::KC, NB><<<NB * parts, 256, 0, stream>>>(X, g.M, g.cols, g.nchunks, is_bf16,
+                                                             parts, vec, xs, yscale);
   count_launch();
   if ((rc = record_cuda_error(cudaGetLastError()))) return rc;
 
@@ -631,35 +737,31 @@ int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* epl
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<C, NB, PC>, rec, eplane,
-                                       (const unsigned char*)xs, Y, partial, counters, g);
+  cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<C, NB>, rec, eplane,
+                                       (const unsigned char*)xs, (const float2*)yscale, Y, partial,
+                                       counters, g);
   if (err != cudaSuccess) return record_cuda_error(err);
   count_launch();
   return record_cuda_error(cudaGetLastError());
 }
 
-template <int C, int PC>
+template <int C>
 int dispatch_nb(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* eplane,
-                const uint16_t* X, float* Y, unsigned char* ws, const TcWorkspace& w,
+                const uint16_t* X, int is_bf16, float* Y, unsigned char* ws, const TcWorkspace& w,
                 cudaStream_t st, const DeviceInfo& dev) {
   switch ((g.M + 15) / 16 * 16) {
-    case 16: return launch_tc<C, 16, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
-    case 32: return launch_tc<C, 32, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
-    case 48: return launch_tc<C, 48, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
-    default: return launch_tc<C, 64, PC>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+    case 16: return launch_tc<C, 16>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    case 32: return launch_tc<C, 32>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    case 48: return launch_tc<C, 48>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    default: return launch_tc<C, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
   }
 }
 
-// bf16 activations take three bf16 pieces of W, fp16 activations two fp16
-// pieces (of 2^6 W): A and B of one MMA always have the same type.
 int dispatch_tc(const seedlm_format& f, const TcGeom& g, int ctas, const uint32_t* rec,
                 const uint8_t* eplane, const uint16_t* X, int is_bf16, float* Y,
                 unsigned char* ws, const TcWorkspace& w, cudaStream_t st, const DeviceInfo& dev) {
-  if (f.C == 8)
-    return is_bf16 ? dispatch_nb<8, 3>(g, ctas, rec, eplane, X, Y, ws, w, st, dev)
-                   : dispatch_nb<8, 2>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
-  return is_bf16 ? dispatch_nb<12, 3>(g, ctas, rec, eplane, X, Y, ws, w, st, dev)
-                 : dispatch_nb<12, 2>(g, ctas, rec, eplane, X, Y, ws, w, st, dev);
+  if (f.C == 8) return dispatch_nb<8>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+  return dispatch_nb<12>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
 }
 
 }  // namespace

@@ -9,21 +9,14 @@
 // arithmetic (seedlm_device.cuh) plus its decode, and the decode's table
 // lookups are random.  The kernel is organised around two facts:
 //
-//   * Lane-replicated tables, conflict-free.  Every decode table (the stream
-//     jump tables, and for C = 8 the coefficient tables) is stored once per
-//     lane, in rows of 256 bytes: row v holds entry v for each lane side by
-//     side (4-byte entries: lanes 0..31; 8-byte entries: lanes 0..15, one
-//     half-warp at a time).  Lane l therefore always reads its own bank (bank
-//     pair) whatever index it looks up: one shared-memory wavefront per
-//     lookup instead of ~3.2 for random indices into a single copy, which
-//     saturated the shared-memory pipe before.
-//   * One-instruction table addresses.  The table rows start at fixed shared
-//     addresses (kTabJump, kTabCoef), so the address of (row v, lane l) is
-//     (v << 8) | lane_offset: one prmt moves the index byte of the record
-//     next to the lane's offset byte, and the table base rides in the load's
-//     immediate offset.  The dynamic shared allocation must start at shared
-//     address kSmemBase for this (checked at entry; a mismatch raises the
-//     device error flag and the kernel does nothing).
+//   * Lane-replicated tables, conflict-free, at fixed shared addresses
+//     (rep_tables.cuh): one shared-memory wavefront per lookup instead of
+//     ~3.2 for random indices into a single copy, which saturated the
+//     shared-memory pipe before, and a one-instruction address (one prmt of
+//     the record's index byte next to the lane's offset; the table base
+//     rides in the load's immediate offset).  The dynamic shared allocation
+//     must start at shared address kSmemBase for this (checked at entry; a
+//     mismatch raises the device error flag and the kernel does nothing).
 //
 // Work decomposition (one CTA per SM, persistent):
 //   * x is converted to fp32 into shared memory in a swizzled "record pair"
@@ -49,6 +42,7 @@
 
 #include <type_traits>
 
+#include "rep_tables.cuh"
 #include "seedlm_device.cuh"
 #include "seedlm_internal.h"
 
@@ -128,11 +122,12 @@ constexpr int kSpanUnits = 32;    // lane units (pairs or quads of blocks) per s
 //     of this launch and of the next one in the stream -- share an SM.  On
 //     a 512 x 512 matrix the replicated tables' setup (128 KB of shared
 //     stores, one CTA per SM) costs more than the product itself.
-constexpr uint32_t kSmemBase = 1024;
-constexpr uint32_t kTabCoef = 0x20000;
+using rep::kSmemBase;
+using rep::lds32;
+using rep::lds64;
 template <int C, int V>
 struct Smem {
-  static constexpr uint32_t kJump = (C == 8) ? 0x10000u : 0x20000u;  // V = 0
+  static constexpr uint32_t kJump = rep::tables_begin<C>();  // V = 0
   // V = 1: jump tables (C = 8: 2 x 256 words; C = 12: 2 x 256 8-byte
   // entries) then, for C = 8, the two coefficient tables (2 x 256 x 8 B).
   static constexpr int kTabBytes = (V == 0) ? 0 : (C == 8) ? 2048 + 4096 : 4096;
@@ -145,7 +140,9 @@ struct Smem {
   static constexpr int kMaxSegSpans = kXBytes / kSpanBytes;
   static constexpr int kPartBytesPerGroup = kRowsPerTask * 4;  // per warp
 };
+#if SEEDLM_GEMV_LFSR == 2
 constexpr uint32_t kTabJump = Smem<8, 0>::kJump;
+#endif
 
 struct GemvGeom {
   int rows, cols, nb, rec_pitch, e_pitch;
@@ -160,20 +157,6 @@ struct GemvGeom {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-template <uint32_t OFF>
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
-  return v;
-}
-
-template <uint32_t OFF>
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
-  return v;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -210,17 +193,8 @@ constexpr CycleSeeds make_cycle_seeds() {
 __device__ const CycleSeeds kCycleSeeds = make_cycle_seeds();
 #endif
 
-// Fills the table rows.  Row v (256 bytes) holds, for C = 8,
-//   jump rows:  ext_lo(v) for lanes 0..31, then ext_hi(v) for lanes 0..31
-//               (4 bytes each: stream bits 16..47 of the seed bytes v and v<<8)
-//   coef rows:  tq1(v) for lanes 0..15, then tq2(v) for lanes 0..15 (8 bytes)
-// and for C = 12 the jump rows only, with 8-byte entries (stream bits 16..79)
-// for lanes 0..15.  Coefficient entries, with q the signed nibble values:
-//   tq1(v), v = q0 | q1 << 4: (kappa0, kappa1) = (q0, 256 q0 + q1) and
-//           bits(1.5 * 2^8) - 32768 (q0 + q1)
-//   tq2(v), v = q1 | q2 << 4: (kappa2, kappa3) = (256 q1 + q2, 256 q2) and
-//           -32768 q2
-// so that the block's integer start value is tq1.y + tq2.y - (e << 23).
+// Fills the decode tables: for V = 1 one copy of each at the start of the
+// allocation, for V = 0 the lane-replicated rows (rep_tables.cuh).
 template <int C, int V>
 __device__ void fill_tables(unsigned char* smem) {
   if constexpr (V == 1) {
@@ -240,52 +214,29 @@ __device__ void fill_tables(unsigned char* smem) {
     }
     return;
   }
-  uint4* jr = reinterpret_cast<uint4*>(smem + (Smem<C, 0>::kJump - kSmemBase));
+  rep::fill_rep_tables<C, 0>(smem, threadIdx.x, blockDim.x);
 #if SEEDLM_GEMV_LFSR == 2
   if constexpr (C == 8) {
     // Cycle-window table: entry k = the seed at position 8k followed by its
-    // stream bits 16..63 (64 KB in place of the jump rows).
-    uint2* cw = reinterpret_cast<uint2*>(jr);
+    // stream bits 16..63, written over the jump rows (64 KB).
+    __syncthreads();
+    uint2* cw = reinterpret_cast<uint2*>(smem + (Smem<C, 0>::kJump - kSmemBase));
     for (int i = threadIdx.x; i < 8192; i += blockDim.x) {
       const uint32_t sd = kCycleSeeds.s[i];
       const uint64_t ext = kStreamTables.lo[sd & 0xffu] ^ kStreamTables.hi[sd >> 8];
       const uint64_t e = (uint64_t)sd | (ext << 16);
       cw[i] = make_uint2((uint32_t)e, (uint32_t)(e >> 32));
     }
-  } else
+  }
 #endif
-  // One thread per (row v, table): one 8-byte read of the jump table, eight
-  // 16-byte stores of its lane copies.
-  for (int t = threadIdx.x; t < 512; t += blockDim.x) {
-    const int v = t & 255, which = t >> 8;
-    const uint64_t e = which ? kStreamTables.hi[v] : kStreamTables.lo[v];
-    const uint32_t lo = (uint32_t)e, hi = (uint32_t)(e >> 32);
-    const uint4 q = (C == 8) ? make_uint4(lo, lo, lo, lo) : make_uint4(lo, hi, lo, hi);
-    uint4* row = jr + v * 16 + which * 8;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) row[k] = q;
-  }
-  if constexpr (C == 8) {
-    uint4* cr = reinterpret_cast<uint4*>(smem + (kTabCoef - kSmemBase));
-    for (int t = threadIdx.x; t < 512; t += blockDim.x) {
-      const int v = t & 255, which = t >> 8;
-      const int32_t a = nibble_value(v), b = nibble_value(v >> 4);
-      const uint2 e = which == 0 ? make_uint2(pack_s16(a, 256 * a + b),
-                                              kMagicBits - (uint32_t)(32768 * (a + b)))
-                                 : make_uint2(pack_s16(256 * a + b, 256 * b),
-                                              (uint32_t)(-32768 * b));
-      const uint4 q = make_uint4(e.x, e.y, e.x, e.y);
-      uint4* row = cr + v * 16 + which * 8;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) row[k] = q;
-    }
-  }
 }
 
-// C = 8 decode from the replicated tables.  The record's byte 2 and byte 3
-// are the seed's low and high bytes, byte 0 is q0 | q1 << 4 and bits 4..11
-// are q1 | q2 << 4.
+// C = 8 decode from the replicated tables (rep_tables.cuh), or by one of the
+// comparison LFSR variants.
 __device__ __forceinline__ BlockC8 decode_c8_rep(uint32_t rec, uint32_t lane4, uint32_t lane8) {
+#if SEEDLM_GEMV_LFSR == 0
+  return rep::decode_c8_rep<0>(rec, lane4, lane8);
+#else
   BlockC8 b;
 #if SEEDLM_GEMV_LFSR == 1
   b.lo = rec;
@@ -293,7 +244,7 @@ __device__ __forceinline__ BlockC8 decode_c8_rep(uint32_t rec, uint32_t lane4, u
   const uint32_t t1 = lfsr_pass(rec);                     // bits 16..26 valid at 16..26
   const uint32_t t2 = lfsr_pass(prmt<0x7632u>(rec, t1));  // stream 0..26 -> 16..37 at 0..21
   b.hi = lfsr_pass(prmt<0x5432u>(rec, t2));               // stream 0..31 -> 16..42 at 0..26
-#elif SEEDLM_GEMV_LFSR == 2
+#else
   // rec bits [16,32) = position P in the cycle; the table entry k holds
   // cycle bits [8k, 8k + 64).
   const uint32_t pos = rec >> 16;
@@ -302,32 +253,20 @@ __device__ __forceinline__ BlockC8 decode_c8_rep(uint32_t rec, uint32_t lane4, u
   const uint32_t s_lo = __funnelshift_r(w.x, w.y, sh), s_hi = w.y >> sh;  // bits [P, P+56)
   b.lo = s_lo << 16;
   b.hi = __funnelshift_r(s_lo, s_hi, 16);
-#else
-  b.lo = rec;
-  b.hi = lds32<kTabJump>(prmt<0x5524u>(rec, lane4)) ^
-         lds32<kTabJump + 128>(prmt<0x5534u>(rec, lane4));
 #endif
-  const uint2 c1 = lds64<kTabCoef>(prmt<0x5504u>(rec, lane8));
-  const uint2 c2 = lds64<kTabCoef + 128>(prmt<0x5514u>(rec << 4, lane8));
+  const uint2 c1 = lds64<rep::kCoef8>(prmt<0x5504u>(rec, lane8));
+  const uint2 c2 = lds64<rep::kCoef8 + 128>(prmt<0x5514u>(rec << 4, lane8));
   b.a01 = c1.x;
   b.a23 = c2.x;
   const uint32_t e23 = (rec << 11) & 0x07800000u;  // e << 23
   b.init = (int32_t)(c1.y + c2.y - e23);
   b.negm = kNegMagicBits - e23;
   return b;
+#endif
 }
 
-// C = 12 decode: stream windows from the replicated 8-byte jump tables, the
-// coefficients computed from the record's nibbles (seedlm_device.cuh).
 __device__ __forceinline__ BlockC12 decode_c12_rep(uint32_t rec, uint32_t e4, uint32_t lane8) {
-  BlockC12 b;
-  b.lo = rec;
-  const uint2 x0 = lds64<Smem<12, 0>::kJump>(prmt<0x5524u>(rec, lane8));
-  const uint2 x1 = lds64<Smem<12, 0>::kJump + 128>(prmt<0x5534u>(rec, lane8));
-  b.mid = x0.x ^ x1.x;
-  b.hi = x0.y ^ x1.y;
-  coef_c12(b, rec, e4);
-  return b;
+  return rep::decode_c12_rep<0>(rec, e4, lane8);
 }
 
 // x slot layout, per lane unit u (kBPL consecutive blocks of a row):

@@ -223,7 +223,9 @@ struct BlockC12 {
 };
 
 // The coefficient part of a C = 12 block: (q_p, 256 q_p) pairs, the integer
-// start value and -M_e.  e4 is the block's exponent in bits [0,4).
+// start value and -M_e.  e4 is the block's exponent in bits [0,4).  SHIFT
+// scales the weights by 2^SHIFT (added to the exponent of M_e).
+template <int SHIFT = 0>
 __device__ __forceinline__ void coef_c12(BlockC12& b, uint32_t rec, uint32_t e4) {
   uint32_t v = prmt<0x5140u>(rec, rec >> 4) & 0x0f0f0f0fu;  // (q0, q1, q2, q3)
   uint32_t s = sext_nibble_bytes(v);
@@ -234,8 +236,8 @@ __device__ __forceinline__ void coef_c12(BlockC12& b, uint32_t rec, uint32_t e4)
   b.a[3] = prmt<0x3cb3u>(s, v);
   int32_t qsum = __dp4a((int)s, 0x01010101, 0);
   uint32_t e23 = (e4 & 15u) << 23;
-  b.init = (int32_t)(kMagicBits - e23) - qsum * 32768;
-  b.negm = kNegMagicBits - e23;
+  b.init = (int32_t)(kMagicBits + ((uint32_t)SHIFT << 23) - e23) - qsum * 32768;
+  b.negm = kNegMagicBits + ((uint32_t)SHIFT << 23) - e23;
 }
 
 // e4 is the block's exponent in bits [0,4).

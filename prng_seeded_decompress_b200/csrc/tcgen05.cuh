@@ -55,6 +55,56 @@ __device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem
       : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
         "r"(0u), "r"(0u));
 }
+// The same MMA without the disable-output-lane mask operand (every lane of
+// D written): fewer operands to move into uniform registers per MMA.
+__device__ __forceinline__ void mma_f16_ts_warp_nomask(uint32_t d_tmem, uint32_t a_tmem,
+                                                       uint64_t b_desc, uint32_t idesc,
+                                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Eight K = 16 steps of two pieces (16 MMAs) in one statement: piece pc of
+// step k reads A at a0 + pc * pcols + 8 k and B at b_desc + 16 k (the
+// descriptor's address field counts 16-byte units).  One elect for all.
+__device__ __forceinline__ void mma_f16_ts_warp_8x2(uint32_t d_tmem, uint32_t a0, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b32 a<16>;\n\t.reg .b64 b<8>;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.u32 a1, %1, 64;\n\t add.u32 a2, %1, 8;\n\t add.u32 a3, %1, 72;\n\t"
+      "add.u32 a4, %1, 16;\n\t add.u32 a5, %1, 80;\n\t add.u32 a6, %1, 24;\n\t add.u32 a7, %1, 88;\n\t"
+      "add.u32 a8, %1, 32;\n\t add.u32 a9, %1, 96;\n\t add.u32 a10, %1, 40;\n\t add.u32 a11, %1, 104;\n\t"
+      "add.u32 a12, %1, 48;\n\t add.u32 a13, %1, 112;\n\t add.u32 a14, %1, 56;\n\t add.u32 a15, %1, 120;\n\t"
+      "add.u64 b1, %2, 16;\n\t add.u64 b2, %2, 32;\n\t add.u64 b3, %2, 48;\n\t add.u64 b4, %2, 64;\n\t"
+      "add.u64 b5, %2, 80;\n\t add.u64 b6, %2, 96;\n\t add.u64 b7, %2, 112;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], %2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a8], b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a9], b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a10], b5, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a11], b5, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a12], b6, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a13], b6, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a14], b7, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a15], b7, %3, t;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a0), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
 __device__ __forceinline__ void mma_commit_warp(uint32_t mbar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -142,6 +192,37 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
                : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
                : "memory");
 }
+// Converts the 32 floats of two pieces of 16 K-consecutive weights to fp16
+// (exact) and stores them, two per 32-bit column with the lower K index in
+// the low half: h into 8 columns at taddr_h, l into 8 columns at taddr_l.
+// The conversions write the store's source registers directly.
+__device__ __forceinline__ void tmem_st_f16_pieces_x8(uint32_t taddr_h, uint32_t taddr_l,
+                                                      const float (&h)[16], const float (&l)[16]) {
+  asm volatile(
+      "{\n\t.reg .b32 q<16>;\n\t"
+      "cvt.rn.f16x2.f32 q0, %3, %2;\n\t"
+      "cvt.rn.f16x2.f32 q1, %5, %4;\n\t"
+      "cvt.rn.f16x2.f32 q2, %7, %6;\n\t"
+      "cvt.rn.f16x2.f32 q3, %9, %8;\n\t"
+      "cvt.rn.f16x2.f32 q4, %11, %10;\n\t"
+      "cvt.rn.f16x2.f32 q5, %13, %12;\n\t"
+      "cvt.rn.f16x2.f32 q6, %15, %14;\n\t"
+      "cvt.rn.f16x2.f32 q7, %17, %16;\n\t"
+      "cvt.rn.f16x2.f32 q8, %19, %18;\n\t"
+      "cvt.rn.f16x2.f32 q9, %21, %20;\n\t"
+      "cvt.rn.f16x2.f32 q10, %23, %22;\n\t"
+      "cvt.rn.f16x2.f32 q11, %25, %24;\n\t"
+      "cvt.rn.f16x2.f32 q12, %27, %26;\n\t"
+      "cvt.rn.f16x2.f32 q13, %29, %28;\n\t"
+      "cvt.rn.f16x2.f32 q14, %31, %30;\n\t"
+      "cvt.rn.f16x2.f32 q15, %33, %32;\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {q0, q1, q2, q3, q4, q5, q6, q7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%1], {q8, q9, q10, q11, q12, q13, q14, q15};\n\t}\n"
+      :
+      : "r"(taddr_h), "r"(taddr_l), "f"(h[0]), "f"(h[1]), "f"(h[2]), "f"(h[3]), "f"(h[4]), "f"(h[5]), "f"(h[6]), "f"(h[7]), "f"(h[8]), "f"(h[9]), "f"(h[10]), "f"(h[11]), "f"(h[12]), "f"(h[13]), "f"(h[14]), "f"(h[15]), "f"(l[0]), "f"(l[1]), "f"(l[2]), "f"(l[3]), "f"(l[4]), "f"(l[5]), "f"(l[6]), "f"(l[7]), "f"(l[8]), "f"(l[9]), "f"(l[10]), "f"(l[11]), "f"(l[12]), "f"(l[13]), "f"(l[14]), "f"(l[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -311,6 +311,32 @@ def test_gemm_many_short_tiles_per_cta(sl, oracle_mod, cp, rows, cols, M):
         assert_within(got[m], ref[m], refabs[m])
 
 
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_gemm_bf16_rows_of_any_magnitude(sl, oracle_mod, cp):
+    # bf16 activations reach the tensor cores as fp16 scaled by a power of two
+    # per row, chosen from the row's largest finite magnitude: rows near the
+    # top and the bottom of bf16's range (subnormal included), a zero row,
+    # and a row spanning 2^40 between its largest and smallest elements.
+    rows, cols = 300, 3000
+    L = inputs.make_layer(rows, cols, *cp, seed=404)
+    rng = np.random.default_rng(405)
+    base = rng.standard_normal((6, cols)).astype(np.float32)
+    scales = np.array([1e30, 1e-30, 0.0, 1.5e-39, 1.0, 1e34], dtype=np.float32)
+    v = base * scales[:, None]
+    v[4] = base[4] * np.float32(1e-6)
+    v[4, 7] = np.float32(1e6)  # one element 2^40 above the rest
+    Xb = inputs.f32_to_bf16_bits(v.astype(np.float32))
+    Xv = inputs.bf16_bits_to_f64(Xb)
+    assert np.all(np.isfinite(Xv)) and np.any(Xv[3] != 0) and np.all(np.abs(Xv[3]) < 2.0 ** -126)
+    got = gpu_gemm(sl, L, Xb)
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv)
+    assert np.array_equal(got[2], np.zeros(rows))
+    for m in range(6):
+        # No absolute floor: the bound scales with the row.
+        err = np.abs(got[m] - ref[m])
+        assert np.all(err <= TOL * refabs[m]), (m, float((err / (refabs[m] + 1e-300)).max()))
+
+
 def test_gemm_workspace_reuse_is_deterministic(sl):
     # The same workspace across calls (counters must be left at zero) and
     # bit-identical results (split-K partials are added in a fixed order).
