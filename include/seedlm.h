@@ -141,16 +141,20 @@ SEEDLM_API int seedlm_gemv_batch(int32_t n, const seedlm_format* fmts,
  * inference uses s and t: the blocks are rebuilt from seed and coefficients
  * and multiplied with the activations; a batch of M activation rows shares
  * every rebuilt block).  M = 1 runs the GEMV kernel; otherwise the rebuilt
- * weight tiles feed the
- * tcgen05 tensor cores (kind::f16
- * MMAs in the activations' type: W split exactly into three bf16 pieces for
- * bf16 X, two fp16 pieces of 2^6 W for fp16 X; exact products, fp32
- * accumulation in TMEM) -- two launches: X is first copied into the operand
- * layout, then one CTA per SM runs the GEMM.
+ * weight tiles feed the tcgen05 tensor cores: kind::f16 MMAs on fp16
+ * operands, W split exactly into two fp16 pieces of 2^6 W, fp32 accumulation
+ * in TMEM.  fp16 X is used as it is; bf16 X is scaled per row by a power of
+ * two that brings the row's largest finite magnitude to [2^15, 2^16) and
+ * stored as fp16, exact for every element of at least 2^-32 times that
+ * largest one (smaller elements round to fp16's subnormal grid, an error
+ * below 2^-40 of the row's largest element); Y is scaled back exactly.  Two
+ * launches: X is first written into the operand layout, then one CTA per SM
+ * runs the GEMM.
  * `workspace` is device memory of at least
  * seedlm_gemm_smallM_workspace_bytes(fmt, M) bytes, 256-byte aligned.  It
- * holds per-tile counters, X in the operand layout and the partial tiles of
- * row tiles shared by several CTAs: it must be zero-filled before its first
+ * holds per-tile counters, the rows' scale factors, X in the operand layout
+ * and the partial tiles of row tiles shared by several CTAs: it must be
+ * zero-filled before its first
  * use, every call leaves the counters at zero for the next, and calls sharing
  * one workspace must not run concurrently (calls on one stream never do). */
 SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,

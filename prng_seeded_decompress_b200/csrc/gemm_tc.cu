@@ -14,7 +14,7 @@
 //   * X: fp16 activations as they are; bf16 activations scaled per row n by
 //     a power of two 2^s_n that brings the row's largest finite magnitude to
 //     [2^15, 2^16) and stored as fp16.  A bf16 value has 8 significant bits,
-//     so every element within a factor 2^33 of its row's largest is exact;
+//     so every element of at least 2^-32 times its row's largest is exact;
 //     smaller ones round to fp16's subnormal grid, an error below 2^-40 of
 //     the row's largest element.
 //   * Y = acc * 2^-(6 + s_n), applied as two exact power-of-two products.
@@ -38,14 +38,19 @@
 //          (rep_tables.cuh: one conflict-free shared-memory wavefront per
 //          lookup), split them into the two fp16 pieces, pack two K
 //          neighbours per 32-bit word and store them straight into tensor
-//          memory with tcgen05.st, one block at a time -- A operand stages,
-//          128 lanes = rows.  Warp w owns TMEM lanes 32(w%4).. and a quarter
-//          (w/4) of the chunk's blocks.
-//        * one thread issues the MMAs (M = 128, N = NB, A from TMEM, B = X
+//          memory with tcgen05.st (the fp16 conversions of two blocks write
+//          the store's source registers directly) -- A operand stages, 128
+//          lanes = rows.  Warp w owns TMEM lanes 32(w%4).. and a quarter
+//          (w/4) of the chunk's blocks.  The producers set the pace: measured
+//          about 1,350 cycles of rebuild per warp and unit plus 250 waiting
+//          for the slowest warp of the stage, at about 60 % issue use.
+//        * one warp issues the MMAs (M = 128, N = NB, A from TMEM, B = X
 //          slab from shared memory), both pieces into the same fp32
-//          accumulator in TMEM.  An MMA of this shape costs the tensor core
-//          about 45 cycles whatever N (<= 64) and K, so the MMA count, not
-//          M*N*K, sets the tensor-core time.
+//          accumulator in TMEM, a unit's MMAs in one asm statement with one
+//          elect.  An MMA of this shape keeps the tensor core busy ~32
+//          cycles whatever N (<= 64) and K, so the MMA count, not M*N*K, sets
+//          the tensor-core time; issuing a unit's 16 takes ~900 cycles of the
+//          warp that shares its scheduler with four producer warps.
 //        * one thread keeps the X slabs coming, a few chunks ahead, with bulk
 //          copies.
 //        * stages are handed over with mbarriers only (A stage full: all 16
@@ -87,17 +92,25 @@ SEEDLM_CHECK_FLAG(gemm_tc)
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kProdWarps = 16;
-constexpr int kMmaWarp = kProdWarps;         // issues the MMAs (one thread)
-constexpr int kLoaderWarp = kProdWarps + 1;  // copies the X slabs (one thread)
-constexpr int kEpiWarp0 = kProdWarps + 2;    // four warps drain the accumulators
-constexpr int kThreads = (kProdWarps + 6) * 32;
+// Warp roles: producer warps (a multiple of 4: each TMEM lane quarter gets
+// the same number), then the MMA warp, the X loader warp and four epilogue
+// warps.  (24 producer warps on 96-column C = 8 units, 64 registers each,
+// measured 13 % slower than 16 on 128-column units.)
+template <int C>
+struct Roles {
+  static constexpr int kProd = 16;
+  static constexpr int kMma = kProd;         // issues the MMAs (one thread)
+  static constexpr int kLoader = kProd + 1;  // copies the X slabs (one thread)
+  static constexpr int kEpi0 = kProd + 2;    // four warps drain the accumulators
+  static constexpr int kThreads = (kProd + 6) * 32;
+  static_assert(kProd % 4 == 0, "whole lane quarters");
+};
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 64;   // one accumulator (N <= 64); there are two
 constexpr int kShift = 6;      // the pieces are of 2^kShift W
 constexpr int kXS = 5;         // X slabs in shared memory
 constexpr int kHdrBytes = 1024;  // mbarriers, TMEM slot, row scales, at the allocation's start
-constexpr int kRecAhead = 2;   // units of records a producer thread has in flight
+constexpr int kRecAhead = 3;   // units of records a producer thread has in flight (2: 1-2 % slower)
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
 // Per format: K columns per unit and blocks per producer thread and unit.
@@ -155,7 +168,7 @@ struct TcSmem {
   static_assert(SLOT + 16 <= YSCALE && YSCALE + 8 * kAccCols <= SLAB_A, "header");
   static_assert(D_COL + 2 * kAccCols <= kTmemCols, "TMEM budget");
   static_assert(NB <= kAccCols, "one accumulator holds N <= 64 columns");
-  static_assert(KC == 4 * BPT * C, "four producer quarters of BPT blocks per unit");
+  static_assert(KC == Roles<C>::kProd / 4 * BPT * C, "each producer warp of a lane quarter takes BPT blocks");
   static_assert(KC % 16 == 0, "whole K = 16 MMA steps");
   static_assert(SLAB_A % 16 == 0 && XB % 16 == 0, "bulk copies and descriptors need 16-byte alignment");
 };
@@ -305,13 +318,16 @@ struct RecUnit {
 };
 
 template <int C, int NB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<C>::kThreads, 1)
 gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ eplane,
                const unsigned char* __restrict__ Xs, const float2* __restrict__ yscale,
                float* __restrict__ Y, float* __restrict__ partial,
                unsigned int* __restrict__ counters, TcGeom g) {
   using L = TcSmem<C, NB>;
+  using R = Roles<C>;
   constexpr int KC = L::KC, AS = L::AS, BPT = L::BPT;
+  constexpr int kThreads = R::kThreads, kProdWarps = R::kProd, kMmaWarp = R::kMma,
+                kLoaderWarp = R::kLoader, kEpiWarp0 = R::kEpi0;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ctas = gridDim.x;
@@ -417,18 +433,14 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         const uint32_t d = tmem + L::D_COL + kAccCols * db;
         const uint64_t bd = tc::smem_desc(L::slab(xs), 128, L::SBO);
         const uint32_t acc0 = first ? 0u : 1u;
-        if constexpr (C == 8) {
-          // The unit's 16 MMAs in one statement with one elect (measured: the
-          // per-MMA form costs the issuing warp 45 % more cycles).
-          static_assert(KC == 128 && L::PIECE_COLS == 64, "mma_f16_ts_warp_8x2's layout");
+        // The unit's MMAs in one statement with one elect (measured: the
+        // per-MMA form costs the issuing warp 45 % more cycles).
+        if constexpr (KC == 128) {
+          static_assert(L::PIECE_COLS == 64, "mma_f16_ts_warp_8x2's layout");
           tc::mma_f16_ts_warp_8x2(d, a0, bd, idesc, acc0);
         } else {
-#pragma unroll
-          for (int kk = 0; kk < KC / 16; ++kk)
-#pragma unroll
-            for (int pc = 0; pc < 2; ++pc)
-              tc::mma_f16_ts_warp_nomask(d, a0 + pc * L::PIECE_COLS + 8 * kk, bd + 16 * kk, idesc,
-                                         (kk == 0 && pc == 0) ? acc0 : 1u);
+          static_assert(KC == 96 && L::PIECE_COLS == 48, "mma_f16_ts_warp_6x2's layout");
+          tc::mma_f16_ts_warp_6x2(d, a0, bd, idesc, acc0);
         }
         tc::mma_commit_warp(afree(as));  // A stage free
         tc::mma_commit_warp(xfree(xs));  // X slab free
@@ -586,11 +598,12 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       const uint32_t col0 = tmem + ((uint32_t)(32 * lq) << 16) + as * L::STAGE_COLS + kq * NPACK;
       if constexpr (C == 8) {
         // Two blocks at a time: eight packed columns of each piece.
+        constexpr int SB = 2;
 #pragma unroll
-        for (int j2 = 0; j2 < BPT; j2 += 2) {
-          float h[16], l[16];
+        for (int j2 = 0; j2 < BPT; j2 += SB) {
+          float h[8 * SB], l[8 * SB];
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
+          for (int jj = 0; jj < SB; ++jj) {
             const BlockC8 blk = rep::decode_c8_rep<kShift>(cur.r[j2 + jj], lane4, lane8);
             const float2 nm = make_float2(__uint_as_float(blk.negm), __uint_as_float(blk.negm));
             float* hh = h + 8 * jj;
@@ -729,7 +742,7 @@ int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* epl
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Roles<C>::kThreads);
   cfg.dynamicSmemBytes = L::TOTAL;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

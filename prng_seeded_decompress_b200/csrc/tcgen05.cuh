@@ -55,20 +55,6 @@ __device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem
       : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u),
         "r"(0u), "r"(0u));
 }
-// The same MMA without the disable-output-lane mask operand (every lane of
-// D written): fewer operands to move into uniform registers per MMA.
-__device__ __forceinline__ void mma_f16_ts_warp_nomask(uint32_t d_tmem, uint32_t a_tmem,
-                                                       uint64_t b_desc, uint32_t idesc,
-                                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
-      :
-      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
 // Eight K = 16 steps of two pieces (16 MMAs) in one statement: piece pc of
 // step k reads A at a0 + pc * pcols + 8 k and B at b_desc + 16 k (the
 // descriptor's address field counts 16-byte units).  One elect for all.
@@ -101,6 +87,48 @@ __device__ __forceinline__ void mma_f16_ts_warp_8x2(uint32_t d_tmem, uint32_t a0
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a13], b6, %3, t;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a14], b7, %3, t;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a15], b7, %3, t;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a0), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Six K = 16 steps of two pieces (12 MMAs) in one statement: piece pc of
+// step k reads A at a0 + pc * 48 + 8 k and B at b_desc + 16 k.  One elect
+// for all.
+__device__ __forceinline__ void mma_f16_ts_warp_6x2(uint32_t d_tmem, uint32_t a0, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b32 a<12>;\n\t.reg .b64 b<6>;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.u32 a1, %1, 48;\n\t"
+      "add.u32 a2, %1, 8;\n\t"
+      "add.u32 a3, %1, 56;\n\t"
+      "add.u32 a4, %1, 16;\n\t"
+      "add.u32 a5, %1, 64;\n\t"
+      "add.u32 a6, %1, 24;\n\t"
+      "add.u32 a7, %1, 72;\n\t"
+      "add.u32 a8, %1, 32;\n\t"
+      "add.u32 a9, %1, 80;\n\t"
+      "add.u32 a10, %1, 40;\n\t"
+      "add.u32 a11, %1, 88;\n\t"
+      "add.u64 b1, %2, 16;\n\t"
+      "add.u64 b2, %2, 32;\n\t"
+      "add.u64 b3, %2, 48;\n\t"
+      "add.u64 b4, %2, 64;\n\t"
+      "add.u64 b5, %2, 80;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], %2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a8], b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a9], b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a10], b5, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a11], b5, %3, t;\n\t}\n"
       :
       : "r"(d_tmem), "r"(a0), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
