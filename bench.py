@@ -427,8 +427,9 @@ def extras(torch, sl, args):
                                   ep=None if base["ep"] is None else base["ep"].clone())
                              for _ in range(ncp - 1)]
             f = sl.Format.from_dict(base["fmt"])
-            # bf16 activations (three bf16 pieces of W) at every M, fp16 (two
-            # fp16 pieces) at M = 16 and 64.
+            # bf16 activations (staged as fp16 with a power-of-two scale per
+            # row) at every M, fp16 at M = 16 and 64; both meet two fp16
+            # pieces of W.
             for M, dt in ((1, "bf16"), (8, "bf16"), (16, "bf16"), (64, "bf16"), (16, "f16"),
                           (64, "f16")):
                 Xb, _ = inputs.make_activations((M, N), dt, 950 + M)
@@ -451,6 +452,24 @@ def extras(torch, sl, args):
             fn(0)
             gemm[f"{tag}/{name}/gemv_bf16"] = {"us_per_call": round(time_median(torch, fn, 4 * ncp)
                                                                     * 1e3, 2)}
+            # Larger batches (prefill) through seedlm_gemm: passes of at most
+            # 256 rows of X, 4-bit gate/up shape only.
+            if tag == "4bit" and name.startswith("up"):
+                for M in (128, 256, 1024):
+                    Xb, _ = inputs.make_activations((M, N), "bf16", 960 + M)
+                    X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+                    Y = torch.empty((M, R), device="cuda")
+                    ws = torch.zeros(max(sl.gemm_any_workspace_bytes(f, M), 256),
+                                     dtype=torch.uint8, device="cuda")
+                    fn = lambda i: sl.gemm(f, mats[i % ncp]["rec"], mats[i % ncp]["ep"], X, Y,  # noqa
+                                           workspace=ws)
+                    fn(0)
+                    us = time_median(torch, fn, 2 * ncp) * 1e3
+                    gemm[f"{tag}/{name}/M={M}"] = {
+                        "us_per_call": round(us, 2), "weights_per_s_e9": round(R * N / us / 1e3, 2),
+                        "tflops_useful": round(2 * M * R * N / us / 1e6, 2), "copies": ncp,
+                        "entry": "seedlm_gemm"}
+                    del ws
             del mats, base
     out["gemm_smallM"] = gemm
 
@@ -463,7 +482,7 @@ def extras(torch, sl, args):
         Wd = torch.randn((R, N), device="cuda", dtype=torch.float16) * 0.02
         ncp = max(2, math.ceil(4 * l2 / (Wd.numel() * 2)))
         Ws = [Wd] + [Wd.clone() for _ in range(ncp - 1)]
-        for M in (1, 8, 16, 64):
+        for M in ((1, 8, 16, 64, 128, 256, 1024) if name.startswith("up") else (1, 8, 16, 64)):
             X = torch.randn((M, N), device="cuda", dtype=torch.float16)
             if M == 1:
                 y = torch.empty(R, device="cuda")
@@ -598,7 +617,7 @@ def summarize(result, hbm_peak):
             out["llama3_8b_speedup_vs_dense_fp16"] = round(d8 / us8, 3)
     g = ex.get("gemm_smallM", {})
     dm = ex.get("dense_fp16_smallM", {})
-    for M in (8, 16, 64):
+    for M in (8, 16, 64, 128, 256, 1024):
         k = f"4bit/up_28672x8192/M={M}"
         if k in g:
             out[f"gemm_4bit_28672x8192_M{M}_us"] = g[k]["us_per_call"]

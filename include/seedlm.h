@@ -166,6 +166,28 @@ SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec,
  * GEMV, negative on error). */
 SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M);
 
+/* Y = X W^T for any batch M >= 1 -- the same product as seedlm_gemm_smallM
+ * (paperhub.cn review thread, authors' reply on how inference uses s and t),
+ * extended to prefill-sized batches, where the rebuild of each weight tile is
+ * shared by many rows of X.  X is M x cols (row-major, type x_dtype), Y is
+ * M x rows fp32 (row-major).  M = 1 runs the GEMV; otherwise the rows of X
+ * go through the tensor-core kernel of seedlm_gemm_smallM (same operand
+ * precision) in passes of at most 256 rows, one after the other on the
+ * stream: up to 64 rows per MMA as there, 65-128 rows as one N = 128 pass,
+ * 129-256 as one N = 256 pass (units of 64 columns at 4 bits, 48 at 3 bits,
+ * one accumulator in TMEM).  For M <= 64 the result is the one
+ * seedlm_gemm_smallM gives.  `workspace`: device memory of at least
+ * seedlm_gemm_workspace_bytes(fmt, M) bytes, 256-byte aligned, zero-filled
+ * before its first use, with the sharing rules of seedlm_gemm_smallM. */
+SEEDLM_API int seedlm_gemm(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane,
+                           const void* X, int x_dtype, int M, float* Y, void* workspace,
+                           int64_t workspace_bytes, seedlm_stream stream);
+
+/* Workspace bytes seedlm_gemm needs for this format and M on the current
+ * device (HOST function; 0 for an empty matrix or when M = 1 runs the GEMV,
+ * negative on error). */
+SEEDLM_API int64_t seedlm_gemm_workspace_bytes(const seedlm_format* fmt, int M);
+
 /* Same result as seedlm_gemm_smallM, for callers that cannot allocate device
  * memory -- e.g. code embedded in a host program that owns all of the GPU's
  * memory through its own pool, or a path where cudaMalloc's implicit device

@@ -98,6 +98,23 @@ int allow_max_smem(const void* kernel, const DeviceInfo& dev) {
 
 using namespace seedlm;
 
+namespace {
+
+// Workspace of seedlm_gemm: the larger of a full pass and the last pass.
+int64_t gemm_any_workspace(const seedlm_format& f, int M, const DeviceInfo& dev) {
+  if (M == 1 && gemv_smem_bytes(f, dev) > 0) return 0;  // the GEMV
+  const int full = M < kGemmPassRows ? M : kGemmPassRows;
+  int64_t need = gemm_tc_workspace_bytes(f, full, dev);
+  const int last = M % kGemmPassRows;
+  if (M > kGemmPassRows && last) {
+    const int64_t l = gemm_tc_workspace_bytes(f, last, dev);
+    if (l > need) need = l;
+  }
+  return need;
+}
+
+}  // namespace
+
 extern "C" {
 
 int seedlm_init(void) {
@@ -209,6 +226,47 @@ int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M) {
   if (rc) return rc;
   if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0) return 0;  // the GEMV
   return gemm_tc_workspace_bytes(*fmt, M, dev);
+}
+
+int seedlm_gemm(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* eplane, const void* X,
+                int x_dtype, int M, float* Y, void* workspace, int64_t workspace_bytes,
+                seedlm_stream stream) {
+  int rc = check_format(fmt);
+  if (rc) return rc;
+  if ((rc = check_planes(fmt, rec, eplane))) return rc;
+  if (x_dtype != SEEDLM_F16 && x_dtype != SEEDLM_BF16) return SEEDLM_EINVAL;
+  if (M < 1 || workspace_bytes < 0) return SEEDLM_EINVAL;
+  if (fmt->rows == 0) return SEEDLM_OK;
+  if (!Y || !aligned(Y, 4)) return SEEDLM_EINVAL;
+  if (fmt->cols > 0 && (!X || !aligned(X, 2))) return SEEDLM_EINVAL;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const cudaStream_t st = (cudaStream_t)stream;
+  if (fmt->cols == 0)
+    return record_cuda_error(cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), st));
+  const uint16_t* Xh = static_cast<const uint16_t*>(X);
+  const int is_bf16 = x_dtype == SEEDLM_BF16;
+  if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0)
+    return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
+  if (workspace_bytes < gemm_any_workspace(*fmt, M, dev)) return SEEDLM_EINVAL;
+  // Passes of up to kGemmPassRows rows of X, one after the other on the
+  // stream, sharing the workspace (each pass leaves its counters at zero).
+  for (int m0 = 0; m0 < M; m0 += kGemmPassRows) {
+    const int mc = M - m0 < kGemmPassRows ? M - m0 : kGemmPassRows;
+    rc = launch_gemm_tc(*fmt, rec, eplane, Xh + (size_t)m0 * fmt->cols, is_bf16, mc,
+                        Y + (size_t)m0 * fmt->rows, workspace, workspace_bytes, st, dev);
+    if (rc) return rc;
+  }
+  return SEEDLM_OK;
+}
+
+int64_t seedlm_gemm_workspace_bytes(const seedlm_format* fmt, int M) {
+  if (check_format(fmt) || M < 1) return SEEDLM_EINVAL;
+  if (fmt->rows == 0 || fmt->cols == 0) return 0;
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  return gemm_any_workspace(*fmt, M, dev);
 }
 
 int seedlm_encode(const seedlm_format* fmt, const float* W, int64_t ldw, uint32_t* rec,

@@ -106,25 +106,22 @@ struct Roles {
   static_assert(kProd % 4 == 0, "whole lane quarters");
 };
 constexpr int kTmemCols = 512;
-constexpr int kAccCols = 64;   // one accumulator (N <= 64); there are two
-constexpr int kShift = 6;      // the pieces are of 2^kShift W
-constexpr int kXS = 5;         // X slabs in shared memory
-constexpr int kHdrBytes = 1024;  // mbarriers, TMEM slot, row scales, at the allocation's start
+constexpr int kMaxNB = 256;      // batch rows of one pass (the MMA's largest N)
+constexpr int kShift = 6;        // the pieces are of 2^kShift W
+constexpr int kMaxXS = 5;        // X slabs in shared memory, at most
+constexpr int kHdrBytes = 2304;  // mbarriers, TMEM slot, row scales, at the allocation's start
+constexpr uint32_t kSmemLimit = rep::kSmemBase + 232448;  // end of the largest allocation (B200)
 constexpr int kRecAhead = 3;   // units of records a producer thread has in flight (2: 1-2 % slower)
 constexpr uint64_t kWaitLimit = 2000000000ull;  // ns an mbarrier wait may take before giving up
 
-// Per format: K columns per unit and blocks per producer thread and unit.
-template <int C>
-struct TcCfg;
-template <>
-struct TcCfg<8> {
-  static constexpr int KC = 128;  // 16 blocks
-  static constexpr int BPT = 4;
-};
-template <>
-struct TcCfg<12> {
-  static constexpr int KC = 96;  // 8 blocks
-  static constexpr int BPT = 2;
+// Batch rows NB (a pass's M rounded up: 16, 32, 48, 64, 128 or 256) ->
+// K columns per unit and blocks per producer thread and unit.  Up to 128
+// rows: units of 128 (C = 8) or 96 (C = 12) columns.  Above: half-width
+// units, so that two X slabs of 32 KB still fit beside the decode tables.
+template <int C, int NB>
+struct TcCfg {
+  static constexpr int BPT = (NB > 128) ? (C == 8 ? 2 : 1) : (C == 8 ? 4 : 2);
+  static constexpr int KC = 4 * BPT * C;  // 128, 64 (C = 8); 96, 48 (C = 12)
 };
 
 struct TcGeom {
@@ -141,33 +138,41 @@ struct TcGeom {
 //   [tables, rep::kEnd)               lane-replicated decode tables
 //   [rep::kEnd, ...)                  the remaining X slabs
 // TMEM: AS A stages of two pieces (KC/2 columns each: two fp16 per 32-bit
-// column), then two accumulators of kAccCols fp32 columns.
+// column), then NACC accumulators of ACC fp32 columns (two, so that one
+// segment's epilogue overlaps the next segment, when they fit).
 template <int C, int NB>
 struct TcSmem {
-  static constexpr int KC = TcCfg<C>::KC;
-  static constexpr int BPT = TcCfg<C>::BPT;
+  static constexpr int KC = TcCfg<C, NB>::KC;
+  static constexpr int BPT = TcCfg<C, NB>::BPT;
   static constexpr int SBO = KC * 16;      // bytes between 8-row groups of X (KC/8 core matrices)
   static constexpr int XB = NB * KC * 2;   // one X slab (fp16)
   static constexpr int PIECE_COLS = KC / 2;
   static constexpr int STAGE_COLS = 2 * PIECE_COLS;
-  static constexpr int AS = (kTmemCols - 2 * kAccCols) / STAGE_COLS;  // C = 8: 3, C = 12: 4
+  static constexpr int ACC = NB < 64 ? 64 : NB;
+  static constexpr int NACC = (2 * ACC + 2 * STAGE_COLS <= kTmemCols) ? 2 : 1;
+  static constexpr int AS = (kTmemCols - NACC * ACC) / STAGE_COLS;
   static constexpr int D_COL = AS * STAGE_COLS;  // first accumulator column
-  // mbarriers: xfull[kXS] xfree[kXS] afull[AS] afree[AS] dfree[2] dfull[2]
-  static constexpr int NBAR = 2 * kXS + 2 * AS + 4;
+  static constexpr uint32_t SLAB_A = rep::kSmemBase + kHdrBytes;
+  static constexpr uint32_t TAB = rep::tables_begin<C>();
+  static constexpr int A_CAP = (int)((TAB - SLAB_A) / XB);          // slabs below the tables
+  static constexpr int B_CAP = (int)((kSmemLimit - rep::kEnd) / XB);  // slabs above them
+  static constexpr int XS = A_CAP + B_CAP < kMaxXS ? A_CAP + B_CAP : kMaxXS;
+  static constexpr int SLABS_A = A_CAP < XS ? A_CAP : XS;
+  // mbarriers: xfull[XS] xfree[XS] afull[AS] afree[AS] dfree[NACC] dfull[NACC]
+  static constexpr int NBAR = 2 * XS + 2 * AS + 2 * NACC;
   static constexpr uint32_t BAR = rep::kSmemBase;
   static constexpr uint32_t SLOT = BAR + 8 * NBAR;  // TMEM base, last-CTA flag, give-up flag
   static constexpr uint32_t YSCALE = rep::kSmemBase + 256;  // NB float2: the rows' output scales
-  static constexpr uint32_t SLAB_A = rep::kSmemBase + kHdrBytes;
-  static constexpr uint32_t TAB = rep::tables_begin<C>();
-  static constexpr int SLABS_A = (int)((TAB - SLAB_A) / XB) < kXS ? (int)((TAB - SLAB_A) / XB) : kXS;
-  static constexpr uint32_t END = rep::kEnd + (uint32_t)(kXS - SLABS_A) * XB;
+  static constexpr uint32_t END = XS > SLABS_A ? rep::kEnd + (uint32_t)(XS - SLABS_A) * XB : rep::kEnd;
   static constexpr int TOTAL = (int)(END - rep::kSmemBase);
   __host__ __device__ static constexpr uint32_t slab(int s) {
     return s < SLABS_A ? SLAB_A + (uint32_t)s * XB : rep::kEnd + (uint32_t)(s - SLABS_A) * XB;
   }
-  static_assert(SLOT + 16 <= YSCALE && YSCALE + 8 * kAccCols <= SLAB_A, "header");
-  static_assert(D_COL + 2 * kAccCols <= kTmemCols, "TMEM budget");
-  static_assert(NB <= kAccCols, "one accumulator holds N <= 64 columns");
+  static_assert(XS >= 2, "X slabs are double-buffered at least");
+  static_assert(AS >= 2, "A stages are double-buffered at least");
+  static_assert(SLOT + 16 <= YSCALE && YSCALE + 8 * kMaxNB <= SLAB_A, "header");
+  static_assert(D_COL + NACC * ACC <= kTmemCols, "TMEM budget");
+  static_assert(NB <= kMaxNB && NB <= ACC, "one accumulator holds the pass");
   static_assert(KC == Roles<C>::kProd / 4 * BPT * C, "each producer warp of a lane quarter takes BPT blocks");
   static_assert(KC % 16 == 0, "whole K = 16 MMA steps");
   static_assert(SLAB_A % 16 == 0 && XB % 16 == 0, "bulk copies and descriptors need 16-byte alignment");
@@ -325,7 +330,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
                unsigned int* __restrict__ counters, TcGeom g) {
   using L = TcSmem<C, NB>;
   using R = Roles<C>;
-  constexpr int KC = L::KC, AS = L::AS, BPT = L::BPT;
+  constexpr int KC = L::KC, AS = L::AS, BPT = L::BPT, XS = L::XS, NACC = L::NACC, ACC = L::ACC;
   constexpr int kThreads = R::kThreads, kProdWarps = R::kProd, kMmaWarp = R::kMma,
                 kLoaderWarp = R::kLoader, kEpiWarp0 = R::kEpi0;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -351,14 +356,14 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   // completed: its A stage may be reused.  dfull: a segment's MMAs completed,
   // its accumulator is final.  dfree: the epilogue warps have read it out.
   auto xfull = [&](int s) { return bar + 8 * s; };
-  auto xfree = [&](int s) { return bar + 8 * (kXS + s); };
-  auto afull = [&](int s) { return bar + 8 * (2 * kXS + s); };
-  auto afree = [&](int s) { return bar + 8 * (2 * kXS + AS + s); };
-  auto dfree = [&](int b) { return bar + 8 * (2 * kXS + 2 * AS + b); };
-  auto dfull = [&](int b) { return bar + 8 * (2 * kXS + 2 * AS + 2 + b); };
+  auto xfree = [&](int s) { return bar + 8 * (XS + s); };
+  auto afull = [&](int s) { return bar + 8 * (2 * XS + s); };
+  auto afree = [&](int s) { return bar + 8 * (2 * XS + AS + s); };
+  auto dfree = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + b); };
+  auto dfull = [&](int b) { return bar + 8 * (2 * XS + 2 * AS + NACC + b); };
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + (L::SLOT - rep::kSmemBase));
   if (tid == 0) {
-    for (int s = 0; s < kXS; ++s) {
+    for (int s = 0; s < XS; ++s) {
       tc::mbar_init(xfull(s), 1);
       tc::mbar_init(xfree(s), 1);
     }
@@ -366,7 +371,7 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       tc::mbar_init(afull(s), kProdWarps);
       tc::mbar_init(afree(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       tc::mbar_init(dfree(b), 4);
       tc::mbar_init(dfull(b), 1);
     }
@@ -388,9 +393,9 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       // Xs is written by the previous kernel on the stream.
       asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j = 0; j < n_units; ++j, xc.next(g.nchunks)) {
-        const int s = j % kXS;
-        if (j >= kXS)  // the slab's previous unit (j - kXS) has finished its MMAs
-          ok = tc::mbar_wait_or_abort(xfree(s), ((j / kXS) - 1) & 1, kWaitLimit, abort_flag) && ok;
+        const int s = j % XS;
+        if (j >= XS)  // the slab's previous unit (j - XS) has finished its MMAs
+          ok = tc::mbar_wait_or_abort(xfree(s), ((j / XS) - 1) & 1, kWaitLimit, abort_flag) && ok;
         if (SEEDLM_IN_BOUNDS(g_check_flag, xc.chunk, g.nchunks)) {
           tc::mbar_arrive_expect_tx(xfull(s), L::XB);
           tc::bulk_g2s(L::slab(s), Xs + (size_t)xc.chunk * L::XB, L::XB, xfull(s));
@@ -400,8 +405,8 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       }
       // Every copy this thread issued has landed before the CTA may exit
       // (bounded, and not cut short by the give-up flag).
-      for (int s = 0; s < kXS && s < n_units; ++s) {
-        const int k = (n_units - 1 - s) / kXS;  // last load into slab s
+      for (int s = 0; s < XS && s < n_units; ++s) {
+        const int k = (n_units - 1 - s) / XS;  // last load into slab s
         ok = tc::mbar_wait(xfull(s), k & 1, kWaitLimit) && ok;
       }
     }
@@ -417,12 +422,12 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       for (int i = 0; i < n_units; ++i, mc.next(g.nchunks)) {
         const bool first = i == 0 || mc.chunk == 0;
         if (first && i > 0) ++seg;
-        const int db = seg & 1;
-        if (first && seg >= 2)  // accumulator db was last used by segment seg - 2
-          ok = tc::mbar_wait_or_abort(dfree(db), ((seg >> 1) - 1) & 1, kWaitLimit, abort_flag) && ok;
-        const int xs = i % kXS, as = i % AS;
-        if (!tc::mbar_try_wait2(xfull(xs), (i / kXS) & 1, afull(as), (i / AS) & 1)) {
-          ok = tc::mbar_wait_or_abort(xfull(xs), (i / kXS) & 1, kWaitLimit, abort_flag) && ok;
+        const int db = seg % NACC;
+        if (first && seg >= NACC)  // accumulator db was last used by segment seg - NACC
+          ok = tc::mbar_wait_or_abort(dfree(db), ((seg / NACC) - 1) & 1, kWaitLimit, abort_flag) && ok;
+        const int xs = i % XS, as = i % AS;
+        if (!tc::mbar_try_wait2(xfull(xs), (i / XS) & 1, afull(as), (i / AS) & 1)) {
+          ok = tc::mbar_wait_or_abort(xfull(xs), (i / XS) & 1, kWaitLimit, abort_flag) && ok;
           ok = tc::mbar_wait_or_abort(afull(as), (i / AS) & 1, kWaitLimit, abort_flag) && ok;
         }
         __syncwarp();  // reconverge before the elected issue
@@ -430,18 +435,21 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
         // The issue rate bounds the tensor core here, so everything but the
         // MMAs is computed up front.
         const uint32_t a0 = tmem + as * L::STAGE_COLS;
-        const uint32_t d = tmem + L::D_COL + kAccCols * db;
+        const uint32_t d = tmem + L::D_COL + ACC * db;
         const uint64_t bd = tc::smem_desc(L::slab(xs), 128, L::SBO);
         const uint32_t acc0 = first ? 0u : 1u;
         // The unit's MMAs in one statement with one elect (measured: the
         // per-MMA form costs the issuing warp 45 % more cycles).
-        if constexpr (KC == 128) {
-          static_assert(L::PIECE_COLS == 64, "mma_f16_ts_warp_8x2's layout");
+        static_assert(L::PIECE_COLS == KC / 2, "the helpers' piece stride");
+        if constexpr (KC == 128)
           tc::mma_f16_ts_warp_8x2(d, a0, bd, idesc, acc0);
-        } else {
-          static_assert(KC == 96 && L::PIECE_COLS == 48, "mma_f16_ts_warp_6x2's layout");
+        else if constexpr (KC == 96)
           tc::mma_f16_ts_warp_6x2(d, a0, bd, idesc, acc0);
-        }
+        else if constexpr (KC == 64)
+          tc::mma_f16_ts_warp_4x2(d, a0, bd, idesc, acc0);
+        else
+          tc::mma_f16_ts_warp_3x2(d, a0, bd, idesc, acc0);
+        static_assert(KC == 128 || KC == 96 || KC == 64 || KC == 48, "a unit's MMA count");
         tc::mma_commit_warp(afree(as));  // A stage free
         tc::mma_commit_warp(xfree(xs));  // X slab free
         if (i == n_units - 1 || mc.chunk == g.nchunks - 1)
@@ -468,12 +476,11 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     // into shared memory once.
     float2* ys = reinterpret_cast<float2*>(smem + (L::YSCALE - rep::kSmemBase));
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int et = tid - kEpiWarp0 * 32;  // 0..127
-    if (et < NB) ys[et] = __ldcg(yscale + et);
+    for (int i = tid - kEpiWarp0 * 32; i < NB; i += 128) ys[i] = __ldcg(yscale + i);
     tc::named_sync(128);
     auto epilogue = [&](int seg, int tile) {
-      const int db = seg & 1;
-      ok = tc::mbar_wait_or_abort(dfull(db), (seg >> 1) & 1, kWaitLimit, abort_flag) && ok;
+      const int db = seg % NACC;
+      ok = tc::mbar_wait_or_abort(dfull(db), (seg / NACC) & 1, kWaitLimit, abort_flag) && ok;
       tc::fence_after_sync();
       const int gr = tile * kTileM + row;
       const int first = unit_owner((long long)tile * g.nchunks, g.units, ctas);
@@ -484,10 +491,10 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       SEEDLM_CHECK_ONLY(const size_t y_n = (size_t)g.M * g.rows;
                         const size_t part_n = (size_t)ctas * g.segs_max * (NB * kTileM);
                         const size_t mine_off = ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);)
-#pragma unroll
+#pragma unroll(NB > 64 ? 2 : 4)
       for (int n16 = 0; n16 < NB / 16; ++n16) {
         float v[16];
-        tc::tmem_ld16(tmem + ((uint32_t)(32 * eq) << 16) + L::D_COL + kAccCols * db + 16 * n16, v);
+        tc::tmem_ld16(tmem + ((uint32_t)(32 * eq) << 16) + L::D_COL + ACC * db + 16 * n16, v);
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const float2 f = ys[16 * n16 + q];
@@ -578,14 +585,28 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
                        SEEDLM_IN_BOUNDS(g_check_flag, b0 + BPT - 1, g.rec_pitch) &&
                        (C == 8 || SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, g.e_pitch));
       const uint32_t* src = rec + (size_t)gr * g.rec_pitch + b0;
-      if constexpr (C == 8) {
+      // b0 is a multiple of BPT, so each load is aligned to its width.
+      if constexpr (C == 8 && BPT == 4) {
         const uint4 v = ok_ ? ld_stream_u4(src) : make_uint4(0u, 0u, 0u, 0u);
         p.r[0] = v.x; p.r[1] = v.y; p.r[2] = v.z; p.r[3] = v.w;
         p.e = 0;
-      } else {
+      } else if constexpr (C == 8) {
+        static_assert(BPT == 2, "C = 8 takes two or four blocks per thread");
+        const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
+        p.r[0] = v.x; p.r[1] = v.y;
+        p.e = 0;
+      } else if constexpr (BPT == 2) {
+        // b0 is even: one 8-byte load; the exponent byte holds block b0 in
+        // its low nibble and b0 + 1 in its high nibble.
         const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
         p.r[0] = v.x; p.r[1] = v.y;
         p.e = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
+      } else {
+        // One block: a 4-byte load, the exponent from the nibble of b0's parity.
+        static_assert(BPT == 1, "C = 12 takes one or two blocks per thread");
+        p.r[0] = ok_ ? ld_stream_u1(src) : 0u;
+        const uint32_t eb = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
+        p.e = eb >> (4 * (b0 & 1));
       }
     };
 
@@ -628,10 +649,19 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
           fp16_pieces(weight_bits_c12<8>(blk), weight_bits_c12<9>(blk), nm, neg1, ph[6 * j + 4], pl[6 * j + 4]);
           fp16_pieces(weight_bits_c12<10>(blk), weight_bits_c12<11>(blk), nm, neg1, ph[6 * j + 5], pl[6 * j + 5]);
         }
+        if constexpr (NPACK % 4 == 0) {  // two blocks: 12 columns from a multiple of 4
 #pragma unroll
-        for (int q = 0; q < NPACK / 4; ++q) {
-          tc::tmem_st4(col0 + 4 * q, ph + 4 * q);
-          tc::tmem_st4(col0 + L::PIECE_COLS + 4 * q, pl + 4 * q);
+          for (int q = 0; q < NPACK / 4; ++q) {
+            tc::tmem_st4(col0 + 4 * q, ph + 4 * q);
+            tc::tmem_st4(col0 + L::PIECE_COLS + 4 * q, pl + 4 * q);
+          }
+        } else {  // one block: 6 columns from an even column
+          static_assert(NPACK == 6, "one 12-weight block");
+#pragma unroll
+          for (int q = 0; q < NPACK / 2; ++q) {
+            tc::tmem_st2(col0 + 2 * q, ph + 2 * q);
+            tc::tmem_st2(col0 + L::PIECE_COLS + 2 * q, pl + 2 * q);
+          }
         }
       }
       tc::tmem_wait_st();
@@ -673,7 +703,13 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   }
 }
 
-int kc_of(int C) { return C == 8 ? TcCfg<8>::KC : TcCfg<12>::KC; }
+// Batch rows of a pass of M rows: M rounded up to 16 up to 64, then 128 or 256.
+int nb_of(int M) { return M <= 64 ? (M + 15) / 16 * 16 : (M <= 128 ? 128 : 256); }
+
+int kc_of(int C, int NB) {
+  if (C == 8) return NB > 128 ? TcCfg<8, 256>::KC : TcCfg<8, 64>::KC;
+  return NB > 128 ? TcCfg<12, 256>::KC : TcCfg<12, 64>::KC;
+}
 
 TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev, int* ctas) {
   TcGeom g;
@@ -683,7 +719,7 @@ TcGeom make_tc_geom(const seedlm_format& f, int M, const DeviceInfo& dev, int* c
   g.rec_pitch = f.rec_pitch;
   g.e_pitch = f.e_pitch;
   g.M = M;
-  const int KC = kc_of(f.C);
+  const int KC = kc_of(f.C, nb_of(M));
   g.nchunks = (f.cols + KC - 1) / KC;
   g.tiles = (f.rows + kTileM - 1) / kTileM;
   g.units = (long long)g.tiles * g.nchunks;
@@ -709,11 +745,11 @@ struct TcWorkspace {
 int64_t round256(int64_t v) { return (v + 255) / 256 * 256; }
 
 TcWorkspace tc_workspace(const TcGeom& g, int C, int ctas) {
-  const int NB = (g.M + 15) / 16 * 16;
+  const int NB = nb_of(g.M);
   TcWorkspace w;
   w.cnt_bytes = round256((int64_t)g.tiles * 4);
   w.scale_bytes = round256((int64_t)NB * 8);
-  w.xs_bytes = round256((int64_t)g.nchunks * NB * kc_of(C) * 2);
+  w.xs_bytes = round256((int64_t)g.nchunks * NB * kc_of(C, NB) * 2);
   w.part_bytes = round256((int64_t)ctas * g.segs_max * NB * kTileM * 4);
   return w;
 }
@@ -762,11 +798,13 @@ template <int C>
 int dispatch_nb(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* eplane,
                 const uint16_t* X, int is_bf16, float* Y, unsigned char* ws, const TcWorkspace& w,
                 cudaStream_t st, const DeviceInfo& dev) {
-  switch ((g.M + 15) / 16 * 16) {
+  switch (nb_of(g.M)) {
     case 16: return launch_tc<C, 16>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
     case 32: return launch_tc<C, 32>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
     case 48: return launch_tc<C, 48>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
-    default: return launch_tc<C, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    case 64: return launch_tc<C, 64>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    case 128: return launch_tc<C, 128>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
+    default: return launch_tc<C, 256>(g, ctas, rec, eplane, X, is_bf16, Y, ws, w, st, dev);
   }
 }
 

@@ -98,6 +98,9 @@ int launch_decompress(const seedlm_format& f, const uint32_t* rec, const uint8_t
                       float* W, int64_t ldw, cudaStream_t stream, const DeviceInfo& dev);
 int launch_dense_gemv_f16(int rows, int cols, const uint16_t* W, int64_t ldw, const uint16_t* x,
                           float* y, cudaStream_t stream, const DeviceInfo& dev);
+// Largest batch of one tensor-core GEMM pass (the MMA's largest N); more
+// rows are run as consecutive passes.
+constexpr int kGemmPassRows = 256;
 int64_t gemm_tc_workspace_bytes(const seedlm_format& f, int M, const DeviceInfo& dev);
 int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                    const uint16_t* X, int is_bf16, int M, float* Y, void* workspace,

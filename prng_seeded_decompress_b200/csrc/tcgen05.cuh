@@ -133,6 +133,65 @@ __device__ __forceinline__ void mma_f16_ts_warp_6x2(uint32_t d_tmem, uint32_t a0
       : "r"(d_tmem), "r"(a0), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
+// Four K = 16 steps of two pieces (8 MMAs) in one statement: piece pc of
+// step k reads A at a0 + pc * 32 + 8 k and B at b_desc + 16 k.  One elect
+// for all.
+__device__ __forceinline__ void mma_f16_ts_warp_4x2(uint32_t d_tmem, uint32_t a0, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b32 a<8>;\n\t.reg .b64 b<4>;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.u32 a1, %1, 32;\n\t"
+      "add.u32 a2, %1, 8;\n\t"
+      "add.u32 a3, %1, 40;\n\t"
+      "add.u32 a4, %1, 16;\n\t"
+      "add.u32 a5, %1, 48;\n\t"
+      "add.u32 a6, %1, 24;\n\t"
+      "add.u32 a7, %1, 56;\n\t"
+      "add.u64 b1, %2, 16;\n\t"
+      "add.u64 b2, %2, 32;\n\t"
+      "add.u64 b3, %2, 48;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], %2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b3, %3, t;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a0), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Three K = 16 steps of two pieces (6 MMAs) in one statement: piece pc of
+// step k reads A at a0 + pc * 24 + 8 k and B at b_desc + 16 k.  One elect
+// for all.
+__device__ __forceinline__ void mma_f16_ts_warp_3x2(uint32_t d_tmem, uint32_t a0, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b32 a<6>;\n\t.reg .b64 b<3>;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.u32 a1, %1, 24;\n\t"
+      "add.u32 a2, %1, 8;\n\t"
+      "add.u32 a3, %1, 32;\n\t"
+      "add.u32 a4, %1, 16;\n\t"
+      "add.u32 a5, %1, 40;\n\t"
+      "add.u64 b1, %2, 16;\n\t"
+      "add.u64 b2, %2, 32;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], %2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b2, %3, t;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a0), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
 __device__ __forceinline__ void mma_commit_warp(uint32_t mbar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -213,6 +272,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
         "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};"
+               :
+               : "r"(taddr), "r"(r[0]), "r"(r[1])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};"

@@ -21,7 +21,8 @@ BF16 = 1
 #: Every symbol include/seedlm.h declares.
 EXPORTS = (
     "seedlm_init", "seedlm_decompress", "seedlm_gemv", "seedlm_gemm_smallM",
-    "seedlm_gemm_smallM_workspace_bytes", "seedlm_gemm_smallM_noalloc", "seedlm_device_error",
+    "seedlm_gemm_smallM_workspace_bytes", "seedlm_gemm_smallM_noalloc", "seedlm_gemm",
+    "seedlm_gemm_workspace_bytes", "seedlm_device_error",
     "seedlm_dense_gemv_f16", "seedlm_row_bytes_ideal", "seedlm_row_bytes_stored",
     "seedlm_strerror", "seedlm_last_cuda_error", "seedlm_launch_count", "seedlm_shutdown",
     "seedlm_encode", "seedlm_selftest_wait_timeout", "seedlm_checked_build",
@@ -61,6 +62,8 @@ def _load():
         "seedlm_gemm_smallM": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp,
                                               vp, i64, vp]),
         "seedlm_gemm_smallM_workspace_bytes": (i64, [fmtp, ctypes.c_int]),
+        "seedlm_gemm": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i64, vp]),
+        "seedlm_gemm_workspace_bytes": (i64, [fmtp, ctypes.c_int]),
         "seedlm_gemm_smallM_noalloc": (ctypes.c_int, [fmtp, vp, vp, vp, ctypes.c_int,
                                                       ctypes.c_int, vp, vp]),
         "seedlm_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
@@ -253,6 +256,31 @@ def gemm_smallM(fmt, rec, eplane, X, Y, workspace=None, stream=None):
         workspace = gemm_workspace(f, M, device=Y.device)
     nbytes = workspace.numel() * workspace.element_size()
     _check("seedlm_gemm_smallM", lib.seedlm_gemm_smallM(
+        ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), M, _ptr(Y),
+        _ptr(workspace), nbytes, _stream(stream, Y)))
+
+
+def gemm_any_workspace_bytes(fmt, M: int) -> int:
+    n = int(lib.seedlm_gemm_workspace_bytes(ctypes.byref(_fmt(fmt)), int(M)))
+    if n < 0:
+        _check("seedlm_gemm_workspace_bytes", n)
+    return n
+
+
+def gemm(fmt, rec, eplane, X, Y, workspace=None, stream=None):
+    """Y = X W^T for any number of rows M of X (seedlm_gemm: passes of at most
+    256 rows on the tensor cores; M = 1 runs the GEMV).  `workspace`: a
+    zero-filled uint8 tensor of at least gemm_any_workspace_bytes(fmt, M)
+    bytes; if omitted a fresh one is made."""
+    import torch
+    f = _fmt(fmt)
+    _dense(X, "X"), _dense(Y, "Y")
+    M = int(X.shape[0])
+    if workspace is None:
+        workspace = torch.zeros(max(gemm_any_workspace_bytes(f, M), 256), dtype=torch.uint8,
+                                device=Y.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("seedlm_gemm", lib.seedlm_gemm(
         ctypes.byref(f), _ptr(rec), _ptr(eplane), _ptr(X), _act_dtype(X), M, _ptr(Y),
         _ptr(workspace), nbytes, _stream(stream, Y)))
 

@@ -28,8 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("seedlm_decompress", "seedlm_gemv", "seedlm_gemm_smallM", "seedlm_init",
-              "seedlm_strerror", "seedlm_shutdown"):
+    for n in ("seedlm_decompress", "seedlm_gemv", "seedlm_gemm_smallM", "seedlm_gemm",
+              "seedlm_init", "seedlm_strerror", "seedlm_shutdown"):
         assert n in names
 
 
@@ -117,6 +117,13 @@ def test_bad_pointers_are_rejected_before_cuda(sl):
         assert L.seedlm_gemm_smallM_workspace_bytes(ctypes.byref(f), M) == -1
     assert L.seedlm_gemm_smallM(ctypes.byref(f), 0x1000, None, 0x2000, 0, 4, 0x3000,
                                 None, -1, None) == -1
+    for M in (0, -1):
+        assert L.seedlm_gemm(ctypes.byref(f), 0x1000, None, 0x2000, 0, M, 0x3000,
+                             None, 0, None) == -1
+        assert L.seedlm_gemm_workspace_bytes(ctypes.byref(f), M) == -1
+    assert L.seedlm_gemm(ctypes.byref(f), 0x1000, None, 0x2000, 0, 300, 0x3000, None, -1, None) == -1
+    assert L.seedlm_gemm(ctypes.byref(f), 0x1000, None, 0x2000, 7, 300, 0x3000, None, 0, None) == -1
+    assert L.seedlm_gemm(ctypes.byref(f), 0x1000, None, 0x2001, 0, 300, 0x3000, None, 0, None) == -1
     assert L.seedlm_device_error(None) == -1
     for limit in (0, 999, 100000001):
         assert L.seedlm_selftest_wait_timeout(limit, None) == -1

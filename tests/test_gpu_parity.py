@@ -337,6 +337,59 @@ def test_gemm_bf16_rows_of_any_magnitude(sl, oracle_mod, cp):
         assert np.all(err <= TOL * refabs[m]), (m, float((err / (refabs[m] + 1e-300)).max()))
 
 
+def gpu_gemm_any(sl, L, Xb, dtype="bf16"):
+    rec, ep = planes(L)
+    M = Xb.shape[0]
+    X = act_tensor(Xb, dtype)
+    Y = torch.full((M, L["fmt"]["rows"]), float("nan"), device="cuda")
+    sl.gemm(L["fmt"], rec, ep, X, Y)
+    torch.cuda.synchronize()
+    assert sl.device_error() == 0
+    return Y.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+@pytest.mark.parametrize("M", [65, 128, 129, 256, 257, 600])
+def test_gemm_large_batches_match_oracle(sl, oracle_mod, cp, M):
+    # seedlm_gemm: one N = 128 pass (65-128 rows), one N = 256 pass with
+    # half-width units (129-256), and several passes sharing one workspace
+    # (257, 600: the last pass narrower than the others).
+    rows, cols = 300, 3000  # 3 row tiles (one ragged), ragged last K chunk
+    L = inputs.make_layer(rows, cols, *cp, seed=700 + M)
+    Xb, Xv = inputs.make_activations((M, cols), "bf16", 701 + M)
+    got = gpu_gemm_any(sl, L, Xb)
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv, threads=os.cpu_count() or 1)
+    for m in range(M):
+        assert_within(got[m], ref[m], refabs[m])
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_gemm_large_batches_fp16_and_small_M_agreement(sl, oracle_mod, cp):
+    L = inputs.make_layer(129, 1000, *cp, seed=711)
+    Xb, Xv = inputs.make_activations((200, 1000), "f16", 712)
+    got = gpu_gemm_any(sl, L, Xb, "f16")
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv, threads=os.cpu_count() or 1)
+    for m in range(200):
+        assert_within(got[m], ref[m], refabs[m])
+    # Up to 64 rows seedlm_gemm is seedlm_gemm_smallM, bit for bit.
+    Xs = Xb[:33]
+    assert np.array_equal(gpu_gemm_any(sl, L, Xs, "f16").view(np.uint64),
+                          gpu_gemm(sl, L, Xs, "f16").view(np.uint64))
+
+
+@pytest.mark.parametrize("cp,rows,cols,M", [(C8, 28672, 8192, 256), (C12, 8192, 28672, 300)])
+def test_gemm_large_batches_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols, M):
+    L = inputs.make_layer(rows, cols, *cp, seed=rows + cols + M)
+    Xb, Xv = inputs.make_activations((M, cols), "bf16", 92)
+    got = gpu_gemm_any(sl, L, Xb)
+    rng = np.random.default_rng(2)
+    sample = np.unique(np.concatenate([np.arange(2), np.arange(rows - 2, rows),
+                                       rng.integers(0, rows, 8)]))
+    ref, refabs = oracle_mod.gemm_rows(L["fmt"], L["rec"], L["eplane"], Xv, sample)
+    for m in range(M):
+        assert_within(got[m, sample], ref[m], refabs[m])
+
+
 def test_gemm_workspace_reuse_is_deterministic(sl):
     # The same workspace across calls (counters must be left at zero) and
     # bit-identical results (split-K partials are added in a fixed order).
