@@ -285,34 +285,62 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
                : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
                : "memory");
 }
-// Converts the 32 floats of two pieces of 16 K-consecutive weights to fp16
-// (exact) and stores them, two per 32-bit column with the lower K index in
-// the low half: h into 8 columns at taddr_h, l into 8 columns at taddr_l.
-// The conversions write the store's source registers directly.
-__device__ __forceinline__ void tmem_st_f16_pieces_x8(uint32_t taddr_h, uint32_t taddr_l,
-                                                      const float (&h)[16], const float (&l)[16]) {
+// Splits 16 K-consecutive weights w (fp32, exact multiples of 2^-24 below
+// 2^11 in magnitude) into two fp16 pieces and stores them, two per 32-bit
+// column with the lower K index in the low half: hi = w rounded toward zero
+// to fp16 (its top 11 significant bits; all of w below fp16's normal range)
+// into 8 columns at taddr_h, lo = w - hi (at most 9 bits, exact) into 8
+// columns at taddr_l.  lo comes from one mixed-precision FMA per weight,
+// (-1) * hi + w with hi in fp16.
+__device__ __forceinline__ void tmem_st_f16_split_x8(uint32_t taddr_h, uint32_t taddr_l,
+                                                     const float (&w)[16]) {
   asm volatile(
-      "{\n\t.reg .b32 q<16>;\n\t"
-      "cvt.rn.f16x2.f32 q0, %3, %2;\n\t"
-      "cvt.rn.f16x2.f32 q1, %5, %4;\n\t"
-      "cvt.rn.f16x2.f32 q2, %7, %6;\n\t"
-      "cvt.rn.f16x2.f32 q3, %9, %8;\n\t"
-      "cvt.rn.f16x2.f32 q4, %11, %10;\n\t"
-      "cvt.rn.f16x2.f32 q5, %13, %12;\n\t"
-      "cvt.rn.f16x2.f32 q6, %15, %14;\n\t"
-      "cvt.rn.f16x2.f32 q7, %17, %16;\n\t"
-      "cvt.rn.f16x2.f32 q8, %19, %18;\n\t"
-      "cvt.rn.f16x2.f32 q9, %21, %20;\n\t"
-      "cvt.rn.f16x2.f32 q10, %23, %22;\n\t"
-      "cvt.rn.f16x2.f32 q11, %25, %24;\n\t"
-      "cvt.rn.f16x2.f32 q12, %27, %26;\n\t"
-      "cvt.rn.f16x2.f32 q13, %29, %28;\n\t"
-      "cvt.rn.f16x2.f32 q14, %31, %30;\n\t"
-      "cvt.rn.f16x2.f32 q15, %33, %32;\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {q0, q1, q2, q3, q4, q5, q6, q7};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%1], {q8, q9, q10, q11, q12, q13, q14, q15};\n\t}\n"
+      "{\n\t.reg .b32 h<8>, l<8>;\n\t.reg .f16 g<16>, m;\n\t.reg .f32 d<16>;\n\t"
+      "mov.b16 m, 0xBC00;\n\t"
+      "cvt.rz.f16x2.f32 h0, %3, %2;\n\t"
+      "mov.b32 {g0, g1}, h0;\n\t"
+      "cvt.rz.f16x2.f32 h1, %5, %4;\n\t"
+      "mov.b32 {g2, g3}, h1;\n\t"
+      "cvt.rz.f16x2.f32 h2, %7, %6;\n\t"
+      "mov.b32 {g4, g5}, h2;\n\t"
+      "cvt.rz.f16x2.f32 h3, %9, %8;\n\t"
+      "mov.b32 {g6, g7}, h3;\n\t"
+      "cvt.rz.f16x2.f32 h4, %11, %10;\n\t"
+      "mov.b32 {g8, g9}, h4;\n\t"
+      "cvt.rz.f16x2.f32 h5, %13, %12;\n\t"
+      "mov.b32 {g10, g11}, h5;\n\t"
+      "cvt.rz.f16x2.f32 h6, %15, %14;\n\t"
+      "mov.b32 {g12, g13}, h6;\n\t"
+      "cvt.rz.f16x2.f32 h7, %17, %16;\n\t"
+      "mov.b32 {g14, g15}, h7;\n\t"
+      "fma.rn.f32.f16 d0, g0, m, %2;\n\t"
+      "fma.rn.f32.f16 d1, g1, m, %3;\n\t"
+      "fma.rn.f32.f16 d2, g2, m, %4;\n\t"
+      "fma.rn.f32.f16 d3, g3, m, %5;\n\t"
+      "fma.rn.f32.f16 d4, g4, m, %6;\n\t"
+      "fma.rn.f32.f16 d5, g5, m, %7;\n\t"
+      "fma.rn.f32.f16 d6, g6, m, %8;\n\t"
+      "fma.rn.f32.f16 d7, g7, m, %9;\n\t"
+      "fma.rn.f32.f16 d8, g8, m, %10;\n\t"
+      "fma.rn.f32.f16 d9, g9, m, %11;\n\t"
+      "fma.rn.f32.f16 d10, g10, m, %12;\n\t"
+      "fma.rn.f32.f16 d11, g11, m, %13;\n\t"
+      "fma.rn.f32.f16 d12, g12, m, %14;\n\t"
+      "fma.rn.f32.f16 d13, g13, m, %15;\n\t"
+      "fma.rn.f32.f16 d14, g14, m, %16;\n\t"
+      "fma.rn.f32.f16 d15, g15, m, %17;\n\t"
+      "cvt.rn.f16x2.f32 l0, d1, d0;\n\t"
+      "cvt.rn.f16x2.f32 l1, d3, d2;\n\t"
+      "cvt.rn.f16x2.f32 l2, d5, d4;\n\t"
+      "cvt.rn.f16x2.f32 l3, d7, d6;\n\t"
+      "cvt.rn.f16x2.f32 l4, d9, d8;\n\t"
+      "cvt.rn.f16x2.f32 l5, d11, d10;\n\t"
+      "cvt.rn.f16x2.f32 l6, d13, d12;\n\t"
+      "cvt.rn.f16x2.f32 l7, d15, d14;\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {h0, h1, h2, h3, h4, h5, h6, h7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%1], {l0, l1, l2, l3, l4, l5, l6, l7};\n\t}\n"
       :
-      : "r"(taddr_h), "r"(taddr_l), "f"(h[0]), "f"(h[1]), "f"(h[2]), "f"(h[3]), "f"(h[4]), "f"(h[5]), "f"(h[6]), "f"(h[7]), "f"(h[8]), "f"(h[9]), "f"(h[10]), "f"(h[11]), "f"(h[12]), "f"(h[13]), "f"(h[14]), "f"(h[15]), "f"(l[0]), "f"(l[1]), "f"(l[2]), "f"(l[3]), "f"(l[4]), "f"(l[5]), "f"(l[6]), "f"(l[7]), "f"(l[8]), "f"(l[9]), "f"(l[10]), "f"(l[11]), "f"(l[12]), "f"(l[13]), "f"(l[14]), "f"(l[15])
+      : "r"(taddr_h), "r"(taddr_l), "f"(w[0]), "f"(w[1]), "f"(w[2]), "f"(w[3]), "f"(w[4]), "f"(w[5]), "f"(w[6]), "f"(w[7]), "f"(w[8]), "f"(w[9]), "f"(w[10]), "f"(w[11]), "f"(w[12]), "f"(w[13]), "f"(w[14]), "f"(w[15])
       : "memory");
 }
 
