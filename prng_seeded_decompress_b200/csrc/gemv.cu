@@ -107,6 +107,15 @@ constexpr int kRowsPerTask = 4;
 constexpr int kMinWarps = 8;      // warps per CTA however few items it has
 constexpr int kSpanUnits = 32;    // lane units (pairs or quads of blocks) per span
 
+// V = 2 is V = 0 with half-warp spans: each half-warp takes 16 units of its
+// own 4 rows, so an item is 8 rows x 16 units.  Chosen where it pads a row's
+// units less (3-bit rows of 4096 columns: 171 pairs fill 176 lanes instead
+// of 192).
+template <int V>
+__host__ __device__ constexpr int span_units() { return V == 2 ? kSpanUnits / 2 : kSpanUnits; }
+template <int V>
+__host__ __device__ constexpr int rows_per_item() { return kRowsPerTask * (kSpanUnits / span_units<V>()); }
+
 // Two variants of the kernel:
 //   V = 0 (large products): the lane-replicated tables at absolute shared
 //     addresses, one CTA per SM.  Shared-memory map:
@@ -116,6 +125,7 @@ constexpr int kSpanUnits = 32;    // lane units (pairs or quads of blocks) per s
 //       C = 12: [kSmemBase, 0x20000)  x slots of one column segment
 //               [0x20000, 0x30000)    stream jump-table rows
 //       both:   [0x30000, ...)        partial row sums of one pass
+//   V = 2: V = 0 with half-warp spans (above), for C = 12.
 //   V = 1 (small products, a few items per CTA): one copy of each table at
 //     the start of the allocation, 32 KB of x slots after it, then the
 //     partial sums; 8 warps and small allocations, so that several CTAs --
@@ -127,18 +137,18 @@ using rep::lds32;
 using rep::lds64;
 template <int C, int V>
 struct Smem {
-  static constexpr uint32_t kJump = rep::tables_begin<C>();  // V = 0
+  static constexpr uint32_t kJump = rep::tables_begin<C>();  // V = 0, 2
   // V = 1: jump tables (C = 8: 2 x 256 words; C = 12: 2 x 256 8-byte
   // entries) then, for C = 8, the two coefficient tables (2 x 256 x 8 B).
-  static constexpr int kTabBytes = (V == 0) ? 0 : (C == 8) ? 2048 + 4096 : 4096;
+  static constexpr int kTabBytes = (V != 1) ? 0 : (C == 8) ? 2048 + 4096 : 4096;
   static constexpr int kXOff = kTabBytes;  // bytes from the allocation's start
-  static constexpr int kXBytes = (V == 0) ? (int)(kJump - kSmemBase) : 32768;
-  static constexpr int kPartOff = (V == 0) ? (int)(0x30000u - kSmemBase) : kXOff + kXBytes;
+  static constexpr int kXBytes = (V != 1) ? (int)(kJump - kSmemBase) : 32768;
+  static constexpr int kPartOff = (V != 1) ? (int)(0x30000u - kSmemBase) : kXOff + kXBytes;
   // x floats per lane unit: C * kBPL, rounded up to 32 for C = 12 (swizzle).
   static constexpr int kSlotFloats = (C == 8) ? 8 * Tune<C, V>::kBPL : 32;
-  static constexpr int kSpanBytes = kSpanUnits * kSlotFloats * 4;
+  static constexpr int kSpanBytes = span_units<V>() * kSlotFloats * 4;
   static constexpr int kMaxSegSpans = kXBytes / kSpanBytes;
-  static constexpr int kPartBytesPerGroup = kRowsPerTask * 4;  // per warp
+  static constexpr int kPartBytesPerGroup = rows_per_item<V>() * 4;  // per warp
 };
 #if SEEDLM_GEMV_LFSR == 2
 constexpr uint32_t kTabJump = Smem<8, 0>::kJump;
@@ -146,9 +156,9 @@ constexpr uint32_t kTabJump = Smem<8, 0>::kJump;
 
 struct GemvGeom {
   int rows, cols, nb, rec_pitch, e_pitch;
-  int n_spans;      // ceil(ceil(nb / kBPL) / 32)
-  int groups;       // ceil(rows / 4)
-  int full_groups;  // groups with all 4 rows inside the matrix
+  int n_spans;      // ceil(ceil(nb / kBPL) / span units)
+  int groups;       // ceil(rows / rows per item)
+  int full_groups;  // groups with all their rows inside the matrix
   int full_spans;   // spans whose every unit lies inside the row pitch
   int seg_spans;    // spans per x segment (the last one may be shorter)
   int n_segs;
@@ -298,8 +308,8 @@ __device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, 
                         int s0, int sl) {
   constexpr int kBPL = Tune<C, V>::kBPL;
   constexpr int kVals = C * kBPL;  // x values of one unit (16, 24 or 32)
-  const int units = sl * kSpanUnits;
-  const int col_base = s0 * kSpanUnits * kVals;
+  const int units = sl * span_units<V>();
+  const int col_base = s0 * span_units<V>() * kVals;
   const bool vec = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
   SEEDLM_CHECK_ONLY(const unsigned int xs_floats = Smem<C, V>::kXBytes / 4;)
   for (int u = threadIdx.x; u < units; u += blockDim.x) {
@@ -352,8 +362,9 @@ __device__ __forceinline__ void load_set(RecSet<C, V>& o, const uint32_t* __rest
                                          const uint8_t* __restrict__ eplane, const GemvGeom& g,
                                          int grp, int span, int lane) {
   constexpr int kBPL = Tune<C, V>::kBPL;
-  const int row0 = grp * kRowsPerTask;
-  const int u = span * kSpanUnits + lane;
+  constexpr int kSU = span_units<V>();
+  const int row0 = grp * rows_per_item<V>() + (lane / kSU) * kRowsPerTask;
+  const int u = span * kSU + lane % kSU;
   const uint32_t* p = rec + (size_t)row0 * g.rec_pitch + kBPL * u;
   if (grp < g.full_groups && span < g.full_spans && !SEEDLM_CHECK) {
     // Every row of the group and every unit of the span is inside the plane.
@@ -430,7 +441,7 @@ __device__ __forceinline__ float2 fma_pair(int32_t bits_a, int32_t bits_b, float
 template <int V>
 __device__ __forceinline__ BlockC8 decode_c8_v(uint32_t rec, uint32_t lane4, uint32_t lane8,
                                                const unsigned char* tabs) {
-  if constexpr (V == 0) {
+  if constexpr (V != 1) {
     return decode_c8_rep(rec, lane4, lane8);
   } else {
     const uint32_t* t = reinterpret_cast<const uint32_t*>(tabs);
@@ -442,7 +453,7 @@ __device__ __forceinline__ BlockC8 decode_c8_v(uint32_t rec, uint32_t lane4, uin
 template <int V>
 __device__ __forceinline__ BlockC12 decode_c12_v(uint32_t rec, uint32_t e4, uint32_t lane8,
                                                  const unsigned char* tabs) {
-  if constexpr (V == 0) {
+  if constexpr (V != 1) {
     return decode_c12_rep(rec, e4, lane8);
   } else {
     const uint2* t = reinterpret_cast<const uint2*>(tabs);
@@ -564,10 +575,11 @@ template <int C, int V, bool kBatch>
 __global__ void __launch_bounds__(Tune<C, V>::kWarps * 32, Tune<C, V>::kMinBlocks)
 gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
   constexpr int kP = Tune<C, V>::kPrefetch;
+  constexpr int kSU = span_units<V>(), kRPI = rows_per_item<V>();
   extern __shared__ __align__(16) unsigned char smem[];
   // V = 0: the table addresses are absolute, so the allocation must start at
   // kSmemBase.
-  if (V == 0 && smem_u32(smem) != kSmemBase) {
+  if (V != 1 && smem_u32(smem) != kSmemBase) {
     if (threadIdx.x == 0) atomicOr(&g_gemv_error, 1u);
     return;
   }
@@ -597,7 +609,7 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
     const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
     for (int p0 = g0; p0 < g1; p0 += g.pass_groups) {
       const int p1 = min(p0 + g.pass_groups, g1);
-      for (int i = threadIdx.x; i < (p1 - p0) * kRowsPerTask * nw; i += blockDim.x)
+      for (int i = threadIdx.x; i < (p1 - p0) * kRPI * nw; i += blockDim.x)
         if (SEEDLM_IN_BOUNDS(g_check_flag, i, part_floats)) part[i] = 0.f;
       for (int sg = 0; sg < g.n_segs; ++sg) {
         const int s0 = sg * g.seg_spans;
@@ -624,7 +636,7 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
           for (;;) {
 #pragma unroll
             for (int k = 0; k <= kP; ++k) {
-              const int ul = span * kSpanUnits + lane;
+              const int ul = span * kSU + lane % kSU;
               // Every x slot of the lane's unit lies in its kSlotFloats row.
               if (SEEDLM_IN_BOUNDS(g_check_flag, (ul + 1) * (Smem<C, V>::kSlotFloats) - 1, xs_floats))
                 rebuild_and_dot<C, V>(buf[k], xs, ul, lane, lane4, lane8, tabs, acc);
@@ -637,9 +649,12 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
               if (end_group || ci == i1) {
 #pragma unroll
                 for (int j = 0; j < kRowsPerTask; ++j) {
-                  const float sum = warp_sum(acc[j].x + acc[j].y);
-                  const int pi = ((grp - p0) * kRowsPerTask + j) * nw + warp;
-                  if (lane == 0 && SEEDLM_IN_BOUNDS(g_check_flag, pi, part_floats)) part[pi] += sum;
+                  // Sum over the lanes of the row's span (the warp, or its half).
+                  float sum = acc[j].x + acc[j].y;
+#pragma unroll
+                  for (int o = kSU / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                  const int pi = ((grp - p0) * kRPI + (lane / kSU) * kRowsPerTask + j) * nw + warp;
+                  if (lane % kSU == 0 && SEEDLM_IN_BOUNDS(g_check_flag, pi, part_floats)) part[pi] += sum;
                   acc[j] = make_float2(0.f, 0.f);
                 }
                 if (end_group) { span = 0; ++grp; }
@@ -655,8 +670,8 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
         // The next kernel in the stream may start its prologue now.
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
       }
-      for (int t = threadIdx.x; t < (p1 - p0) * kRowsPerTask; t += blockDim.x) {
-        const int r = p0 * kRowsPerTask + t;
+      for (int t = threadIdx.x; t < (p1 - p0) * kRPI; t += blockDim.x) {
+        const int r = p0 * kRPI + t;
         if (r < g.rows) {
           float sum = 0.f;
           for (int w = 0; w < nw; ++w)
@@ -692,12 +707,13 @@ GemvGeom make_geom(const seedlm_format& f, int max_smem, int nw, int grid) {
   g.nb = f.nb;
   g.rec_pitch = f.rec_pitch;
   g.e_pitch = f.e_pitch;
-  g.n_spans = ((f.nb + kBPL - 1) / kBPL + kSpanUnits - 1) / kSpanUnits;
+  constexpr int kSU = span_units<V>(), kRPI = rows_per_item<V>();
+  g.n_spans = ((f.nb + kBPL - 1) / kBPL + kSU - 1) / kSU;
   if (g.n_spans < 1) g.n_spans = 1;
-  g.groups = (f.rows + kRowsPerTask - 1) / kRowsPerTask;
-  g.full_groups = f.rows / kRowsPerTask;
+  g.groups = (f.rows + kRPI - 1) / kRPI;
+  g.full_groups = f.rows / kRPI;
   // Units of the pitch: a span is full when its last unit ends inside it.
-  g.full_spans = f.rec_pitch / (kBPL * kSpanUnits);
+  g.full_spans = f.rec_pitch / (kBPL * kSU);
   g.n_segs = (g.n_spans + Smem<C, V>::kMaxSegSpans - 1) / Smem<C, V>::kMaxSegSpans;
   g.seg_spans = (g.n_spans + g.n_segs - 1) / g.n_segs;
   int64_t room = (int64_t)max_smem - Smem<C, V>::kPartOff;
@@ -728,9 +744,10 @@ int max_items_per_cta(const seedlm_format* const* f, int n, int max_ctas, int* m
   constexpr int kBPL = Tune<C, V>::kBPL;
   int mi = 1;
   *max_groups = 1;
+  constexpr int kSU = span_units<V>(), kRPI = rows_per_item<V>();
   for (int k = 0; k < n; ++k) {
-    const int groups = (f[k]->rows + kRowsPerTask - 1) / kRowsPerTask;
-    int n_spans = ((f[k]->nb + kBPL - 1) / kBPL + kSpanUnits - 1) / kSpanUnits;
+    const int groups = (f[k]->rows + kRPI - 1) / kRPI;
+    int n_spans = ((f[k]->nb + kBPL - 1) / kBPL + kSU - 1) / kSU;
     if (n_spans < 1) n_spans = 1;
     if (groups > *max_groups) *max_groups = groups;
     const int grid_k = groups < max_ctas ? groups : max_ctas;
@@ -747,7 +764,7 @@ int max_items_per_cta(const seedlm_format* const* f, int n, int max_ctas, int* m
 template <int C, int V>
 GemvLaunch plan_v(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
   GemvLaunch L{};
-  const int max_ctas = (V == 0) ? dev.num_sms : 2 * dev.num_sms;
+  const int max_ctas = (V != 1) ? dev.num_sms : 2 * dev.num_sms;
   int max_groups = 1;
   const int max_items = max_items_per_cta<C, V>(f, n, max_ctas, &max_groups);
   L.variant = V;
@@ -770,11 +787,33 @@ GemvLaunch plan_v(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
 // The small variant when the large one would give each of its 16 warps
 // fewer than 4 items: there the setup of the replicated tables and the
 // one-CTA-per-SM launch, not the rebuild, set the time.
+// Lane units the busiest of `grid` CTAs walks through in variant V (row
+// groups per CTA rounded up, each row's units padded to whole spans), summed
+// over the batch's products.
+template <int V>
+int64_t busiest_cta_units(const seedlm_format* const* f, int n, int bpl, int grid) {
+  constexpr int kSU = span_units<V>(), kRPI = rows_per_item<V>();
+  int64_t t = 0;
+  for (int k = 0; k < n; ++k) {
+    const int64_t units = (f[k]->nb + bpl - 1) / bpl;
+    const int64_t groups = (f[k]->rows + kRPI - 1) / kRPI;
+    t += (groups + grid - 1) / grid * kRPI * ((units + kSU - 1) / kSU * kSU);
+  }
+  return t;
+}
+
 template <int C>
 GemvLaunch plan(const seedlm_format* const* f, int n, const DeviceInfo& dev) {
   int max_groups = 1;
   const int items = max_items_per_cta<C, 0>(f, n, dev.num_sms, &max_groups);
   if (items < 4 * Tune<C, 0>::kWarps) return plan_v<C, 1>(f, n, dev);
+  if constexpr (C == 12) {
+    // Half-warp spans where the busiest CTA then has less to do: less span
+    // padding, against coarser row groups (8 rows) to spread over the CTAs.
+    constexpr int kBPL = Tune<12, 0>::kBPL;
+    if (busiest_cta_units<2>(f, n, kBPL, dev.num_sms) < busiest_cta_units<0>(f, n, kBPL, dev.num_sms))
+      return plan_v<12, 2>(f, n, dev);
+  }
   return plan_v<C, 0>(f, n, dev);
 }
 
@@ -803,6 +842,7 @@ const void* kernel_for(int C, int V, bool batch) {
     return batch ? (const void*)gemv_kernel<8, 1, true> : (const void*)gemv_kernel<8, 1, false>;
   }
   if (V == 0) return batch ? (const void*)gemv_kernel<12, 0, true> : (const void*)gemv_kernel<12, 0, false>;
+  if (V == 2) return batch ? (const void*)gemv_kernel<12, 2, true> : (const void*)gemv_kernel<12, 2, false>;
   return batch ? (const void*)gemv_kernel<12, 1, true> : (const void*)gemv_kernel<12, 1, false>;
 }
 

@@ -205,14 +205,17 @@ def test_gemm_decompress_encode_empty_shapes(sl):
         X = torch.zeros((3, max(cols, 1)), dtype=torch.bfloat16, device="cuda")
         Y = torch.full((3, max(rows, 1)), float("nan"), device="cuda")
         sl.gemm_smallM(L["fmt"], rec, ep, X, Y)
+        Y2 = torch.full((300, max(rows, 1)), float("nan"), device="cuda")
+        sl.gemm(L["fmt"], rec, ep, torch.zeros((300, max(cols, 1)), dtype=torch.bfloat16,
+                                               device="cuda"), Y2)
         W = torch.full((max(rows, 1), max(cols, 1)), float("nan"), device="cuda")
         sl.decompress(L["fmt"], rec, ep, W, ldw=max(cols, 1))
         sl.encode(L["fmt"], W, rec, ep, ldw=max(cols, 1))
         torch.cuda.synchronize()
         if rows:
-            assert torch.equal(Y, torch.zeros_like(Y))
+            assert torch.equal(Y, torch.zeros_like(Y)) and torch.equal(Y2, torch.zeros_like(Y2))
         else:
-            assert torch.isnan(Y).all()
+            assert torch.isnan(Y).all() and torch.isnan(Y2).all()
         assert torch.isnan(W).all()
     assert sl.device_error() == 0
 
@@ -377,6 +380,27 @@ def test_gemm_large_batches_fp16_and_small_M_agreement(sl, oracle_mod, cp):
                           gpu_gemm(sl, L, Xs, "f16").view(np.uint64))
 
 
+def test_gemm_any_M_one_row_is_the_gemv_and_workspace_query(sl):
+    L = inputs.make_layer(256, 4096, *C8, seed=73)
+    xb, _ = inputs.make_activations((1, 4096), "bf16", 74)
+    assert sl.gemm_any_workspace_bytes(L["fmt"], 1) == 0  # M = 1 runs the GEMV
+    got = gpu_gemm_any(sl, L, xb)
+    assert np.array_equal(got[0], gpu_gemv(sl, L, xb[0], "bf16"))
+    # A full pass and a narrower last pass: the query covers the larger need.
+    need = sl.gemm_any_workspace_bytes(L["fmt"], 300)
+    assert need >= sl.gemm_any_workspace_bytes(L["fmt"], 256)
+    assert need >= sl.gemm_any_workspace_bytes(L["fmt"], 44)
+    assert sl.gemm_any_workspace_bytes(L["fmt"], 64) == sl.gemm_workspace_bytes(L["fmt"], 64)
+    # Too small a workspace is refused before anything runs.
+    rec, ep = planes(L)
+    X = torch.zeros((300, 4096), dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros((300, 256), device="cuda")
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sl.SeedLMError) as exc:
+        sl.gemm(L["fmt"], rec, ep, X, Y, workspace=ws)
+    assert exc.value.code == -1
+
+
 @pytest.mark.parametrize("cp,rows,cols,M", [(C8, 28672, 8192, 256), (C12, 8192, 28672, 300)])
 def test_gemm_large_batches_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols, M):
     L = inputs.make_layer(rows, cols, *cp, seed=rows + cols + M)
@@ -491,6 +515,11 @@ def test_graph_replay_matches_eager_calls(sl):
     # 768 (3 bits) per x segment.
     (C8, 2400, 70000), (C12, 2400, 50000), (C8, 2400, 15360), (C8, 2400, 15361),
     (C12, 2400, 23808), (C12, 2400, 23809),
+    # 3 bits with half-warp spans (chosen where the busiest CTA has fewer
+    # lane units: less span padding against 8-row items): 63 spans of 16
+    # units of 24 columns per segment -- one segment exactly, two, and the
+    # Llama-3-8B width; ragged row counts.
+    (C12, 2365, 24192), (C12, 2365, 24720), (C12, 7101, 4096),
     # Small-product kernel (a few items per CTA): 32 KB of x slots, 16 spans
     # of 512 columns (4 bits, 2 blocks per lane) or 8 of 768 (3 bits).
     (C8, 40, 8192), (C8, 40, 8193), (C12, 40, 6144), (C12, 40, 6145),
