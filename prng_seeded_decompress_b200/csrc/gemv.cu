@@ -34,10 +34,12 @@
 //     warp shuffles and added into a per-warp slot in shared memory; after a
 //     barrier the slots of each row are added in warp order -- the same
 //     order on every call -- and written.
-//   * Launched with programmatic stream serialization: the table fill runs
-//     before griddepcontrol.wait and overlaps the previous kernel's tail;
-//     records and x are read only after the wait, so they may be written by
-//     the previous kernel in the stream.
+//   * Launched with programmatic stream serialization, and every CTA lets
+//     the next kernel launch as soon as it starts: a CTA of the next GEMV
+//     takes its SM when this one's CTA there exits and fills its tables
+//     (before griddepcontrol.wait) while the slowest CTAs of this grid
+//     finish.  Records and x are read only after the wait, so they may be
+//     written by the previous kernel in the stream.
 #include <cuda_runtime.h>
 
 #include <type_traits>
@@ -169,12 +171,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 #if SEEDLM_GEMV_LFSR == 1
 // One pass of the recurrence on a 32-bit word X whose bits [0, n) are stream
 // bits [0, n): bit m of the result is stream bit 16 + m for m + 5 < n.
@@ -302,7 +298,9 @@ __device__ __forceinline__ int x_slot_index(int u, int c, int h) {
 
 // x columns of spans [s0, s0 + sl), zero past cols, into the segment's
 // slots.  One thread per lane unit; 16-byte loads when x is 16-byte aligned
-// and the unit lies inside x.
+// and the unit lies inside x, and one 16-byte store per float4 of the slot:
+// the 8 threads of a quarter-warp then write 8 distinct bank groups (the
+// slot swizzle), where scalar stores met 4-way conflicts.
 template <int C, int V>
 __device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, const GemvGeom& g,
                         int s0, int sl) {
@@ -314,28 +312,39 @@ __device__ void stage_x(float* xs, const uint16_t* __restrict__ x, int is_bf16, 
   SEEDLM_CHECK_ONLY(const unsigned int xs_floats = Smem<C, V>::kXBytes / 4;)
   for (int u = threadIdx.x; u < units; u += blockDim.x) {
     const int col0 = col_base + u * kVals;
-    uint16_t v16[kVals];
+    uint32_t w[kVals / 2];  // value k in the half k % 2 of w[k / 2]
     if (vec && col0 + kVals <= g.cols) {
 #pragma unroll
       for (int k = 0; k < kVals / 8; ++k) {
         const uint4 q = *reinterpret_cast<const uint4*>(x + col0 + 8 * k);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          v16[8 * k + 2 * m] = (uint16_t)w[m];
-          v16[8 * k + 2 * m + 1] = (uint16_t)(w[m] >> 16);
-        }
+        w[4 * k] = q.x;
+        w[4 * k + 1] = q.y;
+        w[4 * k + 2] = q.z;
+        w[4 * k + 3] = q.w;
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < kVals; ++k) v16[k] = col0 + k < g.cols ? x[col0 + k] : (uint16_t)0;
+      for (int k = 0; k < kVals / 2; ++k) {
+        const uint32_t lo = col0 + 2 * k < g.cols ? x[col0 + 2 * k] : 0u;
+        const uint32_t hi = col0 + 2 * k + 1 < g.cols ? x[col0 + 2 * k + 1] : 0u;
+        w[k] = lo | hi << 16;
+      }
     }
+    auto val = [&](int k) { return act_to_float((uint16_t)(w[k >> 1] >> (16 * (k & 1))), is_bf16); };
+    // float4 i of the slot: column i of blocks 0..3 (quads), or columns 2i,
+    // 2i+1 of blocks 0 and 1 (pairs); see x_slot_index.
 #pragma unroll
-    for (int k = 0; k < kVals; ++k) {
-      const int h = k / C, c = k - h * C;
-      const int si = x_slot_index<C, V>(u, c, h);
-      const float f = act_to_float(v16[k], is_bf16);
-      if (SEEDLM_IN_BOUNDS(g_check_flag, si, xs_floats)) xs[si] = f;
+    for (int i = 0; i < kVals / 4; ++i) {
+      float4 f;
+      int si;
+      if constexpr (C == 8 && kBPL == 4) {
+        f = make_float4(val(i), val(8 + i), val(16 + i), val(24 + i));
+        si = x_slot_index<C, V>(u, i, 0);
+      } else {
+        f = make_float4(val(2 * i), val(C + 2 * i), val(2 * i + 1), val(C + 2 * i + 1));
+        si = x_slot_index<C, V>(u, 2 * i, 0);
+      }
+      if (SEEDLM_IN_BOUNDS(g_check_flag, si + 3, xs_floats)) *reinterpret_cast<float4*>(xs + si) = f;
     }
   }
 }
@@ -594,6 +603,11 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
   const uint32_t lane4 = (uint32_t)lane << 2, lane8 = (uint32_t)(lane & 15) << 3;
   RecSet<C, V> buf[kP + 1];
 
+  // The next kernel in the stream may launch now: its CTAs take an SM as
+  // soon as this kernel's CTA there exits, and run their own prologue while
+  // the slower CTAs of this grid finish.  Every CTA of this grid is resident
+  // before the trigger completes, so the early start cannot starve it.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   fill_tables<C, V>(smem);
   // Records and x may be the previous kernel's output: read them only now.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -609,26 +623,31 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
     const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
     for (int p0 = g0; p0 < g1; p0 += g.pass_groups) {
       const int p1 = min(p0 + g.pass_groups, g1);
-      for (int i = threadIdx.x; i < (p1 - p0) * kRPI * nw; i += blockDim.x)
+      // Partial sums of the pass: warp w's sum for row t at part[w * pass_rows + t],
+      // so the final reduction reads consecutive words across the threads.
+      const int pass_rows = (p1 - p0) * kRPI;
+      for (int i = threadIdx.x; i < pass_rows * nw; i += blockDim.x)
         if (SEEDLM_IN_BOUNDS(g_check_flag, i, part_floats)) part[i] = 0.f;
       for (int sg = 0; sg < g.n_segs; ++sg) {
         const int s0 = sg * g.seg_spans;
         const int sl = min(g.seg_spans, g.n_spans - s0);
-        // One segment: x stays staged for every pass of this GEMV.
-        if (g.n_segs > 1 || p0 == g0) stage_x<C, V>(xs, x, is_bf16, g, s0, sl);
-        __syncthreads();  // x, tables and zeroed partials ready
         const int items = (p1 - p0) * sl;
         const int i0 = (int)((int64_t)warp * items / nw);
         const int i1 = (int)((int64_t)(warp + 1) * items / nw);
-        if (i0 < i1) {
-          // Item cursor (grp, span) and load cursor (lgrp, lspan), kP items ahead.
-          int grp = p0 + i0 / sl, span = i0 % sl;
-          int lgrp = grp, lspan = span;
+        // Item cursor (grp, span) and load cursor (lgrp, lspan), kP items
+        // ahead.  The first record sets do not depend on x: they are in
+        // flight while x is staged.
+        int grp = p0 + i0 / sl, span = i0 % sl;
+        int lgrp = grp, lspan = span;
 #pragma unroll
-          for (int k = 0; k <= kP; ++k) {
-            if (i0 + k < i1) load_set<C, V>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
-            if (++lspan == sl) { lspan = 0; ++lgrp; }
-          }
+        for (int k = 0; k <= kP; ++k) {
+          if (i0 + k < i1) load_set<C, V>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+          if (++lspan == sl) { lspan = 0; ++lgrp; }
+        }
+        // One segment: x stays staged for every pass of this GEMV.
+        if (g.n_segs > 1 || p0 == g0) stage_x<C, V>(xs, x, is_bf16, g, s0, sl);
+        __syncthreads();  // x, tables and zeroed partials ready
+        if (i0 < i1) {
           float2 acc[kRowsPerTask];
 #pragma unroll
           for (int j = 0; j < kRowsPerTask; ++j) acc[j] = make_float2(0.f, 0.f);
@@ -653,7 +672,7 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
                   float sum = acc[j].x + acc[j].y;
 #pragma unroll
                   for (int o = kSU / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                  const int pi = ((grp - p0) * kRPI + (lane / kSU) * kRowsPerTask + j) * nw + warp;
+                  const int pi = warp * pass_rows + (grp - p0) * kRPI + (lane / kSU) * kRowsPerTask + j;
                   if (lane % kSU == 0 && SEEDLM_IN_BOUNDS(g_check_flag, pi, part_floats)) part[pi] += sum;
                   acc[j] = make_float2(0.f, 0.f);
                 }
@@ -666,16 +685,12 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
         }
         __syncthreads();  // partials complete; x may be restaged
       }
-      if (bi == nbatch - 1 && p1 == g1) {
-        // The next kernel in the stream may start its prologue now.
-        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-      }
-      for (int t = threadIdx.x; t < (p1 - p0) * kRPI; t += blockDim.x) {
+      for (int t = threadIdx.x; t < pass_rows; t += blockDim.x) {
         const int r = p0 * kRPI + t;
         if (r < g.rows) {
           float sum = 0.f;
           for (int w = 0; w < nw; ++w)
-            if (SEEDLM_IN_BOUNDS(g_check_flag, t * nw + w, part_floats)) sum += part[t * nw + w];
+            if (SEEDLM_IN_BOUNDS(g_check_flag, w * pass_rows + t, part_floats)) sum += part[w * pass_rows + t];
           if (SEEDLM_IN_BOUNDS(g_check_flag, r, g.rows)) y[r] = sum;
         }
       }

@@ -63,31 +63,30 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
 // so that a block's integer start value is tq1.y + tq2.y - (e << 23).
 template <int C, int SHIFT>
 __device__ void fill_rep_tables(unsigned char* smem, int tid, int nthreads) {
-  // One thread per (row v, table): one read of the jump table, eight 16-byte
-  // stores of its lane copies.
+  // 16-byte piece i = 16 v + 8 which + k of the tables: piece k of half-row
+  // (v, which), which = 0 the low 128 bytes of row v, 1 the high ones.  Eight
+  // consecutive threads write one contiguous half-row, so every quarter-warp
+  // store covers the 32 banks once (one thread per half-row would put all 32
+  // lanes of a warp 256 bytes apart, on the same four banks).
   uint4* jr = reinterpret_cast<uint4*>(smem + (tables_begin<C>() - kSmemBase));
-  for (int t = tid; t < 512; t += nthreads) {
-    const int v = t & 255, which = t >> 8;
+#pragma unroll 4
+  for (int i = tid; i < 4096; i += nthreads) {
+    const int v = i >> 4, which = (i >> 3) & 1;
     const uint64_t e = which ? kStreamTables.hi[v] : kStreamTables.lo[v];
     const uint32_t lo = (uint32_t)e, hi = (uint32_t)(e >> 32);
-    const uint4 q = (C == 8) ? make_uint4(lo, lo, lo, lo) : make_uint4(lo, hi, lo, hi);
-    uint4* row = jr + v * 16 + which * 8;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) row[k] = q;
+    jr[i] = (C == 8) ? make_uint4(lo, lo, lo, lo) : make_uint4(lo, hi, lo, hi);
   }
   if constexpr (C == 8) {
     constexpr uint32_t kMagic = kMagicBits + ((uint32_t)SHIFT << 23);
     uint4* cr = reinterpret_cast<uint4*>(smem + (kCoef8 - kSmemBase));
-    for (int t = tid; t < 512; t += nthreads) {
-      const int v = t & 255, which = t >> 8;
+#pragma unroll 4
+    for (int i = tid; i < 4096; i += nthreads) {
+      const int v = i >> 4, which = (i >> 3) & 1;
       const int32_t a = nibble_value(v), b = nibble_value(v >> 4);
       const uint2 e = which == 0
                           ? make_uint2(pack_s16(a, 256 * a + b), kMagic - (uint32_t)(32768 * (a + b)))
                           : make_uint2(pack_s16(256 * a + b, 256 * b), (uint32_t)(-32768 * b));
-      const uint4 q = make_uint4(e.x, e.y, e.x, e.y);
-      uint4* row = cr + v * 16 + which * 8;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) row[k] = q;
+      cr[i] = make_uint4(e.x, e.y, e.x, e.y);
     }
   }
 }
