@@ -359,6 +359,58 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
   const int t_first = (int)(u_begin / g.nchunks);
   const UnitCursor c0{t_first, (int)(u_begin - (long long)t_first * g.nchunks)};
 
+  // Producer warps: their first records are requested before the prologue
+  // (tables, barriers, TMEM), which then hides the memory latency.  The
+  // records are read before griddepcontrol.wait: the kernel before
+  // stage_x_kernel, a plain launch, has finished writing them.
+  const int lq = warp & 3, kq = warp >> 2;
+  const int prow = 32 * lq + lane;  // TMEM lane = row in the tile
+  const uint32_t lane4 = (uint32_t)lane << 2, lane8 = (uint32_t)(lane & 15) << 3;
+  const float2 neg1 = make_float2(-1.f, -1.f);
+  auto load_rec = [&](const UnitCursor& u, RecUnit<C>& p) {
+    const int gr = u.tile * kTileM + prow;
+    const int b0 = u.chunk * (KC / C) + kq * BPT;  // a multiple of BPT
+    // The thread's last record and its exponent byte lie inside row gr.
+    const bool ok_ = gr < g.rows && b0 < g.nb &&
+                     SEEDLM_IN_BOUNDS(g_check_flag, b0 + BPT - 1, g.rec_pitch) &&
+                     (C == 8 || SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, g.e_pitch));
+    const uint32_t* src = rec + (size_t)gr * g.rec_pitch + b0;
+    // b0 is a multiple of BPT, so each load is aligned to its width.
+    if constexpr (C == 8 && BPT == 4) {
+      const uint4 v = ok_ ? ld_stream_u4(src) : make_uint4(0u, 0u, 0u, 0u);
+      p.r[0] = v.x; p.r[1] = v.y; p.r[2] = v.z; p.r[3] = v.w;
+      p.e = 0;
+    } else if constexpr (C == 8) {
+      static_assert(BPT == 2, "C = 8 takes two or four blocks per thread");
+      const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
+      p.r[0] = v.x; p.r[1] = v.y;
+      p.e = 0;
+    } else if constexpr (BPT == 2) {
+      // b0 is even: one 8-byte load; the exponent byte holds block b0 in
+      // its low nibble and b0 + 1 in its high nibble.
+      const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
+      p.r[0] = v.x; p.r[1] = v.y;
+      p.e = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
+    } else {
+      // One block: a 4-byte load, the exponent from the nibble of b0's parity.
+      static_assert(BPT == 1, "C = 12 takes one or two blocks per thread");
+      p.r[0] = ok_ ? ld_stream_u1(src) : 0u;
+      const uint32_t eb = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
+      p.e = eb >> (4 * (b0 & 1));
+    }
+  };
+
+  RecUnit<C> ring[kRecAhead];
+  UnitCursor rc = c0;  // next unit whose records are loaded
+  if (warp < kProdWarps) {
+#pragma unroll
+    for (int k = 0; k < kRecAhead; ++k)
+      if (k < n_units) {
+        load_rec(rc, ring[k]);
+        rc.next(g.nchunks);
+      }
+  }
+
   rep::fill_rep_tables<C, kShift>(smem, tid, kThreads);
   const uint32_t bar = L::BAR;
   // xfull: X slab landed.  xfree: the MMAs that read the slab completed.
@@ -488,10 +540,11 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int i = tid - kEpiWarp0 * 32; i < NB; i += 128) ys[i] = __ldcg(yscale + i);
     tc::named_sync(128);
-    auto epilogue = [&](int seg, int tile) {
+    // Measured: the fast fixup below pays at N = 16, 32 and 256; at 48 to 128
+    // its code costs the producers registers (spills) and the kernel time.
+    constexpr bool kFastFixup = NB <= 32 || NB == 256;
+    auto epilogue = [&](int seg, int tile, bool final_seg) {
       const int db = seg % NACC;
-      ok = tc::mbar_wait_or_abort(dfull(db), (seg / NACC) & 1, kWaitLimit, abort_flag) && ok;
-      tc::fence_after_sync();
       const int gr = tile * kTileM + row;
       const int first = unit_owner((long long)tile * g.nchunks, g.units, ctas);
       const int last = unit_owner((long long)(tile + 1) * g.nchunks - 1, g.units, ctas);
@@ -501,6 +554,61 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       SEEDLM_CHECK_ONLY(const size_t y_n = (size_t)g.M * g.rows;
                         const size_t part_n = (size_t)ctas * g.segs_max * (NB * kTileM);
                         const size_t mine_off = ((size_t)blockIdx.x * g.segs_max + seg) * (NB * kTileM);)
+      // The CTA's last segment, when it starts the tile and other CTAs finish
+      // it: they began with it, so they have usually counted their partials
+      // long before.  If all of them have, this CTA adds the partials straight
+      // away, its own first and from TMEM (no later segment reuses the
+      // accumulator), and neither writes its own partial nor waits for that
+      // write.  Same sum, in the same CTA order, as the general path below.
+      if (kFastFixup && final_seg && first != last && first == (int)blockIdx.x) {
+        if (leader) {
+          const bool all_in = SEEDLM_IN_BOUNDS(g_check_flag, tile, g.tiles) &&
+                              atomicAdd(&counters[tile], 0u) == (unsigned)(last - first);
+          if (all_in) __threadfence();
+          slot[1] = all_in ? 1u : 0u;
+        }
+        tc::named_sync(128);
+        const bool all_in = slot[1] != 0u;
+        tc::named_sync(128);  // slot[1] is rewritten below
+        if (all_in) {
+          ok = tc::mbar_wait_or_abort(dfull(db), (seg / NACC) & 1, kWaitLimit, abort_flag) && ok;
+          tc::fence_after_sync();
+#pragma unroll 1
+          for (int n16 = 0; n16 < NB / 16; ++n16) {
+            float v[16];
+            tc::tmem_ld16(tmem + ((uint32_t)(32 * eq) << 16) + L::D_COL + ACC * db + 16 * n16, v);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float2 f = ys[16 * n16 + q];
+              v[q] = v[q] * f.x * f.y;
+            }
+            // Every later CTA of the tile starts inside it: the tile is its
+            // segment 0.
+#pragma unroll 1
+            for (int c = first + 1; c <= last; ++c) {
+              const size_t off = (size_t)c * g.segs_max * (NB * kTileM) + (size_t)(16 * n16) * kTileM + row;
+              const bool in = SEEDLM_IN_BOUNDS(g_check_flag, off + 15 * kTileM, part_n);
+              const float* p = partial + (in ? off : 0);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) v[q] += __ldcg(p + q * kTileM);
+            }
+            if (gr < g.rows) {
+#pragma unroll
+              for (int q = 0; q < 16; ++q)
+                if (16 * n16 + q < g.M &&
+                    SEEDLM_IN_BOUNDS(g_check_flag, (size_t)(16 * n16 + q) * g.rows + gr, y_n))
+                  Y[(size_t)(16 * n16 + q) * g.rows + gr] = v[q];
+            }
+          }
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(dfree(db));
+          if (leader && SEEDLM_IN_BOUNDS(g_check_flag, tile, g.tiles)) counters[tile] = 0u;
+          return;
+        }
+      }
+      ok = tc::mbar_wait_or_abort(dfull(db), (seg / NACC) & 1, kWaitLimit, abort_flag) && ok;
+      tc::fence_after_sync();
 #pragma unroll(NB > 64 ? 2 : 4)
       for (int n16 = 0; n16 < NB / 16; ++n16) {
         float v[16];
@@ -580,46 +688,9 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
     UnitCursor ec = c0;
     int seg = 0;
     for (int i = 0; i < n_units; ++i, ec.next(g.nchunks))
-      if (i == n_units - 1 || ec.chunk == g.nchunks - 1) epilogue(seg++, ec.tile);
+      if (i == n_units - 1 || ec.chunk == g.nchunks - 1) epilogue(seg++, ec.tile, i == n_units - 1);
   } else {
     // ------------------------------------------------ producers
-    const int lq = warp & 3, kq = warp >> 2;
-    const int prow = 32 * lq + lane;  // TMEM lane = row in the tile
-    const uint32_t lane4 = (uint32_t)lane << 2, lane8 = (uint32_t)(lane & 15) << 3;
-    const float2 neg1 = make_float2(-1.f, -1.f);
-    auto load_rec = [&](const UnitCursor& u, RecUnit<C>& p) {
-      const int gr = u.tile * kTileM + prow;
-      const int b0 = u.chunk * (KC / C) + kq * BPT;  // a multiple of BPT
-      // The thread's last record and its exponent byte lie inside row gr.
-      const bool ok_ = gr < g.rows && b0 < g.nb &&
-                       SEEDLM_IN_BOUNDS(g_check_flag, b0 + BPT - 1, g.rec_pitch) &&
-                       (C == 8 || SEEDLM_IN_BOUNDS(g_check_flag, b0 >> 1, g.e_pitch));
-      const uint32_t* src = rec + (size_t)gr * g.rec_pitch + b0;
-      // b0 is a multiple of BPT, so each load is aligned to its width.
-      if constexpr (C == 8 && BPT == 4) {
-        const uint4 v = ok_ ? ld_stream_u4(src) : make_uint4(0u, 0u, 0u, 0u);
-        p.r[0] = v.x; p.r[1] = v.y; p.r[2] = v.z; p.r[3] = v.w;
-        p.e = 0;
-      } else if constexpr (C == 8) {
-        static_assert(BPT == 2, "C = 8 takes two or four blocks per thread");
-        const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
-        p.r[0] = v.x; p.r[1] = v.y;
-        p.e = 0;
-      } else if constexpr (BPT == 2) {
-        // b0 is even: one 8-byte load; the exponent byte holds block b0 in
-        // its low nibble and b0 + 1 in its high nibble.
-        const uint2 v = ok_ ? ld_stream_u2(src) : make_uint2(0u, 0u);
-        p.r[0] = v.x; p.r[1] = v.y;
-        p.e = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
-      } else {
-        // One block: a 4-byte load, the exponent from the nibble of b0's parity.
-        static_assert(BPT == 1, "C = 12 takes one or two blocks per thread");
-        p.r[0] = ok_ ? ld_stream_u1(src) : 0u;
-        const uint32_t eb = ok_ ? (uint32_t)ld_stream_u8(eplane + (size_t)gr * g.e_pitch + (b0 >> 1)) : 0u;
-        p.e = eb >> (4 * (b0 & 1));
-      }
-    };
-
     auto produce = [&](int i, const RecUnit<C>& cur) {
       const int as = i % AS;
       if (i >= AS) ok = tc::mbar_wait_or_abort(afree(as), ((i / AS) - 1) & 1, kWaitLimit, abort_flag) && ok;
@@ -681,14 +752,6 @@ gemm_tc_kernel(const uint32_t* __restrict__ rec, const uint8_t* __restrict__ epl
       if (lane == 0) tc::mbar_arrive(afull(as));
     };
 
-    RecUnit<C> ring[kRecAhead];
-    UnitCursor rc = c0;  // next unit whose records are loaded
-#pragma unroll
-    for (int k = 0; k < kRecAhead; ++k)
-      if (k < n_units) {
-        load_rec(rc, ring[k]);
-        rc.next(g.nchunks);
-      }
     for (int i0 = 0; i0 < n_units; i0 += kRecAhead) {
 #pragma unroll
       for (int k = 0; k < kRecAhead; ++k) {
