@@ -74,6 +74,7 @@
 //   stage_x_kernel.  The producers read only the records, which the kernel
 //   before stage_x_kernel (a plain launch, so fully finished) may have
 //   written; the X slabs and scale factors are read after griddepcontrol.wait.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -199,27 +200,50 @@ __device__ __forceinline__ uint32_t finite_mag2(uint32_t v) {
 
 // One CTA per (row n of the padded batch, column part).  Writes the row's
 // fp16 slab entries for its part (zeros past M rows and past cols) and, part
-// 0, the row's output scale factors (f1, f2): Y = (acc * f1) * f2.
+// 0, the row's output scale factors (f1, f2): Y = (acc * f1) * f2.  bf16 X
+// needs the row's largest magnitude: every CTA reads the whole row for it,
+// or, when the row's parts form a thread-block cluster (`clustered`), each
+// CTA takes the maximum over its own part and reads the others' from their
+// shared memory, so the row is read once (without: 51 MB and ~10 us for 64
+// rows of 28672 columns in 14 parts).
 template <int KC, int NB>
 __global__ void __launch_bounds__(256)
 stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks, int is_bf16,
-               int parts, int vec, unsigned char* __restrict__ Xs, float2* __restrict__ yscale) {
+               int clustered, int parts, int vec, unsigned char* __restrict__ Xs,
+               float2* __restrict__ yscale) {
   // The GEMM may start its prologue at once; it reads Xs and yscale only after
   // griddepcontrol.wait, i.e. after this grid has finished.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ uint32_t red[8];
+  __shared__ uint32_t part_max;
   const int n = blockIdx.x / parts, part = blockIdx.x - n * parts;
   const uint16_t* row = X + (size_t)n * cols;
+  const int groups = nchunks * (KC / 8);  // 8-column groups of the padded row
+  const int g0 = (int)((long long)part * groups / parts);
+  const int g1e = (int)((long long)(part + 1) * groups / parts);
   int s = 0;  // x is stored as x * 2^s
-  if (is_bf16 && n < M) {
+  if (is_bf16) {
+    namespace cg = cooperative_groups;
+    // The maximum over this CTA's own part when the row's parts form a
+    // cluster, else over the whole row.
     uint32_t m = 0;
-    if (vec) {
+    if (n < M && clustered) {
+      for (int gi = g0 + threadIdx.x; gi < g1e; gi += blockDim.x) {
+        const int col = 8 * gi;
+        if (vec && col + 8 <= cols) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + col));
+          m = max(m, max(max(finite_mag2(v.x), finite_mag2(v.y)), max(finite_mag2(v.z), finite_mag2(v.w))));
+        } else {
+          for (int u = 0; u < 8 && col + u < cols; ++u) m = max(m, finite_mag2(row[col + u]));
+        }
+      }
+    } else if (n < M && vec) {
       const uint4* r4 = reinterpret_cast<const uint4*>(row);
       for (int i = threadIdx.x; i < cols / 8; i += blockDim.x) {
         const uint4 v = __ldg(r4 + i);
         m = max(m, max(max(finite_mag2(v.x), finite_mag2(v.y)), max(finite_mag2(v.z), finite_mag2(v.w))));
       }
-    } else {
+    } else if (n < M) {
       for (int k = threadIdx.x; k < cols; k += blockDim.x) m = max(m, finite_mag2(row[k]));
     }
     m = __reduce_max_sync(0xffffffffu, m);
@@ -228,6 +252,12 @@ stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks, int
     m = red[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) m = max(m, red[w]);
+    if (clustered) {
+      const cg::cluster_group cluster = cg::this_cluster();
+      if (threadIdx.x == 0) part_max = m;
+      cluster.sync();  // every part's maximum is in its CTA's shared memory
+      for (int r = 0; r < parts; ++r) m = max(m, *cluster.map_shared_rank(&part_max, r));
+    }
     if (m) {
       const int E = max((int)(m >> 7), 1) - 127;  // the largest has its leading bit at or below 2^E
       s = 15 - E;                                 // -112 <= s <= 141
@@ -237,9 +267,6 @@ stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks, int
   if (part == 0 && threadIdx.x == 0)
     yscale[n] = make_float2(exp2i(-(kShift + s1)), exp2i(-s2));
   const float g1 = exp2i(s1), g2 = exp2i(s2);
-  const int groups = nchunks * (KC / 8);  // 8-column groups of the padded row
-  const int g0 = (int)((long long)part * groups / parts);
-  const int g1e = (int)((long long)(part + 1) * groups / parts);
   for (int gi = g0 + threadIdx.x; gi < g1e; gi += blockDim.x) {
     const int col = 8 * gi;
     uint16_t h[8];
@@ -269,6 +296,8 @@ stage_x_kernel(const uint16_t* __restrict__ X, int M, int cols, int nchunks, int
     if (SEEDLM_IN_BOUNDS(g_check_flag, xb + 15, (size_t)nchunks * (NB * KC * 2)))
       *reinterpret_cast<uint4*>(Xs + xb) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  // No CTA of the cluster leaves while another may still read its maximum.
+  if (is_bf16 && clustered) cooperative_groups::this_cluster().sync();
 }
 
 __device__ __forceinline__ long long unit_begin(int cta, long long units, int ctas) {
@@ -841,12 +870,34 @@ int launch_tc(const TcGeom& g, int ctas, const uint32_t* rec, const uint8_t* epl
   unsigned char* xs = ws + w.cnt_bytes + w.scale_bytes;
   float* partial = reinterpret_cast<float*>(ws + w.cnt_bytes + w.scale_bytes + w.xs_bytes);
 
-  // stage_x: NB rows x parts CTAs, about 256 column groups of 8 per CTA.
+  // stage_x: NB rows x parts CTAs, about 256 column groups of 8 per CTA (at
+  // most 64 parts).  For bf16 X every CTA reads its whole row for the
+  // maximum unless the row's parts form a cluster; measured, the cluster
+  // pays from 5 parts on (8192 x 28672, M = 64: 140 -> 135 us) and costs
+  // about 1 us below (28672 x 8192, 4 parts), so wide rows take clusters of
+  // up to 8 parts (the portable size) and the rest the plain launch.
   const int groups = g.nchunks * (L::KC / 8);
-  const int parts = groups / 256 < 1 ? 1 : (groups / 256 > 64 ? 64 : groups / 256);
+  int parts = groups / 256 < 1 ? 1 : (groups / 256 > 64 ? 64 : groups / 256);
+  const bool cluster = is_bf16 && parts > 4;
+  if (cluster && parts > 8) parts = 8;
   const int vec = (reinterpret_cast<uintptr_t>(X) % 16 == 0) && (g.cols % 8 == 0);
-  stage_x_kernel<L::KC, NB><<<NB * parts, 256, 0, stream>>>(X, g.M, g.cols, g.nchunks, is_bf16,
-                                                             parts, vec, xs, yscale);
+  {
+    cudaLaunchConfig_t scfg = {};
+    scfg.gridDim = dim3(NB * parts);
+    scfg.blockDim = dim3(256);
+    scfg.stream = stream;
+    cudaLaunchAttribute sattr[1];
+    sattr[0].id = cudaLaunchAttributeClusterDimension;
+    sattr[0].val.clusterDim.x = cluster ? parts : 1;
+    sattr[0].val.clusterDim.y = 1;
+    sattr[0].val.clusterDim.z = 1;
+    scfg.attrs = sattr;
+    scfg.numAttrs = 1;
+    const cudaError_t serr = cudaLaunchKernelEx(&scfg, stage_x_kernel<L::KC, NB>, X, g.M, g.cols,
+                                                g.nchunks, is_bf16, (int)cluster, parts, vec, xs,
+                                                yscale);
+    if (serr != cudaSuccess) return record_cuda_error(serr);
+  }
   count_launch();
   if ((rc = record_cuda_error(cudaGetLastError()))) return rc;
 
