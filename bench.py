@@ -427,11 +427,11 @@ def extras(torch, sl, args):
                                   ep=None if base["ep"] is None else base["ep"].clone())
                              for _ in range(ncp - 1)]
             f = sl.Format.from_dict(base["fmt"])
-            # bf16 activations (staged as fp16 with a power-of-two scale per
-            # row) at every M, fp16 at M = 16 and 64; both meet two fp16
-            # pieces of W.
-            for M, dt in ((1, "bf16"), (8, "bf16"), (16, "bf16"), (64, "bf16"), (16, "f16"),
-                          (64, "f16")):
+            # bf16 activations at every M (M = 2 and 4 run on the CUDA cores;
+            # from M = 5 on the tensor cores take them as fp16 with a
+            # power-of-two scale per row), fp16 at M = 16 and 64.
+            for M, dt in ((1, "bf16"), (2, "bf16"), (4, "bf16"), (8, "bf16"), (16, "bf16"),
+                          (64, "bf16"), (16, "f16"), (64, "f16")):
                 Xb, _ = inputs.make_activations((M, N), dt, 950 + M)
                 X = torch.from_numpy(Xb.view(np.int16)).cuda().view(
                     torch.bfloat16 if dt == "bf16" else torch.float16)
@@ -475,14 +475,14 @@ def extras(torch, sl, args):
 
     # Dense fp16 reference for the crossover on the same shapes: the weights
     # as fp16 (2 bytes each), Y = X W^T through cuBLAS (torch.matmul, fp32
-    # accumulation) at M in {8, 16, 64} and the in-house dense GEMV at M = 1,
+    # accumulation) at M >= 2 and the in-house dense GEMV at M = 1,
     # rotating over copies totalling >= 4x L2.
     dense_mm = {}
     for name, R, N in (("up_28672x8192", 28672, 8192), ("down_8192x28672", 8192, 28672)):
         Wd = torch.randn((R, N), device="cuda", dtype=torch.float16) * 0.02
         ncp = max(2, math.ceil(4 * l2 / (Wd.numel() * 2)))
         Ws = [Wd] + [Wd.clone() for _ in range(ncp - 1)]
-        for M in ((1, 8, 16, 64, 128, 256, 1024) if name.startswith("up") else (1, 8, 16, 64)):
+        for M in ((1, 2, 4, 8, 16, 64, 128, 256, 1024) if name.startswith("up") else (1, 2, 4, 8, 16, 64)):
             X = torch.randn((M, N), device="cuda", dtype=torch.float16)
             if M == 1:
                 y = torch.empty(R, device="cuda")
@@ -617,7 +617,7 @@ def summarize(result, hbm_peak):
             out["llama3_8b_speedup_vs_dense_fp16"] = round(d8 / us8, 3)
     g = ex.get("gemm_smallM", {})
     dm = ex.get("dense_fp16_smallM", {})
-    for M in (8, 16, 64, 128, 256, 1024):
+    for M in (2, 4, 8, 16, 64, 128, 256, 1024):
         k = f"4bit/up_28672x8192/M={M}"
         if k in g:
             out[f"gemm_4bit_28672x8192_M{M}_us"] = g[k]["us_per_call"]

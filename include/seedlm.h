@@ -140,9 +140,12 @@ SEEDLM_API int seedlm_gemv_batch(int32_t n, const seedlm_format* fmts,
  * inference step of the paperhub.cn review thread (authors' reply on how
  * inference uses s and t: the blocks are rebuilt from seed and coefficients
  * and multiplied with the activations; a batch of M activation rows shares
- * every rebuilt block).  M = 1 runs the GEMV kernel; otherwise the rebuilt
- * weight tiles feed the tcgen05 tensor cores: kind::f16 MMAs on fp16
- * operands, W split exactly into two fp16 pieces of 2^6 W, fp32 accumulation
+ * every rebuilt block).  M = 1 runs the GEMV kernel; at 3 bits (C = 12,
+ * P = 4) M = 2 to 4 run its extension on the CUDA cores (each rebuilt
+ * weight pair feeds M packed fp32 FMAs; exact fp32 weights and
+ * activations, the GEMV's accuracy; no workspace is used, so `workspace`
+ * may then be NULL).  Otherwise the rebuilt weight tiles feed the tcgen05
+ * tensor cores: kind::f16 MMAs on fp16 operands, W split exactly into two fp16 pieces of 2^6 W, fp32 accumulation
  * in TMEM.  fp16 X is used as it is; bf16 X is scaled per row by a power of
  * two that brings the row's largest finite magnitude to [2^15, 2^16) and
  * stored as fp16, exact for every element of at least 2^-32 times that
@@ -162,17 +165,19 @@ SEEDLM_API int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec,
                        int64_t workspace_bytes, seedlm_stream stream);
 
 /* Workspace bytes seedlm_gemm_smallM needs for this format and M on the
- * current device (HOST function; 0 for an empty matrix or when M = 1 runs the
- * GEMV, negative on error). */
+ * current device (HOST function; 0 for an empty matrix, for M = 1 (the GEMV)
+ * and for M <= 4 at 3 bits (the CUDA-core kernel), negative on error). */
 SEEDLM_API int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M);
 
 /* Y = X W^T for any batch M >= 1 -- the same product as seedlm_gemm_smallM
  * (paperhub.cn review thread, authors' reply on how inference uses s and t),
  * extended to prefill-sized batches, where the rebuild of each weight tile is
  * shared by many rows of X.  X is M x cols (row-major, type x_dtype), Y is
- * M x rows fp32 (row-major).  M = 1 runs the GEMV; otherwise the rows of X
- * go through the tensor-core kernel of seedlm_gemm_smallM (same operand
- * precision) in passes of at most 256 rows, one after the other on the
+ * M x rows fp32 (row-major).  M = 1, and M <= 4 at 3 bits, run as in
+ * seedlm_gemm_smallM (the GEMV or its CUDA-core extension); otherwise the
+ * rows of X go through the
+ * tensor-core kernel of seedlm_gemm_smallM (same operand precision) in
+ * passes of at most 256 rows, one after the other on the
  * stream: up to 64 rows per MMA as there, 65-128 rows as one N = 128 pass,
  * 129-256 as one N = 256 pass (units of 64 columns at 4 bits, 48 at 3 bits,
  * one accumulator in TMEM).  For M <= 64 the result is the one
@@ -184,8 +189,8 @@ SEEDLM_API int seedlm_gemm(const seedlm_format* fmt, const uint32_t* rec, const 
                            int64_t workspace_bytes, seedlm_stream stream);
 
 /* Workspace bytes seedlm_gemm needs for this format and M on the current
- * device (HOST function; 0 for an empty matrix or when M = 1 runs the GEMV,
- * negative on error). */
+ * device (HOST function; 0 for an empty matrix, for M = 1 (the GEMV) and for
+ * M <= 4 at 3 bits (the CUDA-core kernel), negative on error). */
 SEEDLM_API int64_t seedlm_gemm_workspace_bytes(const seedlm_format* fmt, int M);
 
 /* Same result as seedlm_gemm_smallM, for callers that cannot allocate device

@@ -103,6 +103,7 @@ namespace {
 // Workspace of seedlm_gemm: the larger of a full pass and the last pass.
 int64_t gemm_any_workspace(const seedlm_format& f, int M, const DeviceInfo& dev) {
   if (M == 1 && gemv_smem_bytes(f, dev) > 0) return 0;  // the GEMV
+  if (gemm_cc_applies(f, M)) return 0;                  // the CUDA-core kernel
   const int full = M < kGemmPassRows ? M : kGemmPassRows;
   int64_t need = gemm_tc_workspace_bytes(f, full, dev);
   const int last = M % kGemmPassRows;
@@ -210,10 +211,14 @@ int seedlm_gemm_smallM(const seedlm_format* fmt, const uint32_t* rec, const uint
     return record_cuda_error(
         cudaMemsetAsync(Y, 0, (size_t)M * fmt->rows * sizeof(float), (cudaStream_t)stream));
   const uint16_t* Xh = static_cast<const uint16_t*>(X);
-  // M = 1 runs the GEMV unless x is too wide for its shared memory.
+  // M = 1 runs the GEMV unless x is too wide for its shared memory, 2 to 4
+  // rows the CUDA-core kernel, more rows the tensor cores.
   if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0)
     return launch_gemv(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, Y, (cudaStream_t)stream,
                        dev);
+  if (gemm_cc_applies(*fmt, M))
+    return launch_gemm_cc(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, M, Y, (cudaStream_t)stream,
+                          dev);
   return launch_gemm_tc(*fmt, rec, eplane, Xh, x_dtype == SEEDLM_BF16, M, Y, workspace,
                         workspace_bytes, (cudaStream_t)stream, dev);
 }
@@ -225,6 +230,7 @@ int64_t seedlm_gemm_smallM_workspace_bytes(const seedlm_format* fmt, int M) {
   int rc = device_info(&dev);
   if (rc) return rc;
   if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0) return 0;  // the GEMV
+  if (gemm_cc_applies(*fmt, M)) return 0;                  // the CUDA-core kernel
   return gemm_tc_workspace_bytes(*fmt, M, dev);
 }
 
@@ -248,6 +254,7 @@ int seedlm_gemm(const seedlm_format* fmt, const uint32_t* rec, const uint8_t* ep
   const int is_bf16 = x_dtype == SEEDLM_BF16;
   if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0)
     return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
+  if (gemm_cc_applies(*fmt, M)) return launch_gemm_cc(*fmt, rec, eplane, Xh, is_bf16, M, Y, st, dev);
   if (workspace_bytes < gemm_any_workspace(*fmt, M, dev)) return SEEDLM_EINVAL;
   // Passes of up to kGemmPassRows rows of X, one after the other on the
   // stream, sharing the workspace (each pass leaves its counters at zero).
@@ -310,10 +317,12 @@ int seedlm_device_error(int* flag) {
   if (v) out |= 1;
   if ((rc = read_and_clear_gemv_error(&v))) return rc;
   if (v) out |= 1;
+  if ((rc = read_and_clear_cc_error(&v))) return rc;
+  if (v) out |= 1;
   // Bounds violations recorded by a checked build (always 0 otherwise).
   int (*const readers[])(unsigned int*) = {read_and_clear_check_gemv, read_and_clear_check_decompress,
                                            read_and_clear_check_gemm_tc, read_and_clear_check_encode,
-                                           read_and_clear_check_dense};
+                                           read_and_clear_check_dense, read_and_clear_check_gemm_cc};
   for (auto read : readers) {
     unsigned int c = 0;
     if ((rc = read(&c))) return rc;

@@ -1086,6 +1086,7 @@ extern "C" SEEDLM_API int seedlm_gemm_smallM_noalloc(const seedlm_format* fmt,
   const int is_bf16 = x_dtype == SEEDLM_BF16;
   if (M == 1 && gemv_smem_bytes(*fmt, dev) > 0)
     return launch_gemv(*fmt, rec, eplane, Xh, is_bf16, Y, st, dev);
+  if (gemm_cc_applies(*fmt, M)) return launch_gemm_cc(*fmt, rec, eplane, Xh, is_bf16, M, Y, st, dev);
 
   int ctas = 1;
   const TcGeom g = make_tc_geom(*fmt, M, dev, &ctas);

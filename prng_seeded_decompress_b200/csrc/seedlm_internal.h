@@ -57,6 +57,7 @@ int read_and_clear_check_decompress(unsigned int* out);
 int read_and_clear_check_gemm_tc(unsigned int* out);
 int read_and_clear_check_encode(unsigned int* out);
 int read_and_clear_check_dense(unsigned int* out);
+int read_and_clear_check_gemm_cc(unsigned int* out);
 
 struct DeviceInfo {
   int device;
@@ -106,6 +107,14 @@ int launch_gemm_tc(const seedlm_format& f, const uint32_t* rec, const uint8_t* e
                    const uint16_t* X, int is_bf16, int M, float* Y, void* workspace,
                    int64_t workspace_bytes, cudaStream_t stream, const DeviceInfo& dev);
 int read_and_clear_tc_error(unsigned int* out);
+// 2 <= M <= kGemmCcMaxRows rows of X run on the CUDA cores (gemm_cc.cu): the
+// rebuilt weights feed M packed FMAs each, with no workspace.
+constexpr int kGemmCcMaxRows = 4;
+bool gemm_cc_applies(const seedlm_format& f, int M);
+int launch_gemm_cc(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
+                   const uint16_t* X, int is_bf16, int M, float* Y, cudaStream_t stream,
+                   const DeviceInfo& dev);
+int read_and_clear_cc_error(unsigned int* out);
 int read_and_clear_encode_error(unsigned int* out);
 int launch_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 int launch_bounds_check(int64_t index, int64_t extent, cudaStream_t stream);

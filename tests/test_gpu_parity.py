@@ -279,7 +279,7 @@ def gpu_gemm(sl, L, Xb, dtype="bf16", workspace=None):
 
 
 @pytest.mark.parametrize("cp", [C8, C12])
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 17, 33, 64])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 16, 17, 33, 64])
 def test_gemm_small_matches_oracle(sl, oracle_mod, cp, M):
     rows, cols = 300, 3000  # 3 row tiles (one ragged), ragged last stage, split-K
     L = inputs.make_layer(rows, cols, *cp, seed=50 + M)
@@ -336,6 +336,77 @@ def test_gemm_bf16_rows_of_any_magnitude(sl, oracle_mod, cp):
     assert np.array_equal(got[2], np.zeros(rows))
     for m in range(6):
         # No absolute floor: the bound scales with the row.
+        err = np.abs(got[m] - ref[m])
+        assert np.all(err <= TOL * refabs[m]), (m, float((err / (refabs[m] + 1e-300)).max()))
+
+
+@pytest.mark.parametrize("M", [2, 3, 4])
+def test_gemm_few_rows_on_cuda_cores_match_oracle(sl, oracle_mod, M):
+    # 2 to 4 rows of X at 3 bits run on the CUDA cores: rows not a multiple
+    # of the item height, columns not a multiple of C, x wider than one
+    # shared-memory segment (12,000 columns), a single block, fp16 and bf16;
+    # no workspace.
+    cp = C12
+    assert sl.gemm_workspace_bytes(inputs.make_format(300, 5000, *cp), M) == 0
+    assert sl.gemm_any_workspace_bytes(inputs.make_format(300, 5000, *cp), M) == 0
+    assert sl.gemm_workspace_bytes(inputs.make_format(300, 5000, *C8), M) > 0  # tensor cores
+    for rows, cols, dt in ((301, 12000, "bf16"), (37, 100, "f16"), (5, 12, "bf16"), (2, 9, "f16")):
+        L = inputs.make_layer(rows, cols, *cp, seed=900 + rows + M)
+        Xb, Xv = inputs.make_activations((M, cols), dt, 901 + cols + M)
+        rec, ep = planes(L)
+        X = act_tensor(Xb, dt)
+        Y = torch.full((M, rows), float("nan"), device="cuda")
+        sl.gemm_smallM(L["fmt"], rec, ep, X, Y, workspace=torch.zeros(0, dtype=torch.uint8, device="cuda"))
+        torch.cuda.synchronize()
+        assert sl.device_error() == 0
+        got = Y.cpu().numpy().astype(np.float64)
+        ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv)
+        for m in range(M):
+            assert_within(got[m], ref[m], refabs[m])
+
+
+@pytest.mark.parametrize("cp,rows,cols,M", [(C8, 28672, 8192, 4), (C8, 8192, 28672, 2),
+                                            (C12, 28672, 8192, 3), (C12, 8192, 28672, 4)])
+def test_gemm_few_rows_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols, M):
+    # Full 70B MLP shapes: several partial-sum passes per CTA (28672 rows)
+    # and several x segments (28672 columns); the same call twice gives the
+    # same bits (sums in a fixed order).
+    L = inputs.make_layer(rows, cols, *cp, seed=rows + cols + 7 * M)
+    Xb, Xv = inputs.make_activations((M, cols), "bf16", 93 + M)
+    got = gpu_gemm(sl, L, Xb)
+    again = gpu_gemm(sl, L, Xb)
+    assert np.array_equal(got.view(np.uint64), again.view(np.uint64))
+    rng = np.random.default_rng(3)
+    sample = np.unique(np.concatenate([np.arange(4), np.arange(rows - 4, rows),
+                                       rng.integers(0, rows, 12)]))
+    ref, refabs = oracle_mod.gemm_rows(L["fmt"], L["rec"], L["eplane"], Xv, sample)
+    for m in range(M):
+        assert_within(got[m, sample], ref[m], refabs[m])
+
+
+@pytest.mark.parametrize("cp", [C8, C12])
+def test_gemm_bf16_wide_rows_share_their_maximum(sl, oracle_mod, cp):
+    # Rows wide enough (28672 columns) that the staging kernel splits each
+    # row over several CTAs which exchange their parts' maxima: the row's
+    # largest element sits in the first, a middle or the last part, or the
+    # row spans 2^40; every part must scale by the one row-wide power of two.
+    rows, cols = 200, 28672
+    L = inputs.make_layer(rows, cols, *cp, seed=406)
+    rng = np.random.default_rng(407)
+    v = (rng.standard_normal((6, cols)) * 1e-3).astype(np.float32)
+    v[0, 5] = np.float32(3e4)             # maximum in the first part
+    v[1, cols // 2 + 3] = np.float32(3e4)  # ... in a middle part
+    v[2, cols - 2] = np.float32(3e4)       # ... in the last part
+    v[3] *= np.float32(1e-33)              # the whole row far below 1
+    v[3, cols - 9] = np.float32(2e-30)
+    v[4] = 0.0
+    v[5, cols - 1] = np.float32(1e9)       # 2^40 above the rest, last column
+    Xb = inputs.f32_to_bf16_bits(v)
+    Xv = inputs.bf16_bits_to_f64(Xb)
+    got = gpu_gemm(sl, L, Xb)
+    ref, refabs = oracle_mod.gemm(L["fmt"], L["rec"], L["eplane"], Xv, threads=os.cpu_count() or 1)
+    assert np.array_equal(got[4], np.zeros(rows))
+    for m in range(6):
         err = np.abs(got[m] - ref[m])
         assert np.all(err <= TOL * refabs[m]), (m, float((err / (refabs[m] + 1e-300)).max()))
 
