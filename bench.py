@@ -905,6 +905,17 @@ def profile_case(name: str):
         ws = sl.gemm_workspace(L["fmt"], M)
         for _ in range(3):
             sl.gemm_smallM(L["fmt"], rec, None, X, Y, workspace=ws)
+    elif name == "gemm3x2":
+        # 2 rows of X at 3 bits (the CUDA-core kernel), 28672 x 8192, three
+        # calls (capture with -s 1 -c 1).
+        L = inputs.make_layer(28672, 8192, 12, 4, seed=4)
+        rec = torch.from_numpy(L["rec"].view(np.int32)).cuda()
+        ep = torch.from_numpy(L["eplane"]).cuda()
+        Xb, _ = inputs.make_activations((2, 8192), "bf16", 5)
+        X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+        Y = torch.empty((2, 28672), device="cuda")
+        for _ in range(3):
+            sl.gemm_smallM(L["fmt"], rec, ep, X, Y)
     elif name in ("gemv", "gemv-cycle"):
         # The four GEMVs of one 4-bit Llama-3-70B layer, twice (the first
         # round warms up; capture with -s 4 -c 4).  "gemv-cycle" stores each
@@ -979,7 +990,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
-    ap.add_argument("--case", choices=("gemv", "gemv3", "gemv-cycle", "decompress", "gemm64",
+    ap.add_argument("--case", choices=("gemv", "gemv3", "gemv-cycle", "decompress", "gemm64", "gemm3x2",
                                        "gemm16", "dense", "encode"),
                     help="run one small single-kernel workload (for ncu) and exit")
     args = ap.parse_args()
