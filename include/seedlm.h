@@ -106,7 +106,10 @@ SEEDLM_API int seedlm_decompress(const seedlm_format* fmt, const uint32_t* rec, 
  * SEEDLM_BF16); y: rows fp32.  The blocks are rebuilt on the fly and never
  * written out (paperhub.cn thread, authors' replies on inference and on the
  * custom decoding that avoids full-precision weights in memory).  Any width:
- * x is staged in shared memory as fp32 one column segment at a time.  The
+ * x is staged in shared memory as fp32 one column segment at a time.  Tall
+ * 3-bit matrices (128 to 256 rows per SM) take a kernel that builds tables
+ * of x's contribution per column block once per CTA and shares them across
+ * its rows (same tolerance, a different fp32 summation order).  The
  * kernel is launched with programmatic dependent launch; it reads the
  * records and x only after waiting for the previous kernel in the stream,
  * so that kernel may write them (for example seedlm_encode, or a copy). */

@@ -319,10 +319,13 @@ int seedlm_device_error(int* flag) {
   if (v) out |= 1;
   if ((rc = read_and_clear_cc_error(&v))) return rc;
   if (v) out |= 1;
+  if ((rc = read_and_clear_amort_error(&v))) return rc;
+  if (v) out |= 1;
   // Bounds violations recorded by a checked build (always 0 otherwise).
   int (*const readers[])(unsigned int*) = {read_and_clear_check_gemv, read_and_clear_check_decompress,
                                            read_and_clear_check_gemm_tc, read_and_clear_check_encode,
-                                           read_and_clear_check_dense, read_and_clear_check_gemm_cc};
+                                           read_and_clear_check_dense, read_and_clear_check_gemm_cc,
+                                           read_and_clear_check_gemv_amort};
   for (auto read : readers) {
     unsigned int c = 0;
     if ((rc = read(&c))) return rc;

@@ -900,6 +900,7 @@ int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* epla
                 const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
                 const DeviceInfo& dev) {
   if (f.rows == 0) return SEEDLM_OK;
+  if (gemv_amort_applies(f, dev)) return launch_gemv_amort(f, rec, eplane, x, is_bf16, y, stream, dev);
   const seedlm_format* fp = &f;
   return launch_gemv_batch(1, &fp, &rec, &eplane, &x, is_bf16, &y, stream, dev);
 }

@@ -58,6 +58,7 @@ int read_and_clear_check_gemm_tc(unsigned int* out);
 int read_and_clear_check_encode(unsigned int* out);
 int read_and_clear_check_dense(unsigned int* out);
 int read_and_clear_check_gemm_cc(unsigned int* out);
+int read_and_clear_check_gemv_amort(unsigned int* out);
 
 struct DeviceInfo {
   int device;
@@ -88,6 +89,14 @@ int allow_max_smem(const void* kernel, const DeviceInfo& dev);
 // Shared memory the GEMV kernel needs for f on dev (0: its tables do not fit).
 size_t gemv_smem_bytes(const seedlm_format& f, const DeviceInfo& dev);
 int read_and_clear_gemv_error(unsigned int* out);
+// Tall 3-bit matrices (at least 128 rows per SM, at most 256): the GEMV with
+// the x-dependent part of every block's dot taken from per-column-block
+// tables (gemv_amort.cu).
+bool gemv_amort_applies(const seedlm_format& f, const DeviceInfo& dev);
+int launch_gemv_amort(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
+                      const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
+                      const DeviceInfo& dev);
+int read_and_clear_amort_error(unsigned int* out);
 int launch_gemv(const seedlm_format& f, const uint32_t* rec, const uint8_t* eplane,
                 const uint16_t* x, int is_bf16, float* y, cudaStream_t stream,
                 const DeviceInfo& dev);

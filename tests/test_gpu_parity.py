@@ -238,6 +238,30 @@ def test_gemv_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols):
     assert_within(y[sample], ref, refabs)
 
 
+@pytest.mark.parametrize("rows,cols,dtype", [(19000, 1000, "bf16"), (37888, 385, "f16"),
+                                             (28672, 8192, "f16")])
+def test_gemv_tall_3bit_column_tables(sl, oracle_mod, rows, cols, dtype):
+    # Tall 3-bit matrices (128 to 256 rows per SM) take the column-table
+    # kernel: columns not a multiple of C, a last strip of 32 column blocks
+    # that is partly empty (1000 columns: 84 blocks; 385: 33), rows not a
+    # multiple of the 16 warps, the most rows per CTA it takes (37888), and
+    # the 3-bit MLP shape on sampled rows.  Two calls give the same bits.
+    L = inputs.make_layer(rows, cols, *C12, seed=rows + cols, e_range=(0, 15))
+    xb, xv = inputs.make_activations((cols,), dtype, 18)
+    y = gpu_gemv(sl, L, xb, dtype)
+    again = gpu_gemv(sl, L, xb, dtype)
+    assert np.array_equal(y.view(np.uint64), again.view(np.uint64))
+    if cols <= 1000:
+        ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv, threads=os.cpu_count() or 1)
+        assert_within(y, ref, refabs)
+    else:
+        rng = np.random.default_rng(4)
+        sample = np.unique(np.concatenate([np.arange(8), np.arange(rows - 8, rows),
+                                           rng.integers(0, rows, 48)]))
+        ref, refabs = oracle_mod.gemv_rows(L["fmt"], L["rec"], L["eplane"], xv, sample)
+        assert_within(y[sample], ref, refabs)
+
+
 @pytest.mark.parametrize("cp,rows,cols", [(C8, 100000, 16), (C12, 100000, 24),
                                           (C8, 1800, 56320), (C12, 6000, 42240)])
 def test_gemv_multi_pass_and_wide_x(sl, oracle_mod, cp, rows, cols):
