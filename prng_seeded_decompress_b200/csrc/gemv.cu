@@ -403,6 +403,27 @@ __device__ __forceinline__ void load_set(RecSet<C, V>& o, const uint32_t* __rest
   }
 }
 
+// Record words (32 MiB) from which a 4-bit GEMV prefetches its first record
+// sets into L2 before waiting for the previous kernel.
+constexpr int64_t kL2PrefetchMinWords = (int64_t)8 << 20;
+
+// L2 prefetch of the record lines load_set would read, for full groups and
+// spans only (the addresses the unchecked fast path of load_set reads).
+template <int C, int V>
+__device__ __forceinline__ void prefetch_set(const uint32_t* __restrict__ rec, const GemvGeom& g,
+                                             int grp, int span, int lane) {
+  if (grp >= g.full_groups || span >= g.full_spans) return;
+  constexpr int kSU = span_units<V>(), kBPL = Tune<C, V>::kBPL;
+  const int row0 = grp * rows_per_item<V>() + (lane / kSU) * kRowsPerTask;
+  const int u = span * kSU + lane % kSU;
+#pragma unroll
+  for (int j = 0; j < kRowsPerTask; ++j) {
+    const size_t w = (size_t)(row0 + j) * g.rec_pitch + kBPL * u;
+    if (SEEDLM_IN_BOUNDS(g_check_flag, w + kBPL - 1, (size_t)g.rows * g.rec_pitch))
+      prefetch_l2(rec + w);
+  }
+}
+
 #ifndef SEEDLM_GEMV_C12_ORDER
 #define SEEDLM_GEMV_C12_ORDER 1
 #endif
@@ -608,6 +629,26 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
   // the slower CTAs of this grid finish.  Every CTA of this grid is resident
   // before the trigger completes, so the early start cannot starve it.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (C == 8 && (int64_t)B.g[0].rows * B.g[0].rec_pitch >= kL2PrefetchMinWords) {
+    // The warp's first record sets of the first GEMV head for L2 while the
+    // tables are filled and the previous kernel finishes: after the wait
+    // they come from L2, not from DRAM.  Measured per launch: 0.4-1.7 us
+    // faster on 8192 x 8192 and larger, 0.1-0.7 us slower on smaller
+    // matrices (hence the size floor); at 3 bits (records and exponent
+    // bytes) 0.2-1 us slower.
+    const GemvGeom& g = B.g[0];
+    const int g0 = (int)((int64_t)blockIdx.x * g.groups / gridDim.x);
+    const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
+    const int sl = min(g.seg_spans, g.n_spans);
+    const int items = (min(g0 + g.pass_groups, g1) - g0) * sl;
+    const int i0 = (int)((int64_t)warp * items / nw);
+    const int i1 = (int)((int64_t)(warp + 1) * items / nw);
+    int grp = g0 + (sl > 0 ? i0 / sl : 0), span = sl > 0 ? i0 % sl : 0;
+    for (int k = 0; k < 2 * (kP + 1) && i0 + k < i1; ++k) {
+      prefetch_set<C, V>(B.rec[0], g, grp, span, lane);
+      if (++span == sl) { span = 0; ++grp; }
+    }
+  }
   fill_tables<C, V>(smem);
   // Records and x may be the previous kernel's output: read them only now.
   asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -134,6 +134,14 @@ __device__ __forceinline__ uint8_t ld_stream_u8(const uint8_t* p) {
   return (uint8_t)v;
 }
 
+// Prefetch of one line into L2, nothing returned to the thread.  It may be
+// issued before griddepcontrol.wait even for data the previous kernel writes:
+// the L2 is the point of coherence of the GPU's memory, so a write that lands
+// after the prefetch updates the line in L2, and no copy nearer the SM is made.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // --------------------------------------------------------- block decoding
 
 // Bit pattern of M_e = 1.5 * 2^(8-e) is 0x43C00000 - (e << 23).
