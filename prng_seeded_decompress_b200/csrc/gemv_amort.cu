@@ -17,11 +17,12 @@
 // 48 dp2a.  The tables depend on x only, so a CTA builds them once per strip
 // of 32 column blocks and every row it owns reuses them.
 //
-//   * Lane l of a warp takes column block 32s + l of strip s: its table
-//     entries sit in lane-replicated rows (row v holds entry v of the 32
-//     column blocks side by side, 128 bytes per table, two tables per
-//     256-byte row), so every lookup is one conflict-free wavefront and its
-//     address is one prmt of the stream byte next to the lane's offset.
+//   * Lane l of a warp takes column block 32s + l of strip s: the tables
+//     are interleaved by lane (row v holds entry v of the 32 column blocks
+//     side by side, 128 bytes per table, two tables per 256-byte row), so
+//     lane l always reads its own bank, every lookup is one conflict-free
+//     wavefront, and its address is one prmt of the stream byte next to the
+//     lane's offset.
 //     T0/T1 and T2/T3 take 64 KB each, the lane-replicated stream jump
 //     tables 64 more.
 //   * A CTA owns up to 256 consecutive rows; warp w takes rows w, w + 16, ...
