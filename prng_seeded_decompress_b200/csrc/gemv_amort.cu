@@ -7,12 +7,13 @@
 // the authors' reply on how inference uses s and t).  The dot of block b
 // with its 12 activations is linear in the block's stream bits:
 //
-//   sum_c x_c w_c = 2^-(15+e) (sum_p q_p S_p - 32768 (sum_p q_p) X),
-//   S_p = sum_c x_c state_{12p+c} = sum_{m=0..26} bit_{12p+m} X~_m,
-//   X~_m = sum_c x_c 2^(m-c) (0 <= m - c <= 15),  X = sum_c x_c,
+//   sum_c x_c w_c = 2^-e (sum_p q_p S_p - (sum_p q_p) X),
+//   S_p = 2^-15 sum_c x_c state_{12p+c} = sum_{m=0..26} bit_{12p+m} X~_m,
+//   X~_m = sum_c x_c 2^(m-c-15) (0 <= m - c <= 15),  X = sum_c x_c,
 //
-// where state_j is stream bits [j, j+16).  Cutting the 27 bits behind each
-// S_p into four bytes gives S_p = T0[B0] + T1[B1] + T2[B2] + T3[B3] with
+// where state_j is stream bits [j, j+16) (the 2^-15 keeps X~ within the
+// range of x: |X~_m| <= sum |x_c|).  Cutting the 27 bits behind each S_p into
+// four bytes gives S_p = T0[B0] + T1[B1] + T2[B2] + T3[B3] with
 // T_j[v] = sum_k bit_k(v) X~_{8j+k}: 16 table lookups per block instead of
 // 48 dp2a.  The tables depend on x only, so a CTA builds them once per strip
 // of 32 column blocks and every row it owns reuses them.
@@ -136,22 +137,22 @@ __device__ __forceinline__ void load_strip(StripIn& o, const uint32_t* __restric
 }
 
 // X~_m for m = 8J .. 8J+7 (zero past 26): the first from its definition,
-// the others by X~_m = 2 X~_{m-1} + x_m - 2^16 x_{m-16} (each x_c enters at
-// m = c and leaves past m = c + 15).
+// the others by X~_m = 2 X~_{m-1} + 2^-15 x_m - 2 x_{m-16} (each x_c enters
+// at m = c and leaves past m = c + 15).
 template <int J>
 __device__ __forceinline__ void x_tilde(const float (&xv)[12], float (&xt)[8]) {
   constexpr int m0 = 8 * J;
   float acc = 0.f;
 #pragma unroll
   for (int c = 0; c < 12; ++c)
-    if (m0 - c >= 0 && m0 - c <= 15) acc = fmaf(xv[c], (float)(1u << (m0 - c)), acc);
+    if (m0 - c >= 0 && m0 - c <= 15) acc = fmaf(xv[c], __uint_as_float((uint32_t)(112 + m0 - c) << 23), acc);
   xt[0] = acc;
 #pragma unroll
   for (int k = 1; k < 8; ++k) {
     const int m = m0 + k;
     float v = 2.f * xt[k - 1];
-    if (m < 12) v += xv[m < 12 ? m : 0];
-    if (m >= 16 && m - 16 < 12) v = fmaf(xv[m >= 16 && m - 16 < 12 ? m - 16 : 0], -65536.f, v);
+    if (m < 12) v = fmaf(xv[m < 12 ? m : 0], 0x1p-15f, v);
+    if (m >= 16 && m - 16 < 12) v = fmaf(xv[m >= 16 && m - 16 < 12 ? m - 16 : 0], -2.f, v);
     xt[k] = m <= 26 ? v : 0.f;
   }
 }
@@ -227,8 +228,8 @@ __device__ __forceinline__ float block_dot(uint32_t rec, uint32_t e4, float xsum
   d = fmaf(q1, S1, d);
   d = fmaf(q2, S2, d);
   d = fmaf(q3, S3, d);
-  d = fmaf(qs * -32768.f, xsum, d);
-  return __uint_as_float(0x38000000u - (e4 << 23)) * d;  // 2^-(15+e)
+  d = fmaf(-qs, xsum, d);
+  return __uint_as_float(0x3f800000u - (e4 << 23)) * d;  // 2^-e
 }
 
 __global__ void __launch_bounds__(kWarps * 32, 1)

@@ -263,6 +263,24 @@ def test_gemv_tall_3bit_column_tables(sl, oracle_mod, rows, cols, dtype):
         assert_within(y[sample], ref, refabs)
 
 
+@pytest.mark.parametrize("scale", [1e34, 1e-30])
+def test_gemv_tall_3bit_column_tables_extreme_activations(sl, oracle_mod, scale):
+    # The column tables hold x's partial sums scaled by 2^-15, so they stay
+    # within the range of x itself: bf16 activations near the top of the
+    # range (a 2^15 larger table entry would overflow fp32) and far below 1.
+    rows, cols = 18944, 300
+    L = inputs.make_layer(rows, cols, *C12, seed=77, e_range=(0, 15))
+    base = np.random.default_rng(78).standard_normal(cols).astype(np.float32)
+    xb = inputs.f32_to_bf16_bits((base * np.float32(scale)).astype(np.float32))
+    xv = inputs.bf16_bits_to_f64(xb)
+    assert np.all(np.isfinite(xv))
+    y = gpu_gemv(sl, L, xb, "bf16")
+    ref, refabs = oracle_mod.gemv(L["fmt"], L["rec"], L["eplane"], xv, threads=os.cpu_count() or 1)
+    assert np.all(np.isfinite(y))
+    err = np.abs(y - ref)
+    assert np.all(err <= TOL * refabs), float((err / (refabs + 1e-300)).max())
+
+
 @pytest.mark.parametrize("cp,rows,cols", [(C8, 100000, 16), (C12, 100000, 24),
                                           (C8, 1800, 56320), (C12, 6000, 42240)])
 def test_gemv_multi_pass_and_wide_x(sl, oracle_mod, cp, rows, cols):
