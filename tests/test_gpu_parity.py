@@ -263,13 +263,16 @@ def test_gemv_tall_3bit_column_tables(sl, oracle_mod, rows, cols, dtype):
         assert_within(y[sample], ref, refabs)
 
 
+@pytest.mark.parametrize("cp,rows", [(C12, 18944), (C12, 300), (C8, 300)])
 @pytest.mark.parametrize("scale", [1e34, 1e-30])
-def test_gemv_tall_3bit_column_tables_extreme_activations(sl, oracle_mod, scale):
-    # The column tables hold x's partial sums scaled by 2^-15, so they stay
-    # within the range of x itself: bf16 activations near the top of the
-    # range (a 2^15 larger table entry would overflow fp32) and far below 1.
-    rows, cols = 18944, 300
-    L = inputs.make_layer(rows, cols, *C12, seed=77, e_range=(0, 15))
+def test_gemv_extreme_activations(sl, oracle_mod, cp, rows, scale):
+    # bf16 activations near the top of the range and far below 1.  The
+    # column-table kernel (3 bits, 18944 rows) keeps x's partial sums scaled
+    # by 2^-15, within the range of x itself (a 2^15 larger table entry
+    # would overflow fp32); the per-row kernels multiply x by the weights
+    # themselves (at most P * 8 in magnitude).
+    cols = 300
+    L = inputs.make_layer(rows, cols, *cp, seed=77, e_range=(0, 15))
     base = np.random.default_rng(78).standard_normal(cols).astype(np.float32)
     xb = inputs.f32_to_bf16_bits((base * np.float32(scale)).astype(np.float32))
     xv = inputs.bf16_bits_to_f64(xb)
