@@ -659,10 +659,13 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
     // in registers across the loop it made the 4-bit batch kernel spill, and
     // every variant measured 0.3-0.8 us slower per launch.
     const GemvGeom& g = B.g[bi];
-    const uint32_t* __restrict__ rec = B.rec[bi];
-    const uint8_t* __restrict__ eplane = B.ep[bi];
-    const uint16_t* __restrict__ x = B.x[bi];
-    float* __restrict__ y = B.y[bi];
+    // One GEMV keeps its pointers in registers; a batch reads them from the
+    // parameter where used (each choice measured faster for its kind).
+    const uint32_t* __restrict__ rec_r = kBatch ? nullptr : B.rec[0];
+    const uint8_t* __restrict__ ep_r = kBatch ? nullptr : B.ep[0];
+    const uint16_t* __restrict__ x_r = kBatch ? nullptr : B.x[0];
+    float* __restrict__ y_r = kBatch ? nullptr : B.y[0];
+#define SEEDLM_PTR(reg, field) (kBatch ? B.field[bi] : reg)
     const int g0 = (int)((int64_t)blockIdx.x * g.groups / gridDim.x);
     const int g1 = (int)((int64_t)(blockIdx.x + 1) * g.groups / gridDim.x);
     for (int p0 = g0; p0 < g1; p0 += g.pass_groups) {
@@ -685,11 +688,11 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
         int lgrp = grp, lspan = span;
 #pragma unroll
         for (int k = 0; k <= kP; ++k) {
-          if (i0 + k < i1) load_set<C, V>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+          if (i0 + k < i1) load_set<C, V>(buf[k], SEEDLM_PTR(rec_r, rec), SEEDLM_PTR(ep_r, ep), g, lgrp, s0 + lspan, lane);
           if (++lspan == sl) { lspan = 0; ++lgrp; }
         }
         // One segment: x stays staged for every pass of this GEMV.
-        if (g.n_segs > 1 || p0 == g0) stage_x<C, V>(xs, x, is_bf16, g, s0, sl);
+        if (g.n_segs > 1 || p0 == g0) stage_x<C, V>(xs, SEEDLM_PTR(x_r, x), is_bf16, g, s0, sl);
         __syncthreads();  // x, tables and zeroed partials ready
         if (i0 < i1) {
           float2 acc[kRowsPerTask];
@@ -704,7 +707,7 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
               if (SEEDLM_IN_BOUNDS(g_check_flag, (ul + 1) * (Smem<C, V>::kSlotFloats) - 1, xs_floats))
                 rebuild_and_dot<C, V>(buf[k], xs, ul, lane, lane4, lane8, tabs, acc);
               if (ci + kP + 1 < i1) {
-                load_set<C, V>(buf[k], rec, eplane, g, lgrp, s0 + lspan, lane);
+                load_set<C, V>(buf[k], SEEDLM_PTR(rec_r, rec), SEEDLM_PTR(ep_r, ep), g, lgrp, s0 + lspan, lane);
                 if (++lspan == sl) { lspan = 0; ++lgrp; }
               }
               ++ci;
@@ -735,13 +738,15 @@ gemv_kernel(const __grid_constant__ GemvBatch B, int is_bf16) {
           float sum = 0.f;
           for (int w = 0; w < nw; ++w)
             if (SEEDLM_IN_BOUNDS(g_check_flag, w * pass_rows + t, part_floats)) sum += part[w * pass_rows + t];
-          if (SEEDLM_IN_BOUNDS(g_check_flag, r, g.rows)) y[r] = sum;
+          if (SEEDLM_IN_BOUNDS(g_check_flag, r, g.rows)) SEEDLM_PTR(y_r, y)[r] = sum;
         }
       }
       __syncthreads();  // partials read before the next pass clears them
     }
   }
 }
+
+#undef SEEDLM_PTR
 
 template <int C, int V>
 int warps_for(int items_per_cta) {
