@@ -239,14 +239,18 @@ def test_gemv_full_size_sampled_rows(sl, oracle_mod, cp, rows, cols):
 
 
 @pytest.mark.parametrize("rows,cols,dtype", [(19000, 1000, "bf16"), (37888, 385, "f16"),
-                                             (28672, 8192, "f16"), (18944, 7, "bf16")])
+                                             (28672, 8192, "f16"), (18944, 7, "bf16"),
+                                             (18796, 30, "f16"), (18797, 30, "f16"),
+                                             (37889, 30, "bf16")])
 def test_gemv_tall_3bit_column_tables(sl, oracle_mod, rows, cols, dtype):
     # Tall 3-bit matrices (128 to 256 rows per SM) take the column-table
     # kernel: columns not a multiple of C, a last strip of 32 column blocks
     # that is partly empty (1000 columns: 84 blocks; 385: 33), rows not a
     # multiple of the 16 warps, the most rows per CTA it takes (37888), the
-    # fewest (18944) with one 7-column block per row, and the 3-bit MLP
-    # shape on sampled rows.  Two calls give the same bits.
+    # fewest (18944) with one 7-column block per row, the 3-bit MLP shape on
+    # sampled rows, and both sides of the kernel choice on 148 SMs (18796
+    # rows: 127 per CTA, per-row kernel; 18797: 128; 37889: 257, per-row
+    # kernel again).  Two calls give the same bits.
     L = inputs.make_layer(rows, cols, *C12, seed=rows + cols, e_range=(0, 15))
     xb, xv = inputs.make_activations((cols,), dtype, 18)
     y = gpu_gemv(sl, L, xb, dtype)
